@@ -1,0 +1,211 @@
+"""CPU oracle for one Soft Anisotropic Diagrams fitting iteration.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` are the only callers.  The CUDA library never
+imports, links or runs anything here, and this package imports nothing from
+the CUDA library.
+
+Thin ctypes wrappers over ``sad_oracle.c`` (plain C, fp64 render / backward /
+Adam, fp32 top-K decisions).  Tables are (P, 8) uint32 arrays of site ids,
+images (3, H, W), site parameters (9, N) float32 planes in the order
+x, y, ln tau, r, cr, cg, cb, theta, a.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+SENTINEL = 0xFFFFFFFF
+K = 8
+REC = 16
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        c_int, c_i64, c_u32, c_dbl = ctypes.c_int, ctypes.c_int64, ctypes.c_uint32, ctypes.c_double
+        vp = ctypes.c_void_p
+        L.orc_records.argtypes = [c_int, c_int, c_int, vp, vp, vp]
+        L.orc_score32.argtypes = [vp, c_int, c_int, c_int]
+        L.orc_score32.restype = ctypes.c_float
+        L.orc_topk_exact.argtypes = [c_int, c_int, c_int, vp, vp, c_i64, vp]
+        L.orc_fmix32.argtypes = [c_u32]
+        L.orc_fmix32.restype = c_u32
+        L.orc_xorshift32.argtypes = [c_u32]
+        L.orc_xorshift32.restype = c_u32
+        L.orc_inject_ids.argtypes = [c_u32, c_u32, c_u32, c_int, c_int, vp]
+        L.orc_propagate.argtypes = [c_int, c_int, c_int, vp, vp, vp, c_int, c_int, c_u32, c_u32]
+        L.orc_seed.argtypes = [c_int, c_int, c_int, vp, vp]
+        L.orc_render.argtypes = [c_int, c_int, c_int, vp, vp, vp]
+        L.orc_weights.argtypes = [c_int, c_int, c_int, vp, vp, vp]
+        L.orc_loss_backward.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp]
+        L.orc_loss_backward.restype = c_dbl
+        L.orc_adam.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, c_dbl, c_dbl, c_dbl, c_int]
+        L.orc_num_threads.restype = c_int
+        L.orc_set_threads.argtypes = [c_int]
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _u32(a):
+    return np.ascontiguousarray(a, dtype=np.uint32)
+
+
+def num_threads() -> int:
+    return lib().orc_num_threads()
+
+
+def set_threads(n: int) -> None:
+    lib().orc_set_threads(int(n))
+
+
+def records(H: int, W: int, params: np.ndarray, with64: bool = False):
+    """Per-site score records (N, 16) float32 (and float64 if ``with64``)."""
+    params = _f32(params)
+    N = params.shape[1]
+    r32 = np.empty((N, REC), dtype=np.float32)
+    r64 = np.empty((N, REC), dtype=np.float64) if with64 else None
+    lib().orc_records(H, W, N, _p(params), _p(r32), _p(r64) if with64 else None)
+    return (r32, r64) if with64 else r32
+
+
+def score32(rec32: np.ndarray, site: int, i: int, j: int) -> float:
+    rec32 = _f32(rec32)
+    return float(lib().orc_score32(_p(rec32), int(site), int(i), int(j)))
+
+
+def topk_exact(H: int, W: int, rec32: np.ndarray, pixels: np.ndarray | None = None) -> np.ndarray:
+    """Brute-force top-8 over all active sites; (n_pix, 8) uint32."""
+    rec32 = _f32(rec32)
+    N = rec32.shape[0]
+    if pixels is None:
+        n = H * W
+        out = np.empty((n, K), dtype=np.uint32)
+        lib().orc_topk_exact(H, W, N, _p(rec32), None, n, _p(out))
+    else:
+        pix = np.ascontiguousarray(pixels, dtype=np.int64)
+        out = np.empty((pix.size, K), dtype=np.uint32)
+        lib().orc_topk_exact(H, W, N, _p(rec32), _p(pix), pix.size, _p(out))
+    return out
+
+
+def fmix32(h: int) -> int:
+    return int(lib().orc_fmix32(h & 0xFFFFFFFF))
+
+
+def xorshift32(h: int) -> int:
+    return int(lib().orc_xorshift32(h & 0xFFFFFFFF))
+
+
+def inject_ids(seed: int, pass_index: int, pixel: int, N: int, G: int) -> np.ndarray:
+    out = np.empty(max(G, 1), dtype=np.uint32)
+    lib().orc_inject_ids(seed & 0xFFFFFFFF, pass_index & 0xFFFFFFFF, pixel & 0xFFFFFFFF, N, G, _p(out))
+    return out[:G]
+
+
+def propagate(H: int, W: int, rec32: np.ndarray, table: np.ndarray, jump: int, G: int,
+              seed: int, pass_index: int) -> np.ndarray:
+    """One Jacobi propagation pass; returns the new (P, 8) table."""
+    rec32 = _f32(rec32)
+    tin = _u32(table).reshape(H * W, K)
+    tout = np.empty_like(tin)
+    lib().orc_propagate(H, W, rec32.shape[0], _p(rec32), _p(tin), _p(tout), int(jump), int(G),
+                        seed & 0xFFFFFFFF, pass_index & 0xFFFFFFFF)
+    return tout
+
+
+def seed_table(H: int, W: int, params: np.ndarray) -> np.ndarray:
+    params = _f32(params)
+    out = np.empty((H * W, K), dtype=np.uint32)
+    lib().orc_seed(H, W, params.shape[1], _p(params), _p(out))
+    return out
+
+
+def jump_schedule(H: int, W: int) -> list:
+    """B/2, B/4, ..., 1 with B the largest power of two <= max(H, W)."""
+    B = 1
+    while B * 2 <= max(H, W):
+        B *= 2
+    out = []
+    k = B // 2
+    while k >= 1:
+        out.append(k)
+        k //= 2
+    return out
+
+
+def refresh(H: int, W: int, params: np.ndarray, G: int, seed: int, first_pass: int = 0):
+    """Seed pass then one propagation pass per jump of ``jump_schedule``.
+    Returns (table, number of passes run)."""
+    rec = records(H, W, params)
+    t = seed_table(H, W, params)
+    n = 0
+    for k in jump_schedule(H, W):
+        t = propagate(H, W, rec, t, k, G, seed, first_pass + n)
+        n += 1
+    return t, n
+
+
+def render(H: int, W: int, params: np.ndarray, table: np.ndarray) -> np.ndarray:
+    params = _f32(params)
+    tab = _u32(table).reshape(H * W, K)
+    img = np.empty((3, H, W), dtype=np.float64)
+    lib().orc_render(H, W, params.shape[1], _p(params), _p(tab), _p(img))
+    return img
+
+
+def weights(H: int, W: int, params: np.ndarray, table: np.ndarray) -> np.ndarray:
+    params = _f32(params)
+    tab = _u32(table).reshape(H * W, K)
+    w = np.empty((H * W, K), dtype=np.float64)
+    lib().orc_weights(H, W, params.shape[1], _p(params), _p(tab), _p(w))
+    return w
+
+
+def loss_backward(H: int, W: int, params: np.ndarray, table: np.ndarray, target: np.ndarray,
+                  want_image: bool = False):
+    """Returns (loss, grads (9, N) float64[, image (3, H, W) float64])."""
+    params = _f32(params)
+    tab = _u32(table).reshape(H * W, K)
+    tgt = _f32(target).reshape(3, H * W)
+    N = params.shape[1]
+    g = np.empty((9, N), dtype=np.float64)
+    img = np.empty((3, H, W), dtype=np.float64) if want_image else None
+    L = lib().orc_loss_backward(H, W, N, _p(params), _p(tab), _p(tgt), _p(g),
+                                _p(img) if want_image else None)
+    return (L, g, img) if want_image else (L, g)
+
+
+ADAM_PLANE_GROUP = ("pos", "pos", "log_tau", "r", "color", "color", "color", "theta", "a")
+
+
+def adam(H: int, W: int, params, m, v, grads, lr, t: int, b1: float = 0.9, b2: float = 0.999,
+         eps: float = 1e-8):
+    """One Adam step in double.  ``lr`` is a dict keyed by ADAM_PLANE_GROUP
+    names or a length-9 sequence.  Returns new (params, m, v) float64."""
+    P = np.array(params, dtype=np.float64, order="C", copy=True)
+    M = np.array(m, dtype=np.float64, order="C", copy=True)
+    V = np.array(v, dtype=np.float64, order="C", copy=True)
+    G = np.ascontiguousarray(grads, dtype=np.float64)
+    if isinstance(lr, dict):
+        lrv = np.array([lr[gname] for gname in ADAM_PLANE_GROUP], dtype=np.float64)
+    else:
+        lrv = np.ascontiguousarray(lr, dtype=np.float64)
+    lib().orc_adam(H, W, P.shape[1], _p(P), _p(M), _p(V), _p(G), _p(lrv), b1, b2, eps, int(t))
+    return P, M, V

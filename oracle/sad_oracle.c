@@ -1,0 +1,578 @@
+/*
+ * sad_oracle.c -- plain, slow CPU oracle for one Soft Anisotropic Diagrams
+ * (SAD) fitting iteration.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load this library.  It shares no code,
+ * header, table or constant with the CUDA library, and the CUDA library never
+ * calls it.
+ *
+ * Sources, by page title and section:
+ *   [P1] "Soft Anisotropic Diagrams for Differentiable Image Representation"
+ *        (paperlayer.ai summary of arXiv:2604.21984v2), sections 4, B.2-B.5.
+ *   [P2] reading notes on the same paper (woaixuexisr.github.io), "key
+ *        designs" 1-4: the metric G_i, d_mix, the softmax and the candidate
+ *        update formula.
+ *   [P4] "SAD: Soft Anisotropic Diagrams" project page, "Method".
+ *
+ * Conventions fixed here (the pages leave them open; see the readings list in
+ * the design notes of this repository):
+ *   - pixel (i, j) = (column, row) has centre x = (i + 0.5, j + 0.5) in pixels,
+ *     pixel id = j * W + i; images are planar (3, H, W).
+ *   - site parameters are 9 float32 planes of length N in the order
+ *     x, y, ln tau, r, cr, cg, cb, theta, a.  A site is active iff x >= 0
+ *     ([P1] B.2: inactive sites carry x < 0); a NaN x is inactive.
+ *   - s = 1 / max(H, W); u = (cos theta, sin theta), v = (-sin theta, cos theta)
+ *     and G = e^a u u^T + e^-a v v^T ([P2] key design 1, det G = 1).
+ *   - logit l_i(x) = -tau_i (s ||x - p_i||_G - s r_i) ([P2] key design 2,
+ *     [P4] Method); ranking key (l desc, site id asc); NaN logits drop out.
+ *
+ * Precision: render, loss, backward and Adam are evaluated in double from the
+ * float32 parameters.  The top-K decisions (exact brute force and the
+ * propagation pass) are taken in float32 -- the pages' training precision
+ * ([P1] B.2: float32 site buffer) -- on a float32 per-site score record that
+ * is itself computed in double and rounded once per field, with this fixed
+ * operation order for the score of record R at pixel centre (fx, fy):
+ *     dx = fx - R.x;  dy = fy - R.y
+ *     u1 = fmaf(R.A, dx, R.B * dy);  u2 = fmaf(R.C, dy, R.B * dx)
+ *     q  = fmaf(dx, u1, dy * u2);  q = (q < 0) ? 0 : q
+ *     l  = R.b - sqrtf(q)
+ * where k = tau s, (A, B, C) = k^2 (G11, G12, G22) and b = k r; this is the
+ * same logit as above, rearranged as l = k r - sqrt(k^2 delta^T G delta).
+ *
+ * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (oracle/build.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_SENTINEL 0xFFFFFFFFu
+#define ORC_K 8
+#define ORC_REC 16
+
+enum { P_X = 0, P_Y, P_LT, P_R, P_CR, P_CG, P_CB, P_TH, P_A, P_COUNT };
+
+static int omp_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+static int omp_thread_id(void)
+{
+#ifdef _OPENMP
+    return omp_get_thread_num();
+#else
+    return 0;
+#endif
+}
+
+int orc_num_threads(void) { return omp_threads(); }
+
+void orc_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* Per-site score records                                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Record of site i (16 values): x, y, A, B, C, b, k, 0, cr, cg, cb,
+ * cos theta, sin theta, k^2 e^a, k^2 e^-a, 0 with k = tau s.  An inactive
+ * site gets x = -1 and zeros elsewhere.  Every field is evaluated in double;
+ * rec32 receives each field rounded once to float32, rec64 (optional) the
+ * double values.  Metric from [P2] key design 1; fields follow the packed
+ * candidate-site buffer of [P1] B.2 (position, (ln tau, r), direction, a).
+ */
+void orc_records(int H, int W, int N, const float *params, float *rec32, double *rec64)
+{
+    const double s = 1.0 / (double)(H > W ? H : W);
+    for (int i = 0; i < N; ++i) {
+        double f[ORC_REC];
+        memset(f, 0, sizeof(f));
+        const double px = params[P_X * N + i];
+        if (px >= 0.0) {
+            const double py = params[P_Y * N + i];
+            const double tau = exp((double)params[P_LT * N + i]);
+            const double r = params[P_R * N + i];
+            const double th = params[P_TH * N + i];
+            const double a = params[P_A * N + i];
+            const double k = tau * s;
+            const double ep = exp(a), em = exp(-a);
+            const double c = cos(th), sn = sin(th);
+            const double g11 = ep * c * c + em * sn * sn;
+            const double g12 = (ep - em) * c * sn;
+            const double g22 = ep * sn * sn + em * c * c;
+            const double kk = k * k;
+            f[0] = px;
+            f[1] = py;
+            f[2] = kk * g11;
+            f[3] = kk * g12;
+            f[4] = kk * g22;
+            f[5] = k * r;
+            f[6] = k;
+            f[8] = params[P_CR * N + i];
+            f[9] = params[P_CG * N + i];
+            f[10] = params[P_CB * N + i];
+            f[11] = c;
+            f[12] = sn;
+            f[13] = kk * ep;
+            f[14] = kk * em;
+        } else {
+            f[0] = -1.0;
+        }
+        for (int q = 0; q < ORC_REC; ++q) {
+            rec32[(size_t)i * ORC_REC + q] = (float)f[q];
+            if (rec64) rec64[(size_t)i * ORC_REC + q] = f[q];
+        }
+    }
+}
+
+/* float32 logit of a record at a pixel centre, in the fixed order above */
+static float score32(const float *R, float fx, float fy)
+{
+    const float dx = fx - R[0];
+    const float dy = fy - R[1];
+    const float bdy = R[3] * dy;
+    const float bdx = R[3] * dx;
+    const float u1 = fmaf(R[2], dx, bdy);
+    const float u2 = fmaf(R[4], dy, bdx);
+    const float dyu2 = dy * u2;
+    float q = fmaf(dx, u1, dyu2);
+    if (q < 0.0f) q = 0.0f;
+    return R[5] - sqrtf(q);
+}
+
+float orc_score32(const float *rec32, int id, int i, int j)
+{
+    return score32(rec32 + (size_t)id * ORC_REC, (float)i + 0.5f, (float)j + 0.5f);
+}
+
+/* candidate a ranks above candidate b */
+static int ranks_above(float la, uint32_t ia, float lb, uint32_t ib)
+{
+    return la > lb || (la == lb && ia < ib);
+}
+
+typedef struct {
+    float l[ORC_K];
+    uint32_t id[ORC_K];
+    int n;
+} topk_t;
+
+static void topk_clear(topk_t *t) { t->n = 0; }
+
+static int topk_has(const topk_t *t, uint32_t id)
+{
+    for (int q = 0; q < t->n; ++q)
+        if (t->id[q] == id) return 1;
+    return 0;
+}
+
+/* insert a candidate not present in t; keeps (l desc, id asc) order */
+static void topk_insert(topk_t *t, float l, uint32_t id)
+{
+    if (t->n == ORC_K && !ranks_above(l, id, t->l[ORC_K - 1], t->id[ORC_K - 1])) return;
+    int pos = t->n < ORC_K ? t->n : ORC_K - 1;
+    while (pos > 0 && ranks_above(l, id, t->l[pos - 1], t->id[pos - 1])) {
+        t->l[pos] = t->l[pos - 1];
+        t->id[pos] = t->id[pos - 1];
+        --pos;
+    }
+    t->l[pos] = l;
+    t->id[pos] = id;
+    if (t->n < ORC_K) t->n++;
+}
+
+static void topk_store(const topk_t *t, uint32_t *out)
+{
+    for (int q = 0; q < ORC_K; ++q) out[q] = q < t->n ? t->id[q] : ORC_SENTINEL;
+}
+
+/*
+ * Exact top-K ([P1] abstract: the per-pixel list approximates the nearest
+ * sites under the shading score; this is that quantity): every active site is
+ * scored at every requested pixel.  pix == NULL means all pixels in order.
+ * out: n_pix x 8 site ids, sentinel-padded.
+ */
+void orc_topk_exact(int H, int W, int N, const float *rec32, const int64_t *pix, int64_t n_pix,
+                    uint32_t *out)
+{
+    const int64_t P = (int64_t)H * W;
+    if (!pix) n_pix = P;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t q = 0; q < n_pix; ++q) {
+        const int64_t p = pix ? pix[q] : q;
+        const float fx = (float)(p % W) + 0.5f, fy = (float)(p / W) + 0.5f;
+        topk_t t;
+        topk_clear(&t);
+        for (int i = 0; i < N; ++i) {
+            const float *R = rec32 + (size_t)i * ORC_REC;
+            if (!(R[0] >= 0.0f)) continue;
+            const float l = score32(R, fx, fy);
+            if (l != l) continue;
+            topk_insert(&t, l, (uint32_t)i);
+        }
+        topk_store(&t, out + q * ORC_K);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Candidate propagation ([P2] key design 3, [P1] section 4 and B.3)          */
+/* ------------------------------------------------------------------------ */
+
+/* MurmurHash3 32-bit finaliser (Appleby, public domain) */
+static uint32_t fmix32(uint32_t h)
+{
+    h ^= h >> 16;
+    h *= 0x85ebca6bu;
+    h ^= h >> 13;
+    h *= 0xc2b2ae35u;
+    h ^= h >> 16;
+    return h;
+}
+
+/* Marsaglia, "Xorshift RNGs" (J. Stat. Soft. 2003), shift triple (13, 17, 5) */
+static uint32_t xorshift32(uint32_t x)
+{
+    x ^= x << 13;
+    x ^= x >> 17;
+    x ^= x << 5;
+    return x;
+}
+
+uint32_t orc_fmix32(uint32_t h) { return fmix32(h); }
+uint32_t orc_xorshift32(uint32_t h) { return xorshift32(h); }
+
+/*
+ * The G injected site ids of pixel p in propagation pass number `pass`
+ * ([P1] B.3: xorshift state from the step index and pixel id).  State
+ * h = fmix32(p ^ fmix32(seed ^ pass * 0x9E3779B9)), replaced by 1 if zero;
+ * then h <- xorshift32(h) and id = floor(h * N / 2^32) (Lemire's
+ * multiply-high range reduction) for each injection.
+ */
+void orc_inject_ids(uint32_t seed, uint32_t pass, uint32_t p, int N, int G, uint32_t *out)
+{
+    uint32_t h = fmix32(p ^ fmix32(seed ^ (pass * 0x9E3779B9u)));
+    if (h == 0) h = 1;
+    for (int g = 0; g < G; ++g) {
+        h = xorshift32(h);
+        out[g] = (uint32_t)(((uint64_t)h * (uint64_t)(uint32_t)N) >> 32);
+    }
+}
+
+static void offer(topk_t *t, const float *rec32, int N, uint32_t id, float fx, float fy)
+{
+    if (id == ORC_SENTINEL || id >= (uint32_t)N) return;
+    const float *R = rec32 + (size_t)id * ORC_REC;
+    if (!(R[0] >= 0.0f)) return;
+    if (topk_has(t, id)) return;
+    const float l = score32(R, fx, fy);
+    if (l != l) return;
+    topk_insert(t, l, id);
+}
+
+/*
+ * One Jacobi propagation pass at jump k:
+ *   C_t(x) = topK( C_{t-1}(x) U C_{t-1}(x +- k e_x) U C_{t-1}(x +- k e_y) U G_t(x) )
+ * (temporal reuse + self and 4-neighbour propagation + G stochastic
+ * injections, all re-scored at x).  Out-of-image neighbours are skipped.
+ * Tables are P x 8 site ids.  0 <= G <= 64.
+ */
+void orc_propagate(int H, int W, int N, const float *rec32, const uint32_t *tin, uint32_t *tout,
+                   int jump, int G, uint32_t seed, uint32_t pass)
+{
+    if (G > 64) G = 64;
+    if (G < 0) G = 0;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int j = 0; j < H; ++j) {
+        uint32_t inj[64];
+        for (int i = 0; i < W; ++i) {
+            const int64_t p = (int64_t)j * W + i;
+            const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
+            topk_t t;
+            topk_clear(&t);
+            for (int q = 0; q < ORC_K; ++q) offer(&t, rec32, N, tin[p * ORC_K + q], fx, fy);
+            const int nx[4] = {i - jump, i + jump, i, i};
+            const int ny[4] = {j, j, j - jump, j + jump};
+            for (int d = 0; d < 4; ++d) {
+                if (nx[d] < 0 || nx[d] >= W || ny[d] < 0 || ny[d] >= H) continue;
+                const int64_t pn = (int64_t)ny[d] * W + nx[d];
+                for (int q = 0; q < ORC_K; ++q) offer(&t, rec32, N, tin[pn * ORC_K + q], fx, fy);
+            }
+            if (G > 0) {
+                orc_inject_ids(seed, pass, (uint32_t)p, N, G, inj);
+                for (int q = 0; q < G; ++q) offer(&t, rec32, N, inj[q], fx, fy);
+            }
+            topk_store(&t, tout + p * ORC_K);
+        }
+    }
+}
+
+/*
+ * Seed pass ([P1] B.3: the JFA prepass starts with a seed pass): clear the
+ * table to the sentinel, then every active site whose position lies in the
+ * image writes its id to slot 0 of the pixel containing it; the smallest id
+ * wins where several sites share a pixel.
+ */
+void orc_seed(int H, int W, int N, const float *params, uint32_t *table)
+{
+    const int64_t P = (int64_t)H * W;
+    for (int64_t q = 0; q < P * ORC_K; ++q) table[q] = ORC_SENTINEL;
+    for (int i = 0; i < N; ++i) {
+        const float px = params[P_X * N + i], py = params[P_Y * N + i];
+        if (!(px >= 0.0f) || !(py >= 0.0f)) continue;
+        const int64_t ci = (int64_t)floorf(px), cj = (int64_t)floorf(py);
+        if (ci >= W || cj >= H) continue;
+        uint32_t *slot = table + (cj * W + ci) * ORC_K;
+        if ((uint32_t)i < slot[0]) slot[0] = (uint32_t)i;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Render, loss and backward in double ([P2] key designs 1-2, [P1] B.4)       */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    double px, py, tau, r, c[3], ep, em, ux, uy, vx, vy, g11, g12, g22;
+    int active;
+} site64_t;
+
+static site64_t *sites64(int N, const float *params)
+{
+    site64_t *S = (site64_t *)calloc((size_t)(N > 0 ? N : 1), sizeof(site64_t));
+    for (int i = 0; i < N; ++i) {
+        site64_t *z = &S[i];
+        z->px = params[P_X * N + i];
+        z->active = z->px >= 0.0;
+        z->py = params[P_Y * N + i];
+        z->tau = exp((double)params[P_LT * N + i]);
+        z->r = params[P_R * N + i];
+        for (int ch = 0; ch < 3; ++ch) z->c[ch] = params[(P_CR + ch) * N + i];
+        const double a = params[P_A * N + i], th = params[P_TH * N + i];
+        z->ep = exp(a);
+        z->em = exp(-a);
+        z->ux = cos(th);
+        z->uy = sin(th);
+        z->vx = -z->uy;
+        z->vy = z->ux;
+        /* G = e^a u u^T + e^-a v v^T */
+        z->g11 = z->ep * z->ux * z->ux + z->em * z->vx * z->vx;
+        z->g12 = z->ep * z->ux * z->uy + z->em * z->vx * z->vy;
+        z->g22 = z->ep * z->uy * z->uy + z->em * z->vy * z->vy;
+    }
+    return S;
+}
+
+typedef struct {
+    int n;
+    uint32_t id[ORC_K];
+    double l[ORC_K], w[ORC_K], nrm[ORC_K], dx[ORC_K], dy[ORC_K];
+    double chat[3];
+} pixel64_t;
+
+/*
+ * Soft Apollonius render of one pixel from its candidate slots:
+ * n_i = sqrt(delta^T G_i delta), d_i = s n_i - s r_i, l_i = -tau_i d_i,
+ * w_i = exp(l_i - max l) / sum_j exp(l_j - max l), chat = sum_i w_i c_i.
+ * Slots holding the sentinel, an out-of-range id, an inactive site or a
+ * non-finite logit are skipped; no valid slot gives chat = 0 and n = 0.
+ */
+static void render_pixel(const site64_t *S, int N, double s, const uint32_t *slots, int64_t p, int W,
+                         pixel64_t *o)
+{
+    const double x = (double)(p % W) + 0.5, y = (double)(p / W) + 0.5;
+    o->n = 0;
+    o->chat[0] = o->chat[1] = o->chat[2] = 0.0;
+    for (int q = 0; q < ORC_K; ++q) {
+        const uint32_t id = slots[q];
+        if (id == ORC_SENTINEL || id >= (uint32_t)N || !S[id].active) continue;
+        const site64_t *z = &S[id];
+        const double dx = x - z->px, dy = y - z->py;
+        double qq = z->g11 * dx * dx + 2.0 * z->g12 * dx * dy + z->g22 * dy * dy;
+        if (qq < 0.0) qq = 0.0;
+        const double n = sqrt(qq);
+        const double l = -z->tau * (s * n - s * z->r);
+        if (!isfinite(l)) continue;
+        o->id[o->n] = id;
+        o->l[o->n] = l;
+        o->nrm[o->n] = n;
+        o->dx[o->n] = dx;
+        o->dy[o->n] = dy;
+        o->n++;
+    }
+    if (o->n == 0) return;
+    double M = o->l[0];
+    for (int q = 1; q < o->n; ++q) M = o->l[q] > M ? o->l[q] : M;
+    double Z = 0.0;
+    for (int q = 0; q < o->n; ++q) {
+        o->w[q] = exp(o->l[q] - M);
+        Z += o->w[q];
+    }
+    for (int q = 0; q < o->n; ++q) {
+        o->w[q] /= Z;
+        for (int ch = 0; ch < 3; ++ch) o->chat[ch] += o->w[q] * S[o->id[q]].c[ch];
+    }
+}
+
+/* image: 3 x P doubles */
+void orc_render(int H, int W, int N, const float *params, const uint32_t *table, double *image)
+{
+    const int64_t P = (int64_t)H * W;
+    const double s = 1.0 / (double)(H > W ? H : W);
+    site64_t *S = sites64(N, params);
+#pragma omp parallel for schedule(static)
+    for (int64_t p = 0; p < P; ++p) {
+        pixel64_t o;
+        render_pixel(S, N, s, table + p * ORC_K, p, W, &o);
+        for (int ch = 0; ch < 3; ++ch) image[ch * P + p] = o.chat[ch];
+    }
+    free(S);
+}
+
+/* softmax weights of every pixel's slots (P x 8, zero for skipped slots) */
+void orc_weights(int H, int W, int N, const float *params, const uint32_t *table, double *weights)
+{
+    const int64_t P = (int64_t)H * W;
+    const double s = 1.0 / (double)(H > W ? H : W);
+    site64_t *S = sites64(N, params);
+#pragma omp parallel for schedule(static)
+    for (int64_t p = 0; p < P; ++p) {
+        pixel64_t o;
+        render_pixel(S, N, s, table + p * ORC_K, p, W, &o);
+        for (int q = 0; q < ORC_K; ++q) weights[p * ORC_K + q] = 0.0;
+        int u = 0;
+        for (int q = 0; q < ORC_K && u < o.n; ++q)
+            if (table[p * ORC_K + q] == o.id[u]) weights[p * ORC_K + q] = o.w[u++];
+    }
+    free(S);
+}
+
+/*
+ * MSE loss L = (1/P) sum_x sum_ch (chat - t)^2 ([P2] key design 4: plain MSE;
+ * [P1] B.4: normalised by pixel count) and its analytic gradient with
+ * respect to the stored parameters ([P1] B.4: hand-derived top-K softmax
+ * gradients), accumulated in double:
+ *   g        = 2 (chat - t) / P
+ *   dL/dc_i  = w_i g
+ *   gamma_i  = dL/dl_i = w_i (c_i - chat) . g
+ *   dL/dlntau_i = gamma_i l_i          (l is linear in tau)
+ *   dL/dr_i  = gamma_i tau_i s
+ *   dL/dn_i  = -gamma_i tau_i s, with, for alpha = u.delta, beta = v.delta,
+ *     dn/dp     = -(e^a alpha u + e^-a beta v) / n
+ *     dn/da     = (e^a alpha^2 - e^-a beta^2) / (2 n)
+ *     dn/dtheta = alpha beta (e^a - e^-a) / n
+ *   and all three taken as 0 where n = 0.
+ * grads: 9 x N doubles in parameter-plane order (overwritten).  image
+ * (optional): 3 x P doubles.  Returns L.
+ */
+double orc_loss_backward(int H, int W, int N, const float *params, const uint32_t *table,
+                         const float *target, double *grads, double *image)
+{
+    const int64_t P = (int64_t)H * W;
+    const double s = 1.0 / (double)(H > W ? H : W);
+    site64_t *S = sites64(N, params);
+    const int T = omp_threads();
+    double *acc = (double *)calloc((size_t)T * P_COUNT * (size_t)(N > 0 ? N : 1), sizeof(double));
+    double *lossp = (double *)calloc((size_t)T, sizeof(double));
+#pragma omp parallel
+    {
+        const int tid = omp_thread_id();
+        double *A = acc + (size_t)tid * P_COUNT * N;
+        double lsum = 0.0;
+#pragma omp for schedule(static)
+        for (int64_t p = 0; p < P; ++p) {
+            pixel64_t o;
+            render_pixel(S, N, s, table + p * ORC_K, p, W, &o);
+            double g[3];
+            for (int ch = 0; ch < 3; ++ch) {
+                const double e = o.chat[ch] - (double)target[ch * P + p];
+                lsum += e * e;
+                g[ch] = 2.0 * e / (double)P;
+                if (image) image[ch * P + p] = o.chat[ch];
+            }
+            for (int q = 0; q < o.n; ++q) {
+                const site64_t *z = &S[o.id[q]];
+                const int64_t i = o.id[q];
+                const double w = o.w[q];
+                double gamma = 0.0;
+                for (int ch = 0; ch < 3; ++ch) {
+                    A[(P_CR + ch) * (size_t)N + i] += w * g[ch];
+                    gamma += w * (z->c[ch] - o.chat[ch]) * g[ch];
+                }
+                A[P_LT * (size_t)N + i] += gamma * o.l[q];
+                A[P_R * (size_t)N + i] += gamma * z->tau * s;
+                const double dLdn = -gamma * z->tau * s;
+                const double n = o.nrm[q];
+                if (n > 0.0) {
+                    const double al = z->ux * o.dx[q] + z->uy * o.dy[q];
+                    const double be = z->vx * o.dx[q] + z->vy * o.dy[q];
+                    const double dndx = -(z->ep * al * z->ux + z->em * be * z->vx) / n;
+                    const double dndy = -(z->ep * al * z->uy + z->em * be * z->vy) / n;
+                    const double dnda = (z->ep * al * al - z->em * be * be) / (2.0 * n);
+                    const double dndt = al * be * (z->ep - z->em) / n;
+                    A[P_X * (size_t)N + i] += dLdn * dndx;
+                    A[P_Y * (size_t)N + i] += dLdn * dndy;
+                    A[P_A * (size_t)N + i] += dLdn * dnda;
+                    A[P_TH * (size_t)N + i] += dLdn * dndt;
+                }
+            }
+        }
+        lossp[tid] = lsum;
+    }
+    memset(grads, 0, sizeof(double) * P_COUNT * (size_t)N);
+    double L = 0.0;
+    for (int t = 0; t < T; ++t) {
+        const double *A = acc + (size_t)t * P_COUNT * N;
+        for (size_t q = 0; q < (size_t)P_COUNT * N; ++q) grads[q] += A[q];
+        L += lossp[t];
+    }
+    free(acc);
+    free(lossp);
+    free(S);
+    return L / (double)P;
+}
+
+/*
+ * Adam ([P2] key design 4: Adam on all site parameters; [P1] B.4: the
+ * accumulated gradients are already normalised by the pixel count).  Position
+ * and radius are optimised in the resolution-free units s x and s r, in which
+ * the logit is written, so their gradient is scaled by 1/s and their step by
+ * 1/s.  For every active site (x >= 0) and plane j:
+ *   ghat = grad * sigma_j,  sigma_j = 1/s for x, y, r and 1 otherwise
+ *   m <- b1 m + (1 - b1) ghat;   v <- b2 v + (1 - b2) ghat^2
+ *   param <- param - lr_j sigma_j (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ * Inactive sites are left untouched.  All arrays 9 x N doubles, in place.
+ */
+void orc_adam(int H, int W, int N, double *params, double *m, double *v, const double *grads,
+              const double *lr, double b1, double b2, double eps, int t)
+{
+    const double s = 1.0 / (double)(H > W ? H : W);
+    const double bc1 = 1.0 - pow(b1, (double)t);
+    const double bc2 = 1.0 - pow(b2, (double)t);
+    for (int i = 0; i < N; ++i) {
+        if (!(params[P_X * (size_t)N + i] >= 0.0)) continue;
+        for (int j = 0; j < P_COUNT; ++j) {
+            const size_t q = (size_t)j * N + i;
+            const double sig = (j == P_X || j == P_Y || j == P_R) ? 1.0 / s : 1.0;
+            const double gh = grads[q] * sig;
+            m[q] = b1 * m[q] + (1.0 - b1) * gh;
+            v[q] = b2 * v[q] + (1.0 - b2) * gh * gh;
+            const double mh = m[q] / bc1, vh = v[q] / bc2;
+            params[q] -= lr[j] * sig * mh / (sqrt(vh) + eps);
+        }
+    }
+}
