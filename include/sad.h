@@ -1,0 +1,226 @@
+/*
+ * sad.h -- C ABI of libsad, a B200 (sm_100a) implementation of one fitting
+ * iteration of Soft Anisotropic Diagrams (SAD).
+ *
+ * Source pages (cited by title and section):
+ *   [P1] "Soft Anisotropic Diagrams for Differentiable Image Representation"
+ *        (paperlayer summary of arXiv:2604.21984v2), sections 4, 5, B.2-B.7.
+ *   [P2] reading notes on the same paper, "key designs" 1-4 (formulas for
+ *        G_i, d_mix, the softmax blend, the candidate update, budget control).
+ *   [P4] "SAD: Soft Anisotropic Diagrams" project page, "Method".
+ *
+ * Model.  An image of H x W pixels is represented by up to N_cap sites.  Site
+ * i has position p_i (pixels), log-temperature ln tau_i, radius r_i (pixels),
+ * colour c_i (linear RGB), direction angle theta_i and anisotropy a_i.  With
+ * s = 1 / max(H, W), u = (cos theta, sin theta), v = (-sin theta, cos theta),
+ * G_i = e^a u u^T + e^-a v v^T (det G_i = 1) and n_i(x) = ||x - p_i||_{G_i},
+ * the logit of site i at pixel centre x is
+ *     l_i(x) = -tau_i (s n_i(x) - s r_i)                    ([P2] designs 1-2)
+ * and the pixel colour is the softmax blend of the K = 8 sites held in the
+ * pixel's candidate list ([P2] design 2, [P4] Method).  The candidate list is
+ * maintained by Jacobi propagation passes ([P2] design 3, [P1] section 4).
+ *
+ * Memory.  The library allocates no device memory.  The caller owns every
+ * device buffer (PyTorch tensors in the Python binding) and binds them with
+ * sad_bind(); the library never frees them.  Layouts (all little-endian,
+ * row-major, pixel id p = row * W + column, P = H * W):
+ *   params   float32 [9][N_cap]  planes x, y, ln tau, r, cr, cg, cb, theta, a
+ *                                ([P1] B.2 site buffer, with the direction
+ *                                stored as one angle).  A site is active iff
+ *                                x >= 0 (x < 0 or NaN marks an unused slot).
+ *   grads    float32 [9][N_cap]  dL/d(param), same planes; accumulated by
+ *                                sad_backward, consumed and zeroed by
+ *                                sad_adam_step.
+ *   adam_m, adam_v float32 [9][N_cap]  Adam moments.
+ *   records  float32 [N_cap][16] derived per-site score record (64 bytes).
+ *   table    uint32  [2][2][P][4]  two candidate tables (double buffer), each
+ *                                two planes of uint4 (slots 0-3, slots 4-7)
+ *                                ([P1] B.2: two four-channel uint32 textures,
+ *                                K = 8, 0xffffffff = empty).
+ *   target   float32 [3][P]      planar linear RGB.
+ *   image    float32 [3][P]      planar rendered image (may be NULL).
+ *   workspace bytes >= sad_workspace_bytes(); counters, statistics, loss.
+ * Every pointer must be 16-byte aligned; target and image must not overlap
+ * other buffers.  Which of the two tables is current is kept in device
+ * memory, so a captured CUDA graph of the calls below keeps alternating.
+ *
+ * Calls.  Every call except sad_get_stats, sad_get_loss, sad_get_table and
+ * sad_get_sites is asynchronous on the given stream and returns a status.
+ * Device-side anomalies (hash overflow, skipped non-finite pixels, empty
+ * pixels, ids out of range) are counted in the statistics block; kernels
+ * never trap and contain no waits.
+ */
+#ifndef SAD_H
+#define SAD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *sad_stream_t; /* == cudaStream_t; NULL = legacy default stream */
+
+enum {
+    SAD_OK = 0,
+    SAD_ERR_INVALID_ARG = 1, /* bad size, NULL where a buffer is required, misalignment */
+    SAD_ERR_UNSUPPORTED = 2, /* K != 8, or a flag this build does not implement */
+    SAD_ERR_CUDA = 3,        /* a CUDA call or kernel launch failed; see sad_last_error */
+    SAD_ERR_CAPACITY = 4,    /* more sites than N_cap, too many injections, ... */
+    SAD_ERR_NOT_BOUND = 5    /* buffers not bound yet */
+};
+
+#define SAD_K 8
+#define SAD_N_PARAMS 9
+#define SAD_RECORD_FLOATS 16
+#define SAD_MAX_INJECT 64
+#define SAD_EMPTY 0xFFFFFFFFu
+
+typedef struct sad_ctx sad_ctx;
+
+typedef struct sad_buffers {
+    float *params;
+    float *grads;
+    float *adam_m;
+    float *adam_v;
+    float *records;
+    uint32_t *table;
+    float *target;
+    float *image; /* optional */
+    void *workspace;
+    size_t workspace_bytes;
+} sad_buffers;
+
+/* Adam configuration ([P2] key design 4).  Learning rates per parameter
+ * group; positions and radius are stepped in the resolution-free units s x
+ * and s r in which the logit is written (their gradient is multiplied by
+ * max(H, W) and their step by max(H, W)). */
+typedef struct sad_adam_cfg {
+    float lr_pos, lr_log_tau, lr_r, lr_color, lr_theta, lr_a;
+    float beta1, beta2, eps;
+} sad_adam_cfg;
+
+typedef struct sad_stats {
+    uint64_t hash_overflow;    /* backward contributions that bypassed the tile table */
+    uint64_t nonfinite_pixels; /* pixels skipped by render/backward: sum of weights not finite */
+    uint64_t empty_pixels;     /* pixels without any valid candidate (render writes 0) */
+    uint64_t dropped_ids;      /* table entries >= N_cap met by render/backward */
+    uint32_t pass_counter;     /* propagation passes run (drives injection randomness) */
+    uint32_t adam_step;        /* Adam steps taken (bias-correction t of the next step is +1) */
+    uint32_t current_table;    /* 0 or 1: which table of the double buffer is current */
+    uint32_t reserved;
+    double loss;               /* loss of the last sad_backward / sad_fit_iteration */
+} sad_stats;
+
+/* Bytes of workspace the caller must bind for an H x W image and N_cap sites. */
+int sad_workspace_bytes(int H, int W, int N_cap, size_t *bytes);
+
+/* Create a context.  H, W >= 1, H * W < 2^31, N_cap >= 1, K must be 8
+ * (SAD_ERR_UNSUPPORTED otherwise).  Allocates host memory for the handle
+ * only.  *out is set on success. */
+int sad_create(int H, int W, int N_cap, int K, sad_ctx **out);
+
+/* Destroy a context.  Frees the handle only; bound buffers stay the caller's. */
+int sad_destroy(sad_ctx *ctx);
+
+/* Bind caller-owned device buffers (layouts above).  Checks non-NULL (except
+ * image), 16-byte alignment and the workspace size.  Does not touch their
+ * contents; call sad_reset before first use. */
+int sad_bind(sad_ctx *ctx, const sad_buffers *buf);
+
+/* Zero the counters, statistics, gradients and Adam moments, mark the first
+ * table current and set the injection seed.  Asynchronous. */
+int sad_reset(sad_ctx *ctx, uint32_t seed, sad_stream_t stream);
+
+/* Copy n sites (host or device float32 [9][n] planes) into params slots
+ * 0..n-1, mark slots n..N_cap-1 inactive and rebuild the score records
+ * (step a1).  n <= N_cap else SAD_ERR_CAPACITY.  Asynchronous; a host source
+ * must stay valid until the stream reaches the copy. */
+int sad_set_sites(sad_ctx *ctx, const float *params_9xn, int n, sad_stream_t stream);
+
+/* Copy params slots 0..n-1 into dst (host or device, [9][n]).  Synchronises
+ * the stream when dst is host memory. */
+int sad_get_sites(sad_ctx *ctx, float *dst_9xn, int n, sad_stream_t stream);
+
+/* Copy a target image (host or device float32 [3][P]) into the bound target. */
+int sad_set_target(sad_ctx *ctx, const float *target_3xp, sad_stream_t stream);
+
+/* Step a1: rebuild every score record from params.  Record of site i (fp32
+ * values, each evaluated in double and rounded once): x, y, A, B, C, b, k, 0,
+ * cr, cg, cb, cos theta, sin theta, k^2 e^a, k^2 e^-a, 0 where k = tau s,
+ * (A, B, C) = k^2 (G11, G12, G22), b = k r ([P2] design 1; fields as in the
+ * packed candidate-site buffer of [P1] B.2).  Inactive: x = -1, rest 0. */
+int sad_prep_records(sad_ctx *ctx, sad_stream_t stream);
+
+/* Step a8: exact top-K by brute force over all active sites ([P1] abstract:
+ * the quantity the maintained list approximates).  pixels: device int64
+ * pixel ids (NULL = all P pixels in order); out: device uint32 [n][8],
+ * sorted by (logit desc, id asc), empty slots 0xffffffff.  The logit is
+ * evaluated in float32 as l = b - sqrt(q), q = dx u1 + dy u2 with
+ * u1 = A dx + B dy, u2 = C dy + B dx (fixed IEEE operation order, see the
+ * records above), the pages' logit rearranged. */
+int sad_topk_exact(sad_ctx *ctx, const int64_t *pixels, int64_t n_pix, uint32_t *out,
+                   sad_stream_t stream);
+
+/* Step a9: seed pass + full refresh ([P1] B.3: seed pass, then jump-flood
+ * passes).  Clears the current table, writes each active site's id into slot
+ * 0 of the pixel containing it (smallest id wins), then runs propagation
+ * passes at jumps B/2, B/4, ..., 1 with B the largest power of two
+ * <= max(H, W), each with G injections.  0 <= G <= 64. */
+int sad_refresh(sad_ctx *ctx, int G, sad_stream_t stream);
+
+/* Steps a2/a3: one Jacobi propagation pass at jump >= 1 ([P2] design 3):
+ * for every pixel the new list is the top 8 by (logit desc, id asc) of the
+ * distinct valid ids among its own list, the lists of the four pixels at
+ * (+-jump, 0) and (0, +-jump) that lie inside the image, and G injected ids.
+ * Injection ([P1] B.3: xorshift state from the step index and pixel id):
+ * h = fmix32(p ^ fmix32(seed ^ pass * 0x9E3779B9)), 1 if zero, then G times
+ * h = xorshift32(h) (13, 17, 5), id = (h * N_cap) >> 32.  Reads the current
+ * table, writes the other one, makes it current, advances the pass counter. */
+int sad_propagate(sad_ctx *ctx, int jump, int G, sad_stream_t stream);
+
+/* Step a4: render the current table ([P2] design 2): w = softmax of the valid
+ * slots' logits (max-subtracted), chat = sum w c; a pixel without a valid
+ * slot gets 0.  image: device float32 [3][P], NULL = the bound image. */
+int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream);
+
+/* Steps a4-a6: render, MSE loss L = (1/P) sum_x sum_ch (chat - t)^2 and the
+ * analytic gradient ([P1] B.4), accumulated into grads through a per-tile
+ * shared-memory hash table keyed by site id (multiplicative hash, linear
+ * probing capped at 8, compare-and-swap insert) with one global atomic per
+ * (site, parameter, tile); overflow goes straight to global atomics
+ * ([P1] section 5 and B.4).  Writes the bound image when one is bound and
+ * the loss into the statistics block.  flags must be 0. */
+int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream);
+
+/* Step a7: one Adam step on every active site ([P2] design 4), reading and
+ * zeroing grads, advancing the Adam step counter, and rebuilding the score
+ * records (a1) in the same kernel. */
+int sad_adam_step(sad_ctx *ctx, const sad_adam_cfg *cfg, sad_stream_t stream);
+
+/* One steady-state fitting iteration: a propagation pass at jump 1 with G
+ * injections, then render + loss + backward, then Adam (a2-a7). */
+int sad_fit_iteration(sad_ctx *ctx, int G, const sad_adam_cfg *cfg, sad_stream_t stream);
+
+/* Copy the current table into dst (host or device uint32 [P][8], slot order).
+ * Synchronises the stream. */
+int sad_get_table(sad_ctx *ctx, uint32_t *dst, sad_stream_t stream);
+
+/* Copy a table (host or device uint32 [P][8]) into the current table. */
+int sad_set_table(sad_ctx *ctx, const uint32_t *src, sad_stream_t stream);
+
+/* Read the statistics block (synchronises the stream). */
+int sad_get_stats(sad_ctx *ctx, sad_stats *out, sad_stream_t stream);
+
+/* Loss of the last backward pass, copied to host memory (synchronises). */
+int sad_get_loss(sad_ctx *ctx, double *loss, sad_stream_t stream);
+
+/* Message of the last failing call on this context ("" if none). */
+const char *sad_last_error(const sad_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAD_H */

@@ -1,0 +1,147 @@
+"""B200 (sm_100a) library for one Soft Anisotropic Diagrams fitting iteration.
+
+The computation lives in ``libsad.so`` (CUDA kernels behind the C ABI of
+``include/sad.h``).  ``_lib`` exposes every C entry point under its C name;
+``Sad`` below owns the device buffers as PyTorch tensors (PyTorch is used for
+memory and streams only) and forwards each call to the library.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import _lib
+from ._lib import SadError, adam_cfg  # noqa: F401
+
+__all__ = ["Sad", "SadError", "adam_cfg", "load"]
+
+
+def load():
+    """Load (building if needed) the CUDA library; raises if unavailable."""
+    return _lib.load()
+
+
+class Sad:
+    """A context plus its caller-owned device buffers.
+
+    Buffers (torch tensors on ``device``): params/grads/adam_m/adam_v
+    (9, N) float32, records (N, 16) float32, table (2, 2, P, 4) int32 view of
+    uint32 ids, target/image (3, H, W) float32, workspace bytes.
+    """
+
+    def __init__(self, H: int, W: int, N_cap: int, device="cuda", with_image: bool = True, seed: int = 1):
+        import torch
+
+        if not torch.cuda.is_available():
+            raise SadError(_lib.SAD_ERR_CUDA, "no CUDA device is available")
+        self.torch = torch
+        self.H, self.W, self.N = int(H), int(W), int(N_cap)
+        self.P = self.H * self.W
+        self.device = torch.device(device)
+        _lib.load()
+        f32 = dict(dtype=torch.float32, device=self.device)
+        self.params = torch.zeros((9, self.N), **f32)
+        self.grads = torch.zeros((9, self.N), **f32)
+        self.adam_m = torch.zeros((9, self.N), **f32)
+        self.adam_v = torch.zeros((9, self.N), **f32)
+        self.records = torch.zeros((self.N, 16), **f32)
+        self.table = torch.full((2, 2, self.P, 4), -1, dtype=torch.int32, device=self.device)
+        self.target = torch.zeros((3, self.H, self.W), **f32)
+        self.image = torch.zeros((3, self.H, self.W), **f32) if with_image else None
+        self.ws_bytes = _lib.sad_workspace_bytes(self.H, self.W, self.N)
+        self.workspace = torch.zeros(((self.ws_bytes + 255) // 256 * 256,), dtype=torch.uint8, device=self.device)
+        self.ctx = _lib.sad_create(self.H, self.W, self.N, _lib.SAD_K)
+        _lib.sad_bind(self.ctx, params=self.params, grads=self.grads, adam_m=self.adam_m, adam_v=self.adam_v,
+                      records=self.records, table=self.table, target=self.target, image=self.image,
+                      workspace=self.workspace, workspace_bytes=self.workspace.numel())
+        _lib.sad_reset(self.ctx, seed, self.stream)
+
+    # the stream every call is issued on: torch's current stream
+    @property
+    def stream(self):
+        return self.torch.cuda.current_stream(self.device)
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            _lib.sad_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ---- data in / out ------------------------------------------------------
+    def _dev(self, x, dtype):
+        t = self.torch
+        if isinstance(x, np.ndarray):
+            x = t.from_numpy(np.ascontiguousarray(x))
+        return x.to(device=self.device, dtype=dtype).contiguous()
+
+    def set_sites(self, params):
+        src = self._dev(params, self.torch.float32)
+        _lib.sad_set_sites(self.ctx, src, src.shape[1], self.stream)
+        self._keep = src  # the copy is asynchronous: keep the source alive
+
+    def get_sites(self, n=None):
+        n = self.N if n is None else n
+        out = np.empty((9, n), dtype=np.float32)
+        _lib.sad_get_sites(self.ctx, out, n, self.stream)
+        return out
+
+    def set_target(self, target):
+        src = self._dev(target, self.torch.float32)
+        _lib.sad_set_target(self.ctx, src, self.stream)
+        self._keep_t = src
+
+    def reset(self, seed: int = 1):
+        _lib.sad_reset(self.ctx, seed, self.stream)
+
+    def get_table(self) -> np.ndarray:
+        out = np.empty((self.P, 8), dtype=np.uint32)
+        _lib.sad_get_table(self.ctx, out, self.stream)
+        return out
+
+    def set_table(self, table: np.ndarray):
+        src = np.ascontiguousarray(table, dtype=np.uint32).reshape(self.P, 8)
+        _lib.sad_set_table(self.ctx, src, self.stream)
+
+    def stats(self) -> dict:
+        return _lib.sad_get_stats(self.ctx, self.stream)
+
+    def loss(self) -> float:
+        return _lib.sad_get_loss(self.ctx, self.stream)
+
+    # ---- the hot path ---------------------------------------------------------
+    def prep_records(self):
+        _lib.sad_prep_records(self.ctx, self.stream)
+
+    def topk_exact(self, pixels=None):
+        t = self.torch
+        if pixels is None:
+            out = t.empty((self.P, 8), dtype=t.int32, device=self.device)
+            _lib.sad_topk_exact(self.ctx, None, self.P, out, self.stream)
+        else:
+            pix = self._dev(pixels, t.int64)
+            out = t.empty((pix.numel(), 8), dtype=t.int32, device=self.device)
+            _lib.sad_topk_exact(self.ctx, pix, pix.numel(), out, self.stream)
+        return out
+
+    def refresh(self, G: int):
+        _lib.sad_refresh(self.ctx, G, self.stream)
+
+    def propagate(self, jump: int, G: int):
+        _lib.sad_propagate(self.ctx, jump, G, self.stream)
+
+    def render(self, image=None):
+        _lib.sad_render(self.ctx, image, self.stream)
+        return image if image is not None else self.image
+
+    def backward(self, flags: int = 0):
+        _lib.sad_backward(self.ctx, flags, self.stream)
+
+    def adam_step(self, cfg):
+        _lib.sad_adam_step(self.ctx, cfg, self.stream)
+
+    def fit_iteration(self, G: int, cfg):
+        _lib.sad_fit_iteration(self.ctx, G, cfg, self.stream)

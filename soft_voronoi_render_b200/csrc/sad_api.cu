@@ -1,0 +1,337 @@
+// sad_api.cu -- the C ABI of libsad (declared in include/sad.h).
+//
+// Argument checking, buffer binding, status codes and kernel sequencing.  The
+// library allocates no device memory: every buffer is the caller's.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "../../include/sad.h"
+#include "sad_device.cuh"
+#include "sad_launch.h"
+
+struct sad_ctx {
+    int H, W, N, K;
+    long long P;
+    bool bound;
+    sad_buffers buf;
+    sad::Dev dev;
+    char err[512];
+};
+
+namespace {
+
+int fail(sad_ctx *ctx, int code, const char *fmt, ...) {
+    if (ctx) {
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(ctx->err, sizeof(ctx->err), fmt, ap);
+        va_end(ap);
+    }
+    return code;
+}
+
+int cuda_status(sad_ctx *ctx, cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return SAD_OK;
+    return fail(ctx, SAD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int need_bound(sad_ctx *ctx) {
+    if (!ctx) return SAD_ERR_INVALID_ARG;
+    if (!ctx->bound) return fail(ctx, SAD_ERR_NOT_BOUND, "buffers are not bound (call sad_bind)");
+    return SAD_OK;
+}
+
+cudaStream_t cs(sad_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int read_counters(sad_ctx *ctx, sad::Counters *out, cudaStream_t st) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_status(ctx, e, "stream synchronize");
+    e = cudaMemcpy(out, ctx->buf.workspace, sizeof(sad::Counters), cudaMemcpyDeviceToHost);
+    return cuda_status(ctx, e, "read counters");
+}
+
+int run_refresh(sad_ctx *ctx, int G, cudaStream_t st) {
+    int r = cuda_status(ctx, sad::launch_seed(ctx->dev, st), "seed");
+    if (r) return r;
+    int B = 1;
+    const int m = ctx->H > ctx->W ? ctx->H : ctx->W;
+    while (B * 2 <= m) B *= 2;
+    for (int k = B / 2; k >= 1; k /= 2) {
+        r = cuda_status(ctx, sad::launch_propagate(ctx->dev, k, G, st), "propagate");
+        if (r) return r;
+    }
+    return SAD_OK;
+}
+
+int check_adam(sad_ctx *ctx, const sad_adam_cfg *cfg, sad::AdamHyper &h) {
+    if (!cfg) return fail(ctx, SAD_ERR_INVALID_ARG, "adam config is NULL");
+    if (!(cfg->beta1 >= 0.0f && cfg->beta1 < 1.0f) || !(cfg->beta2 >= 0.0f && cfg->beta2 < 1.0f) ||
+        !(cfg->eps > 0.0f))
+        return fail(ctx, SAD_ERR_INVALID_ARG, "adam betas must lie in [0, 1) and eps > 0");
+    const float lr[9] = {cfg->lr_pos,   cfg->lr_pos,   cfg->lr_log_tau, cfg->lr_r, cfg->lr_color,
+                         cfg->lr_color, cfg->lr_color, cfg->lr_theta,   cfg->lr_a};
+    for (int k = 0; k < 9; ++k) {
+        if (!(lr[k] >= 0.0f)) return fail(ctx, SAD_ERR_INVALID_ARG, "learning rates must be >= 0");
+        h.lr[k] = lr[k];
+    }
+    h.beta1 = cfg->beta1;
+    h.beta2 = cfg->beta2;
+    h.eps = cfg->eps;
+    return SAD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sad_workspace_bytes(int H, int W, int N_cap, size_t *bytes) {
+    if (!bytes || H < 1 || W < 1 || N_cap < 1 || (long long)H * W >= (1ll << 31)) return SAD_ERR_INVALID_ARG;
+    *bytes = sad::workspace_bytes(H, W);
+    return SAD_OK;
+}
+
+int sad_create(int H, int W, int N_cap, int K, sad_ctx **out) {
+    if (!out) return SAD_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (H < 1 || W < 1 || N_cap < 1 || (long long)H * W >= (1ll << 31)) return SAD_ERR_INVALID_ARG;
+    if (K != SAD_K) return SAD_ERR_UNSUPPORTED;
+    sad_ctx *c = new (std::nothrow) sad_ctx();
+    if (!c) return SAD_ERR_CAPACITY;
+    c->H = H;
+    c->W = W;
+    c->N = N_cap;
+    c->K = K;
+    c->P = (long long)H * W;
+    c->bound = false;
+    c->err[0] = 0;
+    *out = c;
+    return SAD_OK;
+}
+
+int sad_destroy(sad_ctx *ctx) {
+    if (!ctx) return SAD_ERR_INVALID_ARG;
+    delete ctx;
+    return SAD_OK;
+}
+
+int sad_bind(sad_ctx *ctx, const sad_buffers *b) {
+    if (!ctx) return SAD_ERR_INVALID_ARG;
+    if (!b) return fail(ctx, SAD_ERR_INVALID_ARG, "buffers struct is NULL");
+    const void *req[] = {b->params, b->grads, b->adam_m, b->adam_v, b->records, b->table, b->target, b->workspace};
+    const char *names[] = {"params", "grads", "adam_m", "adam_v", "records", "table", "target", "workspace"};
+    for (int q = 0; q < 8; ++q) {
+        if (!req[q]) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer %s is NULL", names[q]);
+        if (!aligned16(req[q])) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer %s is not 16-byte aligned", names[q]);
+    }
+    if (b->image && !aligned16(b->image)) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer image is not 16-byte aligned");
+    const size_t need = sad::workspace_bytes(ctx->H, ctx->W);
+    if (b->workspace_bytes < need)
+        return fail(ctx, SAD_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", b->workspace_bytes, need);
+    ctx->buf = *b;
+    sad::Dev &d = ctx->dev;
+    d.H = ctx->H;
+    d.W = ctx->W;
+    d.N = ctx->N;
+    d.P = ctx->P;
+    d.params = b->params;
+    d.grads = b->grads;
+    d.adam_m = b->adam_m;
+    d.adam_v = b->adam_v;
+    d.records = reinterpret_cast<float4 *>(b->records);
+    d.table = b->table;
+    d.target = b->target;
+    d.image = b->image;
+    d.ws = b->workspace;
+    ctx->bound = true;
+    ctx->err[0] = 0;
+    return SAD_OK;
+}
+
+int sad_reset(sad_ctx *ctx, uint32_t seed, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    cudaStream_t st = cs(stream);
+    const size_t pn = sizeof(float) * 9 * (size_t)ctx->N;
+    cudaError_t e = cudaMemsetAsync(ctx->buf.grads, 0, pn, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->buf.adam_m, 0, pn, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->buf.adam_v, 0, pn, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->buf.workspace, 0, sad::COUNTERS_BYTES, st);
+    if (e == cudaSuccess) e = sad::launch_init_counters(ctx->dev, seed, st);
+    return cuda_status(ctx, e, "reset");
+}
+
+int sad_set_sites(sad_ctx *ctx, const float *src, int n, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (n < 0 || (n > 0 && !src)) return fail(ctx, SAD_ERR_INVALID_ARG, "bad site source (n=%d)", n);
+    if (n > ctx->N) return fail(ctx, SAD_ERR_CAPACITY, "%d sites exceed the capacity %d", n, ctx->N);
+    cudaStream_t st = cs(stream);
+    cudaError_t e = cudaSuccess;
+    if (n > 0)
+        e = cudaMemcpy2DAsync(ctx->buf.params, sizeof(float) * (size_t)ctx->N, src, sizeof(float) * (size_t)n,
+                              sizeof(float) * (size_t)n, 9, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = sad::launch_mark_inactive(ctx->dev, n, st);
+    if (e == cudaSuccess) e = sad::launch_records(ctx->dev, st);
+    return cuda_status(ctx, e, "set sites");
+}
+
+int sad_get_sites(sad_ctx *ctx, float *dst, int n, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (n < 0 || n > ctx->N || (n > 0 && !dst)) return fail(ctx, SAD_ERR_INVALID_ARG, "bad site destination");
+    cudaStream_t st = cs(stream);
+    if (n == 0) return SAD_OK;
+    cudaError_t e = cudaMemcpy2DAsync(dst, sizeof(float) * (size_t)n, ctx->buf.params, sizeof(float) * (size_t)ctx->N,
+                                      sizeof(float) * (size_t)n, 9, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(ctx, e, "get sites");
+}
+
+int sad_set_target(sad_ctx *ctx, const float *src, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!src) return fail(ctx, SAD_ERR_INVALID_ARG, "target source is NULL");
+    cudaError_t e = cudaMemcpyAsync(ctx->buf.target, src, sizeof(float) * 3 * (size_t)ctx->P, cudaMemcpyDefault,
+                                    cs(stream));
+    return cuda_status(ctx, e, "set target");
+}
+
+int sad_prep_records(sad_ctx *ctx, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    return cuda_status(ctx, sad::launch_records(ctx->dev, cs(stream)), "records");
+}
+
+int sad_topk_exact(sad_ctx *ctx, const int64_t *pixels, int64_t n_pix, uint32_t *out, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!pixels) n_pix = ctx->P;
+    if (n_pix < 0 || (n_pix > 0 && !out)) return fail(ctx, SAD_ERR_INVALID_ARG, "bad top-K output");
+    if (out && !aligned16(out)) return fail(ctx, SAD_ERR_INVALID_ARG, "top-K output is not 16-byte aligned");
+    return cuda_status(ctx, sad::launch_topk_exact(ctx->dev, pixels, n_pix, out, cs(stream)), "topk_exact");
+}
+
+int sad_refresh(sad_ctx *ctx, int G, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (G < 0 || G > SAD_MAX_INJECT) return fail(ctx, SAD_ERR_CAPACITY, "G=%d outside [0, %d]", G, SAD_MAX_INJECT);
+    return run_refresh(ctx, G, cs(stream));
+}
+
+int sad_propagate(sad_ctx *ctx, int jump, int G, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (jump < 1) return fail(ctx, SAD_ERR_INVALID_ARG, "jump must be >= 1");
+    if (G < 0 || G > SAD_MAX_INJECT) return fail(ctx, SAD_ERR_CAPACITY, "G=%d outside [0, %d]", G, SAD_MAX_INJECT);
+    return cuda_status(ctx, sad::launch_propagate(ctx->dev, jump, G, cs(stream)), "propagate");
+}
+
+int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!image) image = ctx->buf.image;
+    if (!image) return fail(ctx, SAD_ERR_INVALID_ARG, "no image buffer given or bound");
+    if (!aligned16(image)) return fail(ctx, SAD_ERR_INVALID_ARG, "image is not 16-byte aligned");
+    return cuda_status(ctx, sad::launch_render(ctx->dev, image, cs(stream)), "render");
+}
+
+int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (flags != 0) return fail(ctx, SAD_ERR_UNSUPPORTED, "backward flags 0x%x not supported", flags);
+    return cuda_status(ctx, sad::launch_render_backward(ctx->dev, cs(stream)), "backward");
+}
+
+int sad_adam_step(sad_ctx *ctx, const sad_adam_cfg *cfg, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    sad::AdamHyper h;
+    r = check_adam(ctx, cfg, h);
+    if (r) return r;
+    return cuda_status(ctx, sad::launch_adam(ctx->dev, h, cs(stream)), "adam");
+}
+
+int sad_fit_iteration(sad_ctx *ctx, int G, const sad_adam_cfg *cfg, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (G < 0 || G > SAD_MAX_INJECT) return fail(ctx, SAD_ERR_CAPACITY, "G=%d outside [0, %d]", G, SAD_MAX_INJECT);
+    sad::AdamHyper h;
+    r = check_adam(ctx, cfg, h);
+    if (r) return r;
+    cudaStream_t st = cs(stream);
+    r = cuda_status(ctx, sad::launch_propagate(ctx->dev, 1, G, st), "propagate");
+    if (r) return r;
+    r = cuda_status(ctx, sad::launch_render_backward(ctx->dev, st), "backward");
+    if (r) return r;
+    return cuda_status(ctx, sad::launch_adam(ctx->dev, h, st), "adam");
+}
+
+int sad_get_table(sad_ctx *ctx, uint32_t *dst, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!dst) return fail(ctx, SAD_ERR_INVALID_ARG, "table destination is NULL");
+    cudaStream_t st = cs(stream);
+    sad::Counters c;
+    r = read_counters(ctx, &c, st);
+    if (r) return r;
+    const uint32_t *plane0 = ctx->buf.table + (size_t)c.cur * ctx->P * SAD_K;
+    const uint32_t *plane1 = plane0 + (size_t)ctx->P * 4;
+    cudaError_t e = cudaMemcpy2DAsync(dst, 32, plane0, 16, 16, (size_t)ctx->P, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaMemcpy2DAsync(dst + 4, 32, plane1, 16, 16, (size_t)ctx->P, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(ctx, e, "get table");
+}
+
+int sad_set_table(sad_ctx *ctx, const uint32_t *src, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!src) return fail(ctx, SAD_ERR_INVALID_ARG, "table source is NULL");
+    cudaStream_t st = cs(stream);
+    sad::Counters c;
+    r = read_counters(ctx, &c, st);
+    if (r) return r;
+    uint32_t *plane0 = ctx->buf.table + (size_t)c.cur * ctx->P * SAD_K;
+    uint32_t *plane1 = plane0 + (size_t)ctx->P * 4;
+    cudaError_t e = cudaMemcpy2DAsync(plane0, 16, src, 32, 16, (size_t)ctx->P, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaMemcpy2DAsync(plane1, 16, src + 4, 32, 16, (size_t)ctx->P, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(ctx, e, "set table");
+}
+
+int sad_get_stats(sad_ctx *ctx, sad_stats *out, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!out) return fail(ctx, SAD_ERR_INVALID_ARG, "stats destination is NULL");
+    sad::Counters c;
+    r = read_counters(ctx, &c, cs(stream));
+    if (r) return r;
+    out->hash_overflow = c.hash_overflow;
+    out->nonfinite_pixels = c.nonfinite_pixels;
+    out->empty_pixels = c.empty_pixels;
+    out->dropped_ids = c.dropped_ids;
+    out->pass_counter = c.pass_counter;
+    out->adam_step = c.adam_step;
+    out->current_table = c.cur;
+    out->reserved = 0;
+    out->loss = c.loss;
+    return SAD_OK;
+}
+
+int sad_get_loss(sad_ctx *ctx, double *loss, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!loss) return fail(ctx, SAD_ERR_INVALID_ARG, "loss destination is NULL");
+    cudaStream_t st = cs(stream);
+    cudaError_t e = cudaMemcpyAsync(loss, &reinterpret_cast<sad::Counters *>(ctx->buf.workspace)->loss,
+                                    sizeof(double), cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(ctx, e, "get loss");
+}
+
+const char *sad_last_error(const sad_ctx *ctx) { return ctx ? ctx->err : "context is NULL"; }
+
+}  // extern "C"

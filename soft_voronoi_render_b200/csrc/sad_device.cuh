@@ -1,0 +1,150 @@
+// sad_device.cuh -- device-side definitions shared by the libsad kernels.
+//
+// Soft Anisotropic Diagrams ("Soft Anisotropic Diagrams for Differentiable
+// Image Representation"): logit of site i at pixel centre x
+//     l_i(x) = -tau_i (s ||x - p_i||_{G_i} - s r_i),   G_i = e^a u u^T + e^-a v v^T
+// (reading notes, key designs 1-2).  The kernels evaluate it from a per-site
+// record holding k = tau s, (A, B, C) = k^2 (G11, G12, G22) and b = k r as
+//     l = b - sqrt(dx (A dx + B dy) + dy (C dy + B dx)),
+// which is the same quantity; the top-K decisions use exactly the IEEE
+// operation sequence of sad_logit() below.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sad {
+
+constexpr int K = 8;
+constexpr uint32_t EMPTY = 0xFFFFFFFFu;
+constexpr int NPARAM = 9;
+constexpr int REC_F4 = 4;  // a record is 4 float4 = 64 bytes
+
+// parameter planes
+enum : int { PX = 0, PY, PLT, PR, PCR, PCG, PCB, PTH, PA };
+
+// Workspace layout: counters and statistics at offset 0, loss partials after.
+struct Counters {
+    uint32_t pass_counter;   // propagation passes run so far
+    uint32_t adam_step;      // Adam steps taken so far
+    uint32_t cur;            // index (0/1) of the current candidate table
+    uint32_t seed;           // injection seed
+    uint32_t ticket_prop;    // last-block tickets (reset by the last block)
+    uint32_t ticket_bwd;
+    uint32_t ticket_adam;
+    uint32_t pad0;
+    unsigned long long hash_overflow;
+    unsigned long long nonfinite_pixels;
+    unsigned long long empty_pixels;
+    unsigned long long dropped_ids;
+    double loss;
+    double pad1[7];
+};
+static_assert(sizeof(Counters) <= 256, "counter block exceeds its 256-byte slot");
+constexpr size_t COUNTERS_BYTES = 256;
+
+// ---------------------------------------------------------------------------
+// ranking: (logit desc, id asc)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool ranks_above(float la, uint32_t ia, float lb, uint32_t ib) {
+    return la > lb || (la == lb && ia < ib);
+}
+
+// Fixed-order float32 logit; returns NaN for NaN inputs.  Every operation is
+// an explicit round-to-nearest intrinsic so that no contraction or reordering
+// can change the bits that decide the top-K.
+__device__ __forceinline__ float sad_logit(float px, float py, float A, float B, float C, float b,
+                                           float fx, float fy) {
+    const float dx = __fsub_rn(fx, px);
+    const float dy = __fsub_rn(fy, py);
+    const float bdy = __fmul_rn(B, dy);
+    const float bdx = __fmul_rn(B, dx);
+    const float u1 = __fmaf_rn(A, dx, bdy);
+    const float u2 = __fmaf_rn(C, dy, bdx);
+    float q = __fmaf_rn(dx, u1, __fmul_rn(dy, u2));
+    q = (q < 0.0f) ? 0.0f : q;
+    return __fsub_rn(b, __fsqrt_rn(q));
+}
+
+// Same logit, also returning the pieces the backward pass needs:
+// (u1, u2) = G' delta and m = sqrt(delta^T G' delta) = k n.
+__device__ __forceinline__ float sad_logit_parts(float px, float py, float A, float B, float C, float b,
+                                                 float fx, float fy, float &dx, float &dy, float &u1,
+                                                 float &u2, float &m) {
+    dx = __fsub_rn(fx, px);
+    dy = __fsub_rn(fy, py);
+    const float bdy = __fmul_rn(B, dy);
+    const float bdx = __fmul_rn(B, dx);
+    u1 = __fmaf_rn(A, dx, bdy);
+    u2 = __fmaf_rn(C, dy, bdx);
+    float q = __fmaf_rn(dx, u1, __fmul_rn(dy, u2));
+    q = (q < 0.0f) ? 0.0f : q;
+    m = __fsqrt_rn(q);
+    return __fsub_rn(b, m);
+}
+
+// ---------------------------------------------------------------------------
+// injection randomness ("xorshift state from the step index and pixel ID")
+// ---------------------------------------------------------------------------
+// MurmurHash3 32-bit finaliser (Austin Appleby, public domain).
+__device__ __forceinline__ uint32_t fmix32(uint32_t h) {
+    h ^= h >> 16;
+    h *= 0x85ebca6bu;
+    h ^= h >> 13;
+    h *= 0xc2b2ae35u;
+    h ^= h >> 16;
+    return h;
+}
+
+// Marsaglia's xorshift32 with shifts (13, 17, 5).
+__device__ __forceinline__ uint32_t xorshift32(uint32_t x) {
+    x ^= x << 13;
+    x ^= x >> 17;
+    x ^= x << 5;
+    return x;
+}
+
+__device__ __forceinline__ uint32_t inject_state(uint32_t seed, uint32_t pass, uint32_t pixel) {
+    uint32_t h = fmix32(pixel ^ fmix32(seed ^ (pass * 0x9E3779B9u)));
+    return h ? h : 1u;
+}
+
+// ---------------------------------------------------------------------------
+// per-thread top-8 list kept in registers
+// ---------------------------------------------------------------------------
+struct Top8 {
+    float l[K];
+    uint32_t id[K];
+
+    __device__ __forceinline__ void clear() {
+#pragma unroll
+        for (int q = 0; q < K; ++q) {
+            l[q] = -__int_as_float(0x7f800000);  // -inf
+            id[q] = EMPTY;
+        }
+    }
+    __device__ __forceinline__ bool has(uint32_t x) const {
+        bool h = false;
+#pragma unroll
+        for (int q = 0; q < K; ++q) h |= (id[q] == x);
+        return h;
+    }
+    // insert a candidate known not to be in the list (bubble network)
+    __device__ __forceinline__ void insert(float lv, uint32_t iv) {
+#pragma unroll
+        for (int q = 0; q < K; ++q) {
+            const bool a = ranks_above(lv, iv, l[q], id[q]);
+            const float tl = a ? l[q] : lv;
+            const uint32_t ti = a ? id[q] : iv;
+            l[q] = a ? lv : l[q];
+            id[q] = a ? iv : id[q];
+            lv = tl;
+            iv = ti;
+        }
+    }
+    __device__ __forceinline__ bool beats_last(float lv, uint32_t iv) const {
+        return ranks_above(lv, iv, l[K - 1], id[K - 1]);
+    }
+};
+
+}  // namespace sad

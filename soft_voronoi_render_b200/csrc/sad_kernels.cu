@@ -1,0 +1,605 @@
+// sad_kernels.cu -- sm_100a kernels of one Soft Anisotropic Diagrams fitting
+// iteration ("Soft Anisotropic Diagrams for Differentiable Image
+// Representation"; reading notes key designs 1-4; summary sections 4, 5 and
+// B.2-B.5).
+//
+//   records_kernel      a1  per-site score record (fp64 math, fp32 fields)
+//   topk_exact_kernel   a8  brute-force top-8 per pixel
+//   seed_*_kernel       a9  seed pass of a refresh
+//   propagate_kernel    a2/a3  one Jacobi candidate pass (+ injection)
+//   render_kernel       a4  softmax blend of the current candidates
+//   render_bwd_kernel   a4-a6  render + MSE + analytic backward with a per-tile
+//                       shared-memory hash reduction of site gradients
+//   adam_kernel         a7  Adam step + a1 for the updated sites
+#include "sad_device.cuh"
+#include "sad_launch.h"
+
+namespace sad {
+
+namespace {
+
+constexpr int TILE_X = 32;  // image-space blocks: one warp per 32-pixel row segment
+constexpr int TILE_Y = 8;
+constexpr int TILE_THREADS = TILE_X * TILE_Y;
+constexpr int SITE_THREADS = 256;
+
+__device__ __forceinline__ Counters *counters(void *ws) { return reinterpret_cast<Counters *>(ws); }
+__device__ __forceinline__ double *loss_partials(void *ws) {
+    return reinterpret_cast<double *>(reinterpret_cast<char *>(ws) + COUNTERS_BYTES);
+}
+
+// ---------------------------------------------------------------------------
+// a1: per-site record, evaluated in double with the operation order of the
+// definition, each field rounded once to float32.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void write_record(float4 *__restrict__ rec, int i, float px, float py, float lt,
+                                             float r, float cr, float cg, float cb, float th, float a,
+                                             double s) {
+    float4 r0, r1, r2, r3;
+    if (px >= 0.0f) {
+        const double tau = exp((double)lt);
+        const double k = __dmul_rn(tau, s);
+        const double ep = exp((double)a), em = exp(-(double)a);
+        double sn, c;
+        sincos((double)th, &sn, &c);
+        const double g11 = __dadd_rn(__dmul_rn(__dmul_rn(ep, c), c), __dmul_rn(__dmul_rn(em, sn), sn));
+        const double g12 = __dmul_rn(__dmul_rn(__dsub_rn(ep, em), c), sn);
+        const double g22 = __dadd_rn(__dmul_rn(__dmul_rn(ep, sn), sn), __dmul_rn(__dmul_rn(em, c), c));
+        const double kk = __dmul_rn(k, k);
+        r0 = make_float4(px, py, (float)__dmul_rn(kk, g11), (float)__dmul_rn(kk, g12));
+        r1 = make_float4((float)__dmul_rn(kk, g22), (float)__dmul_rn(k, (double)r), (float)k, 0.0f);
+        r2 = make_float4(cr, cg, cb, (float)c);
+        r3 = make_float4((float)sn, (float)__dmul_rn(kk, ep), (float)__dmul_rn(kk, em), 0.0f);
+    } else {
+        r0 = make_float4(-1.0f, 0.0f, 0.0f, 0.0f);
+        r1 = r2 = r3 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+    float4 *o = rec + (size_t)i * REC_F4;
+    o[0] = r0;
+    o[1] = r1;
+    o[2] = r2;
+    o[3] = r3;
+}
+
+__global__ void __launch_bounds__(SITE_THREADS) records_kernel(const float *__restrict__ prm, int N, double s,
+                                                               float4 *__restrict__ rec) {
+    const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
+    if (i >= N) return;
+    const size_t n = (size_t)N;
+    write_record(rec, i, prm[PX * n + i], prm[PY * n + i], prm[PLT * n + i], prm[PR * n + i],
+                 prm[PCR * n + i], prm[PCG * n + i], prm[PCB * n + i], prm[PTH * n + i],
+                 prm[PA * n + i], s);
+}
+
+__global__ void init_counters_kernel(Counters *c, uint32_t seed) {
+    c->pass_counter = 0;
+    c->adam_step = 0;
+    c->cur = 0;
+    c->seed = seed;
+    c->ticket_prop = c->ticket_bwd = c->ticket_adam = 0;
+    c->hash_overflow = c->nonfinite_pixels = c->empty_pixels = c->dropped_ids = 0;
+    c->loss = 0.0;
+}
+
+__global__ void mark_inactive_kernel(float *prm, int N, int from) {
+    const int i = from + blockIdx.x * SITE_THREADS + threadIdx.x;
+    if (i < N) prm[i] = -1.0f;  // x plane
+}
+
+// ---------------------------------------------------------------------------
+// a8: exact top-8 by brute force; records staged through shared memory.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(SITE_THREADS) topk_exact_kernel(const float4 *__restrict__ rec, int N, int H,
+                                                                  int W, const int64_t *__restrict__ pix,
+                                                                  int64_t n_pix, uint32_t *__restrict__ out) {
+    __shared__ float sx[SITE_THREADS], sy[SITE_THREADS], sA[SITE_THREADS], sB[SITE_THREADS],
+        sC[SITE_THREADS], sb[SITE_THREADS];
+    const int64_t q = (int64_t)blockIdx.x * SITE_THREADS + threadIdx.x;
+    const int64_t P = (int64_t)H * W;
+    int64_t p = -1;
+    if (q < n_pix) p = pix ? pix[q] : q;
+    const bool live = p >= 0 && p < P;
+    const float fx = live ? (float)(int)(p % W) + 0.5f : 0.0f;
+    const float fy = live ? (float)(int)(p / W) + 0.5f : 0.0f;
+    Top8 t;
+    t.clear();
+    for (int base = 0; base < N; base += SITE_THREADS) {
+        const int i = base + threadIdx.x;
+        if (i < N) {
+            const float4 r0 = __ldg(rec + (size_t)i * REC_F4);
+            const float4 r1 = __ldg(rec + (size_t)i * REC_F4 + 1);
+            sx[threadIdx.x] = r0.x;
+            sy[threadIdx.x] = r0.y;
+            sA[threadIdx.x] = r0.z;
+            sB[threadIdx.x] = r0.w;
+            sC[threadIdx.x] = r1.x;
+            sb[threadIdx.x] = r1.y;
+        } else {
+            sx[threadIdx.x] = -1.0f;
+        }
+        __syncthreads();
+        const int cnt = min(SITE_THREADS, N - base);
+        if (live) {
+            for (int j = 0; j < cnt; ++j) {
+                if (!(sx[j] >= 0.0f)) continue;
+                const float l = sad_logit(sx[j], sy[j], sA[j], sB[j], sC[j], sb[j], fx, fy);
+                if (l != l) continue;
+                const uint32_t id = (uint32_t)(base + j);
+                if (t.beats_last(l, id)) t.insert(l, id);
+            }
+        }
+        __syncthreads();
+    }
+    if (q < n_pix) {
+        uint4 *o = reinterpret_cast<uint4 *>(out + q * K);
+        o[0] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
+        o[1] = make_uint4(t.id[4], t.id[5], t.id[6], t.id[7]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a9 seed pass: clear the current table, scatter each active site's id into
+// slot 0 of the pixel containing it (atomicMin: smallest id wins).
+// ---------------------------------------------------------------------------
+__global__ void seed_clear_kernel(uint32_t *__restrict__ table, long long P, const Counters *__restrict__ c) {
+    uint4 *t = reinterpret_cast<uint4 *>(table + (size_t)c->cur * (size_t)P * K);
+    const long long n = 2 * P;
+    const uint4 e = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY);
+    for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x)
+        t[q] = e;
+}
+
+__global__ void seed_scatter_kernel(const float *__restrict__ prm, int N, int H, int W, uint32_t *__restrict__ table,
+                                    const Counters *__restrict__ c) {
+    const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
+    if (i >= N) return;
+    const float px = prm[PX * (size_t)N + i], py = prm[PY * (size_t)N + i];
+    if (!(px >= 0.0f) || !(py >= 0.0f)) return;
+    const float fi = floorf(px), fj = floorf(py);
+    if (fi >= (float)W || fj >= (float)H) return;
+    const long long p = (long long)fj * W + (long long)fi;
+    uint32_t *plane0 = table + (size_t)c->cur * (size_t)H * W * K;
+    atomicMin(plane0 + (size_t)p * 4, (uint32_t)i);
+}
+
+// ---------------------------------------------------------------------------
+// a2/a3: one Jacobi propagation pass.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void offer(Top8 &t, uint32_t id, const float4 *__restrict__ rec, uint32_t N,
+                                      float fx, float fy) {
+    if (id >= N) return;  // also rejects the empty marker
+    if (t.has(id)) return;
+    const float4 r0 = __ldg(rec + (size_t)id * REC_F4);
+    if (!(r0.x >= 0.0f)) return;
+    const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
+    const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+    if (l != l) return;
+    if (t.beats_last(l, id)) t.insert(l, id);
+}
+
+__device__ __forceinline__ void offer8(Top8 &t, uint4 a, uint4 b, const float4 *__restrict__ rec, uint32_t N,
+                                       float fx, float fy) {
+    offer(t, a.x, rec, N, fx, fy);
+    offer(t, a.y, rec, N, fx, fy);
+    offer(t, a.z, rec, N, fx, fy);
+    offer(t, a.w, rec, N, fx, fy);
+    offer(t, b.x, rec, N, fx, fy);
+    offer(t, b.y, rec, N, fx, fy);
+    offer(t, b.z, rec, N, fx, fy);
+    offer(t, b.w, rec, N, fx, fy);
+}
+
+__global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *__restrict__ rec, uint32_t *table,
+                                                                 int H, int W, int N, int jump, int G,
+                                                                 Counters *c) {
+    const uint32_t cur = c->cur, pass = c->pass_counter, seed = c->seed;
+    const size_t P = (size_t)H * W;
+    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + cur * P * K);
+    const uint4 *in1 = in0 + P;
+    uint4 *out0 = reinterpret_cast<uint4 *>(table + (cur ^ 1u) * P * K);
+    uint4 *out1 = out0 + P;
+    const int i = blockIdx.x * TILE_X + threadIdx.x;
+    const int j = blockIdx.y * TILE_Y + threadIdx.y;
+    if (i < W && j < H) {
+        const size_t p = (size_t)j * W + i;
+        const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
+        Top8 t;
+        t.clear();
+        offer8(t, in0[p], in1[p], rec, (uint32_t)N, fx, fy);
+        if (i - jump >= 0) offer8(t, in0[p - jump], in1[p - jump], rec, (uint32_t)N, fx, fy);
+        if (i + jump < W) offer8(t, in0[p + jump], in1[p + jump], rec, (uint32_t)N, fx, fy);
+        if (j - jump >= 0) {
+            const size_t pn = p - (size_t)jump * W;
+            offer8(t, in0[pn], in1[pn], rec, (uint32_t)N, fx, fy);
+        }
+        if (j + jump < H) {
+            const size_t pn = p + (size_t)jump * W;
+            offer8(t, in0[pn], in1[pn], rec, (uint32_t)N, fx, fy);
+        }
+        if (G > 0) {
+            uint32_t h = inject_state(seed, pass, (uint32_t)p);
+            for (int g = 0; g < G; ++g) {
+                h = xorshift32(h);
+                offer(t, __umulhi(h, (uint32_t)N), rec, (uint32_t)N, fx, fy);
+            }
+        }
+        out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
+        out1[p] = make_uint4(t.id[4], t.id[5], t.id[6], t.id[7]);
+    }
+    // the last block to finish flips the double buffer and advances the pass
+    // counter; every block has read both before taking its ticket
+    __syncthreads();
+    if (threadIdx.x == 0 && threadIdx.y == 0) {
+        __threadfence();
+        const unsigned total = gridDim.x * gridDim.y;
+        if (atomicAdd(&c->ticket_prop, 1u) == total - 1) {
+            c->cur = cur ^ 1u;
+            c->pass_counter = pass + 1u;
+            c->ticket_prop = 0;
+            __threadfence();
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a4: render
+// ---------------------------------------------------------------------------
+struct PixelSoftmax {
+    float l[K];      // logits, then unnormalised weights e_q
+    uint32_t id[K];
+    unsigned valid;  // bit q set when slot q contributes
+    float Z, cr, cg, cb;
+};
+
+// softmax over the valid slots of one pixel (max-subtracted); returns the
+// number of valid slots
+__device__ __forceinline__ int pixel_softmax(const uint4 a, const uint4 b, const float4 *__restrict__ rec,
+                                             uint32_t N, float fx, float fy, PixelSoftmax &s,
+                                             unsigned &dropped) {
+    s.id[0] = a.x; s.id[1] = a.y; s.id[2] = a.z; s.id[3] = a.w;
+    s.id[4] = b.x; s.id[5] = b.y; s.id[6] = b.z; s.id[7] = b.w;
+    s.valid = 0;
+    float M = -__int_as_float(0x7f800000);
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+        s.l[q] = 0.0f;
+        const uint32_t id = s.id[q];
+        if (id >= N) {
+            dropped += (id != EMPTY);
+            continue;
+        }
+        const float4 r0 = __ldg(rec + (size_t)id * REC_F4);
+        if (!(r0.x >= 0.0f)) continue;
+        const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
+        const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+        if (!isfinite(l)) continue;
+        s.l[q] = l;
+        s.valid |= 1u << q;
+        M = fmaxf(M, l);
+    }
+    s.Z = 0.0f;
+    s.cr = s.cg = s.cb = 0.0f;
+    if (!s.valid) return 0;
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+        if (!(s.valid >> q & 1u)) continue;
+        const float e = __expf(s.l[q] - M);
+        const float4 r2 = __ldg(rec + (size_t)s.id[q] * REC_F4 + 2);
+        s.l[q] = e;
+        s.Z += e;
+        s.cr = fmaf(e, r2.x, s.cr);
+        s.cg = fmaf(e, r2.y, s.cg);
+        s.cb = fmaf(e, r2.z, s.cb);
+    }
+    const float iz = 1.0f / s.Z;
+    s.cr *= iz;
+    s.cg *= iz;
+    s.cb *= iz;
+    return __popc(s.valid);
+}
+
+__global__ void __launch_bounds__(TILE_THREADS) render_kernel(const float4 *__restrict__ rec,
+                                                              const uint32_t *__restrict__ table, int H, int W,
+                                                              int N, float *__restrict__ image, Counters *c) {
+    const size_t P = (size_t)H * W;
+    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * P * K);
+    const uint4 *in1 = in0 + P;
+    const int i = blockIdx.x * TILE_X + threadIdx.x;
+    const int j = blockIdx.y * TILE_Y + threadIdx.y;
+    unsigned dropped = 0;
+    bool empty = false;
+    if (i < W && j < H) {
+        const size_t p = (size_t)j * W + i;
+        PixelSoftmax s;
+        const int nv = pixel_softmax(in0[p], in1[p], rec, (uint32_t)N, (float)i + 0.5f, (float)j + 0.5f, s,
+                                     dropped);
+        empty = nv == 0;
+        image[p] = s.cr;
+        image[P + p] = s.cg;
+        image[2 * P + p] = s.cb;
+    }
+    const int ne = __syncthreads_count(empty);
+    const int nd = __syncthreads_count(dropped != 0);
+    if (threadIdx.x == 0 && threadIdx.y == 0) {
+        if (ne) atomicAdd(&c->empty_pixels, (unsigned long long)ne);
+        if (nd) atomicAdd(&c->dropped_ids, (unsigned long long)nd);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a4-a6: render + MSE + backward, per-tile hash reduction of site gradients.
+// ---------------------------------------------------------------------------
+constexpr int HASH_BITS = 9;
+constexpr int HASH_SLOTS = 1 << HASH_BITS;
+constexpr int HASH_PROBES = 8;  // "linear probing capped at 8 probes"
+
+__device__ __forceinline__ int hash_find_or_insert(uint32_t *keys, uint32_t id) {
+    uint32_t s = (id * 2654435761u) >> (32 - HASH_BITS);
+#pragma unroll 1
+    for (int q = 0; q < HASH_PROBES; ++q) {
+        const uint32_t k = *reinterpret_cast<volatile uint32_t *>(keys + s);
+        if (k == id) return (int)s;
+        if (k == EMPTY) {
+            const uint32_t old = atomicCAS(keys + s, EMPTY, id);
+            if (old == EMPTY || old == id) return (int)s;
+        }
+        s = (s + 1) & (HASH_SLOTS - 1);
+    }
+    return -1;
+}
+
+__global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *__restrict__ rec,
+                                                                  const uint32_t *__restrict__ table,
+                                                                  const float *__restrict__ target, int H, int W,
+                                                                  int N, float *__restrict__ image,
+                                                                  float *__restrict__ grads, void *ws) {
+    __shared__ uint32_t keys[HASH_SLOTS];
+    __shared__ float acc[NPARAM][HASH_SLOTS];
+    __shared__ float warp_loss[TILE_THREADS / 32];
+    Counters *c = counters(ws);
+    const int tid = threadIdx.y * TILE_X + threadIdx.x;
+    for (int q = tid; q < HASH_SLOTS; q += TILE_THREADS) {
+        keys[q] = EMPTY;
+#pragma unroll
+        for (int j = 0; j < NPARAM; ++j) acc[j][q] = 0.0f;
+    }
+    __syncthreads();
+
+    const size_t P = (size_t)H * W;
+    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * P * K);
+    const uint4 *in1 = in0 + P;
+    const int i = blockIdx.x * TILE_X + threadIdx.x;
+    const int j = blockIdx.y * TILE_Y + threadIdx.y;
+    const float invP = 1.0f / (float)P;
+    float lsum = 0.0f;
+    unsigned dropped = 0, overflow = 0;
+    bool empty = false;
+    if (i < W && j < H) {
+        const size_t p = (size_t)j * W + i;
+        const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
+        PixelSoftmax s;
+        const int nv = pixel_softmax(in0[p], in1[p], rec, (uint32_t)N, fx, fy, s, dropped);
+        empty = nv == 0;
+        const float er = s.cr - target[p], eg = s.cg - target[P + p], eb = s.cb - target[2 * P + p];
+        lsum = er * er + eg * eg + eb * eb;
+        if (image) {
+            image[p] = s.cr;
+            image[P + p] = s.cg;
+            image[2 * P + p] = s.cb;
+        }
+        const float gr = 2.0f * er * invP, gg = 2.0f * eg * invP, gb = 2.0f * eb * invP;
+        const float iz = nv ? 1.0f / s.Z : 0.0f;
+#pragma unroll 1
+        for (int q = 0; q < K; ++q) {
+            if (!(s.valid >> q & 1u)) continue;
+            const uint32_t id = s.id[q];
+            const float4 *R = rec + (size_t)id * REC_F4;
+            const float4 r0 = __ldg(R), r1 = __ldg(R + 1), r2 = __ldg(R + 2), r3 = __ldg(R + 3);
+            float dx, dy, u1, u2, m;
+            const float l = sad_logit_parts(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy, dx, dy, u1, u2, m);
+            const float w = s.l[q] * iz;
+            const float gamma = w * ((r2.x - s.cr) * gr + (r2.y - s.cg) * gg + (r2.z - s.cb) * gb);
+            const float im = m > 0.0f ? 1.0f / m : 0.0f;
+            const float gi = gamma * im;
+            const float al = r2.w * dx + r3.x * dy;    // u . delta
+            const float be = -r3.x * dx + r2.w * dy;   // v . delta
+            float v[NPARAM];
+            v[PX] = gi * u1;
+            v[PY] = gi * u2;
+            v[PLT] = gamma * l;
+            v[PR] = gamma * r1.z;
+            v[PCR] = w * gr;
+            v[PCG] = w * gg;
+            v[PCB] = w * gb;
+            v[PTH] = -gi * al * be * (r3.y - r3.z);
+            v[PA] = -0.5f * gi * (r3.y * al * al - r3.z * be * be);
+            const int slot = hash_find_or_insert(keys, id);
+            if (slot >= 0) {
+#pragma unroll
+                for (int k = 0; k < NPARAM; ++k) atomicAdd(&acc[k][slot], v[k]);
+            } else {
+                ++overflow;
+#pragma unroll
+                for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + id, v[k]);
+            }
+        }
+    }
+    // loss partial of this tile
+    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    if ((tid & 31) == 0) warp_loss[tid >> 5] = lsum;
+    const int ne = __syncthreads_count(empty);
+    const int nd = __syncthreads_count(dropped != 0);
+    const int no = __syncthreads_count(overflow != 0);
+    // flush the tile table: one global atomic per (site, parameter)
+    for (int q = tid; q < HASH_SLOTS; q += TILE_THREADS) {
+        const uint32_t id = keys[q];
+        if (id == EMPTY) continue;
+#pragma unroll
+        for (int k = 0; k < NPARAM; ++k) {
+            const float a = acc[k][q];
+            if (a != 0.0f) atomicAdd(grads + (size_t)k * N + id, a);
+        }
+    }
+    if (tid == 0) {
+        float t = 0.0f;
+        for (int q = 0; q < TILE_THREADS / 32; ++q) t += warp_loss[q];
+        const unsigned b = blockIdx.y * gridDim.x + blockIdx.x;
+        loss_partials(ws)[b] = (double)t;
+        if (ne) atomicAdd(&c->empty_pixels, (unsigned long long)ne);
+        if (nd) atomicAdd(&c->dropped_ids, (unsigned long long)nd);
+        if (no) atomicAdd(&c->hash_overflow, (unsigned long long)no);
+        __threadfence();
+    }
+    // the last tile sums the loss partials in double
+    __shared__ bool last;
+    if (tid == 0) {
+        const unsigned total = gridDim.x * gridDim.y;
+        last = atomicAdd(&c->ticket_bwd, 1u) == total - 1;
+    }
+    __syncthreads();
+    if (last) {
+        __shared__ double red[TILE_THREADS];
+        const unsigned total = gridDim.x * gridDim.y;
+        const volatile double *lp = loss_partials(ws);
+        double t = 0.0;
+        for (unsigned q = tid; q < total; q += TILE_THREADS) t += lp[q];
+        red[tid] = t;
+        __syncthreads();
+        for (int o = TILE_THREADS / 2; o > 0; o >>= 1) {
+            if (tid < o) red[tid] += red[tid + o];
+            __syncthreads();
+        }
+        if (tid == 0) {
+            c->loss = red[0] / (double)P;
+            c->ticket_bwd = 0;
+            __threadfence();
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a7: Adam + a1 for every site; zeroes the gradients.
+// ---------------------------------------------------------------------------
+struct AdamArgs {
+    float lr[NPARAM];
+    float beta1, beta2, eps;
+};
+
+__global__ void __launch_bounds__(SITE_THREADS) adam_kernel(float *__restrict__ prm, float *__restrict__ grads,
+                                                            float *__restrict__ m1, float *__restrict__ m2,
+                                                            float4 *__restrict__ rec, int N, int maxHW,
+                                                            AdamArgs a, Counters *c) {
+    const uint32_t t = c->adam_step + 1u;
+    const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
+    if (i < N) {
+        const size_t n = (size_t)N;
+        float v[NPARAM];
+#pragma unroll
+        for (int k = 0; k < NPARAM; ++k) v[k] = prm[k * n + i];
+        if (v[PX] >= 0.0f) {
+            const float bc1 = (float)(1.0 - pow((double)a.beta1, (double)t));
+            const float bc2 = (float)(1.0 - pow((double)a.beta2, (double)t));
+            const float sig_pos = (float)maxHW;
+#pragma unroll
+            for (int k = 0; k < NPARAM; ++k) {
+                const float sig = (k == PX || k == PY || k == PR) ? sig_pos : 1.0f;
+                const float gh = grads[k * n + i] * sig;
+                const float mk = a.beta1 * m1[k * n + i] + (1.0f - a.beta1) * gh;
+                const float vk = a.beta2 * m2[k * n + i] + (1.0f - a.beta2) * gh * gh;
+                m1[k * n + i] = mk;
+                m2[k * n + i] = vk;
+                const float mh = mk / bc1, vh = vk / bc2;
+                v[k] -= a.lr[k] * sig * mh / (sqrtf(vh) + a.eps);
+                prm[k * n + i] = v[k];
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < NPARAM; ++k) grads[k * n + i] = 0.0f;
+        write_record(rec, i, v[PX], v[PY], v[PLT], v[PR], v[PCR], v[PCG], v[PCB], v[PTH], v[PA],
+                     1.0 / (double)maxHW);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&c->ticket_adam, 1u) == gridDim.x - 1) {
+            c->adam_step = t;
+            c->ticket_adam = 0;
+            __threadfence();
+        }
+    }
+}
+
+inline dim3 tile_grid(int H, int W) { return dim3((W + TILE_X - 1) / TILE_X, (H + TILE_Y - 1) / TILE_Y); }
+inline unsigned site_blocks(long long n) { return (unsigned)((n + SITE_THREADS - 1) / SITE_THREADS); }
+inline Counters *host_counters(const Dev &d) { return reinterpret_cast<Counters *>(d.ws); }
+
+}  // namespace
+
+size_t workspace_bytes(int H, int W) {
+    // loss partials sized for 8 x 8 tiles, the smallest tile any kernel uses
+    const size_t tiles = (size_t)((W + 7) / 8) * (size_t)((H + 7) / 8);
+    return COUNTERS_BYTES + tiles * sizeof(double);
+}
+
+cudaError_t launch_init_counters(const Dev &d, uint32_t seed, cudaStream_t st) {
+    init_counters_kernel<<<1, 1, 0, st>>>(host_counters(d), seed);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mark_inactive(const Dev &d, int from, cudaStream_t st) {
+    if (from >= d.N) return cudaSuccess;
+    mark_inactive_kernel<<<site_blocks(d.N - from), SITE_THREADS, 0, st>>>(d.params, d.N, from);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_records(const Dev &d, cudaStream_t st) {
+    records_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.N, 1.0 / (double)(d.H > d.W ? d.H : d.W),
+                                                            d.records);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk_exact(const Dev &d, const int64_t *pix, int64_t n, uint32_t *out, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    topk_exact_kernel<<<site_blocks(n), SITE_THREADS, 0, st>>>(d.records, d.N, d.H, d.W, pix, n, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_seed(const Dev &d, cudaStream_t st) {
+    seed_clear_kernel<<<148 * 8, 256, 0, st>>>(d.table, d.P, host_counters(d));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    seed_scatter_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.N, d.H, d.W, d.table,
+                                                                 host_counters(d));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st) {
+    propagate_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.H, d.W, d.N,
+                                                                           jump, G, host_counters(d));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st) {
+    render_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.H, d.W, d.N, image,
+                                                                        host_counters(d));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_render_backward(const Dev &d, cudaStream_t st) {
+    render_bwd_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.target, d.H,
+                                                                            d.W, d.N, d.image, d.grads, d.ws);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st) {
+    AdamArgs a;
+    for (int k = 0; k < NPARAM; ++k) a.lr[k] = h.lr[k];
+    a.beta1 = h.beta1;
+    a.beta2 = h.beta2;
+    a.eps = h.eps;
+    adam_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.grads, d.adam_m, d.adam_v, d.records, d.N,
+                                                          d.H > d.W ? d.H : d.W, a, host_counters(d));
+    return cudaGetLastError();
+}
+
+}  // namespace sad

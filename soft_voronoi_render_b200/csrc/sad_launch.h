@@ -1,0 +1,37 @@
+// sad_launch.h -- host-side launchers of the libsad kernels (internal).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sad {
+
+struct Dev {
+    int H, W, N;
+    long long P;
+    float *params, *grads, *adam_m, *adam_v;
+    float4 *records;
+    uint32_t *table;  // [2][2][P][4]
+    float *target, *image;
+    void *ws;
+};
+
+struct AdamHyper {
+    float lr[9];
+    float beta1, beta2, eps;
+};
+
+size_t workspace_bytes(int H, int W);
+
+cudaError_t launch_init_counters(const Dev &d, uint32_t seed, cudaStream_t st);
+cudaError_t launch_mark_inactive(const Dev &d, int from, cudaStream_t st);
+cudaError_t launch_records(const Dev &d, cudaStream_t st);
+cudaError_t launch_topk_exact(const Dev &d, const int64_t *pix, int64_t n, uint32_t *out, cudaStream_t st);
+cudaError_t launch_seed(const Dev &d, cudaStream_t st);
+cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st);
+cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st);
+cudaError_t launch_render_backward(const Dev &d, cudaStream_t st);
+cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st);
+
+}  // namespace sad

@@ -1,0 +1,106 @@
+"""The C-ABI library loads and exports every entry point include/sad.h
+declares; host-side argument checks work without a GPU (no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from soft_voronoi_render_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "sad.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:int|const char \*)\s*(sad_\w+)\s*\(", txt, flags=re.M)))
+
+
+def test_header_declares_the_abi():
+    names = _declared()
+    assert set(names) == set(_lib.EXPORTED), set(names) ^ set(_lib.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    L = _lib.load()
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_create_validates_arguments():
+    L = _lib.load()
+    h = ctypes.c_void_p(0)
+    assert L.sad_create(0, 4, 4, 8, ctypes.byref(h)) == _lib.SAD_ERR_INVALID_ARG
+    assert L.sad_create(4, 4, 0, 8, ctypes.byref(h)) == _lib.SAD_ERR_INVALID_ARG
+    assert L.sad_create(65536, 65536, 4, 8, ctypes.byref(h)) == _lib.SAD_ERR_INVALID_ARG
+    assert L.sad_create(4, 4, 4, 4, ctypes.byref(h)) == _lib.SAD_ERR_UNSUPPORTED
+    assert L.sad_create(4, 4, 4, 8, None) == _lib.SAD_ERR_INVALID_ARG
+    ctx = _lib.sad_create(16, 24, 100)
+    try:
+        assert ctx
+    finally:
+        _lib.sad_destroy(ctx)
+
+
+def test_workspace_bytes():
+    b = _lib.sad_workspace_bytes(2048, 2048, 131072)
+    assert b >= 256 + 8 * (2048 // 32) * (2048 // 8)
+    with pytest.raises(_lib.SadError):
+        _lib.sad_workspace_bytes(0, 1, 1)
+
+
+def test_bind_checks_alignment_and_sizes_without_touching_memory():
+    ctx = _lib.sad_create(8, 8, 16)
+    ws = _lib.sad_workspace_bytes(8, 8, 16)
+    fake = dict(params=0x10000, grads=0x20000, adam_m=0x30000, adam_v=0x40000, records=0x50000,
+                table=0x60000, target=0x70000, workspace=0x80000, workspace_bytes=ws)
+    try:
+        # calls that need bound buffers fail before binding
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_render(ctx)
+        assert e.value.status == _lib.SAD_ERR_NOT_BOUND
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_bind(ctx, **{**fake, "records": 0x50004})
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG and "aligned" in str(e.value)
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_bind(ctx, **{**fake, "target": None})
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_bind(ctx, **{**fake, "workspace_bytes": ws - 8})
+        assert "workspace" in str(e.value)
+        _lib.sad_bind(ctx, **fake)  # only checks; no memory is touched
+        # argument checks that precede any launch
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_propagate(ctx, 0, 2)
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_propagate(ctx, 1, 65)
+        assert e.value.status == _lib.SAD_ERR_CAPACITY
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_refresh(ctx, -1)
+        assert e.value.status == _lib.SAD_ERR_CAPACITY
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_set_sites(ctx, 0x90000, 17)
+        assert e.value.status == _lib.SAD_ERR_CAPACITY
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_backward(ctx, 1)
+        assert e.value.status == _lib.SAD_ERR_UNSUPPORTED
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_adam_step(ctx, _lib.adam_cfg(beta1=1.0))
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_adam_step(ctx, _lib.adam_cfg(lr_pos=-1.0))
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+    finally:
+        _lib.sad_destroy(ctx)
+
+
+def test_product_path_has_no_oracle_dependency():
+    """The CUDA package never imports the oracle (test infrastructure)."""
+    pkg = os.path.join(ROOT, "soft_voronoi_render_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "sad_oracle" not in txt and "orc_" not in txt, f

@@ -1,0 +1,330 @@
+"""GPU (C-ABI) versus CPU oracle parity on seeded synthetic inputs.
+
+Tolerances (float32 kernels against the float64 oracle):
+  * records, exact top-K, propagation, refresh: bit-exact (the top-K decision
+    is taken in float32 on both sides with the same IEEE operation order);
+  * render from a fixed table: 1e-5 absolute;
+  * per-site gradients: 1e-4 relative with a 1e-6 absolute floor;
+  * loss: 1e-5 relative;
+  * Adam: 4 float32 ulps of the parameter plus 1e-5 of the step size
+    (three float32 steps against float64 state).
+Oracle inputs always come from the generators or from the oracle itself.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+SENT = 0xFFFFFFFF
+RENDER_ATOL = 1e-5
+GRAD_RTOL, GRAD_ATOL = 1e-4, 1e-6
+LOSS_RTOL = 1e-5
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch
+
+
+def make_ctx(torch_cuda, H, W, N, params, target=None, seed=1, n=None):
+    from soft_voronoi_render_b200 import Sad
+    s = Sad(H, W, N, seed=seed)
+    s.set_sites(params if n is None else params[:, :n])
+    if target is not None:
+        s.set_target(target)
+    return s
+
+
+def u32(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def assert_grads(g_gpu, g_orc, what=""):
+    err = np.abs(g_gpu.astype(np.float64) - g_orc)
+    tol = np.maximum(GRAD_RTOL * np.abs(g_orc), GRAD_ATOL)
+    bad = err > tol
+    assert not bad.any(), (what, int(bad.sum()), float((err / tol).max()))
+
+
+def adam_hyper():
+    from soft_voronoi_render_b200 import adam_cfg
+    lr = dict(pos=1e-3, log_tau=2e-3, r=1.5e-3, color=5e-3, theta=2.5e-3, a=3e-3)
+    cfg = adam_cfg(lr_pos=lr["pos"], lr_log_tau=lr["log_tau"], lr_r=lr["r"], lr_color=lr["color"],
+                   lr_theta=lr["theta"], lr_a=lr["a"])
+    f = lambda x: float(np.float32(x))  # the kernel sees float32 hyper-parameters
+    lr32 = {k: f(v) for k, v in lr.items()}
+    return cfg, lr32, f(0.9), f(0.999), f(1e-8)
+
+
+# ---------------------------------------------------------------------------
+# a1 records and a8 exact top-K
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("wl", ["c1", "c2"])
+def test_records_bitwise(torch_cuda, wl):
+    tgt, prm, w = synth.make_workload(wl, seed=1)
+    prm = prm.copy()
+    prm[0, 5] = -1.0
+    prm[0, 6] = np.nan
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm)
+    rec_gpu = s.records.cpu().numpy()
+    rec_orc = oracle.records(w.H, w.W, prm)
+    assert np.array_equal(rec_gpu.view(np.uint32), rec_orc.view(np.uint32))
+
+
+def test_topk_exact_c1_bit_exact(torch_cuda):
+    tgt, prm, w = synth.make_workload("c1", seed=1)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm)
+    gpu = u32(s.topk_exact())
+    ref = oracle.topk_exact(w.H, w.W, oracle.records(w.H, w.W, prm))
+    np.testing.assert_array_equal(gpu, ref)
+
+
+def test_topk_exact_ragged_and_inactive(torch_cuda):
+    H, W, N = 37, 53, 300
+    prm = synth.uniform_sites(H, W, N, 5)
+    prm[0, ::7] = -1.0
+    s = make_ctx(torch_cuda, H, W, N + 20, prm, n=N)  # capacity beyond n: tail inactive
+    gpu = u32(s.topk_exact())
+    full = np.concatenate([prm, np.zeros((9, 20), np.float32)], 1)
+    full[0, N:] = -1.0
+    ref = oracle.topk_exact(H, W, oracle.records(H, W, full))
+    np.testing.assert_array_equal(gpu, ref)
+
+
+def test_topk_exact_sampled_full_size_c3(torch_cuda):
+    tgt, prm, w = synth.make_workload("c3", seed=1)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm)
+    pix = synth.Stream(3, "c3-sample").integers(1024, w.H * w.W)
+    gpu = u32(s.topk_exact(pix))
+    ref = oracle.topk_exact(w.H, w.W, oracle.records(w.H, w.W, prm), pix)
+    np.testing.assert_array_equal(gpu, ref)
+
+
+# ---------------------------------------------------------------------------
+# a4 render, a5/a6 loss + backward
+# ---------------------------------------------------------------------------
+
+def test_render_fixed_table_c1(torch_cuda):
+    tgt, prm, w = synth.make_workload("c1", seed=1)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt)
+    table = oracle.topk_exact(w.H, w.W, oracle.records(w.H, w.W, prm))
+    s.set_table(table)
+    img = s.render().cpu().numpy()
+    ref = oracle.render(w.H, w.W, prm, table)
+    assert np.abs(img - ref).max() <= RENDER_ATOL
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_backward_c1(torch_cuda, seed):
+    tgt, prm, w = synth.make_workload("c1", seed=seed)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt)
+    table = oracle.topk_exact(w.H, w.W, oracle.records(w.H, w.W, prm))
+    s.set_table(table)
+    s.backward()
+    L_gpu = s.loss()
+    L, g, img = oracle.loss_backward(w.H, w.W, prm, table, tgt, want_image=True)
+    assert abs(L_gpu - L) <= LOSS_RTOL * L
+    assert np.abs(s.image.cpu().numpy() - img).max() <= RENDER_ATOL
+    assert_grads(s.grads.cpu().numpy(), g, "c1")
+    st = s.stats()
+    assert st["hash_overflow"] == 0 and st["empty_pixels"] == 0 and st["dropped_ids"] == 0
+
+
+def test_backward_hash_overflow_path(torch_cuda):
+    """Random tables put ~8 distinct sites on every pixel of a tile, so the
+    per-tile table overflows and contributions take the global-atomic path."""
+    H, W, N = 64, 96, 40000
+    prm = synth.uniform_sites(H, W, N, 9)
+    tgt = synth.make_image(H, W, 10, 0, 9)
+    table = synth.Stream(9, "rand-table").integers(H * W * 8, N).astype(np.uint32).reshape(H * W, 8)
+    s = make_ctx(torch_cuda, H, W, N, prm, tgt)
+    s.set_table(table)
+    s.backward()
+    L, g = oracle.loss_backward(H, W, prm, table, tgt)
+    assert s.stats()["hash_overflow"] > 0
+    assert abs(s.loss() - L) <= LOSS_RTOL * L
+    assert_grads(s.grads.cpu().numpy(), g, "overflow")
+
+
+def test_backward_edge_cases(torch_cuda):
+    H, W, N = 9, 33, 64
+    prm = synth.uniform_sites(H, W, N, 4)
+    tgt = synth.make_image(H, W, 2, 0, 4)
+    table = oracle.topk_exact(H, W, oracle.records(H, W, prm))
+    table[3] = SENT                       # an empty pixel
+    table[5, 6:] = [N + 3, 2 ** 31]       # ids beyond capacity are skipped
+    table[7, 1] = table[7, 0]             # duplicates count twice on both sides
+    prm2 = prm.copy()
+    prm2[0, int(table[10, 0])] = -1.0     # an inactive site referenced by the table
+    s = make_ctx(torch_cuda, H, W, N, prm2, tgt)
+    s.set_table(table)
+    s.backward()
+    L, g, img = oracle.loss_backward(H, W, prm2, table, tgt, want_image=True)
+    assert abs(s.loss() - L) <= LOSS_RTOL * L
+    assert np.abs(s.image.cpu().numpy() - img).max() <= RENDER_ATOL
+    assert_grads(s.grads.cpu().numpy(), g, "edges")
+    st = s.stats()
+    assert st["empty_pixels"] >= 1 and st["dropped_ids"] >= 1
+
+
+def test_all_inactive_renders_zero(torch_cuda):
+    H, W, N = 16, 16, 8
+    prm = synth.uniform_sites(H, W, N, 1)
+    prm[0] = -1.0
+    tgt = synth.make_image(H, W, 1, 0, 1)
+    s = make_ctx(torch_cuda, H, W, N, prm, tgt)
+    s.refresh(2)
+    assert np.all(s.get_table() == SENT)
+    s.backward()
+    assert np.all(s.image.cpu().numpy() == 0.0)
+    assert np.all(s.grads.cpu().numpy() == 0.0)
+    np.testing.assert_allclose(s.loss(), float(np.sum(tgt.astype(np.float64) ** 2) / (H * W)), rtol=1e-6)
+    assert s.stats()["empty_pixels"] == H * W
+
+
+# ---------------------------------------------------------------------------
+# a7 Adam (synthetic gradients: the oracle never takes GPU values)
+# ---------------------------------------------------------------------------
+
+def test_adam_step_parity(torch_cuda):
+    tgt, prm, w = synth.make_workload("c1", seed=3)
+    prm = prm.copy()
+    prm[0, 11] = -1.0
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt)
+    cfg, lr32, b1, b2, eps = adam_hyper()
+    P, M, V = prm.astype(np.float64), np.zeros((9, w.N)), np.zeros((9, w.N))
+    for t in (1, 2, 3):
+        g = synth.random_gradients(w.N, 40 + t)
+        s.grads.copy_(torch_cuda.from_numpy(g))
+        s.adam_step(cfg)
+        P, M, V = oracle.adam(w.H, w.W, P, M, V, g, lr32, t, b1, b2, eps)
+        p_gpu = s.params.cpu().numpy()
+        sig = np.ones(9)
+        sig[[0, 1, 3]] = max(w.H, w.W)
+        lrv = np.array([lr32[k] for k in oracle.ADAM_PLANE_GROUP])
+        tol = 4 * np.spacing(np.abs(P).astype(np.float32)).astype(np.float64) + 1e-5 * (lrv * sig)[:, None]
+        assert np.all(np.abs(p_gpu - P) <= tol)
+        np.testing.assert_allclose(s.adam_m.cpu().numpy(), M, rtol=1e-5, atol=1e-12)
+        np.testing.assert_allclose(s.adam_v.cpu().numpy(), V, rtol=1e-5, atol=1e-18)
+        assert np.all(s.grads.cpu().numpy() == 0.0)
+        assert s.stats()["adam_step"] == t
+    assert np.array_equal(s.params.cpu().numpy()[:, 11], prm[:, 11])
+    # the records rebuilt in Adam's epilogue equal a fresh rebuild of the same params
+    rec_epi = s.records.cpu().numpy().copy()
+    s.prep_records()
+    assert np.array_equal(rec_epi.view(np.uint32), s.records.cpu().numpy().view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# a2/a3 propagation, a9 refresh
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("H,W,N,jump,G", [(37, 53, 300, 1, 2), (37, 53, 300, 4, 0), (64, 40, 500, 16, 5),
+                                          (20, 17, 60, 64, 64), (1, 1, 1, 1, 3), (256, 256, 1024, 1, 2)])
+def test_propagate_bit_exact(torch_cuda, H, W, N, jump, G):
+    prm = synth.uniform_sites(H, W, N, 6)
+    prm[0, ::11] = -1.0
+    st = synth.Stream(H * 1000 + W, "prop-table")
+    table = st.integers(H * W * 8, N + 5).astype(np.uint32).reshape(H * W, 8)
+    table[st.uniform(H * W * 8).reshape(H * W, 8) < 0.3] = SENT
+    s = make_ctx(torch_cuda, H, W, N, prm, seed=1234)
+    s.set_table(table)
+    s.propagate(jump, G)
+    rec = oracle.records(H, W, prm)
+    ref = oracle.propagate(H, W, rec, table, jump, G, seed=1234, pass_index=0)
+    np.testing.assert_array_equal(s.get_table(), ref)
+    s.propagate(1, G)
+    ref2 = oracle.propagate(H, W, rec, ref, 1, G, seed=1234, pass_index=1)
+    np.testing.assert_array_equal(s.get_table(), ref2)
+    assert s.stats()["pass_counter"] == 2
+
+
+def test_refresh_c2_bit_exact(torch_cuda):
+    tgt, prm, w = synth.make_workload("c2", seed=1)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, seed=77)
+    s.refresh(w.G)
+    ref, npass = oracle.refresh(w.H, w.W, prm, w.G, seed=77)
+    np.testing.assert_array_equal(s.get_table(), ref)
+    assert s.stats()["pass_counter"] == npass == 9
+
+
+def test_recall_after_convergence_c2(torch_cuda):
+    """Propagated lists reach recall@8 >= 0.99 against exact top-K after
+    convergence (params frozen; k = 1 passes until no slot changes, cap 64)."""
+    tgt, prm, w = synth.make_workload("c2", seed=2)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, seed=5)
+    s.refresh(w.G)
+    prev = s.get_table()
+    for _ in range(64):
+        s.propagate(1, w.G)
+        cur = s.get_table()
+        if np.array_equal(cur, prev):
+            break
+        prev = cur
+    pix = synth.Stream(2, "recall").integers(8192, w.H * w.W)
+    ex = oracle.topk_exact(w.H, w.W, oracle.records(w.H, w.W, prm), pix)
+    got = prev[pix]
+    hit = [len(set(a.tolist()) & set(b.tolist()) - {SENT}) / max(1, int((b != SENT).sum()))
+           for a, b in zip(got, ex)]
+    assert np.mean(hit) >= 0.99
+
+
+# ---------------------------------------------------------------------------
+# whole iteration and full-size cases
+# ---------------------------------------------------------------------------
+
+def test_fit_iteration_c1(torch_cuda):
+    tgt, prm, w = synth.make_workload("c1", seed=1)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt, seed=9)
+    rec = oracle.records(w.H, w.W, prm)
+    t0 = oracle.topk_exact(w.H, w.W, rec)
+    s.set_table(t0)
+    cfg, lr32, b1, b2, eps = adam_hyper()
+    s.fit_iteration(2, cfg)
+    t1 = oracle.propagate(w.H, w.W, rec, t0, 1, 2, seed=9, pass_index=0)
+    np.testing.assert_array_equal(s.get_table(), t1)
+    L, g = oracle.loss_backward(w.H, w.W, prm, t1, tgt)
+    assert abs(s.loss() - L) <= LOSS_RTOL * L
+    P, _, _ = oracle.adam(w.H, w.W, prm, np.zeros((9, w.N)), np.zeros((9, w.N)), g, lr32, 1, b1, b2, eps)
+    p_gpu = s.params.cpu().numpy()
+    sig = np.ones(9)
+    sig[[0, 1, 3]] = max(w.H, w.W)
+    lrv = np.array([lr32[k] for k in oracle.ADAM_PLANE_GROUP])
+    # first step is -lr sigma sign(g): compare where |g| is far above the
+    # gradient tolerance, so that float32 accumulation cannot flip its sign
+    firm = np.abs(g) > 10 * np.maximum(GRAD_RTOL * np.abs(g), GRAD_ATOL)
+    tol = 2 * np.spacing(np.abs(P).astype(np.float32)) + 1e-3 * (lrv * sig)[:, None]
+    assert np.all((np.abs(p_gpu - P) <= tol)[firm])
+    assert firm.mean() > 0.5
+    assert s.stats()["adam_step"] == 1 and s.stats()["pass_counter"] == 1
+
+
+@pytest.mark.slow
+def test_full_size_c3_iteration_pieces(torch_cuda):
+    """2048 x 2048, N = 131,072 (the benchmark workload), launched as the
+    benchmark launches it: one propagation pass is bit-exact against the
+    oracle, and render + backward agree with the oracle on the oracle's table."""
+    tgt, prm, w = synth.make_workload("c3", seed=1)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt, seed=3)
+    rec = oracle.records(w.H, w.W, prm)
+    t, npass = oracle.refresh(w.H, w.W, prm, w.G, seed=3)
+    s.set_table(t)
+    s.propagate(1, w.G)  # pass number 0 of this context
+    ref = oracle.propagate(w.H, w.W, rec, t, 1, w.G, seed=3, pass_index=0)
+    np.testing.assert_array_equal(s.get_table(), ref)
+    s.backward()
+    L, g, img = oracle.loss_backward(w.H, w.W, prm, ref, tgt, want_image=True)
+    assert abs(s.loss() - L) <= LOSS_RTOL * L
+    assert np.abs(s.image.cpu().numpy() - img).max() <= RENDER_ATOL
+    assert_grads(s.grads.cpu().numpy(), g, "c3")
+    st = s.stats()
+    assert st["empty_pixels"] == 0
