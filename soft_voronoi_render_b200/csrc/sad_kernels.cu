@@ -348,6 +348,48 @@ __device__ __forceinline__ int hash_find_or_insert(uint32_t *keys, uint32_t id) 
     return -1;
 }
 
+// Sum v[0..8] over each maximal run of lanes holding the same key (runs in
+// lane order; a warp covers 32 consecutive pixels of a row, and neighbouring
+// pixels usually hold the same site in the same slot).  Afterwards the last
+// lane of every run holds the run's total.  Returns true on those lanes.
+__device__ __forceinline__ bool warp_run_reduce(uint32_t key, float (&v)[NPARAM], int lane) {
+    constexpr unsigned FULL = 0xffffffffu;
+    const uint32_t key_next = __shfl_down_sync(FULL, key, 1);
+    const bool tail = lane == 31 || key_next != key;
+    const uint32_t tails = __ballot_sync(FULL, tail);
+    const uint32_t cont = ~tails;  // bit L: lanes L and L+1 share a run
+    if (cont) {
+        const uint32_t prev = tails & ((1u << lane) - 1u);
+        const int start = prev ? 32 - __clz(prev) : 0;
+        // doubling steps needed for the longest run (warp-uniform)
+        int levels = 1;
+        uint32_t r = cont & (cont >> 1);
+        if (r) {
+            levels = 2;
+            r &= r >> 2;
+            if (r) {
+                levels = 3;
+                r &= r >> 4;
+                if (r) {
+                    levels = 4;
+                    r &= r >> 8;
+                    if (r) levels = 5;
+                }
+            }
+        }
+        for (int L = 0; L < levels; ++L) {
+            const int off = 1 << L;
+            const bool take = lane - off >= start;
+#pragma unroll
+            for (int k = 0; k < NPARAM; ++k) {
+                const float t = __shfl_up_sync(FULL, v[k], off);
+                if (take) v[k] += t;
+            }
+        }
+    }
+    return tail;
+}
+
 __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *__restrict__ rec,
                                                                   const uint32_t *__restrict__ table,
                                                                   const float *__restrict__ target, int H, int W,
@@ -357,6 +399,7 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
     __shared__ float acc[NPARAM][HASH_SLOTS];
     __shared__ float warp_loss[TILE_THREADS / 32];
     Counters *c = counters(ws);
+    const int lane = threadIdx.x;  // blockDim.x == 32: one warp per row segment
     const int tid = threadIdx.y * TILE_X + threadIdx.x;
     for (int q = tid; q < HASH_SLOTS; q += TILE_THREADS) {
         keys[q] = EMPTY;
@@ -370,14 +413,18 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
     const uint4 *in1 = in0 + P;
     const int i = blockIdx.x * TILE_X + threadIdx.x;
     const int j = blockIdx.y * TILE_Y + threadIdx.y;
+    const bool inside = i < W && j < H;
     const float invP = 1.0f / (float)P;
+    const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
     float lsum = 0.0f;
     unsigned dropped = 0, overflow = 0;
     bool empty = false;
-    if (i < W && j < H) {
+    PixelSoftmax s;
+    s.valid = 0;
+    s.cr = s.cg = s.cb = 0.0f;
+    float gr = 0.0f, gg = 0.0f, gb = 0.0f, iz = 0.0f;
+    if (inside) {
         const size_t p = (size_t)j * W + i;
-        const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
-        PixelSoftmax s;
         const int nv = pixel_softmax(in0[p], in1[p], rec, (uint32_t)N, fx, fy, s, dropped);
         empty = nv == 0;
         const float er = s.cr - target[p], eg = s.cg - target[P + p], eb = s.cb - target[2 * P + p];
@@ -387,13 +434,21 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
             image[P + p] = s.cg;
             image[2 * P + p] = s.cb;
         }
-        const float gr = 2.0f * er * invP, gg = 2.0f * eg * invP, gb = 2.0f * eb * invP;
-        const float iz = nv ? 1.0f / s.Z : 0.0f;
-#pragma unroll 1
-        for (int q = 0; q < K; ++q) {
-            if (!(s.valid >> q & 1u)) continue;
-            const uint32_t id = s.id[q];
-            const float4 *R = rec + (size_t)id * REC_F4;
+        gr = 2.0f * er * invP;
+        gg = 2.0f * eg * invP;
+        gb = 2.0f * eb * invP;
+        iz = nv ? 1.0f / s.Z : 0.0f;
+    }
+    // every lane runs the slot loop (the run reduction needs the whole warp)
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+        const bool vq = (s.valid >> q) & 1u;
+        const uint32_t key = vq ? s.id[q] : EMPTY;
+        float v[NPARAM];
+#pragma unroll
+        for (int k = 0; k < NPARAM; ++k) v[k] = 0.0f;
+        if (vq) {
+            const float4 *R = rec + (size_t)key * REC_F4;
             const float4 r0 = __ldg(R), r1 = __ldg(R + 1), r2 = __ldg(R + 2), r3 = __ldg(R + 3);
             float dx, dy, u1, u2, m;
             const float l = sad_logit_parts(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy, dx, dy, u1, u2, m);
@@ -401,9 +456,8 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
             const float gamma = w * ((r2.x - s.cr) * gr + (r2.y - s.cg) * gg + (r2.z - s.cb) * gb);
             const float im = m > 0.0f ? 1.0f / m : 0.0f;
             const float gi = gamma * im;
-            const float al = r2.w * dx + r3.x * dy;    // u . delta
-            const float be = -r3.x * dx + r2.w * dy;   // v . delta
-            float v[NPARAM];
+            const float al = r2.w * dx + r3.x * dy;   // u . delta
+            const float be = -r3.x * dx + r2.w * dy;  // v . delta
             v[PX] = gi * u1;
             v[PY] = gi * u2;
             v[PLT] = gamma * l;
@@ -413,14 +467,17 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
             v[PCB] = w * gb;
             v[PTH] = -gi * al * be * (r3.y - r3.z);
             v[PA] = -0.5f * gi * (r3.y * al * al - r3.z * be * be);
-            const int slot = hash_find_or_insert(keys, id);
+        }
+        const bool tail = warp_run_reduce(key, v, lane);
+        if (tail && key != EMPTY) {
+            const int slot = hash_find_or_insert(keys, key);
             if (slot >= 0) {
 #pragma unroll
                 for (int k = 0; k < NPARAM; ++k) atomicAdd(&acc[k][slot], v[k]);
             } else {
                 ++overflow;
 #pragma unroll
-                for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + id, v[k]);
+                for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + key, v[k]);
             }
         }
     }
