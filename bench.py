@@ -3,8 +3,8 @@
 One step = one steady-state fitting iteration on the 2048 x 2048, N = 131,072
 workload (c3 of the synthetic workloads): a propagation pass at jump 1 with
 G = 2 injections, render + MSE + analytic backward, and Adam with the record
-rebuild, issued through the C ABI (sad_propagate, sad_backward,
-sad_adam_step -- the three calls sad_fit_iteration makes).
+rebuild, issued through the C ABI as sad_fit_pass + sad_adam_step (the two
+kernels sad_fit_iteration launches).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -37,15 +37,13 @@ WORKLOAD = "c3"
 ADAM_LR = dict(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=5e-3, lr_theta=1e-3, lr_a=1e-3)
 
 # Algorithmic DRAM bytes (compulsory traffic) per launch, per pixel and per site.
-#   propagate : read own 8-id list 32 B + write new list 32 B; read 24 B of each
-#               site record (scoring fields) once
-#   render_bwd: read list 32 B + target 12 B + write image 12 B; read each
-#               64-B record once + one 36-B gradient write-back per site
-#   adam      : params, m, v read+write (3 x 72 B), gradients read + zero
-#               (72 B), record write 64 B
+#   fit_pass: read the 8-id list 32 B + write the new list 32 B + read target
+#             12 B + write image 12 B; read each 64-B record once + one 36-B
+#             gradient write-back per site
+#   adam    : params, m, v read+write (3 x 72 B), gradients read + zero
+#             (72 B), record write 64 B
 BYTES = {
-    "propagate": (64, 24),
-    "render_bwd": (56, 100),
+    "fit_pass": (88, 100),
     "adam": (0, 352),
 }
 # the iteration's own compulsory traffic (fused ideal: the list is read once)
@@ -271,22 +269,19 @@ def run_ours(args):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        _lib.sad_propagate(ctx, 1, G, sp)
+        _lib.sad_fit_pass(ctx, G, sp)
         if ev is not None:
             ev[1].record(stream)
-        _lib.sad_backward(ctx, 0, sp)
-        if ev is not None:
-            ev[2].record(stream)
         _lib.sad_adam_step(ctx, cfg, sp)
         if ev is not None:
-            ev[3].record(stream)
+            ev[2].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize(dev)
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}")
     if local == 0 or world == 1:
@@ -305,11 +300,10 @@ def run_ours(args):
         dist.barrier()
     clocks = sampler.stop() if (local == 0 or world == 1) else None
     ms_total = t_start.elapsed_time(t_end)
-    per_kernel = {n: 0.0 for n in ("propagate", "render_bwd", "adam")}
+    per_kernel = {n: 0.0 for n in ("fit_pass", "adam")}
     for e in evs:
-        per_kernel["propagate"] += e[0].elapsed_time(e[1])
-        per_kernel["render_bwd"] += e[1].elapsed_time(e[2])
-        per_kernel["adam"] += e[2].elapsed_time(e[3])
+        per_kernel["fit_pass"] += e[0].elapsed_time(e[1])
+        per_kernel["adam"] += e[1].elapsed_time(e[2])
     ms_max = ms_total
     if world > 1:
         t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
@@ -366,7 +360,7 @@ def run_ours(args):
                          "algorithmic_bytes": alg_bytes},
             "e2e": {"value": e2e_value, "unit": "Mpix/s", "h2d_bytes_per_step": int(host_tgt.numel() * 4),
                     "d2h_bytes_per_step": 8, "steps": E},
-            "gpu_launches": 3 * K,
+            "gpu_launches": 2 * K,
             "clocks": clocks,
             "device_stats": {k: st[k] for k in ("hash_overflow", "empty_pixels", "dropped_ids")},
             "loss": st["loss"],

@@ -199,8 +199,19 @@ int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream);
  * records (a1) in the same kernel. */
 int sad_adam_step(sad_ctx *ctx, const sad_adam_cfg *cfg, sad_stream_t stream);
 
-/* One steady-state fitting iteration: a propagation pass at jump 1 with G
- * injections, then render + loss + backward, then Adam (a2-a7). */
+/* Steps a2-a6 in one kernel: a propagation pass at jump 1 with G injections
+ * (same result as sad_propagate(ctx, 1, G)), then render, loss and backward
+ * on the new lists (same result as sad_backward, up to the summation order
+ * of the gradients).  Each 32 x 8 tile gathers the distinct sites of its and
+ * its halo's lists into a dense local index (at most 128 sites; tiles with
+ * more take a slower generic path) that serves both to de-duplicate the
+ * candidate union and to accumulate the tile's gradients ([P1] section 5 and
+ * B.4: per-tile shared-memory reduction, one global atomic per site and
+ * parameter).  Writes the bound image when one is bound. */
+int sad_fit_pass(sad_ctx *ctx, int G, sad_stream_t stream);
+
+/* One steady-state fitting iteration: sad_fit_pass then sad_adam_step
+ * (steps a2-a7, two kernels). */
 int sad_fit_iteration(sad_ctx *ctx, int G, const sad_adam_cfg *cfg, sad_stream_t stream);
 
 /* Copy the current table into dst (host or device uint32 [P][8], slot order).

@@ -143,5 +143,8 @@ class Sad:
     def adam_step(self, cfg):
         _lib.sad_adam_step(self.ctx, cfg, self.stream)
 
+    def fit_pass(self, G: int):
+        _lib.sad_fit_pass(self.ctx, G, self.stream)
+
     def fit_iteration(self, G: int, cfg):
         _lib.sad_fit_iteration(self.ctx, G, cfg, self.stream)

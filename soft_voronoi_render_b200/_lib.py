@@ -57,7 +57,7 @@ class sad_stats(ctypes.Structure):
 EXPORTED = (
     "sad_workspace_bytes", "sad_create", "sad_destroy", "sad_bind", "sad_reset", "sad_set_sites",
     "sad_get_sites", "sad_set_target", "sad_prep_records", "sad_topk_exact", "sad_refresh", "sad_propagate",
-    "sad_render", "sad_backward", "sad_adam_step", "sad_fit_iteration", "sad_get_table", "sad_set_table",
+    "sad_render", "sad_backward", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
     "sad_get_stats", "sad_get_loss", "sad_last_error",
 )
 
@@ -97,6 +97,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "sad_render": [vp, vp, vp],
         "sad_backward": [vp, cu32, vp],
         "sad_adam_step": [vp, ctypes.POINTER(sad_adam_cfg), vp],
+        "sad_fit_pass": [vp, ci, vp],
         "sad_fit_iteration": [vp, ci, ctypes.POINTER(sad_adam_cfg), vp],
         "sad_get_table": [vp, vp, vp],
         "sad_set_table": [vp, vp, vp],
@@ -211,6 +212,10 @@ def adam_cfg(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=1e-3, lr_theta=1e
 
 def sad_adam_step(ctx: int, cfg: sad_adam_cfg, stream=None) -> None:
     _check(ctx, load().sad_adam_step(ctx, ctypes.byref(cfg), _stream(stream)))
+
+
+def sad_fit_pass(ctx: int, G: int, stream=None) -> None:
+    _check(ctx, load().sad_fit_pass(ctx, G, _stream(stream)))
 
 
 def sad_fit_iteration(ctx: int, G: int, cfg: sad_adam_cfg, stream=None) -> None:

@@ -7,7 +7,7 @@
 #include <cstring>
 #include <new>
 
-#include "../../include/sad.h"
+#include "sad.h"
 #include "sad_device.cuh"
 #include "sad_launch.h"
 
@@ -263,11 +263,16 @@ int sad_fit_iteration(sad_ctx *ctx, int G, const sad_adam_cfg *cfg, sad_stream_t
     r = check_adam(ctx, cfg, h);
     if (r) return r;
     cudaStream_t st = cs(stream);
-    r = cuda_status(ctx, sad::launch_propagate(ctx->dev, 1, G, st), "propagate");
-    if (r) return r;
-    r = cuda_status(ctx, sad::launch_render_backward(ctx->dev, st), "backward");
+    r = cuda_status(ctx, sad::launch_fit_tile(ctx->dev, G, st), "fit pass");
     if (r) return r;
     return cuda_status(ctx, sad::launch_adam(ctx->dev, h, st), "adam");
+}
+
+int sad_fit_pass(sad_ctx *ctx, int G, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (G < 0 || G > SAD_MAX_INJECT) return fail(ctx, SAD_ERR_CAPACITY, "G=%d outside [0, %d]", G, SAD_MAX_INJECT);
+    return cuda_status(ctx, sad::launch_fit_tile(ctx->dev, G, cs(stream)), "fit pass");
 }
 
 int sad_get_table(sad_ctx *ctx, uint32_t *dst, sad_stream_t stream) {

@@ -147,4 +147,57 @@ struct Top8 {
     }
 };
 
+// Sum v[0..NV-1] over each maximal run of lanes holding the same key (runs in
+// lane order; a warp covers 32 consecutive pixels of a row, and neighbouring
+// pixels usually hold the same site in the same slot).  Afterwards the last
+// lane of every run holds the run's total.  Returns true on those lanes.
+template <int NV>
+__device__ __forceinline__ bool warp_run_reduce(uint32_t key, float (&v)[NV], int lane) {
+    constexpr unsigned FULL = 0xffffffffu;
+    const uint32_t key_next = __shfl_down_sync(FULL, key, 1);
+    const bool tail = lane == 31 || key_next != key;
+    const uint32_t tails = __ballot_sync(FULL, tail);
+    const uint32_t cont = ~tails;  // bit L: lanes L and L+1 share a run
+    if (cont) {
+        const uint32_t prev = tails & ((1u << lane) - 1u);
+        const int start = prev ? 32 - __clz(prev) : 0;
+        // doubling steps needed for the longest run (warp-uniform)
+        int levels = 1;
+        uint32_t r = cont & (cont >> 1);
+        if (r) {
+            levels = 2;
+            r &= r >> 2;
+            if (r) {
+                levels = 3;
+                r &= r >> 4;
+                if (r) {
+                    levels = 4;
+                    r &= r >> 8;
+                    if (r) levels = 5;
+                }
+            }
+        }
+#pragma unroll
+        for (int L = 0; L < 5; ++L) {
+            if (L < levels) {  // warp-uniform
+                const int off = 1 << L;
+                const bool take = lane - off >= start;
+#pragma unroll
+                for (int k = 0; k < NV; ++k) {
+                    const float x = __shfl_up_sync(FULL, v[k], off);
+                    if (take) v[k] += x;
+                }
+            }
+        }
+    }
+    return tail;
+}
+
+
+// workspace views
+__device__ __forceinline__ Counters *ws_counters(void *ws) { return reinterpret_cast<Counters *>(ws); }
+__device__ __forceinline__ double *ws_loss_partials(void *ws) {
+    return reinterpret_cast<double *>(reinterpret_cast<char *>(ws) + COUNTERS_BYTES);
+}
+
 }  // namespace sad

@@ -33,5 +33,6 @@ cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st);
 cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st);
 cudaError_t launch_render_backward(const Dev &d, cudaStream_t st);
 cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st);
+cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st);
 
 }  // namespace sad

@@ -315,23 +315,92 @@ def test_fit_iteration_c1(torch_cuda):
     assert s.stats()["adam_step"] == 1 and s.stats()["pass_counter"] == 1
 
 
+@pytest.mark.parametrize("wl,H,W,N", [("c1", None, None, None), ("c2", None, None, None),
+                                      ("c1", 37, 70, 400), ("c1", 8, 33, 50)])
+def test_fit_pass_matches_oracle(torch_cuda, wl, H, W, N):
+    """The fused pass (propagation at jump 1 + render + loss + backward) gives
+    the oracle's propagated table bit for bit and the oracle's gradients on it."""
+    tgt, prm, w = synth.make_workload(wl, seed=4, H=H, W=W, N=N)
+    H, W, N = tgt.shape[1], tgt.shape[2], prm.shape[1]
+    prm = prm.copy()
+    prm[0, 3] = -1.0
+    t0, npass = oracle.refresh(H, W, prm, 2, seed=21)
+    s = make_ctx(torch_cuda, H, W, N, prm, tgt, seed=21)
+    s.set_table(t0)
+    s.fit_pass(2)
+    rec = oracle.records(H, W, prm)
+    t1 = oracle.propagate(H, W, rec, t0, 1, 2, seed=21, pass_index=0)
+    np.testing.assert_array_equal(s.get_table(), t1)
+    L, g, img = oracle.loss_backward(H, W, prm, t1, tgt, want_image=True)
+    assert abs(s.loss() - L) <= LOSS_RTOL * L
+    assert np.abs(s.image.cpu().numpy() - img).max() <= RENDER_ATOL
+    assert_grads(s.grads.cpu().numpy(), g, "fit_pass")
+    st = s.stats()
+    assert st["pass_counter"] == 1 and st["current_table"] == 1
+
+
+def test_fit_pass_generic_path_for_crowded_tiles(torch_cuda):
+    """Random lists put far more than 128 distinct sites around each tile, so
+    every tile takes the generic path; results must not change."""
+    H, W, N = 40, 70, 30000
+    prm = synth.uniform_sites(H, W, N, 12)
+    tgt = synth.make_image(H, W, 8, 0, 12)
+    st = synth.Stream(12, "crowded")
+    t0 = st.integers(H * W * 8, N).astype(np.uint32).reshape(H * W, 8)
+    t0[st.uniform(H * W * 8).reshape(H * W, 8) < 0.1] = SENT
+    s = make_ctx(torch_cuda, H, W, N, prm, tgt, seed=5)
+    s.set_table(t0)
+    s.fit_pass(3)
+    rec = oracle.records(H, W, prm)
+    t1 = oracle.propagate(H, W, rec, t0, 1, 3, seed=5, pass_index=0)
+    np.testing.assert_array_equal(s.get_table(), t1)
+    L, g = oracle.loss_backward(H, W, prm, t1, tgt)
+    assert abs(s.loss() - L) <= LOSS_RTOL * L
+    assert_grads(s.grads.cpu().numpy(), g, "generic")
+    assert s.stats()["hash_overflow"] > 0
+
+
+def test_fit_pass_duplicate_ids_in_a_list(torch_cuda):
+    H, W, N = 16, 40, 200
+    prm = synth.uniform_sites(H, W, N, 13)
+    tgt = synth.make_image(H, W, 3, 0, 13)
+    t0 = oracle.topk_exact(H, W, oracle.records(H, W, prm))
+    t0[::3, 5] = t0[::3, 1]      # the same id twice in one list
+    t0[::7, 7] = N + 11          # an id beyond capacity
+    s = make_ctx(torch_cuda, H, W, N, prm, tgt, seed=6)
+    s.set_table(t0)
+    s.fit_pass(2)
+    t1 = oracle.propagate(H, W, oracle.records(H, W, prm), t0, 1, 2, seed=6, pass_index=0)
+    np.testing.assert_array_equal(s.get_table(), t1)
+    L, g = oracle.loss_backward(H, W, prm, t1, tgt)
+    assert_grads(s.grads.cpu().numpy(), g, "dups")
+
+
 @pytest.mark.slow
 def test_full_size_c3_iteration_pieces(torch_cuda):
-    """2048 x 2048, N = 131,072 (the benchmark workload), launched as the
-    benchmark launches it: one propagation pass is bit-exact against the
-    oracle, and render + backward agree with the oracle on the oracle's table."""
+    """2048 x 2048, N = 131,072 (the benchmark workload) with the benchmark's
+    launches: the fused pass is bit-exact against the oracle's propagation and
+    agrees with the oracle's render and backward; so do the separate
+    propagate and backward kernels on the next pass."""
     tgt, prm, w = synth.make_workload("c3", seed=1)
     s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt, seed=3)
     rec = oracle.records(w.H, w.W, prm)
     t, npass = oracle.refresh(w.H, w.W, prm, w.G, seed=3)
     s.set_table(t)
-    s.propagate(1, w.G)  # pass number 0 of this context
+    s.fit_pass(w.G)  # pass number 0 of this context
     ref = oracle.propagate(w.H, w.W, rec, t, 1, w.G, seed=3, pass_index=0)
     np.testing.assert_array_equal(s.get_table(), ref)
-    s.backward()
     L, g, img = oracle.loss_backward(w.H, w.W, prm, ref, tgt, want_image=True)
     assert abs(s.loss() - L) <= LOSS_RTOL * L
     assert np.abs(s.image.cpu().numpy() - img).max() <= RENDER_ATOL
-    assert_grads(s.grads.cpu().numpy(), g, "c3")
+    assert_grads(s.grads.cpu().numpy(), g, "c3 fused")
     st = s.stats()
-    assert st["empty_pixels"] == 0
+    assert st["empty_pixels"] == 0 and st["hash_overflow"] == 0
+    s.grads.zero_()
+    s.propagate(1, w.G)  # pass number 1
+    ref2 = oracle.propagate(w.H, w.W, rec, ref, 1, w.G, seed=3, pass_index=1)
+    np.testing.assert_array_equal(s.get_table(), ref2)
+    s.backward()
+    L2, g2 = oracle.loss_backward(w.H, w.W, prm, ref2, tgt)
+    assert abs(s.loss() - L2) <= LOSS_RTOL * L2
+    assert_grads(s.grads.cpu().numpy(), g2, "c3 separate")
