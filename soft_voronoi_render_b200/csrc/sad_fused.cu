@@ -132,9 +132,14 @@ struct FusedSmem {
     uint32_t ulist[UCAP];
     float4 urec[REC_F4][UCAP];   // field-major: conflict-free for distinct sites
     uint4 masks[HN];             // 128-bit membership of every tile + halo pixel
-    float acc[FY][NPARAM][UCAP];  // one private accumulator set per warp
-    uint32_t owner[FY][UCAP];     // per-warp election scratch for the accumulators
+    float acc[NPARAM][UCAP];      // the tile's gradient sums per local site
+    uint32_t cnt[UCAP];           // (pixel, slot) entries per local site
+    uint32_t cursor[UCAP];        // scatter cursor of the counting sort
+    float pix[6][FT];             // per pixel: chat (3) and dL/dchat (3)
+    float2 ent_wl[FT * K];        // entries grouped by site: softmax weight, logit
+    uint16_t ent_pu[FT * K];      //   pixel (low byte) and local site (high byte)
     float warp_loss[FT / 32];
+    uint32_t n_ent;
     uint32_t ucount;
     int overflow;
     int last;
@@ -149,20 +154,44 @@ __device__ __forceinline__ void set_bit(uint4 &m, uint32_t u) {
     m.w |= (w == 3) ? b : 0u;
 }
 
-__device__ __forceinline__ void load_record(const FusedSmem &sm, const float4 *__restrict__ rec, uint32_t id,
-                                            uint32_t lx, float4 &r0, float4 &r1, float4 &r2, float4 &r3) {
-    if (lx != NOLOC) {
-        r0 = sm.urec[0][lx];
-        r1 = sm.urec[1][lx];
-        r2 = sm.urec[2][lx];
-        r3 = sm.urec[3][lx];
-    } else {
-        const float4 *R = rec + (size_t)id * REC_F4;
-        r0 = __ldg(R);
-        r1 = __ldg(R + 1);
-        r2 = __ldg(R + 2);
-        r3 = __ldg(R + 3);
-    }
+// bounds of the run of equal keys (in lane order) that holds this lane
+__device__ __forceinline__ void run_bounds(uint32_t key, int lane, int &start, int &tail_lane) {
+    const uint32_t key_next = __shfl_down_sync(FULL, key, 1);
+    const bool tail = lane == 31 || key_next != key;
+    const uint32_t tails = __ballot_sync(FULL, tail);
+    const uint32_t prev = tails & ((1u << lane) - 1u);
+    start = prev ? 32 - __clz(prev) : 0;
+    tail_lane = __ffs(tails & (0xFFFFFFFFu << lane)) - 1;
+}
+
+// gradient contributions of one (pixel, slot) with softmax weight w and logit
+// l (both 0 for an unused slot, which then contributes exact zeros):
+//   gamma = w (c - chat) . g,  dL/dc = w g,  dL/dln tau = gamma l,
+//   dL/dr = gamma k,  dL/dp = gamma G'delta / m,
+//   dL/da = -gamma (k^2 e^a alpha^2 - k^2 e^-a beta^2) / (2 m),
+//   dL/dtheta = -gamma alpha beta (k^2 e^a - k^2 e^-a) / m
+// with m = sqrt(delta^T G' delta) = k n (0 where m = 0).
+__device__ __forceinline__ void slot_grad(const float4 r0, const float4 r1, const float4 r2, const float4 r3,
+                                          float fx, float fy, float l, float w, float cr, float cg, float cb,
+                                          float gr, float gg, float gb, float (&v)[NPARAM]) {
+    const float dx = fx - r0.x, dy = fy - r0.y;
+    const float u1 = fmaf(r0.z, dx, r0.w * dy);
+    const float u2 = fmaf(r1.x, dy, r0.w * dx);
+    const float qf = fmaf(dx, u1, dy * u2);
+    const float im = qf > 0.0f ? rsqrtf(qf) : 0.0f;
+    const float gamma = w * ((r2.x - cr) * gr + (r2.y - cg) * gg + (r2.z - cb) * gb);
+    const float gi = gamma * im;
+    const float al = r2.w * dx + r3.x * dy;   // u . delta
+    const float be = -r3.x * dx + r2.w * dy;  // v . delta
+    v[PX] = gi * u1;
+    v[PY] = gi * u2;
+    v[PLT] = gamma * l;
+    v[PR] = gamma * r1.z;
+    v[PCR] = w * gr;
+    v[PCG] = w * gg;
+    v[PCB] = w * gb;
+    v[PTH] = -gi * al * be * (r3.y - r3.z);
+    v[PA] = -0.5f * gi * (r3.y * al * al - r3.z * be * be);
 }
 
 // generic candidate offer (no tile index): dedup against the running list
@@ -221,8 +250,8 @@ __global__ void __launch_bounds__(FT, 3) fit_tile_kernel(const float4 *__restric
     const uint32_t Nu = (uint32_t)N;
 
     for (int q = tid; q < UHASH; q += FT) sm.keys[q] = EMPTY;
-    for (int q = tid; q < FY * NPARAM * UCAP / 4; q += FT)
-        reinterpret_cast<float4 *>(&sm.acc[0][0][0])[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int q = tid; q < NPARAM * UCAP; q += FT) (&sm.acc[0][0])[q] = 0.0f;
+    if (tid < UCAP) sm.cnt[tid] = 0;
     if (tid == 0) {
         sm.ucount = 0;
         sm.overflow = 0;
@@ -459,64 +488,119 @@ __global__ void __launch_bounds__(FT, 3) fit_tile_kernel(const float4 *__restric
             image[2 * P + p] = cb;
         }
     }
+    // ---- D2: group the tile's (pixel, slot) entries by site ----------------
+    // Entries whose site has a tile-local index are counted here and summed
+    // site by site below; the rare rest (injected winners, crowded tiles) go
+    // straight to global atomics.
     unsigned global_adds = 0;
+    sm.pix[0][tid] = cr;
+    sm.pix[1][tid] = cg;
+    sm.pix[2][tid] = cb;
+    sm.pix[3][tid] = gr;
+    sm.pix[4][tid] = gg;
+    sm.pix[5][tid] = gb;
 #pragma unroll
     for (int q = 0; q < K; ++q) {
         const bool vq = vmask >> q & 1u;
-        const uint32_t key = vq ? t.id[q] : EMPTY;
-        float v[NPARAM];
-#pragma unroll
-        for (int k = 0; k < NPARAM; ++k) v[k] = 0.0f;
-        if (vq) {
-            float4 r0, r1, r2, r3;
-            load_record(sm, rec, key, t.lx[q], r0, r1, r2, r3);
-            // delta, G' delta and 1/m = 1/sqrt(delta^T G' delta); the logit
-            // itself is the one the propagation computed
-            const float dx = fx - r0.x, dy = fy - r0.y;
-            const float u1 = fmaf(r0.z, dx, r0.w * dy);
-            const float u2 = fmaf(r1.x, dy, r0.w * dx);
-            const float qf = fmaf(dx, u1, dy * u2);
-            const float im = qf > 0.0f ? rsqrtf(qf) : 0.0f;
-            const float w = __expf(t.l[q] - M) * iz;
-            const float gamma = w * ((r2.x - cr) * gr + (r2.y - cg) * gg + (r2.z - cb) * gb);
-            const float gi = gamma * im;
-            const float al = r2.w * dx + r3.x * dy;   // u . delta
-            const float be = -r3.x * dx + r2.w * dy;  // v . delta
-            v[PX] = gi * u1;
-            v[PY] = gi * u2;
-            v[PLT] = gamma * t.l[q];
-            v[PR] = gamma * r1.z;
-            v[PCR] = w * gr;
-            v[PCG] = w * gg;
-            v[PCB] = w * gb;
-            v[PTH] = -gi * al * be * (r3.y - r3.z);
-            v[PA] = -0.5f * gi * (r3.y * al * al - r3.z * be * be);
-        }
-        const bool tail = warp_run_reduce(key, v, lane);
-        // run tails add their totals into this warp's private accumulators.
-        // Tails holding the same site (two separate runs of it in this slot)
-        // must not update it in the same step: each round, every pending tail
-        // writes its lane into the site's election cell, and the lane that
-        // reads itself back does its update.
-        bool todo = tail && key != EMPTY;
-        if (todo && t.lx[q] == NOLOC) {
+        // one counter update per run of equal sites in this slot
+        const uint32_t key = (vq && t.lx[q] != NOLOC) ? t.lx[q] : EMPTY;
+        int start, tail_lane;
+        run_bounds(key, lane, start, tail_lane);
+        if (lane == tail_lane && key != EMPTY) atomicAdd(&sm.cnt[key], (uint32_t)(tail_lane - start + 1));
+        if (vq && t.lx[q] == NOLOC) {
+            const float4 *R = rec + (size_t)t.id[q] * REC_F4;
+            float v[NPARAM];
+            slot_grad(__ldg(R), __ldg(R + 1), __ldg(R + 2), __ldg(R + 3), fx, fy, t.l[q], __expf(t.l[q] - M) * iz,
+                      cr, cg, cb, gr, gg, gb, v);
             ++global_adds;
 #pragma unroll
-            for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + key, v[k]);
-            todo = false;
+            for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + t.id[q], v[k]);
         }
-        while (__any_sync(FULL, todo)) {
-            const uint32_t u = t.lx[q];
-            if (todo) sm.owner[ty][u] = (uint32_t)lane;
-            __syncwarp();
-            const bool win = todo && sm.owner[ty][u] == (uint32_t)lane;
-            if (win) {
-                float *a = &sm.acc[ty][0][u];
+    }
+    __syncthreads();
+    if (ty == 0) {
+        // exclusive scan of the 128 counts by one warp, 4 per lane
+        uint32_t c4[4], run = 0;
 #pragma unroll
-                for (int k = 0; k < NPARAM; ++k) a[k * UCAP] += v[k];
+        for (int e = 0; e < 4; ++e) {
+            c4[e] = sm.cnt[lane * 4 + e];
+            run += c4[e];
+        }
+        uint32_t incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(FULL, incl, o);
+            if (lane >= o) incl += x;
+        }
+        uint32_t base = incl - run;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sm.cursor[lane * 4 + e] = base;
+            base += c4[e];
+        }
+        if (lane == 31) sm.n_ent = incl;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+        const bool vq = (vmask >> q & 1u) && t.lx[q] != NOLOC;
+        const uint32_t key = vq ? t.lx[q] : EMPTY;
+        int start, tail_lane;
+        run_bounds(key, lane, start, tail_lane);
+        uint32_t pos0 = 0;
+        if (lane == tail_lane && key != EMPTY) pos0 = atomicAdd(&sm.cursor[key], (uint32_t)(tail_lane - start + 1));
+        pos0 = __shfl_sync(FULL, pos0, tail_lane);
+        if (vq) {
+            const uint32_t pos = pos0 + (uint32_t)(lane - start);
+            sm.ent_wl[pos] = make_float2(__expf(t.l[q] - M) * iz, t.l[q]);
+            sm.ent_pu[pos] = (uint16_t)(tid | (key << 8));
+        }
+    }
+    __syncthreads();
+    // ---- D3: every thread sums a run of 8 consecutive entries -------------
+    {
+        const uint32_t n_ent = sm.n_ent;
+        const float fx0 = (float)i0 + 0.5f, fy0 = (float)j0 + 0.5f;
+        uint32_t cur = NOLOC;
+        float4 r0 = make_float4(0.f, 0.f, 0.f, 0.f), r1 = r0, r2 = r0, r3 = r0;
+        float a[NPARAM];
+#pragma unroll
+        for (int k = 0; k < NPARAM; ++k) a[k] = 0.0f;
+        const uint32_t e0 = (uint32_t)tid * K;
+#pragma unroll
+        for (int e = 0; e < K; ++e) {
+            const uint32_t idx = e0 + e;
+            if (idx >= n_ent) break;
+            const uint32_t pu = sm.ent_pu[idx];
+            const uint32_t u = pu >> 8, px = pu & 0xFFu;
+            if (u != cur) {
+                if (cur != NOLOC) {
+#pragma unroll
+                    for (int k = 0; k < NPARAM; ++k) {
+                        atomicAdd(&sm.acc[k][cur], a[k]);
+                        a[k] = 0.0f;
+                    }
+                }
+                cur = u;
+                r0 = sm.urec[0][u];
+                r1 = sm.urec[1][u];
+                r2 = sm.urec[2][u];
+                r3 = sm.urec[3][u];
             }
-            todo = todo && !win;
-            __syncwarp();
+            const float2 wl = sm.ent_wl[idx];
+            float v[NPARAM];
+            slot_grad(r0, r1, r2, r3, fx0 + (float)(px & (FX - 1)), fy0 + (float)(px / FX), wl.y, wl.x,
+                      sm.pix[0][px], sm.pix[1][px], sm.pix[2][px], sm.pix[3][px], sm.pix[4][px], sm.pix[5][px], v);
+#pragma unroll
+            for (int k = 0; k < NPARAM; ++k) a[k] += v[k];
+        }
+        // the last sites of consecutive lanes repeat (entries are sorted):
+        // sum each run across lanes first, then one update per run
+        const uint32_t key = cur == NOLOC ? EMPTY : cur;
+        const bool tail = warp_run_reduce(key, a, lane);
+        if (tail && key != EMPTY) {
+#pragma unroll
+            for (int k = 0; k < NPARAM; ++k) atomicAdd(&sm.acc[k][key], a[k]);
         }
     }
 
@@ -527,9 +611,7 @@ __global__ void __launch_bounds__(FT, 3) fit_tile_kernel(const float4 *__restric
     const int n_global = __syncthreads_count(global_adds != 0);
     for (uint32_t e = tid; e < ucount * NPARAM; e += FT) {
         const uint32_t u = e % ucount, k = e / ucount;
-        float a = 0.0f;
-#pragma unroll
-        for (int w = 0; w < FY; ++w) a += sm.acc[w][k][u];
+        const float a = sm.acc[k][u];
         if (a != 0.0f) atomicAdd(grads + (size_t)k * N + sm.ulist[u], a);
     }
     if (tid == 0) {
