@@ -230,6 +230,35 @@ int sad_get_loss(sad_ctx *ctx, double *loss, sad_stream_t stream);
 /* Message of the last failing call on this context ("" if none). */
 const char *sad_last_error(const sad_ctx *ctx);
 
+/* Render, loss and backward (the work of sad_backward) for callers that
+ * cannot allocate device memory -- for example code running inside another
+ * framework's fixed memory budget, or a plugin interface that receives only
+ * input and output pointers and may not request a workspace.  This entry
+ * point has no counterpart in the paper; it exists only for such callers.
+ * It needs no context and no workspace: its scratch (a 256-byte counter block
+ * plus one double per 32 x 8 tile) lives in a device array of
+ * SAD_NOALLOC_SCRATCH_BYTES that the library holds on every GPU that loads
+ * it, until the process exits.  It calls no cudaMalloc or cudaFree.
+ *   records  float32 [N_cap][16] score records (as sad_prep_records writes)
+ *   table    uint32  [2][P][4] the candidate table to render: plane 0 holds
+ *            slots 0-3, plane 1 slots 4-7
+ *   target   float32 [3][P];  image float32 [3][P] or NULL
+ *   grads    float32 [9][N_cap], accumulated into (zero it first)
+ *   loss     one device double, receives L
+ * Pointers 16-byte aligned (loss 8-byte).  Returns SAD_ERR_CAPACITY when
+ * ceil(W/32) * ceil(H/8) exceeds (SAD_NOALLOC_SCRATCH_BYTES - 256) / 8 =
+ * 131,040 tiles (4096 x 8192 fits), SAD_ERR_INVALID_ARG for bad sizes or
+ * pointers, SAD_ERR_CUDA when a CUDA call fails.  The first call on a device
+ * looks up the array's device address (a one-time set-up): make that first
+ * call before capturing a stream.  All calls on a device share the one
+ * array, which keeps the previous call's contents (each call clears what must
+ * start at zero): calls that may overlap on the GPU -- on different streams,
+ * or from several threads -- race on it and must be serialised by the
+ * caller. */
+#define SAD_NOALLOC_SCRATCH_BYTES (1u << 20)
+int sad_backward_noalloc(int H, int W, int N_cap, const float *records, const uint32_t *table,
+                         const float *target, float *image, float *grads, double *loss, sad_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

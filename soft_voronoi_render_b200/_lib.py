@@ -58,7 +58,7 @@ EXPORTED = (
     "sad_workspace_bytes", "sad_create", "sad_destroy", "sad_bind", "sad_reset", "sad_set_sites",
     "sad_get_sites", "sad_set_target", "sad_prep_records", "sad_topk_exact", "sad_refresh", "sad_propagate",
     "sad_render", "sad_backward", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
-    "sad_get_stats", "sad_get_loss", "sad_last_error",
+    "sad_get_stats", "sad_get_loss", "sad_last_error", "sad_backward_noalloc",
 )
 
 _lib = None
@@ -104,6 +104,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "sad_get_stats": [vp, ctypes.POINTER(sad_stats), vp],
         "sad_get_loss": [vp, ctypes.POINTER(ctypes.c_double), vp],
         "sad_last_error": [vp],
+        "sad_backward_noalloc": [ci, ci, ci, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -244,3 +245,11 @@ def sad_get_loss(ctx: int, stream=None) -> float:
 
 def sad_last_error(ctx: int) -> str:
     return load().sad_last_error(ctx).decode()
+
+
+def sad_backward_noalloc(H: int, W: int, N_cap: int, records, table, target, image, grads, loss,
+                         stream=None) -> None:
+    """Render + loss + backward without a context or workspace, for callers
+    that cannot allocate device memory (see include/sad.h)."""
+    _check(None, load().sad_backward_noalloc(H, W, N_cap, _ptr(records), _ptr(table), _ptr(target), _ptr(image),
+                                             _ptr(grads), _ptr(loss), _stream(stream)))

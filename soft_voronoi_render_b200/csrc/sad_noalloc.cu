@@ -1,0 +1,75 @@
+// sad_noalloc.cu -- render + loss + backward for callers that cannot allocate.
+//
+// Every other entry point runs on caller-bound buffers, including a
+// caller-provided workspace.  Some callers cannot provide one: code that runs
+// inside another framework's fixed memory budget, plugin interfaces that hand
+// over only input and output pointers, or latency-critical paths that must
+// not call cudaMalloc (it can synchronise the device).  For them this file
+// keeps the backward pass's scratch (a 256-byte counter block and one double
+// per 32 x 8 tile for the loss partials) in a file-scope device array that the
+// library owns for the life of the process, on every GPU that loads it.
+#include <cstdint>
+
+#include "sad.h"
+#include "sad_device.cuh"
+#include "sad_launch.h"
+
+namespace {
+
+constexpr size_t kScratchBytes = SAD_NOALLOC_SCRATCH_BYTES;
+constexpr int kTileX = 32, kTileY = 8;  // the tile of the render + backward kernel
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+// device address of g_noalloc_scratch per device, filled on first use
+void *g_scratch_addr[kMaxDevices] = {};
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace
+
+extern "C" int sad_backward_noalloc(int H, int W, int N_cap, const float *records, const uint32_t *table,
+                                    const float *target, float *image, float *grads, double *loss,
+                                    sad_stream_t stream) {
+    if (H < 1 || W < 1 || N_cap < 1 || (long long)H * W >= (1ll << 31)) return SAD_ERR_INVALID_ARG;
+    if (!records || !table || !target || !grads || !loss) return SAD_ERR_INVALID_ARG;
+    if (!aligned(records, 16) || !aligned(table, 16) || !aligned(target, 16) || !aligned(grads, 16) ||
+        (image && !aligned(image, 16)) || !aligned(loss, 8))
+        return SAD_ERR_INVALID_ARG;
+    const size_t tiles = (size_t)((W + kTileX - 1) / kTileX) * (size_t)((H + kTileY - 1) / kTileY);
+    if (sad::COUNTERS_BYTES + tiles * sizeof(double) > kScratchBytes) return SAD_ERR_CAPACITY;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SAD_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SAD_ERR_UNSUPPORTED;
+    if (!g_scratch_addr[dev]) {
+        // host code only sees a stand-in for the array: ask for its address on
+        // this device (a one-time set-up; do it before any stream capture)
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SAD_ERR_CUDA;
+        g_scratch_addr[dev] = p;
+    }
+    void *scratch = g_scratch_addr[dev];
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    // the array keeps the previous call's contents: the counters (current
+    // table 0, last-tile ticket, statistics) must start at zero
+    if (cudaMemsetAsync(scratch, 0, sad::COUNTERS_BYTES, st) != cudaSuccess) return SAD_ERR_CUDA;
+
+    sad::Dev d{};
+    d.H = H;
+    d.W = W;
+    d.N = N_cap;
+    d.P = (long long)H * W;
+    d.records = reinterpret_cast<float4 *>(const_cast<float *>(records));
+    d.table = const_cast<uint32_t *>(table);
+    d.target = const_cast<float *>(target);
+    d.image = image;
+    d.grads = grads;
+    d.ws = scratch;
+    if (sad::launch_render_backward(d, st) != cudaSuccess) return SAD_ERR_CUDA;
+    const double *src = &reinterpret_cast<const sad::Counters *>(scratch)->loss;
+    if (cudaMemcpyAsync(loss, src, sizeof(double), cudaMemcpyDeviceToDevice, st) != cudaSuccess) return SAD_ERR_CUDA;
+    return SAD_OK;
+}
