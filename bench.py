@@ -61,6 +61,25 @@ def parse():
     return ap.parse_args()
 
 
+def reduce_max(x: float, device=None) -> float:
+    """Max of a float over the ranks of the current process group (identity
+    without one).  Uses a CPU tensor under gloo and a device tensor under
+    nccl."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    dev = device if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_mpix(world: int, pixels_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's pixels over the slowest rank's time."""
+    return world * pixels_per_rank * steps / (ms_max * 1e-3) / 1e6
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -304,13 +323,9 @@ def run_ours(args):
     for e in evs:
         per_kernel["fit_pass"] += e[0].elapsed_time(e[1])
         per_kernel["adam"] += e[1].elapsed_time(e[2])
-    ms_max = ms_total
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = reduce_max(ms_total, dev)
     ms_step = ms_max / K
-    value = world * P * K / (ms_max * 1e-3) / 1e6
+    value = aggregate_mpix(world, P, K, ms_max)
 
     # end to end through the C ABI: host target copied in, loss read back
     E = max(1, min(args.e2e_steps, K))
@@ -327,12 +342,8 @@ def run_ours(args):
         _lib.sad_get_loss(ctx, sp)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * P * E / (e2e_ms * 1e-3) / 1e6
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
+    e2e_value = aggregate_mpix(world, P, E, e2e_ms)
     st = s.stats()
 
     if rank == 0:
