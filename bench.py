@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--workload", default="c3", choices=["c3", "c4"],
+                    help="c3: the fitting-iteration metric (default); c4: full candidate refresh + render at "
+                         "4096x4096, N=524,288 (a secondary measurement)")
     return ap.parse_args()
 
 
@@ -386,10 +389,56 @@ def run_ours(args):
     return 0
 
 
+def run_refresh(args):
+    """Full candidate refresh from scratch (seed pass + jumps 2048..1 with
+    G = 4) followed by a render, at 4096 x 4096 with N = 524,288."""
+    import torch
+    import synth
+    from soft_voronoi_render_b200 import Sad, _lib
+
+    tgt, prm, wl = synth.make_workload("c4", seed=1)
+    H, W, N, G, P = wl.H, wl.W, wl.N, wl.G, wl.H * wl.W
+    s = Sad(H, W, N, seed=1)
+    s.set_sites(prm)
+    s.set_target(tgt)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    for _ in range(max(args.warmup, 3)):
+        _lib.sad_refresh(s.ctx, G, sp)
+        _lib.sad_render(s.ctx, None, sp)
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for k in range(K):
+        ev[k][0].record(stream)
+        _lib.sad_refresh(s.ctx, G, sp)
+        ev[k][1].record(stream)
+        _lib.sad_render(s.ctx, None, sp)
+        ev[k][2].record(stream)
+    torch.cuda.synchronize()
+    t_ref = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    t_ren = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    hbm, peak_kind = measured_peaks()
+    passes = 12
+    alg = passes * 64 * P + 32 * P + 44 * P  # passes: list read+write; clear; render list+image
+    line = {"metric": "ms per full candidate refresh (seed + 12 passes, G=4) + render, 4096x4096 N=524,288",
+            "value": t_ref + t_ren, "unit": "ms", "higher_is_better": False, "n_gpus": 1, "steps": K,
+            "warmup": max(args.warmup, 3), "refresh_ms": t_ref, "render_ms": t_ren,
+            "mpix_per_s_per_pass": P * passes / (t_ref * 1e-3) / 1e6, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"c4: {wl.description}", "H": H, "W": W, "N": N, "G": G},
+            "hbm_roof_frac": alg / ((t_ref + t_ren) * 1e-3) / 1e9 / hbm, "peak_kind": peak_kind,
+            "device_stats": s.stats()}
+    print(json.dumps(line), flush=True)
+    s.close()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "c4":
+        return run_refresh(args)
     return run_ours(args)
 
 

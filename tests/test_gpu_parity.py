@@ -404,3 +404,31 @@ def test_full_size_c3_iteration_pieces(torch_cuda):
     L2, g2 = oracle.loss_backward(w.H, w.W, prm, ref2, tgt)
     assert abs(s.loss() - L2) <= LOSS_RTOL * L2
     assert_grads(s.grads.cpu().numpy(), g2, "c3 separate")
+
+
+@pytest.mark.slow
+def test_full_size_c4_refresh_and_render(torch_cuda):
+    """4096 x 4096, N = 524,288: the full refresh (seed + jumps 2048..1, G = 4)
+    is bit-exact against the oracle's, the render of it agrees, and the
+    refreshed lists reach the exact top-8 on most sampled pixels."""
+    tgt, prm, w = synth.make_workload("c4", seed=1)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt, seed=17)
+    s.refresh(w.G)
+    ref, npass = oracle.refresh(w.H, w.W, prm, w.G, seed=17)
+    got = s.get_table()
+    np.testing.assert_array_equal(got, ref)
+    assert npass == 12
+    s.render()
+    img = s.image.cpu().numpy()
+    pix = synth.Stream(4, "c4-render").integers(200_000, w.H * w.W)
+    ref_img = oracle.render(w.H, w.W, prm, ref)  # full image in double
+    assert np.abs(img.reshape(3, -1)[:, pix] - ref_img.reshape(3, -1)[:, pix]).max() <= RENDER_ATOL
+    assert np.abs(img - ref_img).max() <= RENDER_ATOL
+    sample = synth.Stream(4, "c4-recall").integers(1024, w.H * w.W)
+    ex = oracle.topk_exact(w.H, w.W, oracle.records(w.H, w.W, prm), sample)
+    hit = [len(set(a.tolist()) & set(b.tolist()) - {SENT}) / max(1, int((b != SENT).sum()))
+           for a, b in zip(got[sample], ex)]
+    # a refresh from scratch, no extra passes: 0.974 recall@8 and 0.909 right
+    # owners for this seed (the lists equal the oracle's bit for bit above)
+    assert np.mean(hit) >= 0.97
+    assert np.mean(got[sample][:, 0] == ex[:, 0]) >= 0.9
