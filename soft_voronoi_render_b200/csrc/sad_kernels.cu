@@ -165,28 +165,28 @@ __global__ void seed_scatter_kernel(const float *__restrict__ prm, int N, int H,
 // ---------------------------------------------------------------------------
 // a2/a3: one Jacobi propagation pass.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void offer(Top8 &t, uint32_t id, const float4 *__restrict__ rec, uint32_t N,
-                                      float fx, float fy) {
-    if (id >= N) return;  // also rejects the empty marker
-    if (t.has(id)) return;
-    const float4 r0 = __ldg(rec + (size_t)id * REC_F4);
-    if (!(r0.x >= 0.0f)) return;
-    const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
-    const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
-    if (l != l) return;
-    if (t.beats_last(l, id)) t.insert(l, id);
-}
-
-__device__ __forceinline__ void offer8(Top8 &t, uint4 a, uint4 b, const float4 *__restrict__ rec, uint32_t N,
-                                       float fx, float fy) {
-    offer(t, a.x, rec, N, fx, fy);
-    offer(t, a.y, rec, N, fx, fy);
-    offer(t, a.z, rec, N, fx, fy);
-    offer(t, a.w, rec, N, fx, fy);
-    offer(t, b.x, rec, N, fx, fy);
-    offer(t, b.y, rec, N, fx, fy);
-    offer(t, b.z, rec, N, fx, fy);
-    offer(t, b.w, rec, N, fx, fy);
+// Offer a batch of up to 8 candidate ids.  Their records are fetched
+// together (independent loads in flight), then the candidates are offered in
+// order; the duplicate check runs at insertion time, so the result is the
+// same as offering them one by one.
+template <int NB>
+__device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], const float4 *__restrict__ rec,
+                                            uint32_t N, float fx, float fy) {
+    float l[NB];
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        l[q] = __int_as_float(0x7fc00000);  // NaN: not a candidate
+        const uint32_t id = ids[q];
+        if (id < N && !t.has(id)) {
+            const float4 r0 = __ldg(rec + (size_t)id * REC_F4);
+            const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
+            if (r0.x >= 0.0f) l[q] = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        if (l[q] == l[q] && t.beats_last(l[q], ids[q]) && !t.has(ids[q])) t.insert(l[q], ids[q]);
+    }
 }
 
 __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *__restrict__ rec, uint32_t *table,
@@ -205,22 +205,32 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
         const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
         Top8 t;
         t.clear();
-        offer8(t, in0[p], in1[p], rec, (uint32_t)N, fx, fy);
-        if (i - jump >= 0) offer8(t, in0[p - jump], in1[p - jump], rec, (uint32_t)N, fx, fy);
-        if (i + jump < W) offer8(t, in0[p + jump], in1[p + jump], rec, (uint32_t)N, fx, fy);
-        if (j - jump >= 0) {
-            const size_t pn = p - (size_t)jump * W;
-            offer8(t, in0[pn], in1[pn], rec, (uint32_t)N, fx, fy);
-        }
-        if (j + jump < H) {
-            const size_t pn = p + (size_t)jump * W;
-            offer8(t, in0[pn], in1[pn], rec, (uint32_t)N, fx, fy);
+        // own list, then the neighbours at (-k, 0), (+k, 0), (0, -k), (0, +k)
+#pragma unroll 1
+        for (int d = 0; d < 5; ++d) {
+            const int ni = i + (d == 1 ? -jump : (d == 2 ? jump : 0));
+            const int nj = j + (d == 3 ? -jump : (d == 4 ? jump : 0));
+            if (ni < 0 || ni >= W || nj < 0 || nj >= H) continue;
+            const size_t pn = (size_t)nj * W + ni;
+            const uint4 a = in0[pn], b = in1[pn];
+            const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            offer_batch<8>(t, ids, rec, (uint32_t)N, fx, fy);
         }
         if (G > 0) {
             uint32_t h = inject_state(seed, pass, (uint32_t)p);
-            for (int g = 0; g < G; ++g) {
-                h = xorshift32(h);
-                offer(t, __umulhi(h, (uint32_t)N), rec, (uint32_t)N, fx, fy);
+#pragma unroll 1
+            for (int g0 = 0; g0 < G; g0 += 4) {
+                uint32_t ids[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (g0 + q < G) {
+                        h = xorshift32(h);
+                        ids[q] = __umulhi(h, (uint32_t)N);
+                    } else {
+                        ids[q] = EMPTY;
+                    }
+                }
+                offer_batch<4>(t, ids, rec, (uint32_t)N, fx, fy);
             }
         }
         out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
