@@ -49,6 +49,12 @@ def lib():
         L.orc_loss_backward.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp]
         L.orc_loss_backward.restype = c_dbl
         L.orc_adam.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, c_dbl, c_dbl, c_dbl, c_int]
+        L.orc_loss_backward_stats.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, vp]
+        L.orc_loss_backward_stats.restype = c_dbl
+        L.orc_split_score.argtypes = [ctypes.c_float] * 4
+        L.orc_split_score.restype = ctypes.c_float
+        L.orc_densify_prune.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp]
+        L.orc_densify_prune.restype = c_int
         L.orc_num_threads.restype = c_int
         L.orc_set_threads.argtypes = [c_int]
         _lib = L
@@ -209,3 +215,88 @@ def adam(H: int, W: int, params, m, v, grads, lr, t: int, b1: float = 0.9, b2: f
         lrv = np.ascontiguousarray(lr, dtype=np.float64)
     lib().orc_adam(H, W, P.shape[1], _p(P), _p(M), _p(V), _p(G), _p(lrv), b1, b2, eps, int(t))
     return P, M, V
+
+
+STAT_NAMES = ("mass", "energy", "sxx", "sxy", "syy", "removal")
+
+
+def loss_backward_stats(H: int, W: int, params, table, target):
+    """Returns (loss, grads (9, N), stats (6, N)) in float64; stats rows are
+    STAT_NAMES."""
+    params = _f32(params)
+    tab = _u32(table).reshape(H * W, K)
+    tgt = _f32(target).reshape(3, H * W)
+    N = params.shape[1]
+    g = np.empty((9, N), dtype=np.float64)
+    st = np.empty((6, N), dtype=np.float64)
+    L = lib().orc_loss_backward_stats(H, W, N, _p(params), _p(tab), _p(tgt), _p(g), None, _p(st))
+    return L, g, st
+
+
+class DensifyCfg(ctypes.Structure):
+    _fields_ = [("grow", ctypes.c_int), ("prune_frac", ctypes.c_float), ("alpha", ctypes.c_float),
+                ("eps", ctypes.c_float), ("r_scale", ctypes.c_float), ("log_tau_shift", ctypes.c_float),
+                ("offset_scale", ctypes.c_float), ("fallback_offset", ctypes.c_float)]
+
+
+def densify_cfg(grow=2500, prune_frac=0.005, alpha=0.5, eps=1e-6, r_scale=0.85, log_tau_shift=0.6931471805599453,
+                offset_scale=0.5, fallback_offset=0.5) -> DensifyCfg:
+    return DensifyCfg(grow, prune_frac, alpha, eps, r_scale, log_tau_shift, offset_scale, fallback_offset)
+
+
+def split_score(m, E, alpha=0.5, eps=1e-6) -> float:
+    return float(lib().orc_split_score(m, E, alpha, eps))
+
+
+def densify_prune(H: int, W: int, params, m, v, stats, target, cfg: DensifyCfg):
+    """One densify/prune event on float32 state (copies).  Returns
+    (params, m, v, n_split, n_pruned)."""
+    P_ = np.array(params, dtype=np.float32, order="C", copy=True)
+    M = np.array(m, dtype=np.float32, order="C", copy=True)
+    V = np.array(v, dtype=np.float32, order="C", copy=True)
+    S = np.ascontiguousarray(stats, dtype=np.float32)
+    T = _f32(target).reshape(3, H * W)
+    npr = ctypes.c_int(0)
+    ns = lib().orc_densify_prune(H, W, P_.shape[1], _p(P_), _p(M), _p(V), _p(S), _p(T), ctypes.byref(cfg),
+                                 ctypes.byref(npr))
+    return P_, M, V, int(ns), int(npr.value)
+
+
+def fit(H: int, W: int, params, target, N_cap: int, iterations: int, events, grow: int, prune_frac: float,
+        lr: dict, G: int, seed: int, on_event=None):
+    """The oracle's fitting schedule, step for step the device driver's: a
+    refresh, then iterations of (propagate k=1, loss + backward, Adam in
+    double stored as float32, records); an event iteration also accumulates
+    the statistics, densifies/prunes and refreshes.  Returns (params float32
+    (9, N_cap), last loss, number of propagation passes run)."""
+    prm = np.zeros((9, N_cap), dtype=np.float32)
+    n0 = params.shape[1]
+    prm[:, :n0] = params
+    prm[0, n0:] = -1.0
+    m = np.zeros((9, N_cap), dtype=np.float32)
+    v = np.zeros((9, N_cap), dtype=np.float32)
+    tab, npass = refresh(H, W, prm, G, seed, 0)
+    rec = records(H, W, prm)
+    dcfg = densify_cfg(grow=grow, prune_frac=prune_frac)
+    events = set(events)
+    step = 0
+    L = None
+    for it in range(1, iterations + 1):
+        tab = propagate(H, W, rec, tab, 1, G, seed, npass)
+        npass += 1
+        if it in events:
+            L, g, st = loss_backward_stats(H, W, prm, tab, target)
+        else:
+            L, g = loss_backward(H, W, prm, tab, target)
+        step += 1
+        P64, M64, V64 = adam(H, W, prm, m, v, g, lr, step, float(np.float32(0.9)), float(np.float32(0.999)),
+                             float(np.float32(1e-8)))
+        prm, m, v = P64.astype(np.float32), M64.astype(np.float32), V64.astype(np.float32)
+        if it in events:
+            prm, m, v, _, _ = densify_prune(H, W, prm, m, v, st.astype(np.float32), target, dcfg)
+            tab, n = refresh(H, W, prm, G, seed, npass)
+            npass += n
+            if on_event is not None:
+                on_event(it, prm)
+        rec = records(H, W, prm)
+    return prm, L, npass

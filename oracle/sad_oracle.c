@@ -479,30 +479,72 @@ void orc_weights(int H, int W, int N, const float *params, const uint32_t *table
  * grads: 9 x N doubles in parameter-plane order (overwritten).  image
  * (optional): 3 x P doubles.  Returns L.
  */
+double orc_loss_backward_stats(int H, int W, int N, const float *params, const uint32_t *table,
+                               const float *target, double *grads, double *image, double *stats);
+
 double orc_loss_backward(int H, int W, int N, const float *params, const uint32_t *table,
                          const float *target, double *grads, double *image)
+{
+    return orc_loss_backward_stats(H, W, N, params, table, target, grads, image, NULL);
+}
+
+/*
+ * As orc_loss_backward, and when stats is not NULL also the per-site
+ * statistics of the budget control ([P1] B.4-B.5: mass, energy, weighted
+ * second moments, removal delta), 6 x N doubles:
+ *   m_i   = sum_x w_i
+ *   E_i   = sum_x w_i e(x),                 e(x) = |chat - t|^2
+ *   Sxx_i, Sxy_i, Syy_i = sum_x w_i e(x) (dx^2, dx dy, dy^2),  (dx, dy) = x - p_i
+ *   D_i   = sum_x [ |(chat - w_i c_i) / max(1 - w_i, 1e-6) - t|^2 - e(x) ]
+ * (D_i: the error after removing site i and renormalising the remaining
+ * weights, minus the error with it).
+ */
+double orc_loss_backward_stats(int H, int W, int N, const float *params, const uint32_t *table,
+                               const float *target, double *grads, double *image, double *stats)
 {
     const int64_t P = (int64_t)H * W;
     const double s = 1.0 / (double)(H > W ? H : W);
     site64_t *S = sites64(N, params);
     const int T = omp_threads();
-    double *acc = (double *)calloc((size_t)T * P_COUNT * (size_t)(N > 0 ? N : 1), sizeof(double));
+    const int NA = P_COUNT + 6; /* gradients, then statistics */
+    double *acc = (double *)calloc((size_t)T * NA * (size_t)(N > 0 ? N : 1), sizeof(double));
     double *lossp = (double *)calloc((size_t)T, sizeof(double));
 #pragma omp parallel
     {
         const int tid = omp_thread_id();
-        double *A = acc + (size_t)tid * P_COUNT * N;
+        double *A = acc + (size_t)tid * NA * N;
+        double *St = A + (size_t)P_COUNT * N;
         double lsum = 0.0;
 #pragma omp for schedule(static)
         for (int64_t p = 0; p < P; ++p) {
             pixel64_t o;
             render_pixel(S, N, s, table + p * ORC_K, p, W, &o);
-            double g[3];
+            double g[3], ex = 0.0;
             for (int ch = 0; ch < 3; ++ch) {
                 const double e = o.chat[ch] - (double)target[ch * P + p];
                 lsum += e * e;
+                ex += e * e;
                 g[ch] = 2.0 * e / (double)P;
                 if (image) image[ch * P + p] = o.chat[ch];
+            }
+            if (stats) {
+                for (int q = 0; q < o.n; ++q) {
+                    const site64_t *z = &S[o.id[q]];
+                    const int64_t i = o.id[q];
+                    const double w = o.w[q];
+                    double rem = 0.0;
+                    const double den = (1.0 - w) > 1e-6 ? (1.0 - w) : 1e-6;
+                    for (int ch = 0; ch < 3; ++ch) {
+                        const double c2 = (o.chat[ch] - w * z->c[ch]) / den - (double)target[ch * P + p];
+                        rem += c2 * c2;
+                    }
+                    St[0 * (size_t)N + i] += w;
+                    St[1 * (size_t)N + i] += w * ex;
+                    St[2 * (size_t)N + i] += w * ex * o.dx[q] * o.dx[q];
+                    St[3 * (size_t)N + i] += w * ex * o.dx[q] * o.dy[q];
+                    St[4 * (size_t)N + i] += w * ex * o.dy[q] * o.dy[q];
+                    St[5 * (size_t)N + i] += rem - ex;
+                }
             }
             for (int q = 0; q < o.n; ++q) {
                 const site64_t *z = &S[o.id[q]];
@@ -534,10 +576,13 @@ double orc_loss_backward(int H, int W, int N, const float *params, const uint32_
         lossp[tid] = lsum;
     }
     memset(grads, 0, sizeof(double) * P_COUNT * (size_t)N);
+    if (stats) memset(stats, 0, sizeof(double) * 6 * (size_t)N);
     double L = 0.0;
     for (int t = 0; t < T; ++t) {
-        const double *A = acc + (size_t)t * P_COUNT * N;
+        const double *A = acc + (size_t)t * NA * N;
         for (size_t q = 0; q < (size_t)P_COUNT * N; ++q) grads[q] += A[q];
+        if (stats)
+            for (size_t q = 0; q < (size_t)6 * N; ++q) stats[q] += A[(size_t)P_COUNT * N + q];
         L += lossp[t];
     }
     free(acc);
@@ -575,4 +620,185 @@ void orc_adam(int H, int W, int N, double *params, double *m, double *v, const d
             params[q] -= lr[j] * sig * mh / (sqrt(vh) + eps);
         }
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Budget control: densify and prune ([P1] B.5, [P2] key design 4)            */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int grow;               /* net sites added per event */
+    float prune_frac;       /* fraction of active sites pruned per event */
+    float alpha;            /* score exponent */
+    float eps;              /* mass floor */
+    float r_scale;          /* child radius factor */
+    float log_tau_shift;    /* subtracted from the children's ln tau */
+    float offset_scale;     /* child offset = offset_scale * sqrt(lambda_max) */
+    float fallback_offset;  /* child offset (px) when the second moment is degenerate */
+} orc_densify_cfg;
+
+typedef struct {
+    float key;
+    uint32_t id;
+} keyed_t;
+
+static int by_key_desc(const void *a, const void *b)
+{
+    const keyed_t *x = (const keyed_t *)a, *y = (const keyed_t *)b;
+    if (x->key > y->key) return -1;
+    if (x->key < y->key) return 1;
+    return (x->id < y->id) ? -1 : (x->id > y->id);
+}
+
+static int by_key_asc(const void *a, const void *b)
+{
+    const keyed_t *x = (const keyed_t *)a, *y = (const keyed_t *)b;
+    if (x->key < y->key) return -1;
+    if (x->key > y->key) return 1;
+    return (x->id < y->id) ? -1 : (x->id > y->id);
+}
+
+static int cmp_u32(const void *a, const void *b)
+{
+    const uint32_t x = *(const uint32_t *)a, y = *(const uint32_t *)b;
+    return (x > y) - (x < y);
+}
+
+/* the float32 split score E / max(m, eps)^alpha (sqrt when alpha = 0.5) */
+float orc_split_score(float m, float E, float alpha, float eps)
+{
+    const float mm = m > eps ? m : eps;
+    return alpha == 0.5f ? E / sqrtf(mm) : E / powf(mm, alpha);
+}
+
+/*
+ * One densify/prune event on float32 state.  stats: 6 x N float32 as
+ * accumulated by the backward pass.  Decisions are taken on the float32
+ * statistics:
+ *   1. prune the floor(prune_frac * n_active) active sites with the smallest
+ *      removal delta D (ties: smaller id first): x = -1.
+ *   2. split the min(n_pruned + grow, free slots, remaining active) active
+ *      sites with the largest score E / max(m, eps)^alpha (ties: smaller id);
+ *      parents in ascending id take the free slots in ascending id.
+ *   3. split geometry in double: C = S / E; major eigenvector e (sign: e.x > 0,
+ *      or e.x == 0 and e.y > 0) with eigenvalue l; offset d = offset_scale *
+ *      sqrt(l) * e; if E <= 0 or l <= 0, d = fallback_offset * (v if a > 0
+ *      else u), the metric's long axis.  Child A (parent slot) at p + d,
+ *      child B (free slot) at p - d, both clamped into the image; colour =
+ *      target at the child's pixel; r *= r_scale; ln tau -= log_tau_shift;
+ *      theta and a kept; Adam moments of both slots zeroed.
+ * Returns the number of splits; *n_pruned receives the number pruned.
+ */
+int orc_densify_prune(int H, int W, int N, float *params, float *m1, float *m2, const float *stats,
+                      const float *target, const orc_densify_cfg *cfg, int *n_pruned)
+{
+    const int64_t P = (int64_t)H * W;
+    keyed_t *keys = (keyed_t *)malloc(sizeof(keyed_t) * (size_t)(N > 0 ? N : 1));
+    uint32_t *freel = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)(N > 0 ? N : 1));
+    uint32_t *parents = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)(N > 0 ? N : 1));
+    int n_active = 0;
+    for (int i = 0; i < N; ++i) n_active += params[P_X * N + i] >= 0.0f;
+    int n_prune = (int)((double)cfg->prune_frac * (double)n_active);
+    /* prune: smallest removal delta among active sites with a number */
+    int nk = 0;
+    for (int i = 0; i < N; ++i) {
+        const float d = stats[5 * N + i];
+        if (params[P_X * N + i] >= 0.0f && d == d) keys[nk++] = (keyed_t){d, (uint32_t)i};
+    }
+    if (n_prune > nk) n_prune = nk;
+    qsort(keys, (size_t)nk, sizeof(keyed_t), by_key_asc);
+    for (int q = 0; q < n_prune; ++q) params[P_X * N + keys[q].id] = -1.0f;
+    /* split: largest score among the remaining active sites */
+    nk = 0;
+    for (int i = 0; i < N; ++i) {
+        if (!(params[P_X * N + i] >= 0.0f)) continue;
+        const float sc = orc_split_score(stats[0 * N + i], stats[1 * N + i], cfg->alpha, cfg->eps);
+        if (sc == sc) keys[nk++] = (keyed_t){sc, (uint32_t)i};
+    }
+    int nf = 0;
+    for (int i = 0; i < N; ++i)
+        if (!(params[P_X * N + i] >= 0.0f)) freel[nf++] = (uint32_t)i;
+    int n_split = n_prune + cfg->grow;
+    if (n_split > nf) n_split = nf;
+    if (n_split > nk) n_split = nk;
+    if (n_split < 0) n_split = 0;
+    qsort(keys, (size_t)nk, sizeof(keyed_t), by_key_desc);
+    for (int q = 0; q < n_split; ++q) parents[q] = keys[q].id;
+    qsort(parents, (size_t)n_split, sizeof(uint32_t), cmp_u32);
+    const double maxx = nextafter((double)(float)W, 0.0), maxy = nextafter((double)(float)H, 0.0);
+    for (int q = 0; q < n_split; ++q) {
+        const uint32_t a_id = parents[q], b_id = freel[q];
+        float pv[P_COUNT];
+        for (int j = 0; j < P_COUNT; ++j) pv[j] = params[j * (size_t)N + a_id];
+        const double E = stats[1 * N + a_id];
+        double dx = 0.0, dy = 0.0;
+        int ok = 0;
+        if (E > 0.0) {
+            const double cxx = stats[2 * N + a_id] / E, cxy = stats[3 * N + a_id] / E, cyy = stats[4 * N + a_id] / E;
+            const double hm = 0.5 * (cxx - cyy);
+            const double lam = 0.5 * (cxx + cyy) + sqrt(hm * hm + cxy * cxy);
+            if (lam > 0.0) {
+                double ex, ey;
+                if (cxy != 0.0) {
+                    ex = lam - cyy;
+                    ey = cxy;
+                } else if (cxx >= cyy) {
+                    ex = 1.0;
+                    ey = 0.0;
+                } else {
+                    ex = 0.0;
+                    ey = 1.0;
+                }
+                const double nrm = sqrt(ex * ex + ey * ey);
+                ex /= nrm;
+                ey /= nrm;
+                if (ex < 0.0 || (ex == 0.0 && ey < 0.0)) {
+                    ex = -ex;
+                    ey = -ey;
+                }
+                const double off = (double)cfg->offset_scale * sqrt(lam);
+                dx = off * ex;
+                dy = off * ey;
+                ok = 1;
+            }
+        }
+        if (!ok) {
+            const double th = pv[P_TH], c = cos(th), sn = sin(th);
+            const double f = (double)cfg->fallback_offset;
+            if (pv[P_A] > 0.0f) {
+                dx = -sn * f;
+                dy = c * f;
+            } else {
+                dx = c * f;
+                dy = sn * f;
+            }
+        }
+        for (int side = 0; side < 2; ++side) {
+            const uint32_t dst = side == 0 ? a_id : b_id;
+            const double sg = side == 0 ? 1.0 : -1.0;
+            double x = (double)pv[P_X] + sg * dx, y = (double)pv[P_Y] + sg * dy;
+            x = x < 0.0 ? 0.0 : (x > maxx ? maxx : x);
+            y = y < 0.0 ? 0.0 : (y > maxy ? maxy : y);
+            float fxv = (float)x, fyv = (float)y;
+            if (fxv >= (float)W) fxv = nextafterf((float)W, 0.0f);
+            if (fyv >= (float)H) fyv = nextafterf((float)H, 0.0f);
+            const int64_t pix = (int64_t)floorf(fyv) * W + (int64_t)floorf(fxv);
+            params[P_X * (size_t)N + dst] = fxv;
+            params[P_Y * (size_t)N + dst] = fyv;
+            params[P_LT * (size_t)N + dst] = pv[P_LT] - cfg->log_tau_shift;
+            params[P_R * (size_t)N + dst] = pv[P_R] * cfg->r_scale;
+            for (int ch = 0; ch < 3; ++ch) params[(P_CR + ch) * (size_t)N + dst] = target[ch * P + pix];
+            params[P_TH * (size_t)N + dst] = pv[P_TH];
+            params[P_A * (size_t)N + dst] = pv[P_A];
+            for (int j = 0; j < P_COUNT; ++j) {
+                m1[j * (size_t)N + dst] = 0.0f;
+                m2[j * (size_t)N + dst] = 0.0f;
+            }
+        }
+    }
+    free(keys);
+    free(freel);
+    free(parents);
+    if (n_pruned) *n_pruned = n_prune;
+    return n_split;
 }
