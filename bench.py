@@ -58,9 +58,11 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
-    ap.add_argument("--workload", default="c3", choices=["c3", "c4"],
+    ap.add_argument("--workload", default="c3", choices=["c3", "c4", "c5"],
                     help="c3: the fitting-iteration metric (default); c4: full candidate refresh + render at "
-                         "4096x4096, N=524,288 (a secondary measurement)")
+                         "4096x4096, N=524,288; c5: end-to-end 768x512 fit with densify/prune (secondary "
+                         "measurements)")
+    ap.add_argument("--oracle-fit", action="store_true", help="c5: also run the CPU oracle's fit (minutes)")
     return ap.parse_args()
 
 
@@ -433,8 +435,57 @@ def run_refresh(args):
     return 0
 
 
+def run_fit(args):
+    """End-to-end fit of the 768 x 512 workload: 10,000 gradient-weighted
+    sites growing to 50,000 (densify/prune events every 100 iterations from
+    100 to 1600, +2,500 net each, 0.5 % pruned), 2000 iterations, Adam
+    (lr 1e-3 positions, 5e-3 colours).  Reports time to fit and final PSNR."""
+    import torch
+    import synth
+    from soft_voronoi_render_b200 import Sad, fit
+
+    tgt, prm, wl = synth.make_workload("c5", seed=1)
+    H, W, N_cap = wl.H, wl.W, 50_000
+    sched = fit.Schedule()
+    s = Sad(H, W, N_cap, seed=1)
+    s.set_sites(prm)
+    s.set_target(tgt)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    fit.run(s, sched)
+    e1.record()
+    torch.cuda.synchronize()
+    t_fit = e0.elapsed_time(e1) * 1e-3
+    L = s.loss()
+    n_final = int((s.get_sites()[0] >= 0).sum())
+    line = {"metric": "time to fit 768x512 (2000 iterations, N 10,000 -> 50,000 by densify/prune) and final PSNR",
+            "value": t_fit, "unit": "s", "higher_is_better": False, "n_gpus": 1,
+            "psnr_db": 10 * math.log10(3.0 / L), "final_loss": L, "n_active_final": n_final,
+            "iterations": sched.iterations, "events": len(sched.events), "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"c5: {wl.description}", "H": H, "W": W, "N_start": prm.shape[1],
+                       "N_cap": N_cap, "G": sched.G}}
+    if args.oracle_fit:
+        import oracle
+        lr = {k[3:] if k.startswith("lr_") else k: float(np.float32(v)) for k, v in sched.lr.items()}
+        lr = {"pos": lr["pos"], "log_tau": lr["log_tau"], "r": lr["r"], "color": lr["color"],
+              "theta": lr["theta"], "a": lr["a"]}
+        t0 = time.perf_counter()
+        P, L_o, _ = oracle.fit(H, W, prm, tgt, N_cap, sched.iterations, sched.events, sched.grow, sched.prune_frac,
+                               lr, sched.G, 1)
+        line["oracle"] = {"time_s": time.perf_counter() - t0, "psnr_db": 10 * math.log10(3.0 / L_o),
+                          "final_loss": L_o, "n_active_final": int((P[0] >= 0).sum()),
+                          "cores": oracle.num_threads()}
+        line["psnr_diff_db"] = line["psnr_db"] - line["oracle"]["psnr_db"]
+    print(json.dumps(line), flush=True)
+    s.close()
+    return 0
+
+
 def main():
     args = parse()
+    if args.workload == "c5" and args.impl == "ours":
+        return run_fit(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.workload == "c4":

@@ -90,7 +90,27 @@ typedef struct sad_buffers {
     float *image; /* optional */
     void *workspace;
     size_t workspace_bytes;
+    float *stats; /* optional [6][N_cap]: budget-control statistics (SAD_STATS, sad_densify_prune) */
 } sad_buffers;
+
+/* sad_backward flag: also accumulate the budget-control statistics into
+ * stats ([P1] B.4-B.5): per site, mass m = sum w, energy E = sum w e,
+ * second moments sum w e (dx^2, dx dy, dy^2) with (dx, dy) = x - p, and the
+ * removal delta D = sum |(chat - w c) / max(1 - w, 1e-6) - t|^2 - e, where
+ * e = |chat - t|^2 at each pixel holding the site. */
+#define SAD_STATS 1u
+
+/* Densify / prune configuration ([P1] B.5, [P2] design 4). */
+typedef struct sad_densify_cfg {
+    int grow;              /* net sites added per event (2500 in the 768x512 schedule) */
+    float prune_frac;      /* fraction of the active sites pruned (0.005) */
+    float alpha;           /* score E / max(m, eps)^alpha (0.5) */
+    float eps;             /* mass floor (1e-6) */
+    float r_scale;         /* children's radius factor (0.85) */
+    float log_tau_shift;   /* subtracted from the children's ln tau (ln 2) */
+    float offset_scale;    /* child offset = offset_scale * sqrt(largest eigenvalue) (0.5) */
+    float fallback_offset; /* offset in pixels along the metric's long axis when the moment is degenerate (0.5) */
+} sad_densify_cfg;
 
 /* Adam configuration ([P2] key design 4).  Learning rates per parameter
  * group; positions and radius are stepped in the resolution-free units s x
@@ -111,6 +131,10 @@ typedef struct sad_stats {
     uint32_t current_table;    /* 0 or 1: which table of the double buffer is current */
     uint32_t reserved;
     double loss;               /* loss of the last sad_backward / sad_fit_iteration */
+    uint32_t n_active;         /* active sites before the last densify event */
+    uint32_t n_split;          /* sites split by the last densify event */
+    uint32_t n_pruned;         /* sites pruned by the last densify event */
+    uint32_t reserved2;
 } sad_stats;
 
 /* Bytes of workspace the caller must bind for an H x W image and N_cap sites. */
@@ -191,12 +215,38 @@ int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream);
  * probing capped at 8, compare-and-swap insert) with one global atomic per
  * (site, parameter, tile); overflow goes straight to global atomics
  * ([P1] section 5 and B.4).  Writes the bound image when one is bound and
- * the loss into the statistics block.  flags must be 0. */
+ * the loss into the statistics block.  flags: 0 or SAD_STATS (needs the stats
+ * buffer; accumulates into it). */
 int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream);
+
+/* One budget-control event, on the device ([P1] B.5: split by the score
+ * E / m^alpha along a covariance-estimated axis; prune by the removal score,
+ * x = -1; [P2] design 4).  Reads the statistics accumulated by
+ * sad_backward(ctx, SAD_STATS, ...) since the last event, then:
+ *   1. prunes the floor(prune_frac * n_active) active sites with the smallest
+ *      removal delta D (ties: smaller id);
+ *   2. splits the min(n_pruned + grow, free slots, active sites left) active
+ *      sites with the largest float32 score E / max(m, eps)^alpha (IEEE
+ *      sqrt/division when alpha = 0.5; ties: smaller id); parents in
+ *      ascending id take the free slots (x < 0) in ascending id;
+ *   3. places the children at p +- d, d = offset_scale * sqrt(l) e with (l, e)
+ *      the largest eigenpair of the second moment / E (e.x > 0, or e.x = 0
+ *      and e.y > 0), or d = fallback_offset times the metric's long axis
+ *      (v if a > 0, else u) when E or l is not positive; child A keeps the
+ *      parent's slot, child B takes the free slot; both are clamped into the
+ *      image, take the target colour at their pixel, r * r_scale,
+ *      ln tau - log_tau_shift, the parent's theta and a, and zero Adam moments;
+ *   4. zeroes the statistics and rebuilds the score records.
+ * The candidate lists are stale afterwards: run sad_refresh before the next
+ * pass.  Needs the stats buffer.  The number of sites never leaves the
+ * device (see sad_get_stats). */
+int sad_densify_prune(sad_ctx *ctx, const sad_densify_cfg *cfg, sad_stream_t stream);
 
 /* Step a7: one Adam step on every active site ([P2] design 4), reading and
  * zeroing grads, advancing the Adam step counter, and rebuilding the score
- * records (a1) in the same kernel. */
+ * records (a1) in the same kernel.  The step keeps positions inside the
+ * image, [0, W^-] x [0, H^-] with W^- the largest float below W (x < 0 is the
+ * marker of a pruned site, not an optimiser outcome). */
 int sad_adam_step(sad_ctx *ctx, const sad_adam_cfg *cfg, sad_stream_t stream);
 
 /* Steps a2-a6 in one kernel: a propagation pass at jump 1 with G injections

@@ -49,7 +49,7 @@ def lib():
         L.orc_loss_backward.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp]
         L.orc_loss_backward.restype = c_dbl
         L.orc_adam.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, c_dbl, c_dbl, c_dbl, c_int]
-        L.orc_loss_backward_stats.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, vp]
+        L.orc_loss_backward_stats.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp]
         L.orc_loss_backward_stats.restype = c_dbl
         L.orc_split_score.argtypes = [ctypes.c_float] * 4
         L.orc_split_score.restype = ctypes.c_float
@@ -220,17 +220,20 @@ def adam(H: int, W: int, params, m, v, grads, lr, t: int, b1: float = 0.9, b2: f
 STAT_NAMES = ("mass", "energy", "sxx", "sxy", "syy", "removal")
 
 
-def loss_backward_stats(H: int, W: int, params, table, target):
-    """Returns (loss, grads (9, N), stats (6, N)) in float64; stats rows are
-    STAT_NAMES."""
+def loss_backward_stats(H: int, W: int, params, table, target, want_abs: bool = False):
+    """Returns (loss, grads (9, N), stats (6, N)[, stats_abs (6, N)]) in
+    float64; stats rows are STAT_NAMES, stats_abs the sums of the terms'
+    absolute values."""
     params = _f32(params)
     tab = _u32(table).reshape(H * W, K)
     tgt = _f32(target).reshape(3, H * W)
     N = params.shape[1]
     g = np.empty((9, N), dtype=np.float64)
     st = np.empty((6, N), dtype=np.float64)
-    L = lib().orc_loss_backward_stats(H, W, N, _p(params), _p(tab), _p(tgt), _p(g), None, _p(st))
-    return L, g, st
+    sa = np.empty((6, N), dtype=np.float64) if want_abs else None
+    L = lib().orc_loss_backward_stats(H, W, N, _p(params), _p(tab), _p(tgt), _p(g), None, _p(st),
+                                      _p(sa) if want_abs else None)
+    return (L, g, st, sa) if want_abs else (L, g, st)
 
 
 class DensifyCfg(ctypes.Structure):

@@ -480,12 +480,13 @@ void orc_weights(int H, int W, int N, const float *params, const uint32_t *table
  * (optional): 3 x P doubles.  Returns L.
  */
 double orc_loss_backward_stats(int H, int W, int N, const float *params, const uint32_t *table,
-                               const float *target, double *grads, double *image, double *stats);
+                               const float *target, double *grads, double *image, double *stats,
+                               double *stats_abs);
 
 double orc_loss_backward(int H, int W, int N, const float *params, const uint32_t *table,
                          const float *target, double *grads, double *image)
 {
-    return orc_loss_backward_stats(H, W, N, params, table, target, grads, image, NULL);
+    return orc_loss_backward_stats(H, W, N, params, table, target, grads, image, NULL, NULL);
 }
 
 /*
@@ -497,16 +498,19 @@ double orc_loss_backward(int H, int W, int N, const float *params, const uint32_
  *   Sxx_i, Sxy_i, Syy_i = sum_x w_i e(x) (dx^2, dx dy, dy^2),  (dx, dy) = x - p_i
  *   D_i   = sum_x [ |(chat - w_i c_i) / max(1 - w_i, 1e-6) - t|^2 - e(x) ]
  * (D_i: the error after removing site i and renormalising the remaining
- * weights, minus the error with it).
+ * weights, minus the error with it).  stats_abs (optional, with stats)
+ * receives the sums of the terms' absolute values, the scale against which
+ * a float32 accumulation of the same sums is accurate.
  */
 double orc_loss_backward_stats(int H, int W, int N, const float *params, const uint32_t *table,
-                               const float *target, double *grads, double *image, double *stats)
+                               const float *target, double *grads, double *image, double *stats,
+                               double *stats_abs)
 {
     const int64_t P = (int64_t)H * W;
     const double s = 1.0 / (double)(H > W ? H : W);
     site64_t *S = sites64(N, params);
     const int T = omp_threads();
-    const int NA = P_COUNT + 6; /* gradients, then statistics */
+    const int NA = P_COUNT + 12; /* gradients, statistics, their absolute sums */
     double *acc = (double *)calloc((size_t)T * NA * (size_t)(N > 0 ? N : 1), sizeof(double));
     double *lossp = (double *)calloc((size_t)T, sizeof(double));
 #pragma omp parallel
@@ -538,12 +542,12 @@ double orc_loss_backward_stats(int H, int W, int N, const float *params, const u
                         const double c2 = (o.chat[ch] - w * z->c[ch]) / den - (double)target[ch * P + p];
                         rem += c2 * c2;
                     }
-                    St[0 * (size_t)N + i] += w;
-                    St[1 * (size_t)N + i] += w * ex;
-                    St[2 * (size_t)N + i] += w * ex * o.dx[q] * o.dx[q];
-                    St[3 * (size_t)N + i] += w * ex * o.dx[q] * o.dy[q];
-                    St[4 * (size_t)N + i] += w * ex * o.dy[q] * o.dy[q];
-                    St[5 * (size_t)N + i] += rem - ex;
+                    const double t6[6] = {w, w * ex, w * ex * o.dx[q] * o.dx[q], w * ex * o.dx[q] * o.dy[q],
+                                          w * ex * o.dy[q] * o.dy[q], rem - ex};
+                    for (int r = 0; r < 6; ++r) {
+                        St[r * (size_t)N + i] += t6[r];
+                        St[(6 + r) * (size_t)N + i] += fabs(t6[r]);
+                    }
                 }
             }
             for (int q = 0; q < o.n; ++q) {
@@ -577,12 +581,15 @@ double orc_loss_backward_stats(int H, int W, int N, const float *params, const u
     }
     memset(grads, 0, sizeof(double) * P_COUNT * (size_t)N);
     if (stats) memset(stats, 0, sizeof(double) * 6 * (size_t)N);
+    if (stats_abs) memset(stats_abs, 0, sizeof(double) * 6 * (size_t)N);
     double L = 0.0;
     for (int t = 0; t < T; ++t) {
         const double *A = acc + (size_t)t * NA * N;
         for (size_t q = 0; q < (size_t)P_COUNT * N; ++q) grads[q] += A[q];
         if (stats)
             for (size_t q = 0; q < (size_t)6 * N; ++q) stats[q] += A[(size_t)P_COUNT * N + q];
+        if (stats_abs)
+            for (size_t q = 0; q < (size_t)6 * N; ++q) stats_abs[q] += A[(size_t)(P_COUNT + 6) * N + q];
         L += lossp[t];
     }
     free(acc);
@@ -600,7 +607,9 @@ double orc_loss_backward_stats(int H, int W, int N, const float *params, const u
  *   ghat = grad * sigma_j,  sigma_j = 1/s for x, y, r and 1 otherwise
  *   m <- b1 m + (1 - b1) ghat;   v <- b2 v + (1 - b2) ghat^2
  *   param <- param - lr_j sigma_j (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
- * Inactive sites are left untouched.  All arrays 9 x N doubles, in place.
+ * then the position is clamped into [0, W^-] x [0, H^-] (W^- the largest
+ * float below W).  Inactive sites are left untouched.  All arrays 9 x N
+ * doubles, in place.
  */
 void orc_adam(int H, int W, int N, double *params, double *m, double *v, const double *grads,
               const double *lr, double b1, double b2, double eps, int t)
@@ -619,6 +628,12 @@ void orc_adam(int H, int W, int N, double *params, double *m, double *v, const d
             const double mh = m[q] / bc1, vh = v[q] / bc2;
             params[q] -= lr[j] * sig * mh / (sqrt(vh) + eps);
         }
+        /* the step keeps the position inside the image: x < 0 is the marker
+           of a pruned site, not something an optimiser step may produce */
+        const double xmax = (double)nextafterf((float)W, 0.0f), ymax = (double)nextafterf((float)H, 0.0f);
+        double *x = &params[P_X * (size_t)N + i], *y = &params[P_Y * (size_t)N + i];
+        *x = *x < 0.0 ? 0.0 : (*x > xmax ? xmax : *x);
+        *y = *y < 0.0 ? 0.0 : (*y > ymax ? ymax : *y);
     }
 }
 

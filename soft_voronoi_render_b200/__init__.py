@@ -10,9 +10,9 @@ from __future__ import annotations
 import numpy as np
 
 from . import _lib
-from ._lib import SadError, adam_cfg  # noqa: F401
+from ._lib import SAD_STATS, SadError, adam_cfg, densify_cfg  # noqa: F401
 
-__all__ = ["Sad", "SadError", "adam_cfg", "load"]
+__all__ = ["Sad", "SadError", "adam_cfg", "densify_cfg", "SAD_STATS", "load"]
 
 
 def load():
@@ -25,10 +25,12 @@ class Sad:
 
     Buffers (torch tensors on ``device``): params/grads/adam_m/adam_v
     (9, N) float32, records (N, 16) float32, table (2, 2, P, 4) int32 view of
-    uint32 ids, target/image (3, H, W) float32, workspace bytes.
+    uint32 ids, target/image (3, H, W) float32, site_stats (6, N) float32,
+    workspace bytes.
     """
 
-    def __init__(self, H: int, W: int, N_cap: int, device="cuda", with_image: bool = True, seed: int = 1):
+    def __init__(self, H: int, W: int, N_cap: int, device="cuda", with_image: bool = True, seed: int = 1,
+                 with_stats: bool = True):
         import torch
 
         if not torch.cuda.is_available():
@@ -47,12 +49,13 @@ class Sad:
         self.table = torch.full((2, 2, self.P, 4), -1, dtype=torch.int32, device=self.device)
         self.target = torch.zeros((3, self.H, self.W), **f32)
         self.image = torch.zeros((3, self.H, self.W), **f32) if with_image else None
+        self.site_stats = torch.zeros((6, self.N), **f32) if with_stats else None
         self.ws_bytes = _lib.sad_workspace_bytes(self.H, self.W, self.N)
         self.workspace = torch.zeros(((self.ws_bytes + 255) // 256 * 256,), dtype=torch.uint8, device=self.device)
         self.ctx = _lib.sad_create(self.H, self.W, self.N, _lib.SAD_K)
         _lib.sad_bind(self.ctx, params=self.params, grads=self.grads, adam_m=self.adam_m, adam_v=self.adam_v,
                       records=self.records, table=self.table, target=self.target, image=self.image,
-                      workspace=self.workspace, workspace_bytes=self.workspace.numel())
+                      workspace=self.workspace, workspace_bytes=self.workspace.numel(), stats=self.site_stats)
         _lib.sad_reset(self.ctx, seed, self.stream)
 
     # the stream every call is issued on: torch's current stream
@@ -139,6 +142,9 @@ class Sad:
 
     def backward(self, flags: int = 0):
         _lib.sad_backward(self.ctx, flags, self.stream)
+
+    def densify_prune(self, cfg):
+        _lib.sad_densify_prune(self.ctx, cfg, self.stream)
 
     def adam_step(self, cfg):
         _lib.sad_adam_step(self.ctx, cfg, self.stream)

@@ -36,7 +36,21 @@ class sad_buffers(ctypes.Structure):
     _fields_ = [("params", ctypes.c_void_p), ("grads", ctypes.c_void_p), ("adam_m", ctypes.c_void_p),
                 ("adam_v", ctypes.c_void_p), ("records", ctypes.c_void_p), ("table", ctypes.c_void_p),
                 ("target", ctypes.c_void_p), ("image", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("stats", ctypes.c_void_p)]
+
+
+class sad_densify_cfg(ctypes.Structure):
+    _fields_ = [("grow", ctypes.c_int), ("prune_frac", ctypes.c_float), ("alpha", ctypes.c_float),
+                ("eps", ctypes.c_float), ("r_scale", ctypes.c_float), ("log_tau_shift", ctypes.c_float),
+                ("offset_scale", ctypes.c_float), ("fallback_offset", ctypes.c_float)]
+
+
+SAD_STATS = 1
+
+
+def densify_cfg(grow=2500, prune_frac=0.005, alpha=0.5, eps=1e-6, r_scale=0.85, log_tau_shift=0.6931471805599453,
+                offset_scale=0.5, fallback_offset=0.5) -> sad_densify_cfg:
+    return sad_densify_cfg(grow, prune_frac, alpha, eps, r_scale, log_tau_shift, offset_scale, fallback_offset)
 
 
 class sad_adam_cfg(ctypes.Structure):
@@ -48,16 +62,18 @@ class sad_stats(ctypes.Structure):
     _fields_ = [("hash_overflow", ctypes.c_uint64), ("nonfinite_pixels", ctypes.c_uint64),
                 ("empty_pixels", ctypes.c_uint64), ("dropped_ids", ctypes.c_uint64),
                 ("pass_counter", ctypes.c_uint32), ("adam_step", ctypes.c_uint32),
-                ("current_table", ctypes.c_uint32), ("reserved", ctypes.c_uint32), ("loss", ctypes.c_double)]
+                ("current_table", ctypes.c_uint32), ("reserved", ctypes.c_uint32), ("loss", ctypes.c_double),
+                ("n_active", ctypes.c_uint32), ("n_split", ctypes.c_uint32), ("n_pruned", ctypes.c_uint32),
+                ("reserved2", ctypes.c_uint32)]
 
     def as_dict(self):
-        return {n: getattr(self, n) for n, _ in self._fields_ if n != "reserved"}
+        return {n: getattr(self, n) for n, _ in self._fields_ if not n.startswith("reserved")}
 
 
 EXPORTED = (
     "sad_workspace_bytes", "sad_create", "sad_destroy", "sad_bind", "sad_reset", "sad_set_sites",
     "sad_get_sites", "sad_set_target", "sad_prep_records", "sad_topk_exact", "sad_refresh", "sad_propagate",
-    "sad_render", "sad_backward", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
+    "sad_render", "sad_backward", "sad_densify_prune", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
     "sad_get_stats", "sad_get_loss", "sad_last_error", "sad_backward_noalloc",
 )
 
@@ -97,6 +113,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "sad_render": [vp, vp, vp],
         "sad_backward": [vp, cu32, vp],
         "sad_adam_step": [vp, ctypes.POINTER(sad_adam_cfg), vp],
+        "sad_densify_prune": [vp, ctypes.POINTER(sad_densify_cfg), vp],
         "sad_fit_pass": [vp, ci, vp],
         "sad_fit_iteration": [vp, ci, ctypes.POINTER(sad_adam_cfg), vp],
         "sad_get_table": [vp, vp, vp],
@@ -160,9 +177,9 @@ def sad_destroy(ctx: int) -> None:
 
 
 def sad_bind(ctx: int, *, params, grads, adam_m, adam_v, records, table, target, workspace,
-             workspace_bytes: int, image=None) -> None:
+             workspace_bytes: int, image=None, stats=None) -> None:
     b = sad_buffers(_ptr(params), _ptr(grads), _ptr(adam_m), _ptr(adam_v), _ptr(records), _ptr(table),
-                    _ptr(target), _ptr(image), _ptr(workspace), workspace_bytes)
+                    _ptr(target), _ptr(image), _ptr(workspace), workspace_bytes, _ptr(stats))
     _check(ctx, load().sad_bind(ctx, ctypes.byref(b)))
 
 
@@ -209,6 +226,10 @@ def sad_backward(ctx: int, flags: int = 0, stream=None) -> None:
 def adam_cfg(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=1e-3, lr_theta=1e-3, lr_a=1e-3,
              beta1=0.9, beta2=0.999, eps=1e-8) -> sad_adam_cfg:
     return sad_adam_cfg(lr_pos, lr_log_tau, lr_r, lr_color, lr_theta, lr_a, beta1, beta2, eps)
+
+
+def sad_densify_prune(ctx: int, cfg: sad_densify_cfg, stream=None) -> None:
+    _check(ctx, load().sad_densify_prune(ctx, ctypes.byref(cfg), _stream(stream)))
 
 
 def sad_adam_step(ctx: int, cfg: sad_adam_cfg, stream=None) -> None:

@@ -90,7 +90,7 @@ extern "C" {
 
 int sad_workspace_bytes(int H, int W, int N_cap, size_t *bytes) {
     if (!bytes || H < 1 || W < 1 || N_cap < 1 || (long long)H * W >= (1ll << 31)) return SAD_ERR_INVALID_ARG;
-    *bytes = sad::workspace_bytes(H, W);
+    *bytes = sad::workspace_bytes(H, W, N_cap);
     return SAD_OK;
 }
 
@@ -128,7 +128,8 @@ int sad_bind(sad_ctx *ctx, const sad_buffers *b) {
         if (!aligned16(req[q])) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer %s is not 16-byte aligned", names[q]);
     }
     if (b->image && !aligned16(b->image)) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer image is not 16-byte aligned");
-    const size_t need = sad::workspace_bytes(ctx->H, ctx->W);
+    if (b->stats && !aligned16(b->stats)) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer stats is not 16-byte aligned");
+    const size_t need = sad::workspace_bytes(ctx->H, ctx->W, ctx->N);
     if (b->workspace_bytes < need)
         return fail(ctx, SAD_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", b->workspace_bytes, need);
     ctx->buf = *b;
@@ -145,6 +146,7 @@ int sad_bind(sad_ctx *ctx, const sad_buffers *b) {
     d.table = b->table;
     d.target = b->target;
     d.image = b->image;
+    d.stats = b->stats;
     d.ws = b->workspace;
     ctx->bound = true;
     ctx->err[0] = 0;
@@ -159,7 +161,8 @@ int sad_reset(sad_ctx *ctx, uint32_t seed, sad_stream_t stream) {
     cudaError_t e = cudaMemsetAsync(ctx->buf.grads, 0, pn, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(ctx->buf.adam_m, 0, pn, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(ctx->buf.adam_v, 0, pn, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->buf.workspace, 0, sad::COUNTERS_BYTES, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->buf.workspace, 0, ctx->buf.workspace_bytes, st);
+    if (e == cudaSuccess && ctx->buf.stats) e = cudaMemsetAsync(ctx->buf.stats, 0, sizeof(float) * 6 * (size_t)ctx->N, st);
     if (e == cudaSuccess) e = sad::launch_init_counters(ctx->dev, seed, st);
     return cuda_status(ctx, e, "reset");
 }
@@ -242,8 +245,37 @@ int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream) {
 int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream) {
     int r = need_bound(ctx);
     if (r) return r;
-    if (flags != 0) return fail(ctx, SAD_ERR_UNSUPPORTED, "backward flags 0x%x not supported", flags);
+    if (flags & ~SAD_STATS) return fail(ctx, SAD_ERR_UNSUPPORTED, "backward flags 0x%x not supported", flags);
+    if (flags & SAD_STATS) {
+        if (!ctx->buf.stats) return fail(ctx, SAD_ERR_NOT_BOUND, "SAD_STATS needs a bound stats buffer");
+        return cuda_status(ctx, sad::launch_render_backward_stats(ctx->dev, cs(stream)), "backward (stats)");
+    }
     return cuda_status(ctx, sad::launch_render_backward(ctx->dev, cs(stream)), "backward");
+}
+
+int sad_densify_prune(sad_ctx *ctx, const sad_densify_cfg *cfg, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!cfg) return fail(ctx, SAD_ERR_INVALID_ARG, "densify config is NULL");
+    if (!ctx->buf.stats) return fail(ctx, SAD_ERR_NOT_BOUND, "densify needs a bound stats buffer");
+    if (!(cfg->prune_frac >= 0.0f && cfg->prune_frac <= 1.0f) || !(cfg->alpha >= 0.0f) || !(cfg->eps > 0.0f) ||
+        !(cfg->r_scale >= 0.0f) || !(cfg->offset_scale >= 0.0f) || !(cfg->fallback_offset >= 0.0f) ||
+        !(cfg->log_tau_shift == cfg->log_tau_shift))
+        return fail(ctx, SAD_ERR_INVALID_ARG, "densify config out of range");
+    sad::DensifyArgs a;
+    a.grow = cfg->grow;
+    a.prune_frac = cfg->prune_frac;
+    a.alpha = cfg->alpha;
+    a.eps = cfg->eps;
+    a.r_scale = cfg->r_scale;
+    a.log_tau_shift = cfg->log_tau_shift;
+    a.offset_scale = cfg->offset_scale;
+    a.fallback_offset = cfg->fallback_offset;
+    cudaStream_t st = cs(stream);
+    cudaError_t e = sad::launch_densify(ctx->dev, a, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->buf.stats, 0, sizeof(float) * 6 * (size_t)ctx->N, st);
+    if (e == cudaSuccess) e = sad::launch_records(ctx->dev, st);
+    return cuda_status(ctx, e, "densify");
 }
 
 int sad_adam_step(sad_ctx *ctx, const sad_adam_cfg *cfg, sad_stream_t stream) {
@@ -323,6 +355,14 @@ int sad_get_stats(sad_ctx *ctx, sad_stats *out, sad_stream_t stream) {
     out->current_table = c.cur;
     out->reserved = 0;
     out->loss = c.loss;
+    uint32_t hdr[4] = {0, 0, 0, 0};
+    cudaError_t e = cudaMemcpy(hdr, reinterpret_cast<char *>(ctx->buf.workspace) + sad::densify_offset(ctx->H, ctx->W),
+                               sizeof(hdr), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(ctx, e, "read densify header");
+    out->n_split = hdr[0];
+    out->n_pruned = hdr[1];
+    out->n_active = hdr[2];
+    out->reserved2 = 0;
     return SAD_OK;
 }
 

@@ -18,6 +18,7 @@ namespace sad {
 constexpr int K = 8;
 constexpr uint32_t EMPTY = 0xFFFFFFFFu;
 constexpr int NPARAM = 9;
+constexpr int NSTAT = 6;  // budget-control statistics per site
 constexpr int REC_F4 = 4;  // a record is 4 float4 = 64 bytes
 
 // parameter planes

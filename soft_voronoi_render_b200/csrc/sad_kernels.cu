@@ -358,13 +358,20 @@ __device__ __forceinline__ int hash_find_or_insert(uint32_t *keys, uint32_t id) 
     return -1;
 }
 
+// STATS additionally accumulates the budget-control statistics per site
+// (summary B.4-B.5): mass sum w, energy sum w e, second moments
+// sum w e (dx^2, dx dy, dy^2) and the removal delta
+// sum |(chat - w c) / max(1 - w, 1e-6) - t|^2 - e, with e = |chat - t|^2.
+template <bool STATS>
 __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *__restrict__ rec,
                                                                   const uint32_t *__restrict__ table,
                                                                   const float *__restrict__ target, int H, int W,
                                                                   int N, float *__restrict__ image,
-                                                                  float *__restrict__ grads, void *ws) {
+                                                                  float *__restrict__ grads,
+                                                                  float *__restrict__ stats, void *ws) {
+    constexpr int NV = STATS ? NPARAM + NSTAT : NPARAM;
     __shared__ uint32_t keys[HASH_SLOTS];
-    __shared__ float acc[NPARAM][HASH_SLOTS];
+    __shared__ float acc[NV][HASH_SLOTS];
     __shared__ float warp_loss[TILE_THREADS / 32];
     Counters *c = counters(ws);
     const int lane = threadIdx.x;  // blockDim.x == 32: one warp per row segment
@@ -372,7 +379,7 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
     for (int q = tid; q < HASH_SLOTS; q += TILE_THREADS) {
         keys[q] = EMPTY;
 #pragma unroll
-        for (int j = 0; j < NPARAM; ++j) acc[j][q] = 0.0f;
+        for (int j = 0; j < NV; ++j) acc[j][q] = 0.0f;
     }
     __syncthreads();
 
@@ -391,11 +398,14 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
     s.valid = 0;
     s.cr = s.cg = s.cb = 0.0f;
     float gr = 0.0f, gg = 0.0f, gb = 0.0f, iz = 0.0f;
+    float er = 0.0f, eg = 0.0f, eb = 0.0f;
     if (inside) {
         const size_t p = (size_t)j * W + i;
         const int nv = pixel_softmax(in0[p], in1[p], rec, (uint32_t)N, fx, fy, s, dropped);
         empty = nv == 0;
-        const float er = s.cr - target[p], eg = s.cg - target[P + p], eb = s.cb - target[2 * P + p];
+        er = s.cr - target[p];
+        eg = s.cg - target[P + p];
+        eb = s.cb - target[2 * P + p];
         lsum = er * er + eg * eg + eb * eb;
         if (image) {
             image[p] = s.cr;
@@ -407,14 +417,37 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
         gb = 2.0f * eb * invP;
         iz = nv ? 1.0f / s.Z : 0.0f;
     }
+    // STATS: the weight and colour sums over all slots but the dominant one,
+    // summed directly (the removal of the dominant site must not subtract
+    // two nearly equal numbers)
+    int qstar = -1;
+    float zmm = 0.0f, cmr = 0.0f, cmg = 0.0f, cmb = 0.0f;
+    if constexpr (STATS) {
+        float emax = -1.0f;
+#pragma unroll
+        for (int q = 0; q < K; ++q)
+            if ((s.valid >> q & 1u) && s.l[q] > emax) {
+                emax = s.l[q];
+                qstar = q;
+            }
+#pragma unroll
+        for (int q = 0; q < K; ++q) {
+            if (!(s.valid >> q & 1u) || q == qstar) continue;
+            const float4 r2 = __ldg(rec + (size_t)s.id[q] * REC_F4 + 2);
+            zmm += s.l[q];
+            cmr = fmaf(s.l[q], r2.x, cmr);
+            cmg = fmaf(s.l[q], r2.y, cmg);
+            cmb = fmaf(s.l[q], r2.z, cmb);
+        }
+    }
     // every lane runs the slot loop (the run reduction needs the whole warp)
 #pragma unroll
     for (int q = 0; q < K; ++q) {
         const bool vq = (s.valid >> q) & 1u;
         const uint32_t key = vq ? s.id[q] : EMPTY;
-        float v[NPARAM];
+        float v[NV];
 #pragma unroll
-        for (int k = 0; k < NPARAM; ++k) v[k] = 0.0f;
+        for (int k = 0; k < NV; ++k) v[k] = 0.0f;
         if (vq) {
             const float4 *R = rec + (size_t)key * REC_F4;
             const float4 r0 = __ldg(R), r1 = __ldg(R + 1), r2 = __ldg(R + 2), r3 = __ldg(R + 3);
@@ -435,17 +468,53 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
             v[PCB] = w * gb;
             v[PTH] = -gi * al * be * (r3.y - r3.z);
             v[PA] = -0.5f * gi * (r3.y * al * al - r3.z * be * be);
+            if constexpr (STATS) {
+                const float ex = er * er + eg * eg + eb * eb;  // e = |chat - t|^2
+                // removal delta |a|^2 - |b|^2 = (a - b) . (a + b) with b = chat - t,
+                // a = (chat - w c) / max(1 - w, 1e-6) - t; the sums over the other
+                // slots come in unnormalised form: sum_{j != q} e_j (and e_j c_j)
+                const float Z = s.Z, eq = s.l[q];
+                const float oz = q == qstar ? zmm : Z - eq;
+                const float ocr = q == qstar ? cmr : fmaf(-eq, r2.x, s.cr * Z);
+                const float ocg = q == qstar ? cmg : fmaf(-eq, r2.y, s.cg * Z);
+                const float ocb = q == qstar ? cmb : fmaf(-eq, r2.z, s.cb * Z);
+                const float rest = oz * iz;  // 1 - w, without cancellation
+                float dr, dg, db;
+                if (rest >= 1e-6f) {
+                    // a - b = w (chat - c) / (1 - w) = w (c_rest - c), with c_rest the
+                    // blend of the other slots (chat - c itself cancels when w -> 1)
+                    const float ioz = 1.0f / oz;
+                    dr = w * (ocr * ioz - r2.x);
+                    dg = w * (ocg * ioz - r2.y);
+                    db = w * (ocb * ioz - r2.z);
+                } else {
+                    dr = ocr * iz * 1e6f - s.cr;
+                    dg = ocg * iz * 1e6f - s.cg;
+                    db = ocb * iz * 1e6f - s.cb;
+                }
+                const float we = w * ex;
+                v[NPARAM + 0] = w;
+                v[NPARAM + 1] = we;
+                v[NPARAM + 2] = we * dx * dx;
+                v[NPARAM + 3] = we * dx * dy;
+                v[NPARAM + 4] = we * dy * dy;
+                v[NPARAM + 5] = dr * (2.0f * er + dr) + dg * (2.0f * eg + dg) + db * (2.0f * eb + db);
+            }
         }
         const bool tail = warp_run_reduce(key, v, lane);
         if (tail && key != EMPTY) {
             const int slot = hash_find_or_insert(keys, key);
             if (slot >= 0) {
 #pragma unroll
-                for (int k = 0; k < NPARAM; ++k) atomicAdd(&acc[k][slot], v[k]);
+                for (int k = 0; k < NV; ++k) atomicAdd(&acc[k][slot], v[k]);
             } else {
                 ++overflow;
 #pragma unroll
                 for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + key, v[k]);
+                if constexpr (STATS) {
+#pragma unroll
+                    for (int k = 0; k < NSTAT; ++k) atomicAdd(stats + (size_t)k * N + key, v[NPARAM + k]);
+                }
             }
         }
     }
@@ -463,6 +532,13 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
         for (int k = 0; k < NPARAM; ++k) {
             const float a = acc[k][q];
             if (a != 0.0f) atomicAdd(grads + (size_t)k * N + id, a);
+        }
+        if constexpr (STATS) {
+#pragma unroll
+            for (int k = 0; k < NSTAT; ++k) {
+                const float a = acc[NPARAM + k][q];
+                if (a != 0.0f) atomicAdd(stats + (size_t)k * N + id, a);
+            }
         }
     }
     if (tid == 0) {
@@ -513,7 +589,7 @@ struct AdamArgs {
 __global__ void __launch_bounds__(SITE_THREADS) adam_kernel(float *__restrict__ prm, float *__restrict__ grads,
                                                             float *__restrict__ m1, float *__restrict__ m2,
                                                             float4 *__restrict__ rec, int N, int maxHW,
-                                                            AdamArgs a, Counters *c) {
+                                                            float xmax, float ymax, AdamArgs a, Counters *c) {
     const uint32_t t = c->adam_step + 1u;
     const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
     if (i < N) {
@@ -535,8 +611,12 @@ __global__ void __launch_bounds__(SITE_THREADS) adam_kernel(float *__restrict__ 
                 m2[k * n + i] = vk;
                 const float mh = mk / bc1, vh = vk / bc2;
                 v[k] -= a.lr[k] * sig * mh / (sqrtf(vh) + a.eps);
-                prm[k * n + i] = v[k];
             }
+            // the step keeps the position inside the image (x < 0 marks a pruned site)
+            v[PX] = fminf(fmaxf(v[PX], 0.0f), xmax);
+            v[PY] = fminf(fmaxf(v[PY], 0.0f), ymax);
+#pragma unroll
+            for (int k = 0; k < NPARAM; ++k) prm[k * n + i] = v[k];
         }
 #pragma unroll
         for (int k = 0; k < NPARAM; ++k) grads[k * n + i] = 0.0f;
@@ -560,10 +640,15 @@ inline Counters *host_counters(const Dev &d) { return reinterpret_cast<Counters 
 
 }  // namespace
 
-size_t workspace_bytes(int H, int W) {
+size_t densify_offset(int H, int W) {
     // loss partials sized for 8 x 8 tiles, the smallest tile any kernel uses
     const size_t tiles = (size_t)((W + 7) / 8) * (size_t)((H + 7) / 8);
-    return COUNTERS_BYTES + tiles * sizeof(double);
+    return (COUNTERS_BYTES + tiles * sizeof(double) + 255) / 256 * 256;
+}
+
+size_t workspace_bytes(int H, int W, int N) {
+    // densify scratch: a 256-byte header, then the parent and free-slot lists
+    return densify_offset(H, W) + 256 + 2 * sizeof(uint32_t) * (size_t)N;
 }
 
 cudaError_t launch_init_counters(const Dev &d, uint32_t seed, cudaStream_t st) {
@@ -611,8 +696,14 @@ cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st) {
 }
 
 cudaError_t launch_render_backward(const Dev &d, cudaStream_t st) {
-    render_bwd_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.target, d.H,
-                                                                            d.W, d.N, d.image, d.grads, d.ws);
+    render_bwd_kernel<false><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
+        d.records, d.table, d.target, d.H, d.W, d.N, d.image, d.grads, nullptr, d.ws);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_render_backward_stats(const Dev &d, cudaStream_t st) {
+    render_bwd_kernel<true><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
+        d.records, d.table, d.target, d.H, d.W, d.N, d.image, d.grads, d.stats, d.ws);
     return cudaGetLastError();
 }
 
@@ -623,7 +714,8 @@ cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st) {
     a.beta2 = h.beta2;
     a.eps = h.eps;
     adam_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.grads, d.adam_m, d.adam_v, d.records, d.N,
-                                                          d.H > d.W ? d.H : d.W, a, host_counters(d));
+                                                          d.H > d.W ? d.H : d.W, nextafterf((float)d.W, 0.0f),
+                                                          nextafterf((float)d.H, 0.0f), a, host_counters(d));
     return cudaGetLastError();
 }
 

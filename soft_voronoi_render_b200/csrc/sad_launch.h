@@ -14,7 +14,13 @@ struct Dev {
     float4 *records;
     uint32_t *table;  // [2][2][P][4]
     float *target, *image;
+    float *stats;  // [6][N] budget-control statistics (optional)
     void *ws;
+};
+
+struct DensifyArgs {
+    int grow;
+    float prune_frac, alpha, eps, r_scale, log_tau_shift, offset_scale, fallback_offset;
 };
 
 struct AdamHyper {
@@ -22,7 +28,8 @@ struct AdamHyper {
     float beta1, beta2, eps;
 };
 
-size_t workspace_bytes(int H, int W);
+size_t workspace_bytes(int H, int W, int N);
+size_t densify_offset(int H, int W);
 
 cudaError_t launch_init_counters(const Dev &d, uint32_t seed, cudaStream_t st);
 cudaError_t launch_mark_inactive(const Dev &d, int from, cudaStream_t st);
@@ -32,6 +39,8 @@ cudaError_t launch_seed(const Dev &d, cudaStream_t st);
 cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st);
 cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st);
 cudaError_t launch_render_backward(const Dev &d, cudaStream_t st);
+cudaError_t launch_render_backward_stats(const Dev &d, cudaStream_t st);
+cudaError_t launch_densify(const Dev &d, const DensifyArgs &a, cudaStream_t st);
 cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st);
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st);
 

@@ -1,0 +1,45 @@
+"""Host-side fitting schedule: every step is a C-ABI call on the device.
+
+A fit starts with a full candidate refresh, then runs fitting iterations.
+An iteration that precedes a budget-control event accumulates the
+statistics (propagate, backward with SAD_STATS, Adam), runs the
+densify/prune event and refreshes the candidate lists; every other
+iteration is one sad_fit_iteration (fused pass + Adam).  The site count
+stays on the device.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+from . import _lib
+
+
+@dataclass
+class Schedule:
+    iterations: int = 2000
+    G: int = 2
+    events: tuple = field(default_factory=lambda: tuple(range(100, 1601, 100)))
+    grow: int = 2500
+    prune_frac: float = 0.005
+    lr: dict = field(default_factory=lambda: dict(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=5e-3,
+                                                  lr_theta=1e-3, lr_a=1e-3))
+
+
+def run(sad, sched: Schedule, on_event=None) -> None:
+    """Fit the bound target with the context's sites (``sad`` is a ``Sad``)."""
+    ctx, st = sad.ctx, sad.stream
+    cfg = _lib.adam_cfg(**sched.lr)
+    dcfg = _lib.densify_cfg(grow=sched.grow, prune_frac=sched.prune_frac)
+    events = set(sched.events)
+    _lib.sad_refresh(ctx, sched.G, st)
+    for it in range(1, sched.iterations + 1):
+        if it in events:
+            _lib.sad_propagate(ctx, 1, sched.G, st)
+            _lib.sad_backward(ctx, _lib.SAD_STATS, st)
+            _lib.sad_adam_step(ctx, cfg, st)
+            _lib.sad_densify_prune(ctx, dcfg, st)
+            _lib.sad_refresh(ctx, sched.G, st)
+            if on_event is not None:
+                on_event(it)
+        else:
+            _lib.sad_fit_iteration(ctx, sched.G, cfg, st)

@@ -83,8 +83,21 @@ def test_bind_checks_alignment_and_sizes_without_touching_memory():
             _lib.sad_set_sites(ctx, 0x90000, 17)
         assert e.value.status == _lib.SAD_ERR_CAPACITY
         with pytest.raises(_lib.SadError) as e:
-            _lib.sad_backward(ctx, 1)
+            _lib.sad_backward(ctx, 2)
         assert e.value.status == _lib.SAD_ERR_UNSUPPORTED
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_backward(ctx, _lib.SAD_STATS)  # no stats buffer bound
+        assert e.value.status == _lib.SAD_ERR_NOT_BOUND
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_densify_prune(ctx, _lib.densify_cfg())
+        assert e.value.status == _lib.SAD_ERR_NOT_BOUND
+        _lib.sad_bind(ctx, **fake, stats=0xA0000)
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_densify_prune(ctx, _lib.densify_cfg(prune_frac=1.5))
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_bind(ctx, **fake, stats=0xA0004)
+        assert "stats" in str(e.value)
         with pytest.raises(_lib.SadError) as e:
             _lib.sad_adam_step(ctx, _lib.adam_cfg(beta1=1.0))
         assert e.value.status == _lib.SAD_ERR_INVALID_ARG

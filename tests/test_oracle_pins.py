@@ -389,6 +389,9 @@ def test_adam_matches_torch_adam(orc):
             gj[~torch.tensor(active)] = 0.0
             rows[j].grad = gj
         opt.step()
+        with torch.no_grad():  # the step keeps positions inside the image
+            rows[0].clamp_(0.0, float(np.nextafter(np.float32(W), np.float32(0))) / sig[0])
+            rows[1].clamp_(0.0, float(np.nextafter(np.float32(H), np.float32(0))) / sig[1])
         ref = np.stack([rows[j].detach().numpy() * sig[j] for j in range(9)])
         np.testing.assert_allclose(P[:, active], ref[:, active], rtol=1e-13, atol=1e-13)
         assert np.array_equal(P[:, ~active], prm[:, ~active])
