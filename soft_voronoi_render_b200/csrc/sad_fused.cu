@@ -145,6 +145,22 @@ struct FusedSmem {
     int last;
 };
 
+// halo ring pixel r (0..83) -> halo coordinates: top row, bottom row, then
+// the left and right columns of the 8 inner rows
+__device__ __forceinline__ void ring_coords(int r, int &hx, int &hy) {
+    if (r < HX) {
+        hx = r;
+        hy = 0;
+    } else if (r < 2 * HX) {
+        hx = r - HX;
+        hy = HY - 1;
+    } else {
+        const int q = r - 2 * HX;
+        hy = 1 + (q >> 1);
+        hx = (q & 1) ? HX - 1 : 0;
+    }
+}
+
 __device__ __forceinline__ void set_bit(uint4 &m, uint32_t u) {
     const uint32_t b = 1u << (u & 31u);
     const uint32_t w = u >> 5;
@@ -229,7 +245,7 @@ __device__ __forceinline__ void generic_pass(Top8L &t, const uint4 *__restrict__
     }
 }
 
-__global__ void __launch_bounds__(FT, 3) fit_tile_kernel(const float4 *__restrict__ rec, uint32_t *table,
+__global__ void __launch_bounds__(FT, 4) fit_tile_kernel(const float4 *__restrict__ rec, uint32_t *table,
                                                          const float *__restrict__ target, int H, int W, int N,
                                                          int G, float *__restrict__ image,
                                                          float *__restrict__ grads, void *ws) {
@@ -250,6 +266,11 @@ __global__ void __launch_bounds__(FT, 3) fit_tile_kernel(const float4 *__restric
     const uint32_t Nu = (uint32_t)N;
 
     for (int q = tid; q < UHASH; q += FT) sm.keys[q] = EMPTY;
+    for (int r = tid; r < RING; r += FT) {
+        int hx, hy;
+        ring_coords(r, hx, hy);
+        sm.masks[hy * HX + hx] = make_uint4(0, 0, 0, 0);
+    }
     for (int q = tid; q < NPARAM * UCAP; q += FT) (&sm.acc[0][0])[q] = 0.0f;
     if (tid < UCAP) sm.cnt[tid] = 0;
     if (tid == 0) {
@@ -286,34 +307,16 @@ __global__ void __launch_bounds__(FT, 3) fit_tile_kernel(const float4 *__restric
         const uint32_t prev = __shfl_up_sync(FULL, id, 1);
         if (id < Nu && !(lane > 0 && prev == id)) ok &= ukey_insert(sm.keys, id);
     }
-    uint32_t ring_ids[K];
-    int rhx = 0, rhy = 0;
-    bool ring_in = false;
-    if (tid < RING) {
-        if (tid < HX) {
-            rhx = tid;
-            rhy = 0;
-        } else if (tid < 2 * HX) {
-            rhx = tid - HX;
-            rhy = HY - 1;
-        } else {
-            const int q = tid - 2 * HX;
-            rhy = 1 + (q >> 1);
-            rhx = (q & 1) ? HX - 1 : 0;
-        }
-        const int gi = i0 - 1 + rhx, gj = j0 - 1 + rhy;
-        ring_in = gi >= 0 && gi < W && gj >= 0 && gj < H;
-        uint4 a = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY), b = a;
-        if (ring_in) {
-            const size_t pn = (size_t)gj * W + gi;
-            a = in0[pn];
-            b = in1[pn];
-        }
-        ring_ids[0] = a.x; ring_ids[1] = a.y; ring_ids[2] = a.z; ring_ids[3] = a.w;
-        ring_ids[4] = b.x; ring_ids[5] = b.y; ring_ids[6] = b.z; ring_ids[7] = b.w;
-#pragma unroll
-        for (int q = 0; q < K; ++q)
-            if (ring_ids[q] < Nu) ok &= ukey_insert(sm.keys, ring_ids[q]);
+    // the 84 halo pixels x 8 slots, spread over all threads: entry e is
+    // halo pixel e % RING, slot e / RING
+    for (int e = tid; e < RING * K; e += FT) {
+        const int r = e % RING, q = e / RING;
+        int hx, hy;
+        ring_coords(r, hx, hy);
+        const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
+        if (gi < 0 || gi >= W || gj < 0 || gj >= H) continue;
+        const uint32_t id = table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
+        if (id < Nu) ok &= ukey_insert(sm.keys, id);
     }
     if (!ok) sm.overflow = 1;
     __syncthreads();
@@ -345,16 +348,17 @@ __global__ void __launch_bounds__(FT, 3) fit_tile_kernel(const float4 *__restric
             else own_lx_hi = (own_lx_hi & m) | b;
         }
         sm.masks[(ty + 1) * HX + lane + 1] = own_mask;
-        if (tid < RING) {
-            uint4 m = make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int q = 0; q < K; ++q) {
-                if (ring_ids[q] < Nu) {
-                    const uint32_t u = ukey_lookup(sm.keys, sm.lid, ring_ids[q]);
-                    if (u != NOLOC) set_bit(m, u);
-                }
-            }
-            sm.masks[rhy * HX + rhx] = m;
+        for (int e = tid; e < RING * K; e += FT) {
+            const int r = e % RING, q = e / RING;
+            int hx, hy;
+            ring_coords(r, hx, hy);
+            const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
+            if (gi < 0 || gi >= W || gj < 0 || gj >= H) continue;
+            const uint32_t id =
+                table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
+            if (id >= Nu) continue;
+            const uint32_t u = ukey_lookup(sm.keys, sm.lid, id);
+            if (u != NOLOC) atomicOr(reinterpret_cast<uint32_t *>(&sm.masks[hy * HX + hx]) + (u >> 5), 1u << (u & 31u));
         }
         // ---- B: stage the tile's site records --------------------------------
         for (uint32_t u = tid; u < ucount; u += FT) {
@@ -458,15 +462,32 @@ __global__ void __launch_bounds__(FT, 3) fit_tile_kernel(const float4 *__restric
         }
     }
     float Z = 0.0f, cr = 0.0f, cg = 0.0f, cb = 0.0f;
+    bool far_slot = false;  // a slot whose site has no tile-local index
 #pragma unroll
     for (int q = 0; q < K; ++q) {
         if (vmask >> q & 1u) {
             const float e = __expf(t.l[q] - M);
-            const float4 r2 = t.lx[q] != NOLOC ? sm.urec[2][t.lx[q]] : __ldg(rec + (size_t)t.id[q] * REC_F4 + 2);
             Z += e;
-            cr = fmaf(e, r2.x, cr);
-            cg = fmaf(e, r2.y, cg);
-            cb = fmaf(e, r2.z, cb);
+            if (t.lx[q] != NOLOC) {
+                const float4 r2 = sm.urec[2][t.lx[q]];
+                cr = fmaf(e, r2.x, cr);
+                cg = fmaf(e, r2.y, cg);
+                cb = fmaf(e, r2.z, cb);
+            } else {
+                far_slot = true;
+            }
+        }
+    }
+    if (__any_sync(FULL, far_slot)) {
+#pragma unroll
+        for (int q = 0; q < K; ++q) {
+            if ((vmask >> q & 1u) && t.lx[q] == NOLOC) {
+                const float e = __expf(t.l[q] - M);
+                const float4 r2 = __ldg(rec + (size_t)t.id[q] * REC_F4 + 2);
+                cr = fmaf(e, r2.x, cr);
+                cg = fmaf(e, r2.y, cg);
+                cb = fmaf(e, r2.z, cb);
+            }
         }
     }
     const float iz = vmask ? __frcp_rn(Z) : 0.0f;
