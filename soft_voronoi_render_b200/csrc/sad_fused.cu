@@ -21,9 +21,8 @@ namespace sad {
 
 namespace {
 
-constexpr int FX = 32, FY = 8, FT = FX * FY;
-constexpr int HX = FX + 2, HY = FY + 2, HN = HX * HY;  // tile plus one-pixel halo
-constexpr int RING = HN - FT;                          // 84 halo pixels
+constexpr int FX = 32;                                 // tile width: one warp per row
+constexpr int HX = FX + 2;                             // halo row length
 constexpr int UCAP = 128;                              // tile-local site capacity
 constexpr int UW = UCAP / 32;                          // mask words
 constexpr int UHASH_BITS = 9;
@@ -126,7 +125,9 @@ __device__ __forceinline__ uint32_t ukey_lookup(const uint32_t *keys, const uint
     return NOLOC;
 }
 
+template <int FY>
 struct FusedSmem {
+    static constexpr int FT = FX * FY, HN = HX * (FY + 2);
     uint32_t keys[UHASH];
     uint32_t lid[UHASH];
     uint32_t ulist[UCAP];
@@ -135,19 +136,22 @@ struct FusedSmem {
     float acc[NPARAM][UCAP];      // the tile's gradient sums per local site
     uint32_t cnt[UCAP];           // (pixel, slot) entries per local site
     uint32_t cursor[UCAP];        // scatter cursor of the counting sort
-    float pix[6][FT];             // per pixel: chat (3) and dL/dchat (3)
+    float4 pix4[FT];              // per pixel: chat (3), dL/dchat red
+    float2 pix2[FT];              //            dL/dchat green, blue
     float2 ent_wl[FT * K];        // entries grouped by site: softmax weight, logit
-    uint16_t ent_pu[FT * K];      //   pixel (low byte) and local site (high byte)
-    float warp_loss[FT / 32];
+    uint16_t ent_pu[FT * K];      //   pixel (low 9 bits) and local site (high 7 bits)
+    float warp_loss[FY];
     uint32_t n_ent;
     uint32_t ucount;
     int overflow;
     int last;
 };
 
-// halo ring pixel r (0..83) -> halo coordinates: top row, bottom row, then
-// the left and right columns of the 8 inner rows
+// halo ring pixel r -> halo coordinates: top row, bottom row, then the left
+// and right columns of the FY inner rows
+template <int FY>
 __device__ __forceinline__ void ring_coords(int r, int &hx, int &hy) {
+    constexpr int HY = FY + 2;
     if (r < HX) {
         hx = r;
         hy = 0;
@@ -245,12 +249,15 @@ __device__ __forceinline__ void generic_pass(Top8L &t, const uint4 *__restrict__
     }
 }
 
-__global__ void __launch_bounds__(FT, 4) fit_tile_kernel(const float4 *__restrict__ rec, uint32_t *table,
+template <int FY>
+__global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(const float4 *__restrict__ rec,
+                                                                            uint32_t *table,
                                                          const float *__restrict__ target, int H, int W, int N,
                                                          int G, float *__restrict__ image,
                                                          float *__restrict__ grads, void *ws) {
+    constexpr int FT = FX * FY, HY = FY + 2, HN = HX * HY, RING = HN - FT;
     extern __shared__ __align__(16) unsigned char fused_smem_raw[];
-    FusedSmem &sm = *reinterpret_cast<FusedSmem *>(fused_smem_raw);
+    FusedSmem<FY> &sm = *reinterpret_cast<FusedSmem<FY> *>(fused_smem_raw);
     Counters *c = ws_counters(ws);
     const uint32_t cur = c->cur, pass = c->pass_counter, seed = c->seed;
     const int lane = threadIdx.x, ty = threadIdx.y;
@@ -268,7 +275,7 @@ __global__ void __launch_bounds__(FT, 4) fit_tile_kernel(const float4 *__restric
     for (int q = tid; q < UHASH; q += FT) sm.keys[q] = EMPTY;
     for (int r = tid; r < RING; r += FT) {
         int hx, hy;
-        ring_coords(r, hx, hy);
+        ring_coords<FY>(r, hx, hy);
         sm.masks[hy * HX + hx] = make_uint4(0, 0, 0, 0);
     }
     for (int q = tid; q < NPARAM * UCAP; q += FT) (&sm.acc[0][0])[q] = 0.0f;
@@ -312,7 +319,7 @@ __global__ void __launch_bounds__(FT, 4) fit_tile_kernel(const float4 *__restric
     for (int e = tid; e < RING * K; e += FT) {
         const int r = e % RING, q = e / RING;
         int hx, hy;
-        ring_coords(r, hx, hy);
+        ring_coords<FY>(r, hx, hy);
         const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
         if (gi < 0 || gi >= W || gj < 0 || gj >= H) continue;
         const uint32_t id = table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
@@ -351,7 +358,7 @@ __global__ void __launch_bounds__(FT, 4) fit_tile_kernel(const float4 *__restric
         for (int e = tid; e < RING * K; e += FT) {
             const int r = e % RING, q = e / RING;
             int hx, hy;
-            ring_coords(r, hx, hy);
+            ring_coords<FY>(r, hx, hy);
             const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
             if (gi < 0 || gi >= W || gj < 0 || gj >= H) continue;
             const uint32_t id =
@@ -514,12 +521,8 @@ __global__ void __launch_bounds__(FT, 4) fit_tile_kernel(const float4 *__restric
     // site by site below; the rare rest (injected winners, crowded tiles) go
     // straight to global atomics.
     unsigned global_adds = 0;
-    sm.pix[0][tid] = cr;
-    sm.pix[1][tid] = cg;
-    sm.pix[2][tid] = cb;
-    sm.pix[3][tid] = gr;
-    sm.pix[4][tid] = gg;
-    sm.pix[5][tid] = gb;
+    sm.pix4[tid] = make_float4(cr, cg, cb, gr);
+    sm.pix2[tid] = make_float2(gg, gb);
 #pragma unroll
     for (int q = 0; q < K; ++q) {
         const bool vq = vmask >> q & 1u;
@@ -574,7 +577,7 @@ __global__ void __launch_bounds__(FT, 4) fit_tile_kernel(const float4 *__restric
         if (vq) {
             const uint32_t pos = pos0 + (uint32_t)(lane - start);
             sm.ent_wl[pos] = make_float2(__expf(t.l[q] - M) * iz, t.l[q]);
-            sm.ent_pu[pos] = (uint16_t)(tid | (key << 8));
+            sm.ent_pu[pos] = (uint16_t)(tid | (key << 9));
         }
     }
     __syncthreads();
@@ -593,7 +596,7 @@ __global__ void __launch_bounds__(FT, 4) fit_tile_kernel(const float4 *__restric
             const uint32_t idx = e0 + e;
             if (idx >= n_ent) break;
             const uint32_t pu = sm.ent_pu[idx];
-            const uint32_t u = pu >> 8, px = pu & 0xFFu;
+            const uint32_t u = pu >> 9, px = pu & 0x1FFu;
             if (u != cur) {
                 if (cur != NOLOC) {
 #pragma unroll
@@ -609,9 +612,11 @@ __global__ void __launch_bounds__(FT, 4) fit_tile_kernel(const float4 *__restric
                 r3 = sm.urec[3][u];
             }
             const float2 wl = sm.ent_wl[idx];
+            const float4 pa = sm.pix4[px];
+            const float2 pb = sm.pix2[px];
             float v[NPARAM];
-            slot_grad(r0, r1, r2, r3, fx0 + (float)(px & (FX - 1)), fy0 + (float)(px / FX), wl.y, wl.x,
-                      sm.pix[0][px], sm.pix[1][px], sm.pix[2][px], sm.pix[3][px], sm.pix[4][px], sm.pix[5][px], v);
+            slot_grad(r0, r1, r2, r3, fx0 + (float)(px & (FX - 1)), fy0 + (float)(px / FX), wl.y, wl.x, pa.x,
+                      pa.y, pa.z, pa.w, pb.x, pb.y, v);
 #pragma unroll
             for (int k = 0; k < NPARAM; ++k) a[k] += v[k];
         }
@@ -667,24 +672,32 @@ __global__ void __launch_bounds__(FT, 4) fit_tile_kernel(const float4 *__restric
     }
 }
 
-}  // namespace
-
-cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st) {
+template <int FY>
+cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
     // the tile state exceeds the 48 KB default: opt in once per device
     static bool attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(fit_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(FusedSmem));
+        e = cudaFuncSetAttribute(fit_tile_kernel<FY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(FusedSmem<FY>));
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
     const dim3 grid((d.W + FX - 1) / FX, (d.H + FY - 1) / FY);
-    fit_tile_kernel<<<grid, dim3(FX, FY), sizeof(FusedSmem), st>>>(d.records, d.table, d.target, d.H, d.W, d.N, G,
-                                                                   d.image, d.grads, d.ws);
+    fit_tile_kernel<FY><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY>), st>>>(d.records, d.table, d.target, d.H, d.W,
+                                                                           d.N, G, d.image, d.grads, d.ws);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st) {
+    // taller tiles amortise the halo and the per-tile work, but hold more
+    // distinct sites: use them where sites are sparse (>= 16 pixels per site)
+    if ((long long)d.H * d.W >= 16ll * d.N) return launch_fit_tile_h<16>(d, G, st);
+    return launch_fit_tile_h<8>(d, G, st);
 }
 
 }  // namespace sad
