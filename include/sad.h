@@ -91,6 +91,8 @@ typedef struct sad_buffers {
     void *workspace;
     size_t workspace_bytes;
     float *stats; /* optional [6][N_cap]: budget-control statistics (SAD_STATS, sad_densify_prune) */
+    const uint8_t *frozen; /* optional [N_cap]: non-zero = frozen site, left untouched by Adam
+                              ([P1] section 7: boundary sites excluded from gradient updates) */
 } sad_buffers;
 
 /* sad_backward flag: also accumulate the budget-control statistics into
@@ -242,9 +244,18 @@ int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream);
  * device (see sad_get_stats). */
 int sad_densify_prune(sad_ctx *ctx, const sad_densify_cfg *cfg, sad_stream_t stream);
 
+/* Tau diffusion ([P1] B.6): one Jacobi step on the ln tau gradients,
+ * g_i <- (1 - lambda) g_i + lambda mean_j g_j over the active sites j != i in
+ * the candidate list of the pixel containing p_i (the site's local candidate
+ * neighbourhood); all neighbours are read before any write; sites with no
+ * such neighbour, or outside the image, keep g_i.  Call between the backward
+ * pass and Adam.  0 <= lambda <= 1. */
+int sad_tau_diffuse(sad_ctx *ctx, float lambda, sad_stream_t stream);
+
 /* Step a7: one Adam step on every active site ([P2] design 4), reading and
  * zeroing grads, advancing the Adam step counter, and rebuilding the score
- * records (a1) in the same kernel.  The step keeps positions inside the
+ * records (a1) in the same kernel.  Frozen sites (the optional frozen
+ * buffer) are left untouched, like inactive ones.  The step keeps positions inside the
  * image, [0, W^-] x [0, H^-] with W^- the largest float below W (x < 0 is the
  * marker of a pruned site, not an optimiser outcome). */
 int sad_adam_step(sad_ctx *ctx, const sad_adam_cfg *cfg, sad_stream_t stream);

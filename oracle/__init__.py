@@ -55,6 +55,8 @@ def lib():
         L.orc_split_score.restype = ctypes.c_float
         L.orc_densify_prune.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp]
         L.orc_densify_prune.restype = c_int
+        L.orc_adam_frozen.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, c_dbl, c_dbl, c_dbl, c_int, vp]
+        L.orc_tau_diffuse.argtypes = [c_int, c_int, c_int, vp, vp, vp, c_dbl]
         L.orc_num_threads.restype = c_int
         L.orc_set_threads.argtypes = [c_int]
         _lib = L
@@ -202,9 +204,10 @@ ADAM_PLANE_GROUP = ("pos", "pos", "log_tau", "r", "color", "color", "color", "th
 
 
 def adam(H: int, W: int, params, m, v, grads, lr, t: int, b1: float = 0.9, b2: float = 0.999,
-         eps: float = 1e-8):
+         eps: float = 1e-8, frozen=None):
     """One Adam step in double.  ``lr`` is a dict keyed by ADAM_PLANE_GROUP
-    names or a length-9 sequence.  Returns new (params, m, v) float64."""
+    names or a length-9 sequence; ``frozen`` an optional per-site uint8 mask
+    of sites left untouched.  Returns new (params, m, v) float64."""
     P = np.array(params, dtype=np.float64, order="C", copy=True)
     M = np.array(m, dtype=np.float64, order="C", copy=True)
     V = np.array(v, dtype=np.float64, order="C", copy=True)
@@ -213,7 +216,11 @@ def adam(H: int, W: int, params, m, v, grads, lr, t: int, b1: float = 0.9, b2: f
         lrv = np.array([lr[gname] for gname in ADAM_PLANE_GROUP], dtype=np.float64)
     else:
         lrv = np.ascontiguousarray(lr, dtype=np.float64)
-    lib().orc_adam(H, W, P.shape[1], _p(P), _p(M), _p(V), _p(G), _p(lrv), b1, b2, eps, int(t))
+    if frozen is None:
+        lib().orc_adam(H, W, P.shape[1], _p(P), _p(M), _p(V), _p(G), _p(lrv), b1, b2, eps, int(t))
+    else:
+        fz = np.ascontiguousarray(frozen, dtype=np.uint8)
+        lib().orc_adam_frozen(H, W, P.shape[1], _p(P), _p(M), _p(V), _p(G), _p(lrv), b1, b2, eps, int(t), _p(fz))
     return P, M, V
 
 
@@ -303,3 +310,12 @@ def fit(H: int, W: int, params, target, N_cap: int, iterations: int, events, gro
                 on_event(it, prm)
         rec = records(H, W, prm)
     return prm, L, npass
+
+
+def tau_diffuse(H: int, W: int, params, table, grads, lam: float):
+    """One Jacobi tau-diffusion step; returns new grads (9, N) float64."""
+    params = _f32(params)
+    tab = _u32(table).reshape(H * W, K)
+    G = np.array(grads, dtype=np.float64, order="C", copy=True)
+    lib().orc_tau_diffuse(H, W, params.shape[1], _p(params), _p(tab), _p(G), float(lam))
+    return G

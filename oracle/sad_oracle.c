@@ -611,14 +611,26 @@ double orc_loss_backward_stats(int H, int W, int N, const float *params, const u
  * float below W).  Inactive sites are left untouched.  All arrays 9 x N
  * doubles, in place.
  */
+void orc_adam_frozen(int H, int W, int N, double *params, double *m, double *v, const double *grads,
+                     const double *lr, double b1, double b2, double eps, int t, const uint8_t *frozen);
+
 void orc_adam(int H, int W, int N, double *params, double *m, double *v, const double *grads,
               const double *lr, double b1, double b2, double eps, int t)
+{
+    orc_adam_frozen(H, W, N, params, m, v, grads, lr, b1, b2, eps, t, NULL);
+}
+
+/* As orc_adam; sites with frozen[i] != 0 are left untouched as well
+ * ([P1] section 7: frozen sites are excluded from gradient updates). */
+void orc_adam_frozen(int H, int W, int N, double *params, double *m, double *v, const double *grads,
+                     const double *lr, double b1, double b2, double eps, int t, const uint8_t *frozen)
 {
     const double s = 1.0 / (double)(H > W ? H : W);
     const double bc1 = 1.0 - pow(b1, (double)t);
     const double bc2 = 1.0 - pow(b2, (double)t);
     for (int i = 0; i < N; ++i) {
         if (!(params[P_X * (size_t)N + i] >= 0.0)) continue;
+        if (frozen && frozen[i]) continue;
         for (int j = 0; j < P_COUNT; ++j) {
             const size_t q = (size_t)j * N + i;
             const double sig = (j == P_X || j == P_Y || j == P_R) ? 1.0 / s : 1.0;
@@ -816,4 +828,43 @@ int orc_densify_prune(int H, int W, int N, float *params, float *m1, float *m2, 
     free(parents);
     if (n_pruned) *n_pruned = n_prune;
     return n_split;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Tau diffusion ([P1] B.6)                                                   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One Jacobi step on the ln tau gradients: for every active site i whose
+ * position lies in the image, with C = the valid active ids other than i in
+ * the candidate list of the pixel containing p_i (the site's local candidate
+ * neighbourhood), g_i <- (1 - lambda) g_i + lambda mean_{j in C} g_j, all
+ * neighbours read before any write.  Sites with an empty C keep g_i.
+ * grads: 9 x N doubles (plane ln tau updated in place); table: P x 8.
+ */
+void orc_tau_diffuse(int H, int W, int N, const float *params, const uint32_t *table, double *grads,
+                     double lambda)
+{
+    double *g = grads + (size_t)P_LT * N;
+    double *out = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+    for (int i = 0; i < N; ++i) {
+        out[i] = g[i];
+        const float px = params[P_X * N + i], py = params[P_Y * N + i];
+        if (!(px >= 0.0f) || !(py >= 0.0f)) continue;
+        const int64_t ci = (int64_t)floorf(px), cj = (int64_t)floorf(py);
+        if (ci >= W || cj >= H) continue;
+        const uint32_t *slots = table + (cj * W + ci) * ORC_K;
+        double sum = 0.0;
+        int n = 0;
+        for (int q = 0; q < ORC_K; ++q) {
+            const uint32_t id = slots[q];
+            if (id == ORC_SENTINEL || id >= (uint32_t)N || id == (uint32_t)i) continue;
+            if (!(params[P_X * N + id] >= 0.0f)) continue;
+            sum += g[id];
+            ++n;
+        }
+        if (n > 0) out[i] = (1.0 - lambda) * g[i] + lambda * (sum / n);
+    }
+    memcpy(g, out, sizeof(double) * (size_t)N);
+    free(out);
 }

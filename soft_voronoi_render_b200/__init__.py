@@ -26,7 +26,7 @@ class Sad:
     Buffers (torch tensors on ``device``): params/grads/adam_m/adam_v
     (9, N) float32, records (N, 16) float32, table (2, 2, P, 4) int32 view of
     uint32 ids, target/image (3, H, W) float32, site_stats (6, N) float32,
-    workspace bytes.
+    frozen (N,) uint8 (non-zero: Adam leaves the site alone), workspace bytes.
     """
 
     def __init__(self, H: int, W: int, N_cap: int, device="cuda", with_image: bool = True, seed: int = 1,
@@ -50,12 +50,14 @@ class Sad:
         self.target = torch.zeros((3, self.H, self.W), **f32)
         self.image = torch.zeros((3, self.H, self.W), **f32) if with_image else None
         self.site_stats = torch.zeros((6, self.N), **f32) if with_stats else None
+        self.frozen = torch.zeros((self.N,), dtype=torch.uint8, device=self.device)
         self.ws_bytes = _lib.sad_workspace_bytes(self.H, self.W, self.N)
         self.workspace = torch.zeros(((self.ws_bytes + 255) // 256 * 256,), dtype=torch.uint8, device=self.device)
         self.ctx = _lib.sad_create(self.H, self.W, self.N, _lib.SAD_K)
         _lib.sad_bind(self.ctx, params=self.params, grads=self.grads, adam_m=self.adam_m, adam_v=self.adam_v,
                       records=self.records, table=self.table, target=self.target, image=self.image,
-                      workspace=self.workspace, workspace_bytes=self.workspace.numel(), stats=self.site_stats)
+                      workspace=self.workspace, workspace_bytes=self.workspace.numel(), stats=self.site_stats,
+                      frozen=self.frozen)
         _lib.sad_reset(self.ctx, seed, self.stream)
 
     # the stream every call is issued on: torch's current stream
@@ -145,6 +147,9 @@ class Sad:
 
     def densify_prune(self, cfg):
         _lib.sad_densify_prune(self.ctx, cfg, self.stream)
+
+    def tau_diffuse(self, lam: float):
+        _lib.sad_tau_diffuse(self.ctx, lam, self.stream)
 
     def adam_step(self, cfg):
         _lib.sad_adam_step(self.ctx, cfg, self.stream)

@@ -36,7 +36,7 @@ class sad_buffers(ctypes.Structure):
     _fields_ = [("params", ctypes.c_void_p), ("grads", ctypes.c_void_p), ("adam_m", ctypes.c_void_p),
                 ("adam_v", ctypes.c_void_p), ("records", ctypes.c_void_p), ("table", ctypes.c_void_p),
                 ("target", ctypes.c_void_p), ("image", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t), ("stats", ctypes.c_void_p)]
+                ("workspace_bytes", ctypes.c_size_t), ("stats", ctypes.c_void_p), ("frozen", ctypes.c_void_p)]
 
 
 class sad_densify_cfg(ctypes.Structure):
@@ -73,7 +73,7 @@ class sad_stats(ctypes.Structure):
 EXPORTED = (
     "sad_workspace_bytes", "sad_create", "sad_destroy", "sad_bind", "sad_reset", "sad_set_sites",
     "sad_get_sites", "sad_set_target", "sad_prep_records", "sad_topk_exact", "sad_refresh", "sad_propagate",
-    "sad_render", "sad_backward", "sad_densify_prune", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
+    "sad_render", "sad_backward", "sad_densify_prune", "sad_tau_diffuse", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
     "sad_get_stats", "sad_get_loss", "sad_last_error", "sad_backward_noalloc",
 )
 
@@ -114,6 +114,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "sad_backward": [vp, cu32, vp],
         "sad_adam_step": [vp, ctypes.POINTER(sad_adam_cfg), vp],
         "sad_densify_prune": [vp, ctypes.POINTER(sad_densify_cfg), vp],
+        "sad_tau_diffuse": [vp, ctypes.c_float, vp],
         "sad_fit_pass": [vp, ci, vp],
         "sad_fit_iteration": [vp, ci, ctypes.POINTER(sad_adam_cfg), vp],
         "sad_get_table": [vp, vp, vp],
@@ -177,9 +178,9 @@ def sad_destroy(ctx: int) -> None:
 
 
 def sad_bind(ctx: int, *, params, grads, adam_m, adam_v, records, table, target, workspace,
-             workspace_bytes: int, image=None, stats=None) -> None:
+             workspace_bytes: int, image=None, stats=None, frozen=None) -> None:
     b = sad_buffers(_ptr(params), _ptr(grads), _ptr(adam_m), _ptr(adam_v), _ptr(records), _ptr(table),
-                    _ptr(target), _ptr(image), _ptr(workspace), workspace_bytes, _ptr(stats))
+                    _ptr(target), _ptr(image), _ptr(workspace), workspace_bytes, _ptr(stats), _ptr(frozen))
     _check(ctx, load().sad_bind(ctx, ctypes.byref(b)))
 
 
@@ -230,6 +231,10 @@ def adam_cfg(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=1e-3, lr_theta=1e
 
 def sad_densify_prune(ctx: int, cfg: sad_densify_cfg, stream=None) -> None:
     _check(ctx, load().sad_densify_prune(ctx, ctypes.byref(cfg), _stream(stream)))
+
+
+def sad_tau_diffuse(ctx: int, lam: float, stream=None) -> None:
+    _check(ctx, load().sad_tau_diffuse(ctx, lam, _stream(stream)))
 
 
 def sad_adam_step(ctx: int, cfg: sad_adam_cfg, stream=None) -> None:

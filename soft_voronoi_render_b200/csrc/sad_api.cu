@@ -147,6 +147,7 @@ int sad_bind(sad_ctx *ctx, const sad_buffers *b) {
     d.target = b->target;
     d.image = b->image;
     d.stats = b->stats;
+    d.frozen = b->frozen;
     d.ws = b->workspace;
     ctx->bound = true;
     ctx->err[0] = 0;
@@ -276,6 +277,13 @@ int sad_densify_prune(sad_ctx *ctx, const sad_densify_cfg *cfg, sad_stream_t str
     if (e == cudaSuccess) e = cudaMemsetAsync(ctx->buf.stats, 0, sizeof(float) * 6 * (size_t)ctx->N, st);
     if (e == cudaSuccess) e = sad::launch_records(ctx->dev, st);
     return cuda_status(ctx, e, "densify");
+}
+
+int sad_tau_diffuse(sad_ctx *ctx, float lambda, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!(lambda >= 0.0f && lambda <= 1.0f)) return fail(ctx, SAD_ERR_INVALID_ARG, "lambda must lie in [0, 1]");
+    return cuda_status(ctx, sad::launch_tau_diffuse(ctx->dev, lambda, cs(stream)), "tau diffusion");
 }
 
 int sad_adam_step(sad_ctx *ctx, const sad_adam_cfg *cfg, sad_stream_t stream) {

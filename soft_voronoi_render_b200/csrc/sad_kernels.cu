@@ -589,7 +589,8 @@ struct AdamArgs {
 __global__ void __launch_bounds__(SITE_THREADS) adam_kernel(float *__restrict__ prm, float *__restrict__ grads,
                                                             float *__restrict__ m1, float *__restrict__ m2,
                                                             float4 *__restrict__ rec, int N, int maxHW,
-                                                            float xmax, float ymax, AdamArgs a, Counters *c) {
+                                                            float xmax, float ymax, AdamArgs a,
+                                                            const uint8_t *__restrict__ frozen, Counters *c) {
     const uint32_t t = c->adam_step + 1u;
     const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
     if (i < N) {
@@ -597,7 +598,8 @@ __global__ void __launch_bounds__(SITE_THREADS) adam_kernel(float *__restrict__ 
         float v[NPARAM];
 #pragma unroll
         for (int k = 0; k < NPARAM; ++k) v[k] = prm[k * n + i];
-        if (v[PX] >= 0.0f) {
+        // frozen sites keep their parameters (summary section 7)
+        if (v[PX] >= 0.0f && !(frozen && frozen[i])) {
             const float bc1 = (float)(1.0 - pow((double)a.beta1, (double)t));
             const float bc2 = (float)(1.0 - pow((double)a.beta2, (double)t));
             const float sig_pos = (float)maxHW;
@@ -634,6 +636,46 @@ __global__ void __launch_bounds__(SITE_THREADS) adam_kernel(float *__restrict__ 
     }
 }
 
+// ---------------------------------------------------------------------------
+// tau diffusion (summary B.6): one Jacobi step on the ln tau gradients, the
+// neighbourhood being the candidate list at the site's own pixel
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(SITE_THREADS) tau_diffuse_kernel(const float *__restrict__ prm,
+                                                                   const uint32_t *__restrict__ table,
+                                                                   const float *__restrict__ grads, int H, int W,
+                                                                   int N, float lambda, float *__restrict__ out,
+                                                                   const Counters *__restrict__ c) {
+    const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
+    if (i >= N) return;
+    const size_t n = (size_t)N;
+    const float *g = grads + PLT * n;
+    const float gi = g[i];
+    float res = gi;
+    const float px = prm[PX * n + i], py = prm[PY * n + i];
+    if (px >= 0.0f && py >= 0.0f) {
+        const float fi = floorf(px), fj = floorf(py);
+        if (fi < (float)W && fj < (float)H) {
+            const size_t P = (size_t)H * W;
+            const size_t p = (size_t)fj * W + (size_t)fi;
+            const uint4 *t0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * P * K);
+            const uint4 a = t0[p], b = t0[P + p];
+            const uint32_t ids[K] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            double sum = 0.0;
+            int cnt = 0;
+#pragma unroll
+            for (int q = 0; q < K; ++q) {
+                const uint32_t id = ids[q];
+                if (id >= (uint32_t)N || id == (uint32_t)i) continue;
+                if (!(prm[PX * n + id] >= 0.0f)) continue;
+                sum += (double)g[id];
+                ++cnt;
+            }
+            if (cnt > 0) res = (float)((1.0 - (double)lambda) * (double)gi + (double)lambda * (sum / cnt));
+        }
+    }
+    out[i] = res;
+}
+
 inline dim3 tile_grid(int H, int W) { return dim3((W + TILE_X - 1) / TILE_X, (H + TILE_Y - 1) / TILE_Y); }
 inline unsigned site_blocks(long long n) { return (unsigned)((n + SITE_THREADS - 1) / SITE_THREADS); }
 inline Counters *host_counters(const Dev &d) { return reinterpret_cast<Counters *>(d.ws); }
@@ -647,8 +689,20 @@ size_t densify_offset(int H, int W) {
 }
 
 size_t workspace_bytes(int H, int W, int N) {
-    // densify scratch: a 256-byte header, then the parent and free-slot lists
-    return densify_offset(H, W) + 256 + 2 * sizeof(uint32_t) * (size_t)N;
+    // densify scratch: a 256-byte header, then the parent and free-slot lists;
+    // then one float per site for tau diffusion
+    return densify_offset(H, W) + 256 + 3 * sizeof(uint32_t) * (size_t)N;
+}
+
+cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st) {
+    float *scratch = reinterpret_cast<float *>(reinterpret_cast<char *>(d.ws) + densify_offset(d.H, d.W) + 256 +
+                                               2 * sizeof(uint32_t) * (size_t)d.N);
+    tau_diffuse_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.table, d.grads, d.H, d.W, d.N, lambda,
+                                                                  scratch, host_counters(d));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyAsync(d.grads + (size_t)PLT * d.N, scratch, sizeof(float) * (size_t)d.N,
+                           cudaMemcpyDeviceToDevice, st);
 }
 
 cudaError_t launch_init_counters(const Dev &d, uint32_t seed, cudaStream_t st) {
@@ -715,7 +769,7 @@ cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st) {
     a.eps = h.eps;
     adam_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.grads, d.adam_m, d.adam_v, d.records, d.N,
                                                           d.H > d.W ? d.H : d.W, nextafterf((float)d.W, 0.0f),
-                                                          nextafterf((float)d.H, 0.0f), a, host_counters(d));
+                                                          nextafterf((float)d.H, 0.0f), a, d.frozen, host_counters(d));
     return cudaGetLastError();
 }
 

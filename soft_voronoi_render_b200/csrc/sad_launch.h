@@ -15,6 +15,7 @@ struct Dev {
     uint32_t *table;  // [2][2][P][4]
     float *target, *image;
     float *stats;  // [6][N] budget-control statistics (optional)
+    const uint8_t *frozen;  // [N] sites Adam leaves untouched (optional)
     void *ws;
 };
 
@@ -41,6 +42,7 @@ cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st);
 cudaError_t launch_render_backward(const Dev &d, cudaStream_t st);
 cudaError_t launch_render_backward_stats(const Dev &d, cudaStream_t st);
 cudaError_t launch_densify(const Dev &d, const DensifyArgs &a, cudaStream_t st);
+cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st);
 cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st);
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st);
 

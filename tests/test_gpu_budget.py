@@ -113,3 +113,32 @@ def test_short_fit_with_densify_events(torch_cuda):
     # drift apart after an event: compare the outcome in PSNR
     psnr = lambda L: 10 * math.log10(3.0 / L)
     assert abs(psnr(L_gpu) - psnr(L_orc)) <= 0.2, (L_gpu, L_orc)
+
+
+def test_frozen_sites_and_tau_diffusion(torch_cuda):
+    """Frozen sites are left alone by Adam (summary section 7); tau diffusion
+    (summary B.6) matches the oracle's Jacobi step on the same lists."""
+    from soft_voronoi_render_b200 import adam_cfg
+    tgt, prm, w = synth.make_workload("c1", seed=6)
+    prm = prm.copy()
+    prm[0, 9] = -1.0
+    s = _ctx(w.H, w.W, w.N, prm, tgt, seed=2)
+    table = oracle.topk_exact(w.H, w.W, oracle.records(w.H, w.W, prm))
+    s.set_table(table)
+    g = synth.random_gradients(w.N, 66)
+    s.grads.copy_(torch_cuda.from_numpy(g))
+    s.tau_diffuse(0.4)
+    ref = oracle.tau_diffuse(w.H, w.W, prm, table, g.astype(np.float64), 0.4)
+    gd = s.grads.cpu().numpy()
+    np.testing.assert_allclose(gd.astype(np.float64), ref, rtol=1e-6, atol=1e-12)
+    assert np.array_equal(np.delete(gd, 2, 0), np.delete(g, 2, 0))
+    frozen = np.zeros(w.N, np.uint8)
+    frozen[::4] = 1
+    s.frozen.copy_(torch_cuda.from_numpy(frozen))
+    s.adam_step(adam_cfg())
+    f = frozen.astype(bool)
+    pg = s.params.cpu().numpy()
+    assert np.array_equal(pg[:, f], prm[:, f])
+    assert np.all(s.adam_m.cpu().numpy()[:, f] == 0) and np.all(s.grads.cpu().numpy() == 0)
+    moved = (np.abs(pg - prm).sum(0) > 0)
+    assert np.all(moved[~f & (prm[0] >= 0)])

@@ -148,3 +148,45 @@ def test_densify_decisions_and_children(orc):
             assert np.all(M2[:, dst] == 0) and np.all(V2[:, dst] == 0)
     assert 7 in parents  # the fallback axis was exercised
     assert int((P2[0] >= 0).sum()) == n_active - n_pruned + n_split
+
+
+# --------------------------------------------------------------------------
+# frozen sites (summary section 7) and tau diffusion (summary B.6)
+# --------------------------------------------------------------------------
+
+def test_adam_frozen_sites_untouched(orc):
+    H, W, N = 20, 30, 40
+    prm = synth.uniform_sites(H, W, N, 61).astype(np.float64)
+    g = synth.random_gradients(N, 61).astype(np.float64)
+    frozen = np.zeros(N, np.uint8)
+    frozen[::3] = 1
+    lr = [1e-3] * 9
+    P1, M1, V1 = orc.adam(H, W, prm, np.zeros_like(prm), np.zeros_like(prm), g, lr, 1, frozen=frozen)
+    P0, M0, V0 = orc.adam(H, W, prm, np.zeros_like(prm), np.zeros_like(prm), g, lr, 1)
+    f = frozen.astype(bool)
+    assert np.array_equal(P1[:, f], prm[:, f]) and np.all(M1[:, f] == 0) and np.all(V1[:, f] == 0)
+    assert np.array_equal(P1[:, ~f], P0[:, ~f]) and np.array_equal(M1[:, ~f], M0[:, ~f])
+
+
+def test_tau_diffusion_against_numpy(orc):
+    H, W, prm, tgt, tab = _case(orc, seed=7)
+    prm = prm.copy()
+    prm[0, 4] = -1.0
+    N = prm.shape[1]
+    g = synth.random_gradients(N, 7).astype(np.float64)
+    for lam in (0.0, 0.3, 1.0):
+        out = orc.tau_diffuse(H, W, prm, tab, g, lam)
+        ref = g.copy()
+        for i in range(N):
+            if prm[0, i] < 0:
+                continue
+            px, py = int(np.floor(prm[0, i])), int(np.floor(prm[1, i]))
+            nb = [int(j) for j in tab[py * W + px] if j != SENT and j < N and j != i and prm[0, j] >= 0]
+            if nb:
+                ref[2, i] = (1 - lam) * g[2, i] + lam * np.mean(g[2, nb])
+        np.testing.assert_allclose(out, ref, rtol=1e-15, atol=0)
+        assert np.array_equal(np.delete(out, 2, 0), np.delete(g, 2, 0))  # only the ln tau plane moves
+    # a constant gradient field is a fixed point
+    gc = np.zeros_like(g)
+    gc[2] = 0.25
+    np.testing.assert_allclose(orc.tau_diffuse(H, W, prm, tab, gc, 0.7)[2], 0.25, rtol=1e-15)
