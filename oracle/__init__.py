@@ -13,6 +13,7 @@ x, y, ln tau, r, cr, cg, cb, theta, a.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import numpy as np
@@ -57,6 +58,7 @@ def lib():
         L.orc_densify_prune.restype = c_int
         L.orc_adam_frozen.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, c_dbl, c_dbl, c_dbl, c_int, vp]
         L.orc_tau_diffuse.argtypes = [c_int, c_int, c_int, vp, vp, vp, c_dbl]
+        L.orc_jfa3x3.argtypes = [c_int, c_int, c_int, vp, vp, vp, c_int]
         L.orc_num_threads.restype = c_int
         L.orc_set_threads.argtypes = [c_int]
         _lib = L
@@ -273,12 +275,15 @@ def densify_prune(H: int, W: int, params, m, v, stats, target, cfg: DensifyCfg):
 
 
 def fit(H: int, W: int, params, target, N_cap: int, iterations: int, events, grow: int, prune_frac: float,
-        lr: dict, G: int, seed: int, on_event=None):
+        lr: dict, G: int, seed: int, on_event=None, update_every: int = 1):
     """The oracle's fitting schedule, step for step the device driver's: a
     refresh, then iterations of (propagate k=1, loss + backward, Adam in
     double stored as float32, records); an event iteration also accumulates
-    the statistics, densifies/prunes and refreshes.  Returns (params float32
-    (9, N_cap), last loss, number of propagation passes run)."""
+    the statistics, densifies/prunes and refreshes.  With update_every = U
+    the lists are propagated only on iterations 1, 1 + U, 1 + 2U, ... and on
+    event iterations; the others reuse the cached lists (summary B.3).
+    Returns (params float32 (9, N_cap), last loss, number of propagation
+    passes run)."""
     prm = np.zeros((9, N_cap), dtype=np.float32)
     n0 = params.shape[1]
     prm[:, :n0] = params
@@ -292,8 +297,9 @@ def fit(H: int, W: int, params, target, N_cap: int, iterations: int, events, gro
     step = 0
     L = None
     for it in range(1, iterations + 1):
-        tab = propagate(H, W, rec, tab, 1, G, seed, npass)
-        npass += 1
+        if it in events or (it - 1) % update_every == 0:
+            tab = propagate(H, W, rec, tab, 1, G, seed, npass)
+            npass += 1
         if it in events:
             L, g, st = loss_backward_stats(H, W, prm, tab, target)
         else:
@@ -319,3 +325,27 @@ def tau_diffuse(H: int, W: int, params, table, grads, lam: float):
     G = np.array(grads, dtype=np.float64, order="C", copy=True)
     lib().orc_tau_diffuse(H, W, params.shape[1], _p(params), _p(tab), _p(G), float(lam))
     return G
+
+
+def jfa3x3(H: int, W: int, rec32, table, jump: int):
+    """One 3x3 flood pass keeping the 4 best ids in slots 0-3."""
+    rec32 = _f32(rec32)
+    tin = _u32(table).reshape(H * W, K)
+    tout = np.empty_like(tin)
+    lib().orc_jfa3x3(H, W, rec32.shape[0], _p(rec32), _p(tin), _p(tout), int(jump))
+    return tout
+
+
+def flood_schedule(H: int, W: int) -> list:
+    """ceil(log2 max(W, H)) jumps: 2^(n-1), ..., 1."""
+    n = max(1, math.ceil(math.log2(max(H, W))))
+    return [1 << (n - 1 - q) for q in range(n)]
+
+
+def jfa_prepass(H: int, W: int, params):
+    """Seed pass, then one 3x3 flood pass per jump of flood_schedule."""
+    rec = records(H, W, params)
+    t = seed_table(H, W, params)
+    for k in flood_schedule(H, W):
+        t = jfa3x3(H, W, rec, t, k)
+    return t

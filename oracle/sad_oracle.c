@@ -868,3 +868,34 @@ void orc_tau_diffuse(int H, int W, int N, const float *params, const uint32_t *t
     memcpy(g, out, sizeof(double) * (size_t)N);
     free(out);
 }
+
+/* ------------------------------------------------------------------------ */
+/* JFA prepass ([P1] B.3, optional prepass)                                   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One 3x3 flood pass at jump k: for each pixel, the distinct valid ids of the
+ * lists at (i + a k, j + b k), a, b in {-1, 0, 1}, inside the image, re-scored
+ * at the pixel; the 4 best by (logit desc, id asc) go to slots 0-3 and slots
+ * 4-7 are emptied ("four closest sites into the first candidate texture").
+ */
+void orc_jfa3x3(int H, int W, int N, const float *rec32, const uint32_t *tin, uint32_t *tout, int jump)
+{
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int j = 0; j < H; ++j) {
+        for (int i = 0; i < W; ++i) {
+            const int64_t p = (int64_t)j * W + i;
+            const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
+            topk_t t;
+            topk_clear(&t);
+            for (int b = -1; b <= 1; ++b)
+                for (int a = -1; a <= 1; ++a) {
+                    const int ni = i + a * jump, nj = j + b * jump;
+                    if (ni < 0 || ni >= W || nj < 0 || nj >= H) continue;
+                    const int64_t pn = (int64_t)nj * W + ni;
+                    for (int q = 0; q < ORC_K; ++q) offer(&t, rec32, N, tin[pn * ORC_K + q], fx, fy);
+                }
+            for (int q = 0; q < ORC_K; ++q) tout[p * ORC_K + q] = (q < 4 && q < t.n) ? t.id[q] : ORC_SENTINEL;
+        }
+    }
+}

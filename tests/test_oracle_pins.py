@@ -545,3 +545,35 @@ def test_refresh_reaches_pages_accuracy_at_1024(orc):
     ex = orc.topk_exact(H, W, rec, pix)
     exact = np.all(np.sort(t[pix], 1) == np.sort(ex, 1), axis=1)
     assert exact.mean() > claim["min_fraction_exact"]
+
+
+def test_jfa3x3_prepass(orc):
+    """The optional 3x3 flood prepass ([P1] B.3): each pass keeps the 4 best
+    distinct candidates of the 9 lists at jump k, re-scored at the pixel
+    (checked against an independent restatement); on Euclidean sites the
+    prepass finds the nearest site on most pixels (jump flooding is
+    approximate) and only ever fills slots 0-3."""
+    H, W, N = 48, 40, 90
+    prm = _params(N, H, W, 81)                  # a = 0, r = 0, uniform tau
+    rec = orc.records(H, W, prm)
+    assert orc.flood_schedule(48, 40) == [32, 16, 8, 4, 2, 1]
+    t = orc.jfa_prepass(H, W, prm)
+    assert np.all(t[:, 4:] == SENT)
+    ex = orc.topk_exact(H, W, rec)
+    assert np.mean(t[:, 0] == ex[:, 0]) > 0.95
+    # one pass against an independent restatement
+    st = synth.Stream(5, "jfa")
+    tin = st.integers(H * W * 8, N + 3).astype(np.uint32).reshape(H * W, 8)
+    for k in (1, 3, 7):
+        got = orc.jfa3x3(H, W, rec, tin, k)
+        for p in range(0, H * W, 37):
+            j, i = divmod(p, W)
+            cand = [tin[(j + b * k) * W + i + a * k] for b in (-1, 0, 1) for a in (-1, 0, 1)
+                    if 0 <= i + a * k < W and 0 <= j + b * k < H]
+            ids = np.unique(np.concatenate(cand).astype(np.int64))
+            ids = ids[ids < N]
+            sc = np.array([orc.score32(rec, int(q), i, j) for q in ids])
+            order = np.lexsort((ids, -sc))[:4]
+            want = np.full(8, SENT, np.uint32)
+            want[:order.size] = ids[order]
+            np.testing.assert_array_equal(got[p], want)
