@@ -196,6 +196,14 @@ int sad_topk_exact(sad_ctx *ctx, const int64_t *pixels, int64_t n_pix, uint32_t 
  * <= max(H, W), each with G injections.  0 <= G <= 64. */
 int sad_refresh(sad_ctx *ctx, int G, sad_stream_t stream);
 
+/* Optional JFA prepass ([P1] B.3, for reinitialisation or after large
+ * edits): the seed pass, then ceil(log2 max(H, W)) flood passes at jumps
+ * 2^(n-1), ..., 1, each taking for every pixel the 4 best distinct candidates
+ * of the 9 lists at (i + a k, j + b k), a, b in {-1, 0, 1}, into slots 0-3
+ * ("four closest sites into the first candidate texture"; slots 4-7 empty).
+ * Propagation passes then fill the lists. */
+int sad_jfa_prepass(sad_ctx *ctx, sad_stream_t stream);
+
 /* Steps a2/a3: one Jacobi propagation pass at jump >= 1 ([P2] design 3):
  * for every pixel the new list is the top 8 by (logit desc, id asc) of the
  * distinct valid ids among its own list, the lists of the four pixels at
@@ -270,6 +278,12 @@ int sad_adam_step(sad_ctx *ctx, const sad_adam_cfg *cfg, sad_stream_t stream);
  * B.4: per-tile shared-memory reduction, one global atomic per site and
  * parameter).  Writes the bound image when one is bound. */
 int sad_fit_pass(sad_ctx *ctx, int G, sad_stream_t stream);
+
+/* Steps a4-a6 on the cached candidate lists, tiled like sad_fit_pass but
+ * without the propagation: for the iterations between candidate updates
+ * ([P1] B.3: updating every 8-16 iterations did not change the final PSNR).
+ * Same results as sad_backward; the current table is not changed. */
+int sad_fit_pass_cached(sad_ctx *ctx, sad_stream_t stream);
 
 /* One steady-state fitting iteration: sad_fit_pass then sad_adam_step
  * (steps a2-a7, two kernels). */

@@ -135,6 +135,12 @@ class Sad:
     def refresh(self, G: int):
         _lib.sad_refresh(self.ctx, G, self.stream)
 
+    def jfa_prepass(self):
+        _lib.sad_jfa_prepass(self.ctx, self.stream)
+
+    def fit_pass_cached(self):
+        _lib.sad_fit_pass_cached(self.ctx, self.stream)
+
     def propagate(self, jump: int, G: int):
         _lib.sad_propagate(self.ctx, jump, G, self.stream)
 

@@ -72,7 +72,8 @@ class sad_stats(ctypes.Structure):
 
 EXPORTED = (
     "sad_workspace_bytes", "sad_create", "sad_destroy", "sad_bind", "sad_reset", "sad_set_sites",
-    "sad_get_sites", "sad_set_target", "sad_prep_records", "sad_topk_exact", "sad_refresh", "sad_propagate",
+    "sad_get_sites", "sad_set_target", "sad_prep_records", "sad_topk_exact", "sad_refresh", "sad_jfa_prepass",
+    "sad_propagate", "sad_fit_pass_cached",
     "sad_render", "sad_backward", "sad_densify_prune", "sad_tau_diffuse", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
     "sad_get_stats", "sad_get_loss", "sad_last_error", "sad_backward_noalloc",
 )
@@ -110,6 +111,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "sad_topk_exact": [vp, vp, ci64, vp, vp],
         "sad_refresh": [vp, ci, vp],
         "sad_propagate": [vp, ci, ci, vp],
+        "sad_jfa_prepass": [vp, vp],
+        "sad_fit_pass_cached": [vp, vp],
         "sad_render": [vp, vp, vp],
         "sad_backward": [vp, cu32, vp],
         "sad_adam_step": [vp, ctypes.POINTER(sad_adam_cfg), vp],
@@ -210,6 +213,14 @@ def sad_topk_exact(ctx: int, pixels, n_pix: int, out, stream=None) -> None:
 
 def sad_refresh(ctx: int, G: int, stream=None) -> None:
     _check(ctx, load().sad_refresh(ctx, G, _stream(stream)))
+
+
+def sad_jfa_prepass(ctx: int, stream=None) -> None:
+    _check(ctx, load().sad_jfa_prepass(ctx, _stream(stream)))
+
+
+def sad_fit_pass_cached(ctx: int, stream=None) -> None:
+    _check(ctx, load().sad_fit_pass_cached(ctx, _stream(stream)))
 
 
 def sad_propagate(ctx: int, jump: int, G: int, stream=None) -> None:

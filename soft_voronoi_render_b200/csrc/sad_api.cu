@@ -226,6 +226,23 @@ int sad_refresh(sad_ctx *ctx, int G, sad_stream_t stream) {
     return run_refresh(ctx, G, cs(stream));
 }
 
+int sad_jfa_prepass(sad_ctx *ctx, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    cudaStream_t st = cs(stream);
+    r = cuda_status(ctx, sad::launch_seed(ctx->dev, st), "seed");
+    if (r) return r;
+    int n = 0;
+    const int m = ctx->H > ctx->W ? ctx->H : ctx->W;
+    while ((1 << n) < m) ++n;
+    if (n == 0) n = 1;
+    for (int q = n - 1; q >= 0; --q) {
+        r = cuda_status(ctx, sad::launch_jfa3x3(ctx->dev, 1 << q, st), "jfa pass");
+        if (r) return r;
+    }
+    return SAD_OK;
+}
+
 int sad_propagate(sad_ctx *ctx, int jump, int G, sad_stream_t stream) {
     int r = need_bound(ctx);
     if (r) return r;
@@ -306,6 +323,12 @@ int sad_fit_iteration(sad_ctx *ctx, int G, const sad_adam_cfg *cfg, sad_stream_t
     r = cuda_status(ctx, sad::launch_fit_tile(ctx->dev, G, st), "fit pass");
     if (r) return r;
     return cuda_status(ctx, sad::launch_adam(ctx->dev, h, st), "adam");
+}
+
+int sad_fit_pass_cached(sad_ctx *ctx, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    return cuda_status(ctx, sad::launch_fit_tile_cached(ctx->dev, cs(stream)), "fit pass (cached lists)");
 }
 
 int sad_fit_pass(sad_ctx *ctx, int G, sad_stream_t stream) {

@@ -14,6 +14,11 @@
 // built once per tile from the lists instead of by probing per contribution.
 // A tile whose lists hold more than 128 distinct sites takes a generic path
 // (per-candidate de-duplication against the running top-8, global atomics).
+//
+// The same kernel without the propagation (PROP = false) renders and
+// differentiates the cached lists as they stand, for the iterations between
+// candidate updates (summary B.3): no halo, no new lists, the pass counter
+// and the current table are left alone.
 #include "sad_device.cuh"
 #include "sad_launch.h"
 
@@ -249,7 +254,7 @@ __device__ __forceinline__ void generic_pass(Top8L &t, const uint4 *__restrict__
     }
 }
 
-template <int FY>
+template <int FY, bool PROP>
 __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(const float4 *__restrict__ rec,
                                                                             uint32_t *table,
                                                          const float *__restrict__ target, int H, int W, int N,
@@ -273,6 +278,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     const uint32_t Nu = (uint32_t)N;
 
     for (int q = tid; q < UHASH; q += FT) sm.keys[q] = EMPTY;
+    if (PROP)
     for (int r = tid; r < RING; r += FT) {
         int hx, hy;
         ring_coords<FY>(r, hx, hy);
@@ -314,8 +320,9 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         const uint32_t prev = __shfl_up_sync(FULL, id, 1);
         if (id < Nu && !(lane > 0 && prev == id)) ok &= ukey_insert(sm.keys, id);
     }
-    // the 84 halo pixels x 8 slots, spread over all threads: entry e is
-    // halo pixel e % RING, slot e / RING
+    // the halo pixels x 8 slots, spread over all threads: entry e is halo
+    // pixel e % RING, slot e / RING
+    if (PROP)
     for (int e = tid; e < RING * K; e += FT) {
         const int r = e % RING, q = e / RING;
         int hx, hy;
@@ -354,7 +361,8 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             if (q < 4) own_lx_lo = (own_lx_lo & m) | b;
             else own_lx_hi = (own_lx_hi & m) | b;
         }
-        sm.masks[(ty + 1) * HX + lane + 1] = own_mask;
+        if (PROP) sm.masks[(ty + 1) * HX + lane + 1] = own_mask;
+        if (PROP)
         for (int e = tid; e < RING * K; e += FT) {
             const int r = e % RING, q = e / RING;
             int hx, hy;
@@ -382,7 +390,34 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
     Top8L t;
     t.clear();
-    if (inside) {
+    unsigned dropped = 0;
+    if (inside && !PROP) {
+        // cached lists: every slot as it stands, like the standalone backward
+        // (a repeated id counts twice, an id >= N is reported as dropped)
+#pragma unroll
+        for (int q = 0; q < K; ++q) {
+            const uint32_t id = own[q];
+            dropped += (id >= Nu && id != EMPTY);
+            if (id >= Nu) continue;
+            uint32_t u = NOLOC;
+            float4 r0;
+            float2 r1;
+            if (fast) u = ((q < 4 ? own_lx_lo : own_lx_hi) >> ((q & 3) * 8)) & 0xFFu;
+            if (u < UCAP) {
+                r0 = sm.urec[0][u];
+                r1 = make_float2(sm.urec[1][u].x, sm.urec[1][u].y);
+            } else {
+                u = NOLOC;
+                r0 = __ldg(rec + (size_t)id * REC_F4);
+                r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
+            }
+            if (!(r0.x >= 0.0f)) continue;
+            t.l[q] = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+            t.id[q] = id;
+            t.lx[q] = u;
+        }
+    }
+    if (inside && PROP) {
         if (fast) {
             // the pixel's own list re-scored in its previous order, which the
             // new scores rarely change
@@ -635,6 +670,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     if (lane == 0) sm.warp_loss[ty] = lsum;
     const int n_empty = __syncthreads_count(inside && !vmask);
     const int n_global = __syncthreads_count(global_adds != 0);
+    const int n_dropped = PROP ? 0 : __syncthreads_count(dropped != 0);
     for (uint32_t e = tid; e < ucount * NPARAM; e += FT) {
         const uint32_t u = e % ucount, k = e / ucount;
         const float a = sm.acc[k][u];
@@ -646,6 +682,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         ws_loss_partials(ws)[blockIdx.y * gridDim.x + blockIdx.x] = (double)tl;
         if (n_empty) atomicAdd(&c->empty_pixels, (unsigned long long)n_empty);
         if (n_global) atomicAdd(&c->hash_overflow, (unsigned long long)n_global);
+        if (n_dropped) atomicAdd(&c->dropped_ids, (unsigned long long)n_dropped);
         __threadfence();
         sm.last = atomicAdd(&c->ticket_bwd, 1u) == gridDim.x * gridDim.y - 1;
     }
@@ -664,15 +701,17 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             double tsum = 0.0;
             for (int q = 0; q < FY; ++q) tsum += red[q];
             c->loss = tsum / (double)P;
-            c->cur = cur ^ 1u;
-            c->pass_counter = pass + 1u;
+            if (PROP) {
+                c->cur = cur ^ 1u;
+                c->pass_counter = pass + 1u;
+            }
             c->ticket_bwd = 0;
             __threadfence();
         }
     }
 }
 
-template <int FY>
+template <int FY, bool PROP>
 cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
     // the tile state exceeds the 48 KB default: opt in once per device
     static bool attr_set[64] = {};
@@ -680,13 +719,13 @@ cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(fit_tile_kernel<FY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(fit_tile_kernel<FY, PROP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sizeof(FusedSmem<FY>));
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
     const dim3 grid((d.W + FX - 1) / FX, (d.H + FY - 1) / FY);
-    fit_tile_kernel<FY><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY>), st>>>(d.records, d.table, d.target, d.H, d.W,
+    fit_tile_kernel<FY, PROP><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY>), st>>>(d.records, d.table, d.target, d.H, d.W,
                                                                            d.N, G, d.image, d.grads, d.ws);
     return cudaGetLastError();
 }
@@ -696,8 +735,13 @@ cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st) {
     // taller tiles amortise the halo and the per-tile work, but hold more
     // distinct sites: use them where sites are sparse (>= 16 pixels per site)
-    if ((long long)d.H * d.W >= 16ll * d.N) return launch_fit_tile_h<16>(d, G, st);
-    return launch_fit_tile_h<8>(d, G, st);
+    if ((long long)d.H * d.W >= 16ll * d.N) return launch_fit_tile_h<16, true>(d, G, st);
+    return launch_fit_tile_h<8, true>(d, G, st);
+}
+
+cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st) {
+    if ((long long)d.H * d.W >= 16ll * d.N) return launch_fit_tile_h<16, false>(d, 0, st);
+    return launch_fit_tile_h<8, false>(d, 0, st);
 }
 
 }  // namespace sad

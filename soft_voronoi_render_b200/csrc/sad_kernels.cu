@@ -251,6 +251,49 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
     }
 }
 
+// One 3x3 flood pass of the optional JFA prepass (summary B.3): the 4 best
+// distinct candidates of the lists at (i + a k, j + b k), a, b in {-1, 0, 1},
+// go to slots 0-3; slots 4-7 are emptied.
+__global__ void __launch_bounds__(TILE_THREADS) jfa3x3_kernel(const float4 *__restrict__ rec, uint32_t *table,
+                                                              int H, int W, int N, int jump, Counters *c) {
+    const uint32_t cur = c->cur, pass = c->pass_counter;
+    const size_t P = (size_t)H * W;
+    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + cur * P * K);
+    const uint4 *in1 = in0 + P;
+    uint4 *out0 = reinterpret_cast<uint4 *>(table + (cur ^ 1u) * P * K);
+    uint4 *out1 = out0 + P;
+    const int i = blockIdx.x * TILE_X + threadIdx.x;
+    const int j = blockIdx.y * TILE_Y + threadIdx.y;
+    if (i < W && j < H) {
+        const size_t p = (size_t)j * W + i;
+        const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
+        Top8 t;
+        t.clear();
+#pragma unroll 1
+        for (int d = 0; d < 9; ++d) {
+            const int ni = i + (d % 3 - 1) * jump, nj = j + (d / 3 - 1) * jump;
+            if (ni < 0 || ni >= W || nj < 0 || nj >= H) continue;
+            const size_t pn = (size_t)nj * W + ni;
+            const uint4 a = in0[pn], b = in1[pn];
+            const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            offer_batch<8>(t, ids, rec, (uint32_t)N, fx, fy);
+        }
+        out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
+        out1[p] = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && threadIdx.y == 0) {
+        __threadfence();
+        const unsigned total = gridDim.x * gridDim.y;
+        if (atomicAdd(&c->ticket_prop, 1u) == total - 1) {
+            c->cur = cur ^ 1u;
+            c->pass_counter = pass + 1u;
+            c->ticket_prop = 0;
+            __threadfence();
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // a4: render
 // ---------------------------------------------------------------------------
@@ -740,6 +783,12 @@ cudaError_t launch_seed(const Dev &d, cudaStream_t st) {
 cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st) {
     propagate_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.H, d.W, d.N,
                                                                            jump, G, host_counters(d));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st) {
+    jfa3x3_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.H, d.W, d.N, jump,
+                                                                        host_counters(d));
     return cudaGetLastError();
 }
 

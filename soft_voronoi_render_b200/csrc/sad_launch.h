@@ -43,6 +43,8 @@ cudaError_t launch_render_backward(const Dev &d, cudaStream_t st);
 cudaError_t launch_render_backward_stats(const Dev &d, cudaStream_t st);
 cudaError_t launch_densify(const Dev &d, const DensifyArgs &a, cudaStream_t st);
 cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st);
+cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st);
+cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st);
 cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st);
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st);
 

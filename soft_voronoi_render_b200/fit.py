@@ -4,8 +4,12 @@ A fit starts with a full candidate refresh, then runs fitting iterations.
 An iteration that precedes a budget-control event accumulates the
 statistics (propagate, backward with SAD_STATS, Adam), runs the
 densify/prune event and refreshes the candidate lists; every other
-iteration is one sad_fit_iteration (fused pass + Adam).  The site count
-stays on the device.
+iteration is one sad_fit_iteration (fused pass + Adam).  With
+``update_every`` = U > 1 the lists are propagated only on iterations 1,
+1 + U, 1 + 2U, ... (and event iterations); in between the pass renders and
+differentiates the cached lists (sad_fit_pass_cached), the infrequent
+candidate update of the pages' section B.3.  The site count stays on the
+device.
 """
 from __future__ import annotations
 
@@ -21,6 +25,7 @@ class Schedule:
     events: tuple = field(default_factory=lambda: tuple(range(100, 1601, 100)))
     grow: int = 2500
     prune_frac: float = 0.005
+    update_every: int = 1
     lr: dict = field(default_factory=lambda: dict(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=5e-3,
                                                   lr_theta=1e-3, lr_a=1e-3))
 
@@ -31,6 +36,8 @@ def run(sad, sched: Schedule, on_event=None) -> None:
     cfg = _lib.adam_cfg(**sched.lr)
     dcfg = _lib.densify_cfg(grow=sched.grow, prune_frac=sched.prune_frac)
     events = set(sched.events)
+    if sched.update_every < 1:
+        raise ValueError("update_every must be >= 1")
     _lib.sad_refresh(ctx, sched.G, st)
     for it in range(1, sched.iterations + 1):
         if it in events:
@@ -41,5 +48,8 @@ def run(sad, sched: Schedule, on_event=None) -> None:
             _lib.sad_refresh(ctx, sched.G, st)
             if on_event is not None:
                 on_event(it)
-        else:
+        elif (it - 1) % sched.update_every == 0:
             _lib.sad_fit_iteration(ctx, sched.G, cfg, st)
+        else:
+            _lib.sad_fit_pass_cached(ctx, st)
+            _lib.sad_adam_step(ctx, cfg, st)
