@@ -275,13 +275,14 @@ def densify_prune(H: int, W: int, params, m, v, stats, target, cfg: DensifyCfg):
 
 
 def fit(H: int, W: int, params, target, N_cap: int, iterations: int, events, grow: int, prune_frac: float,
-        lr: dict, G: int, seed: int, on_event=None, update_every: int = 1):
+        lr: dict, G: int, seed: int, on_event=None, update_every: int = 1, passes_per_update: int = 1):
     """The oracle's fitting schedule, step for step the device driver's: a
     refresh, then iterations of (propagate k=1, loss + backward, Adam in
     double stored as float32, records); an event iteration also accumulates
     the statistics, densifies/prunes and refreshes.  With update_every = U
     the lists are propagated only on iterations 1, 1 + U, 1 + 2U, ... and on
-    event iterations; the others reuse the cached lists (summary B.3).
+    event iterations; the others reuse the cached lists (summary B.3).  An
+    update outside an event runs passes_per_update jump-1 passes.
     Returns (params float32 (9, N_cap), last loss, number of propagation
     passes run)."""
     prm = np.zeros((9, N_cap), dtype=np.float32)
@@ -298,8 +299,9 @@ def fit(H: int, W: int, params, target, N_cap: int, iterations: int, events, gro
     L = None
     for it in range(1, iterations + 1):
         if it in events or (it - 1) % update_every == 0:
-            tab = propagate(H, W, rec, tab, 1, G, seed, npass)
-            npass += 1
+            for _ in range(1 if it in events else passes_per_update):
+                tab = propagate(H, W, rec, tab, 1, G, seed, npass)
+                npass += 1
         if it in events:
             L, g, st = loss_backward_stats(H, W, prm, tab, target)
         else:

@@ -8,8 +8,9 @@ iteration is one sad_fit_iteration (fused pass + Adam).  With
 ``update_every`` = U > 1 the lists are propagated only on iterations 1,
 1 + U, 1 + 2U, ... (and event iterations); in between the pass renders and
 differentiates the cached lists (sad_fit_pass_cached), the infrequent
-candidate update of the pages' section B.3.  The site count stays on the
-device.
+candidate update of the pages' section B.3; ``passes_per_update`` jump-1
+passes run at each such update (the last one fused with the render).  The
+site count stays on the device.
 """
 from __future__ import annotations
 
@@ -26,6 +27,7 @@ class Schedule:
     grow: int = 2500
     prune_frac: float = 0.005
     update_every: int = 1
+    passes_per_update: int = 1
     lr: dict = field(default_factory=lambda: dict(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=5e-3,
                                                   lr_theta=1e-3, lr_a=1e-3))
 
@@ -36,8 +38,8 @@ def run(sad, sched: Schedule, on_event=None) -> None:
     cfg = _lib.adam_cfg(**sched.lr)
     dcfg = _lib.densify_cfg(grow=sched.grow, prune_frac=sched.prune_frac)
     events = set(sched.events)
-    if sched.update_every < 1:
-        raise ValueError("update_every must be >= 1")
+    if sched.update_every < 1 or sched.passes_per_update < 1:
+        raise ValueError("update_every and passes_per_update must be >= 1")
     _lib.sad_refresh(ctx, sched.G, st)
     for it in range(1, sched.iterations + 1):
         if it in events:
@@ -49,6 +51,8 @@ def run(sad, sched: Schedule, on_event=None) -> None:
             if on_event is not None:
                 on_event(it)
         elif (it - 1) % sched.update_every == 0:
+            for _ in range(sched.passes_per_update - 1):
+                _lib.sad_propagate(ctx, 1, sched.G, st)
             _lib.sad_fit_iteration(ctx, sched.G, cfg, st)
         else:
             _lib.sad_fit_pass_cached(ctx, st)

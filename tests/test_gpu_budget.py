@@ -108,9 +108,11 @@ def test_short_fit_with_densify_events(torch_cuda):
                                  on_event=lambda it, p: ocounts.append(int((p[0] >= 0).sum())))
     assert counts == ocounts == [1000 - 10 + 410, 1400 - 14 + 414]
     assert s.stats()["pass_counter"] == npass
-    # the statistics are float32 atomic sums on the GPU and doubles in the
-    # oracle, so selections near a threshold can differ and the two fits
-    # drift apart after an event: compare the outcome in PSNR
+    # the two agree step for step, not along a whole fit: Adam's first steps
+    # divide gradients of order 1e-8 by |g| + eps, turning float32 rounding
+    # into small position differences that later iterations carry on, and
+    # float32 statistics can flip densify selections near a threshold:
+    # compare the outcome in PSNR
     psnr = lambda L: 10 * math.log10(3.0 / L)
     assert abs(psnr(L_gpu) - psnr(L_orc)) <= 0.2, (L_gpu, L_orc)
 

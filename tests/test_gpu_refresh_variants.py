@@ -113,22 +113,55 @@ def test_fit_pass_cached_crowded_tiles(torch_cuda):
     assert s.stats()["hash_overflow"] > 0
 
 
+def test_infrequent_updates_step_by_step(torch_cuda):
+    """Propagating only every 3rd iteration (summary B.3): each iteration,
+    checked against the oracle on the GPU's own state before it, gives the
+    oracle's propagated table (or leaves the cached one alone) and its loss."""
+    from soft_voronoi_render_b200 import _lib, adam_cfg
+    H, W, N, G, U = 64, 96, 600, 2, 3
+    tgt = synth.make_image(H, W, 8, 0, 41)
+    prm = synth.gradient_sites(tgt, N, 41)
+    s = _ctx(H, W, N, prm, tgt, seed=4)
+    cfg = adam_cfg(lr_color=5e-3)
+    s.refresh(G)
+    npass = len(oracle.jump_schedule(H, W))
+    for it in range(1, 8):
+        P, T = s.get_sites(), s.get_table()
+        if (it - 1) % U == 0:
+            s.fit_pass(G)
+            T = oracle.propagate(H, W, oracle.records(H, W, P), T, 1, G, seed=4, pass_index=npass)
+            npass += 1
+        else:
+            s.fit_pass_cached()
+        np.testing.assert_array_equal(s.get_table(), T)
+        L, g = oracle.loss_backward(H, W, P, T, tgt)
+        assert abs(s.loss() - L) <= LOSS_RTOL * L
+        _assert_grads(s.grads.cpu().numpy(), g, f"iteration {it}")
+        _lib.sad_adam_step(s.ctx, cfg, s.stream)
+    assert s.stats()["pass_counter"] == npass
+
+
 def test_infrequent_updates_schedule(torch_cuda):
-    """A fit that propagates only every 4th iteration (summary B.3) against
-    the oracle's schedule: the same number of propagation passes, the lists
-    unchanged in between, and the same loss within 0.05 dB PSNR."""
+    """fit.run with update_every = 4 and two passes per update against the
+    oracle's schedule: the same propagation passes, and the same outcome
+    within 0.2 dB PSNR.  The two agree step for step (previous test), but
+    not along a whole fit: Adam's
+    first steps divide gradients of order 1e-8 by |g| + eps, which turns
+    float32 rounding into position differences of a few hundredths of a
+    pixel that the following iterations carry on."""
     import math
     from soft_voronoi_render_b200 import fit
     H, W, N, G = 64, 96, 600, 2
     tgt = synth.make_image(H, W, 8, 0, 41)
     prm = synth.gradient_sites(tgt, N, 41)
     s = _ctx(H, W, N, prm, tgt, seed=4)
-    sched = fit.Schedule(iterations=12, G=G, events=(), update_every=4)
+    sched = fit.Schedule(iterations=12, G=G, events=(), update_every=4, passes_per_update=2)
     fit.run(s, sched)
     lr = dict(pos=1e-3, log_tau=1e-3, r=1e-3, color=5e-3, theta=1e-3, a=1e-3)
     lr32 = {k: float(np.float32(x)) for k, x in lr.items()}
-    _, L_orc, npass = oracle.fit(H, W, prm, tgt, N, 12, (), 0, 0.0, lr32, G, 4, update_every=4)
-    assert s.stats()["pass_counter"] == npass == len(oracle.jump_schedule(H, W)) + 3
+    _, L_orc, npass = oracle.fit(H, W, prm, tgt, N, 12, (), 0, 0.0, lr32, G, 4, update_every=4,
+                                 passes_per_update=2)
+    assert s.stats()["pass_counter"] == npass == len(oracle.jump_schedule(H, W)) + 6
     assert s.stats()["adam_step"] == 12
     psnr = lambda L: 10 * math.log10(3.0 / L)
-    assert abs(psnr(s.loss()) - psnr(L_orc)) <= 0.05, (s.loss(), L_orc)
+    assert abs(psnr(s.loss()) - psnr(L_orc)) <= 0.2, (s.loss(), L_orc)
