@@ -38,6 +38,12 @@ def lib():
         L.orc_score32.argtypes = [vp, c_int, c_int, c_int]
         L.orc_score32.restype = ctypes.c_float
         L.orc_topk_exact.argtypes = [c_int, c_int, c_int, vp, vp, c_i64, vp]
+        L.orc_topk_exact_cell.argtypes = [c_int, c_int, c_int, c_int, vp, vp, c_i64, vp]
+        L.orc_propagate_cell.argtypes = [c_int, c_int, c_int, c_int, vp, vp, vp, c_int, c_int, c_u32, c_u32]
+        L.orc_seed_cell.argtypes = [c_int, c_int, c_int, c_int, vp, vp]
+        L.orc_jfa3x3_cell.argtypes = [c_int, c_int, c_int, c_int, vp, vp, vp, c_int]
+        L.orc_score32_at.argtypes = [vp, c_int, ctypes.c_float, ctypes.c_float]
+        L.orc_score32_at.restype = ctypes.c_float
         L.orc_fmix32.argtypes = [c_u32]
         L.orc_fmix32.restype = c_u32
         L.orc_xorshift32.argtypes = [c_u32]
@@ -100,18 +106,40 @@ def score32(rec32: np.ndarray, site: int, i: int, j: int) -> float:
     return float(lib().orc_score32(_p(rec32), int(site), int(i), int(j)))
 
 
-def topk_exact(H: int, W: int, rec32: np.ndarray, pixels: np.ndarray | None = None) -> np.ndarray:
-    """Brute-force top-8 over all active sites; (n_pix, 8) uint32."""
+def score32_at(rec32: np.ndarray, site: int, fx: float, fy: float) -> float:
+    rec32 = _f32(rec32)
+    return float(lib().orc_score32_at(_p(rec32), int(site), float(fx), float(fy)))
+
+
+def grid_dims(H: int, W: int, cell: int = 1):
+    """Candidate grid of an H x W image with cells of cell x cell pixels
+    ("Candidate field", summary B.3): (ceil(H / cell), ceil(W / cell))."""
+    return (H + cell - 1) // cell, (W + cell - 1) // cell
+
+
+def expand_table(H: int, W: int, table: np.ndarray, cell: int) -> np.ndarray:
+    """Per-pixel view of a candidate-grid table: pixel (x, y) takes the list
+    of cell (x // cell, y // cell)."""
+    GH, GW = grid_dims(H, W, cell)
+    tab = _u32(table).reshape(GH * GW, K)
+    jj, ii = np.mgrid[0:H, 0:W]
+    return np.ascontiguousarray(tab[((jj // cell) * GW + ii // cell).ravel()])
+
+
+def topk_exact(H: int, W: int, rec32: np.ndarray, pixels: np.ndarray | None = None, cell: int = 1) -> np.ndarray:
+    """Brute-force top-8 over all active sites at each requested pixel (cell
+    centre when cell > 1); (n_pix, 8) uint32."""
     rec32 = _f32(rec32)
     N = rec32.shape[0]
+    GH, GW = grid_dims(H, W, cell)
     if pixels is None:
-        n = H * W
+        n = GH * GW
         out = np.empty((n, K), dtype=np.uint32)
-        lib().orc_topk_exact(H, W, N, _p(rec32), None, n, _p(out))
+        lib().orc_topk_exact_cell(GH, GW, cell, N, _p(rec32), None, n, _p(out))
     else:
         pix = np.ascontiguousarray(pixels, dtype=np.int64)
         out = np.empty((pix.size, K), dtype=np.uint32)
-        lib().orc_topk_exact(H, W, N, _p(rec32), _p(pix), pix.size, _p(out))
+        lib().orc_topk_exact_cell(GH, GW, cell, N, _p(rec32), _p(pix), pix.size, _p(out))
     return out
 
 
@@ -130,20 +158,23 @@ def inject_ids(seed: int, pass_index: int, pixel: int, N: int, G: int) -> np.nda
 
 
 def propagate(H: int, W: int, rec32: np.ndarray, table: np.ndarray, jump: int, G: int,
-              seed: int, pass_index: int) -> np.ndarray:
-    """One Jacobi propagation pass; returns the new (P, 8) table."""
+              seed: int, pass_index: int, cell: int = 1) -> np.ndarray:
+    """One Jacobi propagation pass on the candidate grid of an H x W image;
+    returns the new (cells, 8) table."""
     rec32 = _f32(rec32)
-    tin = _u32(table).reshape(H * W, K)
+    GH, GW = grid_dims(H, W, cell)
+    tin = _u32(table).reshape(GH * GW, K)
     tout = np.empty_like(tin)
-    lib().orc_propagate(H, W, rec32.shape[0], _p(rec32), _p(tin), _p(tout), int(jump), int(G),
-                        seed & 0xFFFFFFFF, pass_index & 0xFFFFFFFF)
+    lib().orc_propagate_cell(GH, GW, cell, rec32.shape[0], _p(rec32), _p(tin), _p(tout), int(jump), int(G),
+                             seed & 0xFFFFFFFF, pass_index & 0xFFFFFFFF)
     return tout
 
 
-def seed_table(H: int, W: int, params: np.ndarray) -> np.ndarray:
+def seed_table(H: int, W: int, params: np.ndarray, cell: int = 1) -> np.ndarray:
     params = _f32(params)
-    out = np.empty((H * W, K), dtype=np.uint32)
-    lib().orc_seed(H, W, params.shape[1], _p(params), _p(out))
+    GH, GW = grid_dims(H, W, cell)
+    out = np.empty((GH * GW, K), dtype=np.uint32)
+    lib().orc_seed_cell(H, W, cell, params.shape[1], _p(params), _p(out))
     return out
 
 
@@ -160,14 +191,14 @@ def jump_schedule(H: int, W: int) -> list:
     return out
 
 
-def refresh(H: int, W: int, params: np.ndarray, G: int, seed: int, first_pass: int = 0):
-    """Seed pass then one propagation pass per jump of ``jump_schedule``.
-    Returns (table, number of passes run)."""
+def refresh(H: int, W: int, params: np.ndarray, G: int, seed: int, first_pass: int = 0, cell: int = 1):
+    """Seed pass then one propagation pass per jump of ``jump_schedule`` of
+    the candidate grid.  Returns (table, number of passes run)."""
     rec = records(H, W, params)
-    t = seed_table(H, W, params)
+    t = seed_table(H, W, params, cell)
     n = 0
-    for k in jump_schedule(H, W):
-        t = propagate(H, W, rec, t, k, G, seed, first_pass + n)
+    for k in jump_schedule(*grid_dims(H, W, cell)):
+        t = propagate(H, W, rec, t, k, G, seed, first_pass + n, cell)
         n += 1
     return t, n
 
@@ -329,12 +360,13 @@ def tau_diffuse(H: int, W: int, params, table, grads, lam: float):
     return G
 
 
-def jfa3x3(H: int, W: int, rec32, table, jump: int):
+def jfa3x3(H: int, W: int, rec32, table, jump: int, cell: int = 1):
     """One 3x3 flood pass keeping the 4 best ids in slots 0-3."""
     rec32 = _f32(rec32)
-    tin = _u32(table).reshape(H * W, K)
+    GH, GW = grid_dims(H, W, cell)
+    tin = _u32(table).reshape(GH * GW, K)
     tout = np.empty_like(tin)
-    lib().orc_jfa3x3(H, W, rec32.shape[0], _p(rec32), _p(tin), _p(tout), int(jump))
+    lib().orc_jfa3x3_cell(GH, GW, cell, rec32.shape[0], _p(rec32), _p(tin), _p(tout), int(jump))
     return tout
 
 
@@ -344,10 +376,11 @@ def flood_schedule(H: int, W: int) -> list:
     return [1 << (n - 1 - q) for q in range(n)]
 
 
-def jfa_prepass(H: int, W: int, params):
-    """Seed pass, then one 3x3 flood pass per jump of flood_schedule."""
+def jfa_prepass(H: int, W: int, params, cell: int = 1):
+    """Seed pass, then one 3x3 flood pass per jump of flood_schedule of the
+    candidate grid."""
     rec = records(H, W, params)
-    t = seed_table(H, W, params)
-    for k in flood_schedule(H, W):
-        t = jfa3x3(H, W, rec, t, k)
+    t = seed_table(H, W, params, cell)
+    for k in flood_schedule(*grid_dims(H, W, cell)):
+        t = jfa3x3(H, W, rec, t, k, cell)
     return t

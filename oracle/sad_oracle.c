@@ -161,6 +161,21 @@ float orc_score32(const float *rec32, int id, int i, int j)
     return score32(rec32 + (size_t)id * ORC_REC, (float)i + 0.5f, (float)j + 0.5f);
 }
 
+/* the same score at an arbitrary point (a candidate-grid cell centre) */
+float orc_score32_at(const float *rec32, int id, float fx, float fy)
+{
+    return score32(rec32 + (size_t)id * ORC_REC, fx, fy);
+}
+
+/*
+ * Candidate grid ([P1] B.3, "Candidate field"): the lists live on a grid of
+ * ceil(W/cell) x ceil(H/cell) cells; cell (i, j) holds the pixels with
+ * floor(x/cell) = i, floor(y/cell) = j and scores its candidates at its
+ * centre ((i + 0.5) cell, (j + 0.5) cell).  cell = 1 is the pixel grid.
+ * The functions below that take (GH, GW, cell) work on that grid.
+ */
+static float cell_centre(int i, int cell) { return ((float)i + 0.5f) * (float)cell; }
+
 /* candidate a ranks above candidate b */
 static int ranks_above(float la, uint32_t ia, float lb, uint32_t ib)
 {
@@ -208,15 +223,15 @@ static void topk_store(const topk_t *t, uint32_t *out)
  * scored at every requested pixel.  pix == NULL means all pixels in order.
  * out: n_pix x 8 site ids, sentinel-padded.
  */
-void orc_topk_exact(int H, int W, int N, const float *rec32, const int64_t *pix, int64_t n_pix,
-                    uint32_t *out)
+void orc_topk_exact_cell(int GH, int GW, int cell, int N, const float *rec32, const int64_t *pix, int64_t n_pix,
+                         uint32_t *out)
 {
-    const int64_t P = (int64_t)H * W;
+    const int64_t P = (int64_t)GH * GW;
     if (!pix) n_pix = P;
 #pragma omp parallel for schedule(dynamic, 64)
     for (int64_t q = 0; q < n_pix; ++q) {
         const int64_t p = pix ? pix[q] : q;
-        const float fx = (float)(p % W) + 0.5f, fy = (float)(p / W) + 0.5f;
+        const float fx = cell_centre((int)(p % GW), cell), fy = cell_centre((int)(p / GW), cell);
         topk_t t;
         topk_clear(&t);
         for (int i = 0; i < N; ++i) {
@@ -290,10 +305,12 @@ static void offer(topk_t *t, const float *rec32, int N, uint32_t id, float fx, f
  *   C_t(x) = topK( C_{t-1}(x) U C_{t-1}(x +- k e_x) U C_{t-1}(x +- k e_y) U G_t(x) )
  * (temporal reuse + self and 4-neighbour propagation + G stochastic
  * injections, all re-scored at x).  Out-of-image neighbours are skipped.
- * Tables are P x 8 site ids.  0 <= G <= 64.
+ * Here H x W is the candidate grid and x a cell centre (cell = 1: pixels);
+ * injections are keyed on the cell index.  Tables are H W x 8 site ids.
+ * 0 <= G <= 64.
  */
-void orc_propagate(int H, int W, int N, const float *rec32, const uint32_t *tin, uint32_t *tout,
-                   int jump, int G, uint32_t seed, uint32_t pass)
+void orc_propagate_cell(int H, int W, int cell, int N, const float *rec32, const uint32_t *tin, uint32_t *tout,
+                        int jump, int G, uint32_t seed, uint32_t pass)
 {
     if (G > 64) G = 64;
     if (G < 0) G = 0;
@@ -302,7 +319,7 @@ void orc_propagate(int H, int W, int N, const float *rec32, const uint32_t *tin,
         uint32_t inj[64];
         for (int i = 0; i < W; ++i) {
             const int64_t p = (int64_t)j * W + i;
-            const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
+            const float fx = cell_centre(i, cell), fy = cell_centre(j, cell);
             topk_t t;
             topk_clear(&t);
             for (int q = 0; q < ORC_K; ++q) offer(&t, rec32, N, tin[p * ORC_K + q], fx, fy);
@@ -328,16 +345,17 @@ void orc_propagate(int H, int W, int N, const float *rec32, const uint32_t *tin,
  * image writes its id to slot 0 of the pixel containing it; the smallest id
  * wins where several sites share a pixel.
  */
-void orc_seed(int H, int W, int N, const float *params, uint32_t *table)
+void orc_seed_cell(int H, int W, int cell, int N, const float *params, uint32_t *table)
 {
-    const int64_t P = (int64_t)H * W;
+    const int GW = (W + cell - 1) / cell, GH = (H + cell - 1) / cell;
+    const int64_t P = (int64_t)GH * GW;
     for (int64_t q = 0; q < P * ORC_K; ++q) table[q] = ORC_SENTINEL;
     for (int i = 0; i < N; ++i) {
         const float px = params[P_X * N + i], py = params[P_Y * N + i];
         if (!(px >= 0.0f) || !(py >= 0.0f)) continue;
         const int64_t ci = (int64_t)floorf(px), cj = (int64_t)floorf(py);
         if (ci >= W || cj >= H) continue;
-        uint32_t *slot = table + (cj * W + ci) * ORC_K;
+        uint32_t *slot = table + ((cj / cell) * GW + ci / cell) * ORC_K;
         if ((uint32_t)i < slot[0]) slot[0] = (uint32_t)i;
     }
 }
@@ -879,13 +897,14 @@ void orc_tau_diffuse(int H, int W, int N, const float *params, const uint32_t *t
  * at the pixel; the 4 best by (logit desc, id asc) go to slots 0-3 and slots
  * 4-7 are emptied ("four closest sites into the first candidate texture").
  */
-void orc_jfa3x3(int H, int W, int N, const float *rec32, const uint32_t *tin, uint32_t *tout, int jump)
+void orc_jfa3x3_cell(int H, int W, int cell, int N, const float *rec32, const uint32_t *tin, uint32_t *tout,
+                     int jump)
 {
 #pragma omp parallel for schedule(dynamic, 4)
     for (int j = 0; j < H; ++j) {
         for (int i = 0; i < W; ++i) {
             const int64_t p = (int64_t)j * W + i;
-            const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
+            const float fx = cell_centre(i, cell), fy = cell_centre(j, cell);
             topk_t t;
             topk_clear(&t);
             for (int b = -1; b <= 1; ++b)
@@ -898,4 +917,26 @@ void orc_jfa3x3(int H, int W, int N, const float *rec32, const uint32_t *tin, ui
             for (int q = 0; q < ORC_K; ++q) tout[p * ORC_K + q] = (q < 4 && q < t.n) ? t.id[q] : ORC_SENTINEL;
         }
     }
+}
+
+/* pixel-grid (cell = 1) forms of the candidate-grid functions */
+void orc_topk_exact(int H, int W, int N, const float *rec32, const int64_t *pix, int64_t n_pix, uint32_t *out)
+{
+    orc_topk_exact_cell(H, W, 1, N, rec32, pix, n_pix, out);
+}
+
+void orc_propagate(int H, int W, int N, const float *rec32, const uint32_t *tin, uint32_t *tout, int jump, int G,
+                   uint32_t seed, uint32_t pass)
+{
+    orc_propagate_cell(H, W, 1, N, rec32, tin, tout, jump, G, seed, pass);
+}
+
+void orc_seed(int H, int W, int N, const float *params, uint32_t *table)
+{
+    orc_seed_cell(H, W, 1, N, params, table);
+}
+
+void orc_jfa3x3(int H, int W, int N, const float *rec32, const uint32_t *tin, uint32_t *tout, int jump)
+{
+    orc_jfa3x3_cell(H, W, 1, N, rec32, tin, tout, jump);
 }
