@@ -196,6 +196,24 @@ int sad_topk_exact(sad_ctx *ctx, const int64_t *pixels, int64_t n_pix, uint32_t 
  * <= max(H, W), each with G injections.  0 <= G <= 64. */
 int sad_refresh(sad_ctx *ctx, int G, sad_stream_t stream);
 
+/* Candidate grid ([P1] B.3, "Candidate field"): keep the candidate lists on
+ * a ceil(H/cell) x ceil(W/cell) grid of cell x cell pixel cells instead of
+ * one list per pixel.  Cell (i, j) holds the pixels with floor(x/cell) = i,
+ * floor(y/cell) = j (integer mapping, no interpolation); propagation, seed,
+ * exact top-K and the JFA prepass work on the grid and score candidates at
+ * the cell centre ((i + 0.5) cell, (j + 0.5) cell) ("centred cell UVs");
+ * render and backward score each pixel's cell list at the pixel centre.
+ * Injections are keyed on the cell index.  cell = 1 (the default) is the
+ * pixel grid; the fused tile passes run only there, a coarser grid runs
+ * sad_propagate + sad_backward for sad_fit_pass and sad_backward for
+ * sad_fit_pass_cached.  The table buffer bound for H x W holds any grid.
+ * After the call the current table is empty (sentinels): call sad_refresh,
+ * sad_jfa_prepass or sad_set_table next.  sad_get_table, sad_set_table and
+ * sad_topk_exact (pixels = NULL, or cell indices) then use GH x GW lists.
+ * Errors: SAD_ERR_INVALID_ARG when cell < 1 or cell > max(H, W).  May be
+ * called before sad_bind (no launch then). */
+int sad_set_candidate_grid(sad_ctx *ctx, int cell, sad_stream_t stream);
+
 /* Optional JFA prepass ([P1] B.3, for reinitialisation or after large
  * edits): the seed pass, then ceil(log2 max(H, W)) flood passes at jumps
  * 2^(n-1), ..., 1, each taking for every pixel the 4 best distinct candidates

@@ -38,6 +38,7 @@ class Sad:
         self.torch = torch
         self.H, self.W, self.N = int(H), int(W), int(N_cap)
         self.P = self.H * self.W
+        self.cell, self.PT = 1, self.P  # candidate grid (set_candidate_grid)
         self.device = torch.device(device)
         _lib.load()
         f32 = dict(dtype=torch.float32, device=self.device)
@@ -102,13 +103,19 @@ class Sad:
     def reset(self, seed: int = 1):
         _lib.sad_reset(self.ctx, seed, self.stream)
 
+    def set_candidate_grid(self, cell: int):
+        """Lists on a ceil(H/cell) x ceil(W/cell) grid; the table starts empty."""
+        _lib.sad_set_candidate_grid(self.ctx, cell, self.stream)
+        self.cell = cell
+        self.PT = ((self.H + cell - 1) // cell) * ((self.W + cell - 1) // cell)
+
     def get_table(self) -> np.ndarray:
-        out = np.empty((self.P, 8), dtype=np.uint32)
+        out = np.empty((self.PT, 8), dtype=np.uint32)
         _lib.sad_get_table(self.ctx, out, self.stream)
         return out
 
     def set_table(self, table: np.ndarray):
-        src = np.ascontiguousarray(table, dtype=np.uint32).reshape(self.P, 8)
+        src = np.ascontiguousarray(table, dtype=np.uint32).reshape(self.PT, 8)
         _lib.sad_set_table(self.ctx, src, self.stream)
 
     def stats(self) -> dict:
@@ -124,8 +131,8 @@ class Sad:
     def topk_exact(self, pixels=None):
         t = self.torch
         if pixels is None:
-            out = t.empty((self.P, 8), dtype=t.int32, device=self.device)
-            _lib.sad_topk_exact(self.ctx, None, self.P, out, self.stream)
+            out = t.empty((self.PT, 8), dtype=t.int32, device=self.device)
+            _lib.sad_topk_exact(self.ctx, None, self.PT, out, self.stream)
         else:
             pix = self._dev(pixels, t.int64)
             out = t.empty((pix.numel(), 8), dtype=t.int32, device=self.device)

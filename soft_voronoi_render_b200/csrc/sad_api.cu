@@ -14,6 +14,8 @@
 struct sad_ctx {
     int H, W, N, K;
     long long P;
+    int cell, GH, GW;
+    long long PT;
     bool bound;
     sad_buffers buf;
     sad::Dev dev;
@@ -58,13 +60,22 @@ int run_refresh(sad_ctx *ctx, int G, cudaStream_t st) {
     int r = cuda_status(ctx, sad::launch_seed(ctx->dev, st), "seed");
     if (r) return r;
     int B = 1;
-    const int m = ctx->H > ctx->W ? ctx->H : ctx->W;
+    const int m = ctx->GH > ctx->GW ? ctx->GH : ctx->GW;
     while (B * 2 <= m) B *= 2;
     for (int k = B / 2; k >= 1; k /= 2) {
         r = cuda_status(ctx, sad::launch_propagate(ctx->dev, k, G, st), "propagate");
         if (r) return r;
     }
     return SAD_OK;
+}
+
+// the fused tile kernel works on the pixel grid; a coarser candidate grid
+// runs the separate propagation and backward kernels
+int run_fit_pass(sad_ctx *ctx, int G, cudaStream_t st) {
+    if (ctx->cell == 1) return cuda_status(ctx, sad::launch_fit_tile(ctx->dev, G, st), "fit pass");
+    int r = cuda_status(ctx, sad::launch_propagate(ctx->dev, 1, G, st), "propagate");
+    if (r) return r;
+    return cuda_status(ctx, sad::launch_render_backward(ctx->dev, st), "backward");
 }
 
 int check_adam(sad_ctx *ctx, const sad_adam_cfg *cfg, sad::AdamHyper &h) {
@@ -106,6 +117,10 @@ int sad_create(int H, int W, int N_cap, int K, sad_ctx **out) {
     c->N = N_cap;
     c->K = K;
     c->P = (long long)H * W;
+    c->cell = 1;
+    c->GH = H;
+    c->GW = W;
+    c->PT = c->P;
     c->bound = false;
     c->err[0] = 0;
     *out = c;
@@ -138,6 +153,10 @@ int sad_bind(sad_ctx *ctx, const sad_buffers *b) {
     d.W = ctx->W;
     d.N = ctx->N;
     d.P = ctx->P;
+    d.cell = ctx->cell;
+    d.GH = ctx->GH;
+    d.GW = ctx->GW;
+    d.PT = ctx->PT;
     d.params = b->params;
     d.grads = b->grads;
     d.adam_m = b->adam_m;
@@ -213,7 +232,7 @@ int sad_prep_records(sad_ctx *ctx, sad_stream_t stream) {
 int sad_topk_exact(sad_ctx *ctx, const int64_t *pixels, int64_t n_pix, uint32_t *out, sad_stream_t stream) {
     int r = need_bound(ctx);
     if (r) return r;
-    if (!pixels) n_pix = ctx->P;
+    if (!pixels) n_pix = ctx->PT;
     if (n_pix < 0 || (n_pix > 0 && !out)) return fail(ctx, SAD_ERR_INVALID_ARG, "bad top-K output");
     if (out && !aligned16(out)) return fail(ctx, SAD_ERR_INVALID_ARG, "top-K output is not 16-byte aligned");
     return cuda_status(ctx, sad::launch_topk_exact(ctx->dev, pixels, n_pix, out, cs(stream)), "topk_exact");
@@ -233,7 +252,7 @@ int sad_jfa_prepass(sad_ctx *ctx, sad_stream_t stream) {
     r = cuda_status(ctx, sad::launch_seed(ctx->dev, st), "seed");
     if (r) return r;
     int n = 0;
-    const int m = ctx->H > ctx->W ? ctx->H : ctx->W;
+    const int m = ctx->GH > ctx->GW ? ctx->GH : ctx->GW;
     while ((1 << n) < m) ++n;
     if (n == 0) n = 1;
     for (int q = n - 1; q >= 0; --q) {
@@ -320,7 +339,7 @@ int sad_fit_iteration(sad_ctx *ctx, int G, const sad_adam_cfg *cfg, sad_stream_t
     r = check_adam(ctx, cfg, h);
     if (r) return r;
     cudaStream_t st = cs(stream);
-    r = cuda_status(ctx, sad::launch_fit_tile(ctx->dev, G, st), "fit pass");
+    r = run_fit_pass(ctx, G, st);
     if (r) return r;
     return cuda_status(ctx, sad::launch_adam(ctx->dev, h, st), "adam");
 }
@@ -328,6 +347,7 @@ int sad_fit_iteration(sad_ctx *ctx, int G, const sad_adam_cfg *cfg, sad_stream_t
 int sad_fit_pass_cached(sad_ctx *ctx, sad_stream_t stream) {
     int r = need_bound(ctx);
     if (r) return r;
+    if (ctx->cell != 1) return cuda_status(ctx, sad::launch_render_backward(ctx->dev, cs(stream)), "backward");
     return cuda_status(ctx, sad::launch_fit_tile_cached(ctx->dev, cs(stream)), "fit pass (cached lists)");
 }
 
@@ -335,7 +355,25 @@ int sad_fit_pass(sad_ctx *ctx, int G, sad_stream_t stream) {
     int r = need_bound(ctx);
     if (r) return r;
     if (G < 0 || G > SAD_MAX_INJECT) return fail(ctx, SAD_ERR_CAPACITY, "G=%d outside [0, %d]", G, SAD_MAX_INJECT);
-    return cuda_status(ctx, sad::launch_fit_tile(ctx->dev, G, cs(stream)), "fit pass");
+    return run_fit_pass(ctx, G, cs(stream));
+}
+
+int sad_set_candidate_grid(sad_ctx *ctx, int cell, sad_stream_t stream) {
+    if (!ctx) return SAD_ERR_INVALID_ARG;
+    const int m = ctx->H > ctx->W ? ctx->H : ctx->W;
+    if (cell < 1 || cell > m) return fail(ctx, SAD_ERR_INVALID_ARG, "cell size %d outside [1, %d]", cell, m);
+    ctx->cell = cell;
+    ctx->GH = (ctx->H + cell - 1) / cell;
+    ctx->GW = (ctx->W + cell - 1) / cell;
+    ctx->PT = (long long)ctx->GH * ctx->GW;
+    if (!ctx->bound) return SAD_OK;
+    sad::Dev &d = ctx->dev;
+    d.cell = ctx->cell;
+    d.GH = ctx->GH;
+    d.GW = ctx->GW;
+    d.PT = ctx->PT;
+    // the lists of the old grid mean nothing on the new one: start empty
+    return cuda_status(ctx, sad::launch_clear_table(d, cs(stream)), "clear table");
 }
 
 int sad_get_table(sad_ctx *ctx, uint32_t *dst, sad_stream_t stream) {
@@ -346,10 +384,10 @@ int sad_get_table(sad_ctx *ctx, uint32_t *dst, sad_stream_t stream) {
     sad::Counters c;
     r = read_counters(ctx, &c, st);
     if (r) return r;
-    const uint32_t *plane0 = ctx->buf.table + (size_t)c.cur * ctx->P * SAD_K;
-    const uint32_t *plane1 = plane0 + (size_t)ctx->P * 4;
-    cudaError_t e = cudaMemcpy2DAsync(dst, 32, plane0, 16, 16, (size_t)ctx->P, cudaMemcpyDefault, st);
-    if (e == cudaSuccess) e = cudaMemcpy2DAsync(dst + 4, 32, plane1, 16, 16, (size_t)ctx->P, cudaMemcpyDefault, st);
+    const uint32_t *plane0 = ctx->buf.table + (size_t)c.cur * ctx->PT * SAD_K;
+    const uint32_t *plane1 = plane0 + (size_t)ctx->PT * 4;
+    cudaError_t e = cudaMemcpy2DAsync(dst, 32, plane0, 16, 16, (size_t)ctx->PT, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaMemcpy2DAsync(dst + 4, 32, plane1, 16, 16, (size_t)ctx->PT, cudaMemcpyDefault, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     return cuda_status(ctx, e, "get table");
 }
@@ -362,10 +400,10 @@ int sad_set_table(sad_ctx *ctx, const uint32_t *src, sad_stream_t stream) {
     sad::Counters c;
     r = read_counters(ctx, &c, st);
     if (r) return r;
-    uint32_t *plane0 = ctx->buf.table + (size_t)c.cur * ctx->P * SAD_K;
-    uint32_t *plane1 = plane0 + (size_t)ctx->P * 4;
-    cudaError_t e = cudaMemcpy2DAsync(plane0, 16, src, 32, 16, (size_t)ctx->P, cudaMemcpyDefault, st);
-    if (e == cudaSuccess) e = cudaMemcpy2DAsync(plane1, 16, src + 4, 32, 16, (size_t)ctx->P, cudaMemcpyDefault, st);
+    uint32_t *plane0 = ctx->buf.table + (size_t)c.cur * ctx->PT * SAD_K;
+    uint32_t *plane1 = plane0 + (size_t)ctx->PT * 4;
+    cudaError_t e = cudaMemcpy2DAsync(plane0, 16, src, 32, 16, (size_t)ctx->PT, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaMemcpy2DAsync(plane1, 16, src + 4, 32, 16, (size_t)ctx->PT, cudaMemcpyDefault, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     return cuda_status(ctx, e, "set table");
 }

@@ -23,6 +23,17 @@ constexpr int TILE_Y = 8;
 constexpr int TILE_THREADS = TILE_X * TILE_Y;
 constexpr int SITE_THREADS = 256;
 
+// Where a pixel's candidate list lives: the list of its cell on a grid of
+// cell x cell pixel cells (summary B.3, "Candidate field"; cell = 1 is the
+// pixel grid).  PT is the number of lists, the stride of a table plane.
+struct TableGrid {
+    int cell, GW;
+    size_t PT;
+    __device__ __forceinline__ size_t cell_of(int i, int j, size_t p) const {
+        return cell == 1 ? p : (size_t)(j / cell) * GW + (size_t)(i / cell);
+    }
+};
+
 __device__ __forceinline__ Counters *counters(void *ws) { return reinterpret_cast<Counters *>(ws); }
 __device__ __forceinline__ double *loss_partials(void *ws) {
     return reinterpret_cast<double *>(reinterpret_cast<char *>(ws) + COUNTERS_BYTES);
@@ -90,7 +101,7 @@ __global__ void mark_inactive_kernel(float *prm, int N, int from) {
 // a8: exact top-8 by brute force; records staged through shared memory.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(SITE_THREADS) topk_exact_kernel(const float4 *__restrict__ rec, int N, int H,
-                                                                  int W, const int64_t *__restrict__ pix,
+                                                                  int W, float cs, const int64_t *__restrict__ pix,
                                                                   int64_t n_pix, uint32_t *__restrict__ out) {
     __shared__ float sx[SITE_THREADS], sy[SITE_THREADS], sA[SITE_THREADS], sB[SITE_THREADS],
         sC[SITE_THREADS], sb[SITE_THREADS];
@@ -99,8 +110,8 @@ __global__ void __launch_bounds__(SITE_THREADS) topk_exact_kernel(const float4 *
     int64_t p = -1;
     if (q < n_pix) p = pix ? pix[q] : q;
     const bool live = p >= 0 && p < P;
-    const float fx = live ? (float)(int)(p % W) + 0.5f : 0.0f;
-    const float fy = live ? (float)(int)(p / W) + 0.5f : 0.0f;
+    const float fx = live ? ((float)(int)(p % W) + 0.5f) * cs : 0.0f;
+    const float fy = live ? ((float)(int)(p / W) + 0.5f) * cs : 0.0f;
     Top8 t;
     t.clear();
     for (int base = 0; base < N; base += SITE_THREADS) {
@@ -139,7 +150,8 @@ __global__ void __launch_bounds__(SITE_THREADS) topk_exact_kernel(const float4 *
 
 // ---------------------------------------------------------------------------
 // a9 seed pass: clear the current table, scatter each active site's id into
-// slot 0 of the pixel containing it (atomicMin: smallest id wins).
+// slot 0 of the pixel (candidate-grid cell) containing it (atomicMin:
+// smallest id wins).
 // ---------------------------------------------------------------------------
 __global__ void seed_clear_kernel(uint32_t *__restrict__ table, long long P, const Counters *__restrict__ c) {
     uint4 *t = reinterpret_cast<uint4 *>(table + (size_t)c->cur * (size_t)P * K);
@@ -149,16 +161,16 @@ __global__ void seed_clear_kernel(uint32_t *__restrict__ table, long long P, con
         t[q] = e;
 }
 
-__global__ void seed_scatter_kernel(const float *__restrict__ prm, int N, int H, int W, uint32_t *__restrict__ table,
-                                    const Counters *__restrict__ c) {
+__global__ void seed_scatter_kernel(const float *__restrict__ prm, int N, int H, int W, int cell, int GW,
+                                    long long PT, uint32_t *__restrict__ table, const Counters *__restrict__ c) {
     const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
     if (i >= N) return;
     const float px = prm[PX * (size_t)N + i], py = prm[PY * (size_t)N + i];
     if (!(px >= 0.0f) || !(py >= 0.0f)) return;
     const float fi = floorf(px), fj = floorf(py);
     if (fi >= (float)W || fj >= (float)H) return;
-    const long long p = (long long)fj * W + (long long)fi;
-    uint32_t *plane0 = table + (size_t)c->cur * (size_t)H * W * K;
+    const long long p = (long long)((int)fj / cell) * GW + (long long)((int)fi / cell);
+    uint32_t *plane0 = table + (size_t)c->cur * (size_t)PT * K;
     atomicMin(plane0 + (size_t)p * 4, (uint32_t)i);
 }
 
@@ -189,8 +201,10 @@ __device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], 
     }
 }
 
+// H x W is the candidate grid; a cell is scored at its centre, (i + 0.5) cs
+// (cs = 1: the pixel grid)
 __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *__restrict__ rec, uint32_t *table,
-                                                                 int H, int W, int N, int jump, int G,
+                                                                 int H, int W, float cs, int N, int jump, int G,
                                                                  Counters *c) {
     const uint32_t cur = c->cur, pass = c->pass_counter, seed = c->seed;
     const size_t P = (size_t)H * W;
@@ -202,7 +216,7 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
     const int j = blockIdx.y * TILE_Y + threadIdx.y;
     if (i < W && j < H) {
         const size_t p = (size_t)j * W + i;
-        const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
+        const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
         Top8 t;
         t.clear();
         // own list, then the neighbours at (-k, 0), (+k, 0), (0, -k), (0, +k)
@@ -255,7 +269,7 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
 // distinct candidates of the lists at (i + a k, j + b k), a, b in {-1, 0, 1},
 // go to slots 0-3; slots 4-7 are emptied.
 __global__ void __launch_bounds__(TILE_THREADS) jfa3x3_kernel(const float4 *__restrict__ rec, uint32_t *table,
-                                                              int H, int W, int N, int jump, Counters *c) {
+                                                              int H, int W, float cs, int N, int jump, Counters *c) {
     const uint32_t cur = c->cur, pass = c->pass_counter;
     const size_t P = (size_t)H * W;
     const uint4 *in0 = reinterpret_cast<const uint4 *>(table + cur * P * K);
@@ -266,7 +280,7 @@ __global__ void __launch_bounds__(TILE_THREADS) jfa3x3_kernel(const float4 *__re
     const int j = blockIdx.y * TILE_Y + threadIdx.y;
     if (i < W && j < H) {
         const size_t p = (size_t)j * W + i;
-        const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
+        const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
         Top8 t;
         t.clear();
 #pragma unroll 1
@@ -353,18 +367,20 @@ __device__ __forceinline__ int pixel_softmax(const uint4 a, const uint4 b, const
 
 __global__ void __launch_bounds__(TILE_THREADS) render_kernel(const float4 *__restrict__ rec,
                                                               const uint32_t *__restrict__ table, int H, int W,
-                                                              int N, float *__restrict__ image, Counters *c) {
+                                                              TableGrid tg, int N, float *__restrict__ image,
+                                                              Counters *c) {
     const size_t P = (size_t)H * W;
-    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * P * K);
-    const uint4 *in1 = in0 + P;
+    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * tg.PT * K);
+    const uint4 *in1 = in0 + tg.PT;
     const int i = blockIdx.x * TILE_X + threadIdx.x;
     const int j = blockIdx.y * TILE_Y + threadIdx.y;
     unsigned dropped = 0;
     bool empty = false;
     if (i < W && j < H) {
         const size_t p = (size_t)j * W + i;
+        const size_t pt = tg.cell_of(i, j, p);
         PixelSoftmax s;
-        const int nv = pixel_softmax(in0[p], in1[p], rec, (uint32_t)N, (float)i + 0.5f, (float)j + 0.5f, s,
+        const int nv = pixel_softmax(in0[pt], in1[pt], rec, (uint32_t)N, (float)i + 0.5f, (float)j + 0.5f, s,
                                      dropped);
         empty = nv == 0;
         image[p] = s.cr;
@@ -409,7 +425,7 @@ template <bool STATS>
 __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *__restrict__ rec,
                                                                   const uint32_t *__restrict__ table,
                                                                   const float *__restrict__ target, int H, int W,
-                                                                  int N, float *__restrict__ image,
+                                                                  TableGrid tg, int N, float *__restrict__ image,
                                                                   float *__restrict__ grads,
                                                                   float *__restrict__ stats, void *ws) {
     constexpr int NV = STATS ? NPARAM + NSTAT : NPARAM;
@@ -427,8 +443,8 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
     __syncthreads();
 
     const size_t P = (size_t)H * W;
-    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * P * K);
-    const uint4 *in1 = in0 + P;
+    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * tg.PT * K);
+    const uint4 *in1 = in0 + tg.PT;
     const int i = blockIdx.x * TILE_X + threadIdx.x;
     const int j = blockIdx.y * TILE_Y + threadIdx.y;
     const bool inside = i < W && j < H;
@@ -444,7 +460,8 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
     float er = 0.0f, eg = 0.0f, eb = 0.0f;
     if (inside) {
         const size_t p = (size_t)j * W + i;
-        const int nv = pixel_softmax(in0[p], in1[p], rec, (uint32_t)N, fx, fy, s, dropped);
+        const size_t pt = tg.cell_of(i, j, p);
+        const int nv = pixel_softmax(in0[pt], in1[pt], rec, (uint32_t)N, fx, fy, s, dropped);
         empty = nv == 0;
         er = s.cr - target[p];
         eg = s.cg - target[P + p];
@@ -686,7 +703,8 @@ __global__ void __launch_bounds__(SITE_THREADS) adam_kernel(float *__restrict__ 
 __global__ void __launch_bounds__(SITE_THREADS) tau_diffuse_kernel(const float *__restrict__ prm,
                                                                    const uint32_t *__restrict__ table,
                                                                    const float *__restrict__ grads, int H, int W,
-                                                                   int N, float lambda, float *__restrict__ out,
+                                                                   TableGrid tg, int N, float lambda,
+                                                                   float *__restrict__ out,
                                                                    const Counters *__restrict__ c) {
     const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
     if (i >= N) return;
@@ -698,10 +716,9 @@ __global__ void __launch_bounds__(SITE_THREADS) tau_diffuse_kernel(const float *
     if (px >= 0.0f && py >= 0.0f) {
         const float fi = floorf(px), fj = floorf(py);
         if (fi < (float)W && fj < (float)H) {
-            const size_t P = (size_t)H * W;
-            const size_t p = (size_t)fj * W + (size_t)fi;
-            const uint4 *t0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * P * K);
-            const uint4 a = t0[p], b = t0[P + p];
+            const size_t p = tg.cell_of((int)fi, (int)fj, (size_t)fj * W + (size_t)fi);
+            const uint4 *t0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * tg.PT * K);
+            const uint4 a = t0[p], b = t0[tg.PT + p];
             const uint32_t ids[K] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
             double sum = 0.0;
             int cnt = 0;
@@ -722,6 +739,7 @@ __global__ void __launch_bounds__(SITE_THREADS) tau_diffuse_kernel(const float *
 inline dim3 tile_grid(int H, int W) { return dim3((W + TILE_X - 1) / TILE_X, (H + TILE_Y - 1) / TILE_Y); }
 inline unsigned site_blocks(long long n) { return (unsigned)((n + SITE_THREADS - 1) / SITE_THREADS); }
 inline Counters *host_counters(const Dev &d) { return reinterpret_cast<Counters *>(d.ws); }
+inline TableGrid grid_of(const Dev &d) { return TableGrid{d.cell, d.GW, (size_t)d.PT}; }
 
 }  // namespace
 
@@ -740,8 +758,8 @@ size_t workspace_bytes(int H, int W, int N) {
 cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st) {
     float *scratch = reinterpret_cast<float *>(reinterpret_cast<char *>(d.ws) + densify_offset(d.H, d.W) + 256 +
                                                2 * sizeof(uint32_t) * (size_t)d.N);
-    tau_diffuse_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.table, d.grads, d.H, d.W, d.N, lambda,
-                                                                  scratch, host_counters(d));
+    tau_diffuse_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.table, d.grads, d.H, d.W, grid_of(d),
+                                                                  d.N, lambda, scratch, host_counters(d));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return cudaMemcpyAsync(d.grads + (size_t)PLT * d.N, scratch, sizeof(float) * (size_t)d.N,
@@ -767,46 +785,52 @@ cudaError_t launch_records(const Dev &d, cudaStream_t st) {
 
 cudaError_t launch_topk_exact(const Dev &d, const int64_t *pix, int64_t n, uint32_t *out, cudaStream_t st) {
     if (n <= 0) return cudaSuccess;
-    topk_exact_kernel<<<site_blocks(n), SITE_THREADS, 0, st>>>(d.records, d.N, d.H, d.W, pix, n, out);
+    topk_exact_kernel<<<site_blocks(n), SITE_THREADS, 0, st>>>(d.records, d.N, d.GH, d.GW, (float)d.cell, pix, n,
+                                                              out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_clear_table(const Dev &d, cudaStream_t st) {
+    seed_clear_kernel<<<148 * 8, 256, 0, st>>>(d.table, d.PT, host_counters(d));
     return cudaGetLastError();
 }
 
 cudaError_t launch_seed(const Dev &d, cudaStream_t st) {
-    seed_clear_kernel<<<148 * 8, 256, 0, st>>>(d.table, d.P, host_counters(d));
+    seed_clear_kernel<<<148 * 8, 256, 0, st>>>(d.table, d.PT, host_counters(d));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    seed_scatter_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.N, d.H, d.W, d.table,
-                                                                 host_counters(d));
+    seed_scatter_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.N, d.H, d.W, d.cell, d.GW, d.PT,
+                                                                 d.table, host_counters(d));
     return cudaGetLastError();
 }
 
 cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st) {
-    propagate_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.H, d.W, d.N,
-                                                                           jump, G, host_counters(d));
+    propagate_kernel<<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
+        d.records, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d));
     return cudaGetLastError();
 }
 
 cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st) {
-    jfa3x3_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.H, d.W, d.N, jump,
-                                                                        host_counters(d));
+    jfa3x3_kernel<<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.GH, d.GW,
+                                                                          (float)d.cell, d.N, jump, host_counters(d));
     return cudaGetLastError();
 }
 
 cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st) {
-    render_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.H, d.W, d.N, image,
-                                                                        host_counters(d));
+    render_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.H, d.W, grid_of(d),
+                                                                        d.N, image, host_counters(d));
     return cudaGetLastError();
 }
 
 cudaError_t launch_render_backward(const Dev &d, cudaStream_t st) {
     render_bwd_kernel<false><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.target, d.H, d.W, d.N, d.image, d.grads, nullptr, d.ws);
+        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, nullptr, d.ws);
     return cudaGetLastError();
 }
 
 cudaError_t launch_render_backward_stats(const Dev &d, cudaStream_t st) {
     render_bwd_kernel<true><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.target, d.H, d.W, d.N, d.image, d.grads, d.stats, d.ws);
+        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, d.stats, d.ws);
     return cudaGetLastError();
 }
 

@@ -10,9 +10,11 @@ namespace sad {
 struct Dev {
     int H, W, N;
     long long P;
+    int cell, GH, GW;  // candidate grid: ceil(H/cell) x ceil(W/cell) lists
+    long long PT;      // GH * GW
     float *params, *grads, *adam_m, *adam_v;
     float4 *records;
-    uint32_t *table;  // [2][2][P][4]
+    uint32_t *table;  // [2][2][PT][4]
     float *target, *image;
     float *stats;  // [6][N] budget-control statistics (optional)
     const uint8_t *frozen;  // [N] sites Adam leaves untouched (optional)
@@ -37,6 +39,7 @@ cudaError_t launch_mark_inactive(const Dev &d, int from, cudaStream_t st);
 cudaError_t launch_records(const Dev &d, cudaStream_t st);
 cudaError_t launch_topk_exact(const Dev &d, const int64_t *pix, int64_t n, uint32_t *out, cudaStream_t st);
 cudaError_t launch_seed(const Dev &d, cudaStream_t st);
+cudaError_t launch_clear_table(const Dev &d, cudaStream_t st);
 cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st);
 cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st);
 cudaError_t launch_render_backward(const Dev &d, cudaStream_t st);

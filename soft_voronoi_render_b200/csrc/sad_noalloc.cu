@@ -62,6 +62,10 @@ extern "C" int sad_backward_noalloc(int H, int W, int N_cap, const float *record
     d.W = W;
     d.N = N_cap;
     d.P = (long long)H * W;
+    d.cell = 1;  // lists on the pixel grid
+    d.GH = H;
+    d.GW = W;
+    d.PT = d.P;
     d.records = reinterpret_cast<float4 *>(const_cast<float *>(records));
     d.table = const_cast<uint32_t *>(table);
     d.target = const_cast<float *>(target);

@@ -165,3 +165,49 @@ def test_infrequent_updates_schedule(torch_cuda):
     assert s.stats()["adam_step"] == 12
     psnr = lambda L: 10 * math.log10(3.0 / L)
     assert abs(psnr(s.loss()) - psnr(L_orc)) <= 0.2, (s.loss(), L_orc)
+
+
+@pytest.mark.parametrize("H,W,N,cell", [(96, 128, 800, 2), (37, 70, 400, 3), (64, 64, 300, 4), (9, 33, 40, 8)])
+def test_candidate_grid_parity(torch_cuda, H, W, N, cell):
+    """Lists on a ceil(H/s) x ceil(W/s) grid scored at the cell centres
+    (summary B.3): refresh, exact top-K, the JFA prepass and a fitting pass
+    bit-exact on the grid; render, loss and gradients with every pixel using
+    its cell's list; tau diffusion on the site's cell list."""
+    tgt, prm, _ = synth.make_workload("c1", seed=7, H=H, W=W, N=N)
+    prm = prm.copy()
+    prm[0, 4] = -1.0
+    G = 2
+    s = _ctx(H, W, N, prm, tgt, seed=31)
+    s.set_candidate_grid(cell)
+    GH, GW = oracle.grid_dims(H, W, cell)
+    assert s.get_table().shape == (GH * GW, 8) and np.all(s.get_table() == SENT)
+    rec = oracle.records(H, W, prm)
+    s.refresh(G)
+    t0, npass = oracle.refresh(H, W, prm, G, seed=31, cell=cell)
+    np.testing.assert_array_equal(s.get_table(), t0)
+    ex = s.topk_exact().cpu().numpy().view(np.uint32)
+    np.testing.assert_array_equal(ex, oracle.topk_exact(H, W, rec, cell=cell))
+    # one fitting pass: propagation on the grid, backward per pixel
+    s.fit_pass(G)
+    t1 = oracle.propagate(H, W, rec, t0, 1, G, seed=31, pass_index=npass, cell=cell)
+    np.testing.assert_array_equal(s.get_table(), t1)
+    L, g, img = oracle.loss_backward(H, W, prm, oracle.expand_table(H, W, t1, cell), tgt, want_image=True)
+    assert abs(s.loss() - L) <= LOSS_RTOL * L
+    assert np.abs(s.image.cpu().numpy() - img).max() <= RENDER_ATOL
+    _assert_grads(s.grads.cpu().numpy(), g, "grid fit pass")
+    # the cached pass on the grid and tau diffusion on the site's cell list
+    s.grads.zero_()
+    s.fit_pass_cached()
+    _assert_grads(s.grads.cpu().numpy(), g, "grid cached pass")
+    gr = synth.random_gradients(N, 8)
+    s.grads.copy_(torch_cuda.from_numpy(gr))
+    s.tau_diffuse(0.5)
+    ref = oracle.tau_diffuse(H, W, prm, oracle.expand_table(H, W, t1, cell), gr.astype(np.float64), 0.5)
+    np.testing.assert_allclose(s.grads.cpu().numpy().astype(np.float64), ref, rtol=1e-6, atol=1e-12)
+    # the prepass on the grid
+    s.jfa_prepass()
+    np.testing.assert_array_equal(s.get_table(), oracle.jfa_prepass(H, W, prm, cell=cell))
+    # back to the pixel grid
+    s.set_candidate_grid(1)
+    s.refresh(G)
+    assert s.get_table().shape == (H * W, 8)
