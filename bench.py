@@ -63,6 +63,13 @@ def parse():
                          "4096x4096, N=524,288; c5: end-to-end 768x512 fit with densify/prune (secondary "
                          "measurements)")
     ap.add_argument("--oracle-fit", action="store_true", help="c5: also run the CPU oracle's fit (minutes)")
+    ap.add_argument("--cell", type=int, default=1,
+                    help="c4/c5: candidate lists on a grid of cell x cell pixel cells (1: per pixel)")
+    ap.add_argument("--refresh", default="jump", choices=["jump", "jfa"],
+                    help="c4: jump-flooding refresh (seed + propagation passes) or the 3x3 JFA prepass")
+    ap.add_argument("--update-every", type=int, default=1,
+                    help="c5: propagate the candidate lists every U iterations (cached lists between)")
+    ap.add_argument("--passes-per-update", type=int, default=1, help="c5: propagation passes per update")
     return ap.parse_args()
 
 
@@ -393,7 +400,10 @@ def run_ours(args):
 
 def run_refresh(args):
     """Full candidate refresh from scratch (seed pass + jumps 2048..1 with
-    G = 4) followed by a render, at 4096 x 4096 with N = 524,288."""
+    G = 4, or with --refresh jfa the seed pass + 3x3 flood passes) followed
+    by a render, at 4096 x 4096 with N = 524,288; with --cell the lists live
+    on the downscaled candidate grid.  Also reports how often slot 0 holds
+    the exact owner, on 4096 sampled cells (exact top-K on the device)."""
     import torch
     import synth
     from soft_voronoi_render_b200 import Sad, _lib
@@ -403,17 +413,27 @@ def run_refresh(args):
     s = Sad(H, W, N, seed=1)
     s.set_sites(prm)
     s.set_target(tgt)
+    if args.cell != 1:
+        s.set_candidate_grid(args.cell)
+    GH, GW = (H + args.cell - 1) // args.cell, (W + args.cell - 1) // args.cell
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
+
+    def refresh():
+        if args.refresh == "jfa":
+            _lib.sad_jfa_prepass(s.ctx, sp)
+        else:
+            _lib.sad_refresh(s.ctx, G, sp)
+
     for _ in range(max(args.warmup, 3)):
-        _lib.sad_refresh(s.ctx, G, sp)
+        refresh()
         _lib.sad_render(s.ctx, None, sp)
     torch.cuda.synchronize()
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     for k in range(K):
         ev[k][0].record(stream)
-        _lib.sad_refresh(s.ctx, G, sp)
+        refresh()
         ev[k][1].record(stream)
         _lib.sad_render(s.ctx, None, sp)
         ev[k][2].record(stream)
@@ -421,13 +441,28 @@ def run_refresh(args):
     t_ref = sum(e[0].elapsed_time(e[1]) for e in ev) / K
     t_ren = sum(e[1].elapsed_time(e[2]) for e in ev) / K
     hbm, peak_kind = measured_peaks()
-    passes = 12
-    alg = passes * 64 * P + 32 * P + 44 * P  # passes: list read+write; clear; render list+image
-    line = {"metric": "ms per full candidate refresh (seed + 12 passes, G=4) + render, 4096x4096 N=524,288",
+    PT = GH * GW
+    m = max(GH, GW)
+    if args.refresh == "jfa":
+        passes = max(1, (m - 1).bit_length())
+    else:
+        passes = max(0, m.bit_length() - 1)
+    # passes: list read + write; clear; render: the cell lists + image
+    alg = passes * 64 * PT + 32 * PT + 32 * PT + 12 * P
+    # slot 0 against the exact owner on sampled cells
+    tab = s.get_table()
+    cells = np.random.default_rng(1).choice(PT, size=min(4096, PT), replace=False)
+    ex = s.topk_exact(cells).cpu().numpy().view(np.uint32)
+    owner_right = float(np.mean(tab[cells, 0] == ex[:, 0]))
+    what = "3x3 JFA prepass (seed + flood passes)" if args.refresh == "jfa" else f"seed + {passes} passes, G={G}"
+    line = {"metric": f"ms per full candidate refresh ({what}) + render, 4096x4096 N=524,288"
+                      + (f", {args.cell}x{args.cell} candidate cells" if args.cell != 1 else ""),
             "value": t_ref + t_ren, "unit": "ms", "higher_is_better": False, "n_gpus": 1, "steps": K,
             "warmup": max(args.warmup, 3), "refresh_ms": t_ref, "render_ms": t_ren,
-            "mpix_per_s_per_pass": P * passes / (t_ref * 1e-3) / 1e6, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": f"c4: {wl.description}", "H": H, "W": W, "N": N, "G": G},
+            "mpix_per_s_per_pass": PT * passes / (t_ref * 1e-3) / 1e6 if passes else None,
+            "owner_right_sampled": owner_right, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"c4: {wl.description}", "H": H, "W": W, "N": N, "G": G, "cell": args.cell,
+                       "refresh": args.refresh},
             "hbm_roof_frac": alg / ((t_ref + t_ren) * 1e-3) / 1e9 / hbm, "peak_kind": peak_kind,
             "device_stats": s.stats()}
     print(json.dumps(line), flush=True)
@@ -446,14 +481,16 @@ def run_fit(args):
 
     tgt, prm, wl = synth.make_workload("c5", seed=1)
     H, W, N_cap = wl.H, wl.W, 50_000
-    sched = fit.Schedule()
+    sched = fit.Schedule(update_every=args.update_every, passes_per_update=args.passes_per_update)
     s = Sad(H, W, N_cap, seed=1)
     s.set_sites(prm)
     s.set_target(tgt)
+    if args.cell != 1:
+        s.set_candidate_grid(args.cell)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    fit.run(s, sched)
+    info = fit.run(s, sched)
     e1.record()
     torch.cuda.synchronize()
     t_fit = e0.elapsed_time(e1) * 1e-3
@@ -462,17 +499,22 @@ def run_fit(args):
     line = {"metric": "time to fit 768x512 (2000 iterations, N 10,000 -> 50,000 by densify/prune) and final PSNR",
             "value": t_fit, "unit": "s", "higher_is_better": False, "n_gpus": 1,
             "psnr_db": 10 * math.log10(3.0 / L), "final_loss": L, "n_active_final": n_final,
-            "iterations": sched.iterations, "events": len(sched.events), "dtype": "f32", "data": "synthetic",
+            "iterations": sched.iterations, "events": len(sched.events), "schedule_run": info,
+            "dtype": "f32", "data": "synthetic",
             "config": {"workload": f"c5: {wl.description}", "H": H, "W": W, "N_start": prm.shape[1],
-                       "N_cap": N_cap, "G": sched.G}}
+                       "N_cap": N_cap, "G": sched.G, "cell": args.cell, "update_every": sched.update_every,
+                       "passes_per_update": sched.passes_per_update}}
     if args.oracle_fit:
         import oracle
         lr = {k[3:] if k.startswith("lr_") else k: float(np.float32(v)) for k, v in sched.lr.items()}
         lr = {"pos": lr["pos"], "log_tau": lr["log_tau"], "r": lr["r"], "color": lr["color"],
               "theta": lr["theta"], "a": lr["a"]}
         t0 = time.perf_counter()
+        if args.cell != 1:
+            raise SystemExit("--oracle-fit runs the oracle's schedule on the pixel grid only")
         P, L_o, _ = oracle.fit(H, W, prm, tgt, N_cap, sched.iterations, sched.events, sched.grow, sched.prune_frac,
-                               lr, sched.G, 1)
+                               lr, sched.G, 1, update_every=sched.update_every,
+                               passes_per_update=sched.passes_per_update)
         line["oracle"] = {"time_s": time.perf_counter() - t0, "psnr_db": 10 * math.log10(3.0 / L_o),
                           "final_loss": L_o, "n_active_final": int((P[0] >= 0).sum()),
                           "cores": oracle.num_threads()}

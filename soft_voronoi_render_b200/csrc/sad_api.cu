@@ -168,6 +168,9 @@ int sad_bind(sad_ctx *ctx, const sad_buffers *b) {
     d.stats = b->stats;
     d.frozen = b->frozen;
     d.ws = b->workspace;
+    // best effort: the launchers set the attributes themselves when this
+    // fails (binding needs no device, only valid pointers)
+    if (sad::prepare_fused() != cudaSuccess) (void)cudaGetLastError();
     ctx->bound = true;
     ctx->err[0] = 0;
     return SAD_OK;

@@ -711,9 +711,10 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     }
 }
 
+// the tile state exceeds the 48 KB default: opt in once per device (done
+// when buffers are bound, so that a stream capture sees launches only)
 template <int FY, bool PROP>
-cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
-    // the tile state exceeds the 48 KB default: opt in once per device
+cudaError_t ensure_smem_attr() {
     static bool attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -724,6 +725,13 @@ cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
+    return cudaSuccess;
+}
+
+template <int FY, bool PROP>
+cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
+    cudaError_t e = ensure_smem_attr<FY, PROP>();
+    if (e != cudaSuccess) return e;
     const dim3 grid((d.W + FX - 1) / FX, (d.H + FY - 1) / FY);
     fit_tile_kernel<FY, PROP><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY>), st>>>(d.records, d.table, d.target, d.H, d.W,
                                                                            d.N, G, d.image, d.grads, d.ws);
@@ -731,6 +739,14 @@ cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
 }
 
 }  // namespace
+
+cudaError_t prepare_fused() {
+    cudaError_t e = ensure_smem_attr<8, true>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, true>();
+    if (e == cudaSuccess) e = ensure_smem_attr<8, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, false>();
+    return e;
+}
 
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st) {
     // taller tiles amortise the halo and the per-tile work, but hold more

@@ -50,5 +50,6 @@ cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st);
 cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st);
 cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st);
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st);
+cudaError_t prepare_fused();
 
 }  // namespace sad

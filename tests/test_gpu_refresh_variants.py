@@ -211,3 +211,29 @@ def test_candidate_grid_parity(torch_cuda, H, W, N, cell):
     s.set_candidate_grid(1)
     s.refresh(G)
     assert s.get_table().shape == (H * W, 8)
+
+
+@pytest.mark.parametrize("U,events", [(4, ()), (1, (30,))])
+def test_fit_graph_replay_matches_eager(torch_cuda, U, events):
+    """fit.run replaying captured CUDA graphs of 16 iterations advances the
+    device counters exactly as the eager schedule does and reaches the same
+    loss (float32 atomics order the sums differently between runs, so the
+    loss is compared in PSNR)."""
+    import math
+    from soft_voronoi_render_b200 import fit
+    H, W, N, N_cap = 64, 96, 600, 900
+    tgt = synth.make_image(H, W, 8, 0, 43)
+    prm = synth.gradient_sites(tgt, N, 43)
+    out = {}
+    for graphs in (True, False):
+        s = _ctx(H, W, N_cap, prm, tgt, seed=6)
+        sched = fit.Schedule(iterations=60, G=2, events=events, grow=100, prune_frac=0.01, update_every=U)
+        info = fit.run(s, sched, graphs=graphs)
+        st = s.stats()
+        out[graphs] = (info, st["pass_counter"], st["adam_step"], st["n_active"], s.loss())
+    (gi, gp, ga, gn, gl), (ei, ep, ea, en, el) = out[True], out[False]
+    assert gi["graph_replays"] >= 2 and ei["graph_replays"] == 0
+    assert gi["eager_iterations"] + 16 * gi["graph_replays"] + len(events) == 60
+    assert (gp, ga, gn) == (ep, ea, en) and ga == 60
+    psnr = lambda L: 10 * math.log10(3.0 / L)
+    assert abs(psnr(gl) - psnr(el)) <= 0.2, (gl, el)
