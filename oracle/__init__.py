@@ -65,6 +65,9 @@ def lib():
         L.orc_adam_frozen.argtypes = [c_int, c_int, c_int, vp, vp, vp, vp, vp, c_dbl, c_dbl, c_dbl, c_int, vp]
         L.orc_tau_diffuse.argtypes = [c_int, c_int, c_int, vp, vp, vp, c_dbl]
         L.orc_jfa3x3.argtypes = [c_int, c_int, c_int, vp, vp, vp, c_int]
+        L.orc_pack_ranges.argtypes = [c_int, vp, vp]
+        L.orc_pack_sites.argtypes = [c_int, c_int, c_int, vp, vp, vp]
+        L.orc_unpack_sites.argtypes = [c_int, c_int, c_int, vp, vp, vp]
         L.orc_num_threads.restype = c_int
         L.orc_set_threads.argtypes = [c_int]
         _lib = L
@@ -384,3 +387,34 @@ def jfa_prepass(H: int, W: int, params, cell: int = 1):
     for k in flood_schedule(*grid_dims(H, W, cell)):
         t = jfa3x3(H, W, rec, t, k, cell)
     return t
+
+
+PACK_FIELDS = {"x": (0, 18), "y": (18, 18), "cr": (36, 10), "cg": (46, 10), "cb": (56, 10), "ln_tau": (66, 16),
+               "r": (82, 14), "theta": (96, 14), "a": (110, 14), "active": (127, 1)}
+
+
+def pack_ranges(params) -> np.ndarray:
+    """Per-image (lo, hi) of ln tau, r and a over the active sites, as
+    float32 (lo_lt, lo_r, lo_a, hi_lt, hi_r, hi_a)."""
+    params = _f32(params)
+    out = np.empty(6, dtype=np.float32)
+    lib().orc_pack_ranges(params.shape[1], _p(params), _p(out))
+    return out
+
+
+def pack_sites(H: int, W: int, params, lohi=None):
+    """16-byte evaluation records (N, 4) uint32 and the ranges they use."""
+    params = _f32(params)
+    lohi = pack_ranges(params) if lohi is None else np.ascontiguousarray(lohi, dtype=np.float32)
+    out = np.empty((params.shape[1], 4), dtype=np.uint32)
+    lib().orc_pack_sites(H, W, params.shape[1], _p(params), _p(lohi), _p(out))
+    return out, lohi
+
+
+def unpack_sites(H: int, W: int, packed, lohi) -> np.ndarray:
+    """Decode 16-byte records to float32 parameters (9, N)."""
+    packed = _u32(packed).reshape(-1, 4)
+    lohi = np.ascontiguousarray(lohi, dtype=np.float32)
+    out = np.empty((9, packed.shape[0]), dtype=np.float32)
+    lib().orc_unpack_sites(H, W, packed.shape[0], _p(packed), _p(lohi), _p(out))
+    return out

@@ -940,3 +940,148 @@ void orc_jfa3x3(int H, int W, int N, const float *rec32, const uint32_t *tin, ui
 {
     orc_jfa3x3_cell(H, W, 1, N, rec32, tin, tout, jump);
 }
+
+/* ------------------------------------------------------------------------ */
+/* 16-byte evaluation record ([P1] B.2, "Packed storage for evaluation")     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Four 32-bit words per site, one little-endian 128-bit field string, bit
+ * offset (width): x 0 (18), y 18 (18), cr 36 (10), cg 46 (10), cb 56 (10),
+ * ln tau 66 (16), r 82 (14), theta 96 (14), a 110 (14), bits 124-126 zero,
+ * bit 127 = active.  An inactive site packs to four zero words.
+ *   x, y:   cell index floor(x / W 2^18) (clamped), decoded at the cell centre
+ *           (q + 1/2) W / 2^18 (same with H for y);
+ *   colour: round(clamp(c, 0, 1) 1023), decoded q / 1023;
+ *   ln tau, r, a: round((v - lo) / (hi - lo) (2^b - 1)) with the per-image
+ *           lo, hi of the active sites ([P1] B.2: per-image min/scale for
+ *           ln tau and radius; the same for a), decoded lo + q (hi - lo) /
+ *           (2^b - 1);
+ *   theta:  the axis angle theta mod pi (G depends on the axis only),
+ *           round(theta_m / pi 2^14) mod 2^14, decoded q pi / 2^14.
+ * Rounding is floor(t + 1/2) in double; every decoded value is computed in
+ * double and rounded once to float32.
+ */
+enum { PK_X = 0, PK_Y = 18, PK_CR = 36, PK_CG = 46, PK_CB = 56, PK_LT = 66, PK_R = 82, PK_TH = 96, PK_A = 110,
+       PK_ACTIVE = 127 };
+enum { PKW_XY = 18, PKW_C = 10, PKW_LT = 16, PKW_R = 14, PKW_TH = 14, PKW_A = 14 };
+
+static void pk_put(uint32_t w[4], int off, int n, uint32_t v)
+{
+    for (int b = 0; b < n; ++b)
+        if ((v >> b) & 1u) w[(off + b) >> 5] |= 1u << ((off + b) & 31);
+}
+
+static uint32_t pk_get(const uint32_t w[4], int off, int n)
+{
+    uint32_t v = 0;
+    for (int b = 0; b < n; ++b) v |= ((w[(off + b) >> 5] >> ((off + b) & 31)) & 1u) << b;
+    return v;
+}
+
+static uint32_t pk_round(double t, double top)
+{
+    if (t != t) return 0;
+    t = floor(t + 0.5);
+    if (t < 0.0) t = 0.0;
+    if (t > top) t = top;
+    return (uint32_t)t;
+}
+
+static const double PK_PI = 3.14159265358979323846;
+
+/* cell index floor(t), clamped to [0, cells - 1] */
+static uint32_t pk_cell(double t, double cells)
+{
+    if (t != t) return 0;
+    t = floor(t);
+    if (t < 0.0) t = 0.0;
+    if (t > cells - 1.0) t = cells - 1.0;
+    return (uint32_t)t;
+}
+
+static uint32_t pk_range_q(float v, float lo, float hi, int bits)
+{
+    const double top = (double)((1u << bits) - 1u);
+    if (!((double)hi > (double)lo)) return 0;
+    return pk_round(((double)v - (double)lo) / ((double)hi - (double)lo) * top, top);
+}
+
+static float pk_range_v(uint32_t q, float lo, float hi, int bits)
+{
+    const double top = (double)((1u << bits) - 1u);
+    return (float)((double)lo + (double)q * (((double)hi - (double)lo) / top));
+}
+
+/* lohi = (lo ln tau, lo r, lo a, hi ln tau, hi r, hi a) over the active
+ * sites (NaN values skipped, -0 taken as +0); all zero without any. */
+void orc_pack_ranges(int N, const float *params, float *lohi)
+{
+    const int planes[3] = {P_LT, P_R, P_A};
+    for (int f = 0; f < 3; ++f) {
+        int any = 0;
+        float lo = 0.0f, hi = 0.0f;
+        for (int i = 0; i < N; ++i) {
+            if (!(params[P_X * N + i] >= 0.0f)) continue;
+            const float v = params[planes[f] * N + i] + 0.0f;
+            if (v != v) continue;
+            if (!any || v < lo) lo = v;
+            if (!any || v > hi) hi = v;
+            any = 1;
+        }
+        lohi[f] = lo;
+        lohi[3 + f] = hi;
+    }
+}
+
+void orc_pack_sites(int H, int W, int N, const float *params, const float *lohi, uint32_t *packed)
+{
+    const double cells = (double)(1u << PKW_XY), top_c = (double)((1u << PKW_C) - 1u);
+    const double tq = (double)(1u << PKW_TH);
+    for (int i = 0; i < N; ++i) {
+        uint32_t *w = packed + (size_t)i * 4;
+        w[0] = w[1] = w[2] = w[3] = 0;
+        const float x = params[P_X * N + i], y = params[P_Y * N + i];
+        if (!(x >= 0.0f)) continue;
+        pk_put(w, PK_X, PKW_XY, pk_cell((double)x / (double)W * cells, cells));
+        pk_put(w, PK_Y, PKW_XY, pk_cell((double)y / (double)H * cells, cells));
+        const int cp[3] = {P_CR, P_CG, P_CB}, co[3] = {PK_CR, PK_CG, PK_CB};
+        for (int c = 0; c < 3; ++c) {
+            double v = (double)params[cp[c] * N + i];
+            if (v < 0.0) v = 0.0;
+            if (v > 1.0) v = 1.0;
+            pk_put(w, co[c], PKW_C, pk_round(v * top_c, top_c));
+        }
+        pk_put(w, PK_LT, PKW_LT, pk_range_q(params[P_LT * N + i] + 0.0f, lohi[0], lohi[3], PKW_LT));
+        pk_put(w, PK_R, PKW_R, pk_range_q(params[P_R * N + i] + 0.0f, lohi[1], lohi[4], PKW_R));
+        pk_put(w, PK_A, PKW_A, pk_range_q(params[P_A * N + i] + 0.0f, lohi[2], lohi[5], PKW_A));
+        double th = fmod((double)params[P_TH * N + i], PK_PI);
+        if (th < 0.0) th += PK_PI;
+        const uint32_t qt = th == th ? (uint32_t)floor(th / PK_PI * tq + 0.5) : 0u;
+        pk_put(w, PK_TH, PKW_TH, qt & ((1u << PKW_TH) - 1u));
+        pk_put(w, PK_ACTIVE, 1, 1u);
+    }
+}
+
+void orc_unpack_sites(int H, int W, int N, const uint32_t *packed, const float *lohi, float *params)
+{
+    const double cells = (double)(1u << PKW_XY), top_c = (double)((1u << PKW_C) - 1u);
+    const double tq = (double)(1u << PKW_TH);
+    for (int i = 0; i < N; ++i) {
+        const uint32_t *w = packed + (size_t)i * 4;
+        for (int p = 0; p < P_COUNT; ++p) params[p * N + i] = 0.0f;
+        if (!pk_get(w, PK_ACTIVE, 1)) {
+            params[P_X * N + i] = -1.0f;
+            continue;
+        }
+        params[P_X * N + i] = (float)(((double)pk_get(w, PK_X, PKW_XY) + 0.5) * (double)W / cells);
+        params[P_Y * N + i] = (float)(((double)pk_get(w, PK_Y, PKW_XY) + 0.5) * (double)H / cells);
+        params[P_CR * N + i] = (float)((double)pk_get(w, PK_CR, PKW_C) / top_c);
+        params[P_CG * N + i] = (float)((double)pk_get(w, PK_CG, PKW_C) / top_c);
+        params[P_CB * N + i] = (float)((double)pk_get(w, PK_CB, PKW_C) / top_c);
+        params[P_LT * N + i] = pk_range_v(pk_get(w, PK_LT, PKW_LT), lohi[0], lohi[3], PKW_LT);
+        params[P_R * N + i] = pk_range_v(pk_get(w, PK_R, PKW_R), lohi[1], lohi[4], PKW_R);
+        params[P_A * N + i] = pk_range_v(pk_get(w, PK_A, PKW_A), lohi[2], lohi[5], PKW_A);
+        params[P_TH * N + i] = (float)((double)pk_get(w, PK_TH, PKW_TH) * (PK_PI / tq));
+    }
+}
