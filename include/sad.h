@@ -196,6 +196,29 @@ int sad_topk_exact(sad_ctx *ctx, const int64_t *pixels, int64_t n_pix, uint32_t 
  * <= max(H, W), each with G injections.  0 <= G <= 64. */
 int sad_refresh(sad_ctx *ctx, int G, sad_stream_t stream);
 
+/* 16-byte evaluation record ([P1] B.2, "Packed storage for evaluation": the
+ * site's semantic values quantised into four 32-bit words, per-image
+ * min/scale for ln tau and radius).  Field string, little-endian over the
+ * four words, bit offset (width):
+ *   x 0 (18), y 18 (18), cr 36 (10), cg 46 (10), cb 56 (10),
+ *   ln tau 66 (16), r 82 (14), theta 96 (14), a 110 (14), active 127 (1).
+ * x, y: cell floor(x / W 2^18) of 2^18 across the image (clamped), decoded
+ * at the cell centre.  Colours: clamped to [0, 1], 1023 steps.  ln tau, r,
+ * a: 2^b - 1 steps over the range [lo, hi] of the active sites.  theta: the
+ * axis angle theta mod pi in 2^14 steps.  Rounding half up in double;
+ * decoded values rounded once to float32.  Inactive sites pack to zeros.
+ * 128 bits per site: 16.3 bits per pixel at 768 x 512 with 50,000 sites.
+ *
+ * sad_pack_sites: packed = device uint32 [N_cap][4] (16-byte aligned),
+ * written in stream order; range = 6 floats (host or device, may be NULL)
+ * receiving (lo ln tau, lo r, lo a, hi ln tau, hi r, hi a).
+ * sad_unpack_sites: decodes packed + range into params and rebuilds the
+ * records; grads, Adam moments and candidate lists are left alone (call
+ * sad_reset and sad_refresh for a fresh fit or a decode-only render).
+ * Errors: SAD_ERR_INVALID_ARG for NULL or misaligned pointers. */
+int sad_pack_sites(sad_ctx *ctx, uint32_t *packed, float *range, sad_stream_t stream);
+int sad_unpack_sites(sad_ctx *ctx, const uint32_t *packed, const float *range, sad_stream_t stream);
+
 /* Candidate grid ([P1] B.3, "Candidate field"): keep the candidate lists on
  * a ceil(H/cell) x ceil(W/cell) grid of cell x cell pixel cells instead of
  * one list per pixel.  Cell (i, j) holds the pixels with floor(x/cell) = i,

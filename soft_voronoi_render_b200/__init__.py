@@ -103,6 +103,22 @@ class Sad:
     def reset(self, seed: int = 1):
         _lib.sad_reset(self.ctx, seed, self.stream)
 
+    def pack_sites(self):
+        """16-byte evaluation records: (packed (N, 4) int32 device tensor,
+        range (6,) float32 numpy array)."""
+        t = self.torch
+        packed = t.empty((self.N, 4), dtype=t.int32, device=self.device)
+        rng = t.empty(6, dtype=t.float32, device=self.device)
+        _lib.sad_pack_sites(self.ctx, packed, rng, self.stream)
+        return packed, rng.cpu().numpy()
+
+    def unpack_sites(self, packed, rng):
+        t = self.torch
+        src = self._dev(np.asarray(packed).view(np.int32) if isinstance(packed, np.ndarray) else packed, t.int32)
+        r = self._dev(np.asarray(rng, dtype=np.float32), t.float32)
+        _lib.sad_unpack_sites(self.ctx, src, r, self.stream)
+        self.torch.cuda.current_stream(self.device).synchronize()
+
     def set_candidate_grid(self, cell: int):
         """Lists on a ceil(H/cell) x ceil(W/cell) grid; the table starts empty."""
         _lib.sad_set_candidate_grid(self.ctx, cell, self.stream)

@@ -361,6 +361,31 @@ int sad_fit_pass(sad_ctx *ctx, int G, sad_stream_t stream) {
     return run_fit_pass(ctx, G, cs(stream));
 }
 
+int sad_pack_sites(sad_ctx *ctx, uint32_t *packed, float *range, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!packed) return fail(ctx, SAD_ERR_INVALID_ARG, "packed destination is NULL");
+    if (!aligned16(packed)) return fail(ctx, SAD_ERR_INVALID_ARG, "packed destination is not 16-byte aligned");
+    cudaStream_t st = cs(stream);
+    cudaError_t e = sad::launch_pack(ctx->dev, packed, st);
+    if (e == cudaSuccess && range)
+        e = cudaMemcpyAsync(range, sad::pack_range_device(ctx->dev), 6 * sizeof(float), cudaMemcpyDefault, st);
+    return cuda_status(ctx, e, "pack sites");
+}
+
+int sad_unpack_sites(sad_ctx *ctx, const uint32_t *packed, const float *range, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!packed || !range) return fail(ctx, SAD_ERR_INVALID_ARG, "packed source or range is NULL");
+    if (!aligned16(packed)) return fail(ctx, SAD_ERR_INVALID_ARG, "packed source is not 16-byte aligned");
+    cudaStream_t st = cs(stream);
+    float *dr = sad::pack_range_device(ctx->dev);
+    cudaError_t e = cudaMemcpyAsync(dr, range, 6 * sizeof(float), cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = sad::launch_unpack(ctx->dev, packed, dr, st);
+    if (e == cudaSuccess) e = sad::launch_records(ctx->dev, st);
+    return cuda_status(ctx, e, "unpack sites");
+}
+
 int sad_set_candidate_grid(sad_ctx *ctx, int cell, sad_stream_t stream) {
     if (!ctx) return SAD_ERR_INVALID_ARG;
     const int m = ctx->H > ctx->W ? ctx->H : ctx->W;

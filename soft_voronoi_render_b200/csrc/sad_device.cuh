@@ -40,6 +40,8 @@ struct Counters {
     unsigned long long dropped_ids;
     double loss;
     double pad1[7];
+    uint32_t pack_ord[6];    // order-preserving encodings of the pack ranges
+    float pack_range[6];     // lo ln tau, lo r, lo a, hi ln tau, hi r, hi a
 };
 static_assert(sizeof(Counters) <= 256, "counter block exceeds its 256-byte slot");
 constexpr size_t COUNTERS_BYTES = 256;

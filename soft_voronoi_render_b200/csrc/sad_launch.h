@@ -51,5 +51,8 @@ cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st);
 cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st);
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st);
 cudaError_t prepare_fused();
+float *pack_range_device(const Dev &d);
+cudaError_t launch_pack(const Dev &d, uint32_t *packed, cudaStream_t st);
+cudaError_t launch_unpack(const Dev &d, const uint32_t *packed, const float *range, cudaStream_t st);
 
 }  // namespace sad
