@@ -196,6 +196,15 @@ int sad_topk_exact(sad_ctx *ctx, const int64_t *pixels, int64_t n_pix, uint32_t 
  * <= max(H, W), each with G injections.  0 <= G <= 64. */
 int sad_refresh(sad_ctx *ctx, int G, sad_stream_t stream);
 
+/* Rebind the target image to another caller-owned device buffer (float32
+ * [3][H][W], 16-byte aligned) without copying: kernels launched after the
+ * call read the new buffer, earlier launches keep the old one.  This lets a
+ * caller stream targets in: copy the next target into a second buffer on
+ * another stream while the current iteration runs, then bind it.  The
+ * library never frees either buffer.  Errors: SAD_ERR_NOT_BOUND before
+ * sad_bind, SAD_ERR_INVALID_ARG for NULL or misaligned pointers. */
+int sad_bind_target(sad_ctx *ctx, const float *target);
+
 /* 16-byte evaluation record ([P1] B.2, "Packed storage for evaluation": the
  * site's semantic values quantised into four 32-bit words, per-image
  * min/scale for ln tau and radius).  Field string, little-endian over the

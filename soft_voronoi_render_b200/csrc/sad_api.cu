@@ -226,6 +226,16 @@ int sad_set_target(sad_ctx *ctx, const float *src, sad_stream_t stream) {
     return cuda_status(ctx, e, "set target");
 }
 
+int sad_bind_target(sad_ctx *ctx, const float *target) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!target) return fail(ctx, SAD_ERR_INVALID_ARG, "target is NULL");
+    if (!aligned16(target)) return fail(ctx, SAD_ERR_INVALID_ARG, "target is not 16-byte aligned");
+    ctx->buf.target = const_cast<float *>(target);
+    ctx->dev.target = const_cast<float *>(target);
+    return SAD_OK;
+}
+
 int sad_prep_records(sad_ctx *ctx, sad_stream_t stream) {
     int r = need_bound(ctx);
     if (r) return r;

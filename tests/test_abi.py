@@ -104,6 +104,23 @@ def test_bind_checks_alignment_and_sizes_without_touching_memory():
         with pytest.raises(_lib.SadError) as e:
             _lib.sad_adam_step(ctx, _lib.adam_cfg(lr_pos=-1.0))
         assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        # rebinding the target, the candidate grid and packed records check
+        # their pointers and sizes before any launch
+        for bad in (None, 0xB0004):
+            with pytest.raises(_lib.SadError) as e:
+                _lib.sad_bind_target(ctx, bad)
+            assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        _lib.sad_bind_target(ctx, 0xB0000)
+        for bad in (0, 65):
+            with pytest.raises(_lib.SadError) as e:
+                _lib.sad_set_candidate_grid(ctx, bad)
+            assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_pack_sites(ctx, 0xC0008)
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_unpack_sites(ctx, 0xC0000, None)
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG
     finally:
         _lib.sad_destroy(ctx)
 

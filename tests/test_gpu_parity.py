@@ -432,3 +432,26 @@ def test_full_size_c4_refresh_and_render(torch_cuda):
     # owners for this seed (the lists equal the oracle's bit for bit above)
     assert np.mean(hit) >= 0.97
     assert np.mean(got[sample][:, 0] == ex[:, 0]) >= 0.9
+
+
+def test_bind_target_switches_buffers(torch_cuda):
+    """sad_bind_target points the context at another device target without a
+    copy; the next pass's loss is the oracle's loss against that target."""
+    from soft_voronoi_render_b200 import _lib
+    tgt, prm, w = synth.make_workload("c1", seed=3)
+    tgt2 = synth.make_image(w.H, w.W, 6, 0, 99)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt, seed=3)
+    table = oracle.topk_exact(w.H, w.W, oracle.records(w.H, w.W, prm))
+    other = torch_cuda.from_numpy(np.ascontiguousarray(tgt2)).cuda()
+    _lib.sad_bind_target(s.ctx, other.data_ptr())
+    s.set_table(table)
+    s.backward()
+    L2, _ = oracle.loss_backward(w.H, w.W, prm, table, tgt2)
+    assert abs(s.loss() - L2) <= LOSS_RTOL * L2
+    _lib.sad_bind_target(s.ctx, s.target.data_ptr())
+    s.grads.zero_()
+    s.backward()
+    L1, _ = oracle.loss_backward(w.H, w.W, prm, table, tgt)
+    assert abs(s.loss() - L1) <= LOSS_RTOL * L1
+    with pytest.raises(_lib.SadError):
+        _lib.sad_bind_target(s.ctx, other.data_ptr() + 4)
