@@ -160,12 +160,16 @@ class ClockSampler:
 # committed ncu traffic for the dominant kernel (null when the source changed)
 # ---------------------------------------------------------------------------
 def kernel_source_digest() -> str:
-    """Digest of the sources the fused-pass kernel is compiled from: its own
-    file and the two headers it includes."""
+    """Digest of the code the fused-pass kernel is compiled from (its own
+    file and the two headers it includes), comments and blank lines removed,
+    so that only a change of code makes committed counters stale."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "soft_voronoi_render_b200", "csrc")
     for f in ("sad_device.cuh", "sad_fused.cu", "sad_launch.h"):
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        txt = open(os.path.join(csrc, f)).read()
+        txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+        lines = (re.sub(r"//.*", "", ln).rstrip() for ln in txt.splitlines())
+        h.update("\n".join(ln for ln in lines if ln.strip()).encode())
     return h.hexdigest()[:16]
 
 

@@ -3,11 +3,12 @@
 // summary section 4 "Candidate maintenance") fused with the soft Apollonius
 // render, the MSE loss and the analytic backward (summary B.4).
 //
-// A block owns a 32 x 8 pixel tile.  It first gathers the distinct site ids
-// that appear in the candidate lists of the tile and of its one-pixel halo
-// (the only lists a jump-1 pass can read) into a tile-local dense index of at
-// most 128 sites, stages those sites' records in shared memory and gives each
-// pixel a 128-bit membership mask.  The candidate union of a pixel is then the
+// A block owns a 32 x FY pixel tile (FY = 16 where there are at least 16
+// pixels per site, else 8; one warp per row).  It first gathers the distinct
+// site ids that appear in the candidate lists of the tile and of its
+// one-pixel halo (the only lists a jump-1 pass can read) into a tile-local
+// dense index of at most 128 sites, stages those sites' records in shared
+// memory and gives each pixel a 128-bit membership mask.  The candidate union of a pixel is then the
 // OR of five masks, so every distinct candidate is scored exactly once.  The
 // same dense index is the per-tile gradient accumulator: the role the pages
 // give to a hashed shared-memory table (summary section 5 and B.4), here
