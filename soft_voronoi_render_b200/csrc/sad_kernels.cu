@@ -646,13 +646,21 @@ struct AdamArgs {
     float beta1, beta2, eps;
 };
 
-__global__ void __launch_bounds__(SITE_THREADS) adam_kernel(float *__restrict__ prm, float *__restrict__ grads,
+// 4 blocks/SM (64 registers): the kernel is latency-bound, more warps hide it
+__global__ void __launch_bounds__(SITE_THREADS, 4) adam_kernel(float *__restrict__ prm, float *__restrict__ grads,
                                                             float *__restrict__ m1, float *__restrict__ m2,
                                                             float4 *__restrict__ rec, int N, int maxHW,
                                                             float xmax, float ymax, AdamArgs a,
                                                             const uint8_t *__restrict__ frozen, Counters *c) {
     const uint32_t t = c->adam_step + 1u;
     const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
+    // bias corrections 1 - beta^t, once per block
+    __shared__ float bc[2];
+    if (threadIdx.x == 0) {
+        bc[0] = (float)(1.0 - pow((double)a.beta1, (double)t));
+        bc[1] = (float)(1.0 - pow((double)a.beta2, (double)t));
+    }
+    __syncthreads();
     if (i < N) {
         const size_t n = (size_t)N;
         float v[NPARAM];
@@ -660,8 +668,7 @@ __global__ void __launch_bounds__(SITE_THREADS) adam_kernel(float *__restrict__ 
         for (int k = 0; k < NPARAM; ++k) v[k] = prm[k * n + i];
         // frozen sites keep their parameters (summary section 7)
         if (v[PX] >= 0.0f && !(frozen && frozen[i])) {
-            const float bc1 = (float)(1.0 - pow((double)a.beta1, (double)t));
-            const float bc2 = (float)(1.0 - pow((double)a.beta2, (double)t));
+            const float bc1 = bc[0], bc2 = bc[1];
             const float sig_pos = (float)maxHW;
 #pragma unroll
             for (int k = 0; k < NPARAM; ++k) {
