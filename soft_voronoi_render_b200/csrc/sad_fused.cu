@@ -93,12 +93,6 @@ struct Top8L {
         for (int q = 0; q + 1 < K; ++q) o &= !ranks_above(l[q + 1], id[q + 1], l[q], id[q]);
         return o;
     }
-    // Batcher's odd-even merge sort for 8 entries (19 compare-exchanges)
-    __device__ __forceinline__ void sort() {
-        cx(0, 1); cx(2, 3); cx(4, 5); cx(6, 7);
-        cx(0, 2); cx(1, 3); cx(1, 2); cx(4, 6); cx(5, 7); cx(5, 6);
-        cx(0, 4); cx(1, 5); cx(2, 6); cx(3, 7); cx(2, 4); cx(3, 5); cx(1, 2); cx(3, 4); cx(5, 6);
-    }
 };
 
 __device__ __forceinline__ uint32_t uhash(uint32_t id) { return (id * 2654435761u) >> (32 - UHASH_BITS); }
@@ -455,7 +449,13 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
                             t.lx[q] = NOLOC;
                         }
             }
-            if (!t.in_order()) t.sort();
+            // the list is nearly sorted: odd-even transposition rounds until it
+            // is in order (4 rounds = 8 passes always sort 8 entries)
+#pragma unroll 1
+            for (int round = 0; round < 4 && !t.in_order(); ++round) {
+                t.cx(0, 1); t.cx(2, 3); t.cx(4, 5); t.cx(6, 7);
+                t.cx(1, 2); t.cx(3, 4); t.cx(5, 6);
+            }
             // candidates the four neighbours add
             const int hc = (ty + 1) * HX + lane + 1;
             const uint4 mL = sm.masks[hc - 1], mR = sm.masks[hc + 1], mU = sm.masks[hc - HX],
