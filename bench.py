@@ -173,16 +173,36 @@ def kernel_source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def committed_traffic(kernel: str):
+def committed_counter(kernel: str, key: str):
+    """A per-launch counter from the committed ncu summary of the kernel, or
+    None when the summary is missing or the kernel's code changed since."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_c3.md")
     if not os.path.exists(path):
         return None
     txt = open(path).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    m = re.search(key + r":\s*([0-9.eE+]+)", txt)
     d = re.search(r"kernel_source_digest:\s*([0-9a-f]+)", txt)
     if not m or not d or d.group(1) != kernel_source_digest():
         return None
     return float(m.group(1))
+
+
+def committed_traffic(kernel: str):
+    return committed_counter(kernel, "traffic_bytes_per_launch")
+
+
+def issue_roofline(kernel: str, ms: float, clocks):
+    """The fused pass is bound by instruction issue, not by HBM: its warp
+    instructions per launch (committed ncu count) over the live launch time,
+    against 148 SMs x 4 schedulers x one warp instruction per cycle at the SM
+    clock sampled during the run."""
+    inst = committed_counter(kernel, "inst_executed_per_launch")
+    if inst is None or not clocks or not clocks.get("sm_mhz"):
+        return None
+    peak = 148 * 4 * clocks["sm_mhz"] * 1e6
+    achieved = inst / (ms * 1e-3)
+    return {"bound": "issue", "achieved": achieved, "peak": peak, "unit": "warp instructions/s",
+            "frac": achieved / peak, "inst_per_launch": inst, "peak_from": "148 SMs x 4 schedulers x sampled SM clock"}
 
 
 def measured_peaks():
@@ -421,6 +441,7 @@ def run_ours(args):
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
                          "algorithmic_bytes": alg_bytes},
+            "issue_roofline": issue_roofline(dom, avg[dom], clocks),
             "e2e": {"value": e2e_value, "unit": "Mpix/s", "h2d_bytes_per_step": int(host_tgt.numel() * 4),
                     "d2h_bytes_per_step": 8, "steps": E,
                     "how": "per step: pinned host target -> device (copy stream, double-buffered, overlapping the "
