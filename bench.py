@@ -264,6 +264,13 @@ def cpu_baseline(tgt, prm, wl, budget_s=15.0, rows=256):
                       f"{wl.W} band of the {wl.H}x{wl.W} N={wl.N} workload, {dt:.1f} s"}
 
 
+def workload_config(wl, world: int) -> dict:
+    """The benchmark's config, shared by both arms."""
+    return {"workload": f"{WORKLOAD}: {wl.description}", "H": wl.H, "W": wl.W, "N": wl.N, "K": 8, "G": wl.G,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "working set > L2 (two 134 MB candidate tables + 50 MB target + 50 MB image); no flush"}
+
+
 def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
@@ -281,8 +288,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "Mpix/s", "n_gpus": args.gpus,
         "steps": done, "warmup": args.warmup, "ms_per_step": dt / max(done, 1) * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD}: {wl.description}", "H": wl.H, "W": wl.W, "N": wl.N, "G": wl.G,
-                   "sample_rows": rows},
+        "config": workload_config(wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": "Mpix/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": f"each step: one oracle fit iteration on a {rows}-row band "
                                    f"of the {wl.H}x{wl.W} workload"},
@@ -431,10 +437,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "Mpix/s", "n_gpus": world, "steps": K,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": f"{WORKLOAD}: {wl.description}", "H": H, "W": W, "N": N, "K": 8, "G": G,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "working set > L2 (two 134 MB candidate tables + 50 MB target + 50 MB image); "
-                             "no flush"},
+            "config": workload_config(wl, world),
             "hbm_roof_frac_iter": (iter_bytes / (ms_step * 1e-3) / 1e9) / hbm,
             "iter_algorithmic_bytes": iter_bytes,
             "kernels_ms": {k: round(v, 5) for k, v in avg.items()},
