@@ -95,6 +95,14 @@ struct Top8L {
     }
 };
 
+// storage slot of sorted entry idx: the low three bits are XORed with bits of
+// the owning thread (idx >> 3), so that the 32 lanes reading entry 8 t + e
+// of their own runs hit distinct banks
+__device__ __forceinline__ uint32_t ent_slot(uint32_t idx) {
+    const uint32_t t = idx >> 3;
+    return idx ^ ((((t >> 3) & 3u) << 1) | ((t >> 1) & 1u));
+}
+
 __device__ __forceinline__ uint32_t uhash(uint32_t id) { return (id * 2654435761u) >> (32 - UHASH_BITS); }
 
 // insert a site id into the tile's key table (linear probing, compare-and-swap)
@@ -612,8 +620,9 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         pos0 = __shfl_sync(FULL, pos0, tail_lane);
         if (vq) {
             const uint32_t pos = pos0 + (uint32_t)(lane - start);
-            sm.ent_wl[pos] = make_float2(__expf(t.l[q] - M) * iz, t.l[q]);
-            sm.ent_pu[pos] = (uint16_t)(tid | (key << 9));
+            const uint32_t slot = ent_slot(pos);
+            sm.ent_wl[slot] = make_float2(__expf(t.l[q] - M) * iz, t.l[q]);
+            sm.ent_pu[slot] = (uint16_t)(tid | (key << 9));
         }
     }
     __syncthreads();
@@ -631,7 +640,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         for (int e = 0; e < K; ++e) {
             const uint32_t idx = e0 + e;
             if (idx >= n_ent) break;
-            const uint32_t pu = sm.ent_pu[idx];
+            const uint32_t pu = sm.ent_pu[ent_slot(idx)];
             const uint32_t u = pu >> 9, px = pu & 0x1FFu;
             if (u != cur) {
                 if (cur != NOLOC) {
@@ -647,7 +656,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
                 r2 = sm.urec[2][u];
                 r3 = sm.urec[3][u];
             }
-            const float2 wl = sm.ent_wl[idx];
+            const float2 wl = sm.ent_wl[ent_slot(idx)];
             const float4 pa = sm.pix4[px];
             const float2 pb = sm.pix2[px];
             float v[NPARAM];
