@@ -144,8 +144,7 @@ struct FusedSmem {
     float acc[NPARAM][UCAP];      // the tile's gradient sums per local site
     uint32_t cnt[UCAP];           // (pixel, slot) entries per local site
     uint32_t cursor[UCAP];        // scatter cursor of the counting sort
-    float4 pix4[FT];              // per pixel: chat (3), dL/dchat red
-    float2 pix2[FT];              //            dL/dchat green, blue
+    float4 pixg[FT];              // per pixel: dL/dchat (3), chat . dL/dchat
     float2 ent_wl[FT * K];        // entries grouped by site: softmax weight, logit
     uint16_t ent_pu[FT * K];      //   pixel (low 9 bits) and local site (high 7 bits)
     float warp_loss[FY];
@@ -194,20 +193,20 @@ __device__ __forceinline__ void run_bounds(uint32_t key, int lane, int &start, i
 
 // gradient contributions of one (pixel, slot) with softmax weight w and logit
 // l (both 0 for an unused slot, which then contributes exact zeros):
-//   gamma = w (c - chat) . g,  dL/dc = w g,  dL/dln tau = gamma l,
+//   gamma = w (c . g - chat . g),  dL/dc = w g,  dL/dln tau = gamma l,
 //   dL/dr = gamma k,  dL/dp = gamma G'delta / m,
 //   dL/da = -gamma (k^2 e^a alpha^2 - k^2 e^-a beta^2) / (2 m),
 //   dL/dtheta = -gamma alpha beta (k^2 e^a - k^2 e^-a) / m
 // with m = sqrt(delta^T G' delta) = k n (0 where m = 0).
 __device__ __forceinline__ void slot_grad(const float4 r0, const float4 r1, const float4 r2, const float4 r3,
-                                          float fx, float fy, float l, float w, float cr, float cg, float cb,
-                                          float gr, float gg, float gb, float (&v)[NPARAM]) {
+                                          float fx, float fy, float l, float w, float gr, float gg, float gb,
+                                          float cdg, float (&v)[NPARAM]) {
     const float dx = fx - r0.x, dy = fy - r0.y;
     const float u1 = fmaf(r0.z, dx, r0.w * dy);
     const float u2 = fmaf(r1.x, dy, r0.w * dx);
     const float qf = fmaf(dx, u1, dy * u2);
     const float im = qf > 0.0f ? rsqrtf(qf) : 0.0f;
-    const float gamma = w * ((r2.x - cr) * gr + (r2.y - cg) * gg + (r2.z - cb) * gb);
+    const float gamma = w * (fmaf(r2.x, gr, fmaf(r2.y, gg, r2.z * gb)) - cdg);
     const float gi = gamma * im;
     const float al = r2.w * dx + r3.x * dy;   // u . delta
     const float be = -r3.x * dx + r2.w * dy;  // v . delta
@@ -565,8 +564,8 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     // site by site below; the rare rest (injected winners, crowded tiles) go
     // straight to global atomics.
     unsigned global_adds = 0;
-    sm.pix4[tid] = make_float4(cr, cg, cb, gr);
-    sm.pix2[tid] = make_float2(gg, gb);
+    const float cdg = fmaf(cr, gr, fmaf(cg, gg, cb * gb));
+    sm.pixg[tid] = make_float4(gr, gg, gb, cdg);
 #pragma unroll
     for (int q = 0; q < K; ++q) {
         const bool vq = vmask >> q & 1u;
@@ -579,7 +578,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             const float4 *R = rec + (size_t)t.id[q] * REC_F4;
             float v[NPARAM];
             slot_grad(__ldg(R), __ldg(R + 1), __ldg(R + 2), __ldg(R + 3), fx, fy, t.l[q], __expf(t.l[q] - M) * iz,
-                      cr, cg, cb, gr, gg, gb, v);
+                      gr, gg, gb, cdg, v);
             ++global_adds;
 #pragma unroll
             for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + t.id[q], v[k]);
@@ -657,11 +656,10 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
                 r3 = sm.urec[3][u];
             }
             const float2 wl = sm.ent_wl[ent_slot(idx)];
-            const float4 pa = sm.pix4[px];
-            const float2 pb = sm.pix2[px];
+            const float4 pa = sm.pixg[px];
             float v[NPARAM];
             slot_grad(r0, r1, r2, r3, fx0 + (float)(px & (FX - 1)), fy0 + (float)(px / FX), wl.y, wl.x, pa.x,
-                      pa.y, pa.z, pa.w, pb.x, pb.y, v);
+                      pa.y, pa.z, pa.w, v);
 #pragma unroll
             for (int k = 0; k < NPARAM; ++k) a[k] += v[k];
         }
