@@ -147,6 +147,7 @@ struct FusedSmem {
     float4 pixg[FT];              // per pixel: dL/dchat (3), chat . dL/dchat
     float2 ent_wl[FT * K];        // entries grouped by site: softmax weight, logit
     uint16_t ent_pu[FT * K];      //   pixel (low 9 bits) and local site (high 7 bits)
+    uint32_t ring_id[(HN - FT) * K];  // the halo lists, read once from the table
     float warp_loss[FY];
     uint32_t n_ent;
     uint32_t ucount;
@@ -330,8 +331,10 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         int hx, hy;
         ring_coords<FY>(r, hx, hy);
         const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
-        if (gi < 0 || gi >= W || gj < 0 || gj >= H) continue;
-        const uint32_t id = table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
+        uint32_t id = EMPTY;
+        if (gi >= 0 && gi < W && gj >= 0 && gj < H)
+            id = table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
+        sm.ring_id[e] = id;
         if (id < Nu) ok &= ukey_insert(sm.keys, id);
     }
     if (!ok) sm.overflow = 1;
@@ -367,13 +370,10 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         if (PROP)
         for (int e = tid; e < RING * K; e += FT) {
             const int r = e % RING, q = e / RING;
+            const uint32_t id = sm.ring_id[e];
+            if (id >= Nu) continue;  // also the halo pixels outside the image
             int hx, hy;
             ring_coords<FY>(r, hx, hy);
-            const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
-            if (gi < 0 || gi >= W || gj < 0 || gj >= H) continue;
-            const uint32_t id =
-                table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
-            if (id >= Nu) continue;
             const uint32_t u = ukey_lookup(sm.keys, sm.lid, id);
             if (u != NOLOC) atomicOr(reinterpret_cast<uint32_t *>(&sm.masks[hy * HX + hx]) + (u >> 5), 1u << (u & 31u));
         }
