@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         if (PROP) sm.masks[(ty + 1) * HX + lane + 1] = own_mask;
         if (PROP)
         for (int e = tid; e < RING * K; e += FT) {
-            const int r = e % RING, q = e / RING;
+            const int r = e % RING;
             const uint32_t id = sm.ring_id[e];
             if (id >= Nu) continue;  // also the halo pixels outside the image
             int hx, hy;
