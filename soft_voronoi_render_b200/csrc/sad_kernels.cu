@@ -219,9 +219,50 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
         const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
         Top8 t;
         t.clear();
-        // own list, then the neighbours at (-k, 0), (+k, 0), (0, -k), (0, +k)
+        // own list first: re-scored in its previous order it is usually still
+        // sorted and free of repeats, and then it is the top-8 of its own
+        // candidates as it stands; otherwise it is offered like the others
+        {
+            const uint4 a = in0[p], b = in1[p];
+            const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            float l[8];
+            uint32_t id[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                l[q] = -__int_as_float(0x7f800000);
+                id[q] = EMPTY;
+                if (ids[q] < (uint32_t)N) {
+                    const float4 r0 = __ldg(rec + (size_t)ids[q] * REC_F4);
+                    const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)ids[q] * REC_F4 + 1));
+                    if (r0.x >= 0.0f) {
+                        const float lv = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+                        if (lv == lv) {
+                            l[q] = lv;
+                            id[q] = ids[q];
+                        }
+                    }
+                }
+            }
+            bool clean = true;
+#pragma unroll
+            for (int q = 1; q < 8; ++q) {
+                clean &= !ranks_above(l[q], id[q], l[q - 1], id[q - 1]);
+#pragma unroll
+                for (int r = 0; r < q; ++r) clean &= (id[q] == EMPTY) || (id[q] != id[r]);
+            }
+            if (clean) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    t.l[q] = l[q];
+                    t.id[q] = id[q];
+                }
+            } else {
+                offer_batch<8>(t, ids, rec, (uint32_t)N, fx, fy);
+            }
+        }
+        // the neighbours at (-k, 0), (+k, 0), (0, -k), (0, +k)
 #pragma unroll 1
-        for (int d = 0; d < 5; ++d) {
+        for (int d = 1; d < 5; ++d) {
             const int ni = i + (d == 1 ? -jump : (d == 2 ? jump : 0));
             const int nj = j + (d == 3 ? -jump : (d == 4 ? jump : 0));
             if (ni < 0 || ni >= W || nj < 0 || nj >= H) continue;
