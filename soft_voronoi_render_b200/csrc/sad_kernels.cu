@@ -201,6 +201,50 @@ __device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], 
     }
 }
 
+// The pixel's own list as the first candidates of a pass into an empty list:
+// re-scored in its previous order it is usually still sorted and free of
+// repeats (the records do not change between refresh passes), and then it is
+// the top-8 of its own candidates as it stands; otherwise its ids are offered
+// one by one like any other list.  Same result either way.
+__device__ __forceinline__ void take_own_list(Top8 &t, const uint4 a, const uint4 b, const float4 *__restrict__ rec,
+                                              uint32_t N, float fx, float fy) {
+    const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    float l[8];
+    uint32_t id[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        l[q] = -__int_as_float(0x7f800000);
+        id[q] = EMPTY;
+        if (ids[q] < N) {
+            const float4 r0 = __ldg(rec + (size_t)ids[q] * REC_F4);
+            const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)ids[q] * REC_F4 + 1));
+            if (r0.x >= 0.0f) {
+                const float lv = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+                if (lv == lv) {
+                    l[q] = lv;
+                    id[q] = ids[q];
+                }
+            }
+        }
+    }
+    bool clean = true;
+#pragma unroll
+    for (int q = 1; q < 8; ++q) {
+        clean &= !ranks_above(l[q], id[q], l[q - 1], id[q - 1]);
+#pragma unroll
+        for (int r = 0; r < q; ++r) clean &= (id[q] == EMPTY) || (id[q] != id[r]);
+    }
+    if (clean) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            t.l[q] = l[q];
+            t.id[q] = id[q];
+        }
+    } else {
+        offer_batch<8>(t, ids, rec, N, fx, fy);
+    }
+}
+
 // H x W is the candidate grid; a cell is scored at its centre, (i + 0.5) cs
 // (cs = 1: the pixel grid)
 __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *__restrict__ rec, uint32_t *table,
@@ -219,47 +263,7 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
         const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
         Top8 t;
         t.clear();
-        // own list first: re-scored in its previous order it is usually still
-        // sorted and free of repeats, and then it is the top-8 of its own
-        // candidates as it stands; otherwise it is offered like the others
-        {
-            const uint4 a = in0[p], b = in1[p];
-            const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            float l[8];
-            uint32_t id[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                l[q] = -__int_as_float(0x7f800000);
-                id[q] = EMPTY;
-                if (ids[q] < (uint32_t)N) {
-                    const float4 r0 = __ldg(rec + (size_t)ids[q] * REC_F4);
-                    const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)ids[q] * REC_F4 + 1));
-                    if (r0.x >= 0.0f) {
-                        const float lv = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
-                        if (lv == lv) {
-                            l[q] = lv;
-                            id[q] = ids[q];
-                        }
-                    }
-                }
-            }
-            bool clean = true;
-#pragma unroll
-            for (int q = 1; q < 8; ++q) {
-                clean &= !ranks_above(l[q], id[q], l[q - 1], id[q - 1]);
-#pragma unroll
-                for (int r = 0; r < q; ++r) clean &= (id[q] == EMPTY) || (id[q] != id[r]);
-            }
-            if (clean) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    t.l[q] = l[q];
-                    t.id[q] = id[q];
-                }
-            } else {
-                offer_batch<8>(t, ids, rec, (uint32_t)N, fx, fy);
-            }
-        }
+        take_own_list(t, in0[p], in1[p], rec, (uint32_t)N, fx, fy);
         // the neighbours at (-k, 0), (+k, 0), (0, -k), (0, +k)
 #pragma unroll 1
         for (int d = 1; d < 5; ++d) {
@@ -324,8 +328,10 @@ __global__ void __launch_bounds__(TILE_THREADS) jfa3x3_kernel(const float4 *__re
         const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
         Top8 t;
         t.clear();
+        take_own_list(t, in0[p], in1[p], rec, (uint32_t)N, fx, fy);
 #pragma unroll 1
         for (int d = 0; d < 9; ++d) {
+            if (d == 4) continue;  // the own list, taken above
             const int ni = i + (d % 3 - 1) * jump, nj = j + (d / 3 - 1) * jump;
             if (ni < 0 || ni >= W || nj < 0 || nj >= H) continue;
             const size_t pn = (size_t)nj * W + ni;
