@@ -328,10 +328,8 @@ __global__ void __launch_bounds__(TILE_THREADS) jfa3x3_kernel(const float4 *__re
         const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
         Top8 t;
         t.clear();
-        take_own_list(t, in0[p], in1[p], rec, (uint32_t)N, fx, fy);
 #pragma unroll 1
         for (int d = 0; d < 9; ++d) {
-            if (d == 4) continue;  // the own list, taken above
             const int ni = i + (d % 3 - 1) * jump, nj = j + (d / 3 - 1) * jump;
             if (ni < 0 || ni >= W || nj < 0 || nj >= H) continue;
             const size_t pn = (size_t)nj * W + ni;
