@@ -236,9 +236,9 @@ int sad_unpack_sites(sad_ctx *ctx, const uint32_t *packed, const float *range, s
  * the cell centre ((i + 0.5) cell, (j + 0.5) cell) ("centred cell UVs");
  * render and backward score each pixel's cell list at the pixel centre.
  * Injections are keyed on the cell index.  cell = 1 (the default) is the
- * pixel grid; the fused tile passes run only there, a coarser grid runs
- * sad_propagate + sad_backward for sad_fit_pass and sad_backward for
- * sad_fit_pass_cached.  The table buffer bound for H x W holds any grid.
+ * pixel grid.  On a coarser grid sad_fit_pass runs a propagation pass on the
+ * grid and then the tile pass of sad_fit_pass_cached, which reads each
+ * pixel's cell list.  The table buffer bound for H x W holds any grid.
  * After the call the current table is empty (sentinels): call sad_refresh,
  * sad_jfa_prepass or sad_set_table next.  sad_get_table, sad_set_table and
  * sad_topk_exact (pixels = NULL, or cell indices) then use GH x GW lists.

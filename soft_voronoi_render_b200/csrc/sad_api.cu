@@ -69,13 +69,14 @@ int run_refresh(sad_ctx *ctx, int G, cudaStream_t st) {
     return SAD_OK;
 }
 
-// the fused tile kernel works on the pixel grid; a coarser candidate grid
-// runs the separate propagation and backward kernels
+// the fused propagating pass works on the pixel grid; on a coarser candidate
+// grid the propagation runs on the grid, then the tile pass on the cached
+// lists renders and differentiates every pixel from its cell's list
 int run_fit_pass(sad_ctx *ctx, int G, cudaStream_t st) {
     if (ctx->cell == 1) return cuda_status(ctx, sad::launch_fit_tile(ctx->dev, G, st), "fit pass");
     int r = cuda_status(ctx, sad::launch_propagate(ctx->dev, 1, G, st), "propagate");
     if (r) return r;
-    return cuda_status(ctx, sad::launch_render_backward(ctx->dev, st), "backward");
+    return cuda_status(ctx, sad::launch_fit_tile_cached(ctx->dev, st), "fit pass (cached lists)");
 }
 
 int check_adam(sad_ctx *ctx, const sad_adam_cfg *cfg, sad::AdamHyper &h) {
@@ -360,7 +361,6 @@ int sad_fit_iteration(sad_ctx *ctx, int G, const sad_adam_cfg *cfg, sad_stream_t
 int sad_fit_pass_cached(sad_ctx *ctx, sad_stream_t stream) {
     int r = need_bound(ctx);
     if (r) return r;
-    if (ctx->cell != 1) return cuda_status(ctx, sad::launch_render_backward(ctx->dev, cs(stream)), "backward");
     return cuda_status(ctx, sad::launch_fit_tile_cached(ctx->dev, cs(stream)), "fit pass (cached lists)");
 }
 

@@ -46,6 +46,17 @@ struct Counters {
 static_assert(sizeof(Counters) <= 256, "counter block exceeds its 256-byte slot");
 constexpr size_t COUNTERS_BYTES = 256;
 
+// Where a pixel's candidate list lives: the list of its cell on a grid of
+// cell x cell pixel cells (summary B.3, "Candidate field"; cell = 1 is the
+// pixel grid).  PT is the number of lists, the stride of a table plane.
+struct TableGrid {
+    int cell, GW;
+    size_t PT;
+    __device__ __forceinline__ size_t cell_of(int i, int j, size_t p) const {
+        return cell == 1 ? p : (size_t)(j / cell) * GW + (size_t)(i / cell);
+    }
+};
+
 // ---------------------------------------------------------------------------
 // ranking: (logit desc, id asc)
 // ---------------------------------------------------------------------------

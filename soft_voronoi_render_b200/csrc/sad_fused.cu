@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
                                                                             uint32_t *table,
                                                          const float *__restrict__ target, int H, int W, int N,
                                                          int G, float *__restrict__ image,
-                                                         float *__restrict__ grads, void *ws) {
+                                                         float *__restrict__ grads, void *ws, TableGrid lists) {
     constexpr int FT = FX * FY, HY = FY + 2, HN = HX * HY, RING = HN - FT;
     extern __shared__ __align__(16) unsigned char fused_smem_raw[];
     FusedSmem<FY> &sm = *reinterpret_cast<FusedSmem<FY> *>(fused_smem_raw);
@@ -274,8 +274,10 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     const int i = i0 + lane, j = j0 + ty;
     const bool inside = i < W && j < H;
     const size_t P = (size_t)H * W;
-    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + cur * P * K);
-    const uint4 *in1 = in0 + P;
+    // the cached-list form also reads lists kept per cell of a coarser grid
+    const size_t PT = PROP ? P : lists.PT;
+    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + cur * PT * K);
+    const uint4 *in1 = in0 + PT;
     uint4 *out0 = reinterpret_cast<uint4 *>(table + (cur ^ 1u) * P * K);
     uint4 *out1 = out0 + P;
     const uint32_t Nu = (uint32_t)N;
@@ -309,8 +311,9 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         uint4 a = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY), b = a;
         if (inside) {
             const size_t p = (size_t)j * W + i;
-            a = in0[p];
-            b = in1[p];
+            const size_t pt = PROP ? p : lists.cell_of(i, j, p);
+            a = in0[pt];
+            b = in1[pt];
         }
         own[0] = a.x; own[1] = a.y; own[2] = a.z; own[3] = a.w;
         own[4] = b.x; own[5] = b.y; own[6] = b.z; own[7] = b.w;
@@ -738,11 +741,14 @@ cudaError_t ensure_smem_attr() {
 
 template <int FY, bool PROP>
 cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
+    // the propagating form works on the pixel grid only
+    if (PROP && d.cell != 1) return cudaErrorInvalidValue;
+    const TableGrid lists{d.cell, d.GW, (size_t)d.PT};
     cudaError_t e = ensure_smem_attr<FY, PROP>();
     if (e != cudaSuccess) return e;
     const dim3 grid((d.W + FX - 1) / FX, (d.H + FY - 1) / FY);
     fit_tile_kernel<FY, PROP><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY>), st>>>(d.records, d.table, d.target, d.H, d.W,
-                                                                           d.N, G, d.image, d.grads, d.ws);
+                                                                           d.N, G, d.image, d.grads, d.ws, lists);
     return cudaGetLastError();
 }
 

@@ -23,16 +23,6 @@ constexpr int TILE_Y = 8;
 constexpr int TILE_THREADS = TILE_X * TILE_Y;
 constexpr int SITE_THREADS = 256;
 
-// Where a pixel's candidate list lives: the list of its cell on a grid of
-// cell x cell pixel cells (summary B.3, "Candidate field"; cell = 1 is the
-// pixel grid).  PT is the number of lists, the stride of a table plane.
-struct TableGrid {
-    int cell, GW;
-    size_t PT;
-    __device__ __forceinline__ size_t cell_of(int i, int j, size_t p) const {
-        return cell == 1 ? p : (size_t)(j / cell) * GW + (size_t)(i / cell);
-    }
-};
 
 __device__ __forceinline__ Counters *counters(void *ws) { return reinterpret_cast<Counters *>(ws); }
 __device__ __forceinline__ double *loss_partials(void *ws) {
