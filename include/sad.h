@@ -172,6 +172,14 @@ int sad_get_sites(sad_ctx *ctx, float *dst_9xn, int n, sad_stream_t stream);
 /* Copy a target image (host or device float32 [3][P]) into the bound target. */
 int sad_set_target(sad_ctx *ctx, const float *target_3xp, sad_stream_t stream);
 
+/* Convert an 8-bit RGB image into the bound target: src is DEVICE memory
+ * holding H x W pixels of 3 interleaved bytes (row-major, the usual image
+ * layout); channel c of pixel p becomes src[3 p + c] / 255 (IEEE float32
+ * division) in the planar float32 target.  Streamed 8-bit inputs move a
+ * quarter of the bytes of float32 ones.  Errors: SAD_ERR_INVALID_ARG for
+ * NULL. */
+int sad_set_target_u8(sad_ctx *ctx, const uint8_t *src_hw3, sad_stream_t stream);
+
 /* Step a1: rebuild every score record from params.  Record of site i (fp32
  * values, each evaluated in double and rounded once): x, y, A, B, C, b, k, 0,
  * cr, cg, cb, cos theta, sin theta, k^2 e^a, k^2 e^-a, 0 where k = tau s,

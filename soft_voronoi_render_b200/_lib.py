@@ -73,7 +73,7 @@ class sad_stats(ctypes.Structure):
 EXPORTED = (
     "sad_workspace_bytes", "sad_create", "sad_destroy", "sad_bind", "sad_reset", "sad_set_sites",
     "sad_get_sites", "sad_set_target", "sad_prep_records", "sad_topk_exact", "sad_refresh", "sad_jfa_prepass",
-    "sad_propagate", "sad_fit_pass_cached", "sad_set_candidate_grid", "sad_pack_sites", "sad_unpack_sites", "sad_bind_target",
+    "sad_propagate", "sad_fit_pass_cached", "sad_set_candidate_grid", "sad_pack_sites", "sad_unpack_sites", "sad_bind_target", "sad_set_target_u8",
     "sad_render", "sad_backward", "sad_densify_prune", "sad_tau_diffuse", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
     "sad_get_stats", "sad_get_loss", "sad_last_error", "sad_backward_noalloc",
 )
@@ -116,6 +116,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "sad_set_candidate_grid": [vp, ci, vp],
         "sad_pack_sites": [vp, vp, vp, vp],
         "sad_bind_target": [vp, vp],
+        "sad_set_target_u8": [vp, vp, vp],
         "sad_unpack_sites": [vp, vp, vp, vp],
         "sad_render": [vp, vp, vp],
         "sad_backward": [vp, cu32, vp],
@@ -221,6 +222,10 @@ def sad_refresh(ctx: int, G: int, stream=None) -> None:
 
 def sad_jfa_prepass(ctx: int, stream=None) -> None:
     _check(ctx, load().sad_jfa_prepass(ctx, _stream(stream)))
+
+
+def sad_set_target_u8(ctx: int, src, stream=None) -> None:
+    _check(ctx, load().sad_set_target_u8(ctx, _ptr(src), _stream(stream)))
 
 
 def sad_bind_target(ctx: int, target) -> None:

@@ -227,6 +227,13 @@ int sad_set_target(sad_ctx *ctx, const float *src, sad_stream_t stream) {
     return cuda_status(ctx, e, "set target");
 }
 
+int sad_set_target_u8(sad_ctx *ctx, const uint8_t *src, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!src) return fail(ctx, SAD_ERR_INVALID_ARG, "target source is NULL");
+    return cuda_status(ctx, sad::launch_target_u8(ctx->dev, src, cs(stream)), "set target (8-bit)");
+}
+
 int sad_bind_target(sad_ctx *ctx, const float *target) {
     int r = need_bound(ctx);
     if (r) return r;

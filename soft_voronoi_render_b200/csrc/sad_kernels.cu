@@ -778,6 +778,17 @@ __global__ void __launch_bounds__(SITE_THREADS) tau_diffuse_kernel(const float *
     out[i] = res;
 }
 
+// 8-bit interleaved RGB -> planar float32 target, one pixel per thread
+__global__ void __launch_bounds__(SITE_THREADS) target_u8_kernel(const uint8_t *__restrict__ src, long long P,
+                                                                 float *__restrict__ target) {
+    const long long p = (long long)blockIdx.x * SITE_THREADS + threadIdx.x;
+    if (p >= P) return;
+    const uint8_t *px = src + 3 * p;
+    target[p] = __fdiv_rn((float)px[0], 255.0f);
+    target[P + p] = __fdiv_rn((float)px[1], 255.0f);
+    target[2 * P + p] = __fdiv_rn((float)px[2], 255.0f);
+}
+
 inline dim3 tile_grid(int H, int W) { return dim3((W + TILE_X - 1) / TILE_X, (H + TILE_Y - 1) / TILE_Y); }
 inline unsigned site_blocks(long long n) { return (unsigned)((n + SITE_THREADS - 1) / SITE_THREADS); }
 inline Counters *host_counters(const Dev &d) { return reinterpret_cast<Counters *>(d.ws); }
@@ -816,6 +827,11 @@ cudaError_t launch_init_counters(const Dev &d, uint32_t seed, cudaStream_t st) {
 cudaError_t launch_mark_inactive(const Dev &d, int from, cudaStream_t st) {
     if (from >= d.N) return cudaSuccess;
     mark_inactive_kernel<<<site_blocks(d.N - from), SITE_THREADS, 0, st>>>(d.params, d.N, from);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_target_u8(const Dev &d, const uint8_t *src, cudaStream_t st) {
+    target_u8_kernel<<<site_blocks(d.P), SITE_THREADS, 0, st>>>(src, d.P, d.target);
     return cudaGetLastError();
 }
 

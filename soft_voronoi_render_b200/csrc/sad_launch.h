@@ -37,6 +37,7 @@ size_t densify_offset(int H, int W);
 cudaError_t launch_init_counters(const Dev &d, uint32_t seed, cudaStream_t st);
 cudaError_t launch_mark_inactive(const Dev &d, int from, cudaStream_t st);
 cudaError_t launch_records(const Dev &d, cudaStream_t st);
+cudaError_t launch_target_u8(const Dev &d, const uint8_t *src, cudaStream_t st);
 cudaError_t launch_topk_exact(const Dev &d, const int64_t *pix, int64_t n, uint32_t *out, cudaStream_t st);
 cudaError_t launch_seed(const Dev &d, cudaStream_t st);
 cudaError_t launch_clear_table(const Dev &d, cudaStream_t st);

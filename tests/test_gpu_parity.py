@@ -484,3 +484,18 @@ def test_pages_propagation_accuracy_claim_at_1024(torch_cuda):
     assert exact.mean() > claim["min_fraction_exact"], exact.mean()
     # and the device lists are the oracle's, bit for bit, on the sample
     np.testing.assert_array_equal(ex, oracle.topk_exact(H, W, oracle.records(H, W, prm), pix))
+
+
+def test_set_target_u8(torch_cuda):
+    """sad_set_target_u8 turns interleaved 8-bit RGB into the planar float
+    target c / 255, bit for bit."""
+    from soft_voronoi_render_b200 import _lib
+    H, W, N = 37, 53, 50
+    prm = synth.uniform_sites(H, W, N, 2)
+    s = make_ctx(torch_cuda, H, W, N, prm)
+    img = synth.Stream(5, "u8").integers(H * W * 3, 256).astype(np.uint8).reshape(H, W, 3)
+    img[0, 0] = (0, 128, 255)
+    dev = torch_cuda.from_numpy(img).cuda()
+    _lib.sad_set_target_u8(s.ctx, dev.data_ptr(), s.stream)
+    want = (img.transpose(2, 0, 1).astype(np.float32) / np.float32(255.0))
+    np.testing.assert_array_equal(s.target.cpu().numpy(), want)
