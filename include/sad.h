@@ -361,6 +361,11 @@ int sad_get_stats(sad_ctx *ctx, sad_stats *out, sad_stream_t stream);
 /* Loss of the last backward pass, copied to host memory (synchronises). */
 int sad_get_loss(sad_ctx *ctx, double *loss, sad_stream_t stream);
 
+/* The same loss copied in stream order without synchronising: dst (one
+ * double, host-pinned or device memory) holds it once the stream reaches the
+ * copy.  Lets a caller read step k's loss while step k + 1 runs. */
+int sad_copy_loss(sad_ctx *ctx, double *dst, sad_stream_t stream);
+
 /* Message of the last failing call on this context ("" if none). */
 const char *sad_last_error(const sad_ctx *ctx);
 

@@ -75,7 +75,7 @@ EXPORTED = (
     "sad_get_sites", "sad_set_target", "sad_prep_records", "sad_topk_exact", "sad_refresh", "sad_jfa_prepass",
     "sad_propagate", "sad_fit_pass_cached", "sad_set_candidate_grid", "sad_pack_sites", "sad_unpack_sites", "sad_bind_target", "sad_set_target_u8",
     "sad_render", "sad_backward", "sad_densify_prune", "sad_tau_diffuse", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
-    "sad_get_stats", "sad_get_loss", "sad_last_error", "sad_backward_noalloc",
+    "sad_get_stats", "sad_get_loss", "sad_copy_loss", "sad_last_error", "sad_backward_noalloc",
 )
 
 _lib = None
@@ -129,6 +129,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "sad_set_table": [vp, vp, vp],
         "sad_get_stats": [vp, ctypes.POINTER(sad_stats), vp],
         "sad_get_loss": [vp, ctypes.POINTER(ctypes.c_double), vp],
+        "sad_copy_loss": [vp, vp, vp],
         "sad_last_error": [vp],
         "sad_backward_noalloc": [ci, ci, ci, vp, vp, vp, vp, vp, vp, vp],
     }
@@ -298,6 +299,10 @@ def sad_get_stats(ctx: int, stream=None) -> dict:
     s = sad_stats()
     _check(ctx, load().sad_get_stats(ctx, ctypes.byref(s), _stream(stream)))
     return s.as_dict()
+
+
+def sad_copy_loss(ctx: int, dst, stream=None) -> None:
+    _check(ctx, load().sad_copy_loss(ctx, _ptr(dst), _stream(stream)))
 
 
 def sad_get_loss(ctx: int, stream=None) -> float:

@@ -491,6 +491,15 @@ int sad_get_loss(sad_ctx *ctx, double *loss, sad_stream_t stream) {
     return cuda_status(ctx, e, "get loss");
 }
 
+int sad_copy_loss(sad_ctx *ctx, double *dst, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!dst) return fail(ctx, SAD_ERR_INVALID_ARG, "loss destination is NULL");
+    cudaError_t e = cudaMemcpyAsync(dst, &reinterpret_cast<sad::Counters *>(ctx->buf.workspace)->loss,
+                                    sizeof(double), cudaMemcpyDefault, cs(stream));
+    return cuda_status(ctx, e, "copy loss");
+}
+
 const char *sad_last_error(const sad_ctx *ctx) { return ctx ? ctx->err : "context is NULL"; }
 
 }  // extern "C"

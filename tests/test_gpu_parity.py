@@ -499,3 +499,20 @@ def test_set_target_u8(torch_cuda):
     _lib.sad_set_target_u8(s.ctx, dev.data_ptr(), s.stream)
     want = (img.transpose(2, 0, 1).astype(np.float32) / np.float32(255.0))
     np.testing.assert_array_equal(s.target.cpu().numpy(), want)
+
+
+def test_copy_loss_in_stream_order(torch_cuda):
+    """sad_copy_loss puts the loss of the last pass into caller memory in
+    stream order; after a synchronise it equals sad_get_loss."""
+    from soft_voronoi_render_b200 import _lib
+    tgt, prm, w = synth.make_workload("c1", seed=4)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt, seed=4)
+    s.refresh(2)
+    host = torch_cuda.zeros(1, dtype=torch_cuda.float64).pin_memory()
+    devbuf = torch_cuda.zeros(1, dtype=torch_cuda.float64, device="cuda")
+    s.fit_pass(2)
+    _lib.sad_copy_loss(s.ctx, host.data_ptr(), s.stream)
+    _lib.sad_copy_loss(s.ctx, devbuf.data_ptr(), s.stream)
+    torch_cuda.cuda.synchronize()
+    L = s.loss()
+    assert float(host[0]) == L == float(devbuf.cpu()[0]) and L > 0
