@@ -100,6 +100,17 @@ class Sad:
         _lib.sad_set_target(self.ctx, src, self.stream)
         self._keep_t = src
 
+    def set_target_u8(self, rgb):
+        """Target from an 8-bit RGB image (H, W, 3), converted on the device."""
+        src = self._dev(rgb, self.torch.uint8)
+        _lib.sad_set_target_u8(self.ctx, src, self.stream)
+        self._keep_t = src
+
+    def bind_target(self, target):
+        """Point the context at another device target tensor (3, H, W) float32
+        without copying; the caller keeps it alive while kernels read it."""
+        _lib.sad_bind_target(self.ctx, target)
+
     def reset(self, seed: int = 1):
         _lib.sad_reset(self.ctx, seed, self.stream)
 
