@@ -102,6 +102,15 @@ typedef struct sad_buffers {
  * e = |chat - t|^2 at each pixel holding the site. */
 #define SAD_STATS 1u
 
+/* sad_backward flag: gradients that do not depend on the order of the
+ * atomic additions (bit-identical from run to run).  Every per-warp run sum
+ * is rounded to a multiple of 2^-40 and accumulated in 64-bit fixed point
+ * with integer atomics (exact, hence order-free), then added to grads; the
+ * pages accumulate scaled integer gradients the same way on WebGPU
+ * ([P1] B.4).  Magnitudes up to 2^23 per site and parameter; terms below
+ * 2^-41 vanish.  Not combinable with SAD_STATS. */
+#define SAD_DETERMINISTIC 2u
+
 /* Densify / prune configuration ([P1] B.5, [P2] design 4). */
 typedef struct sad_densify_cfg {
     int grow;              /* net sites added per event (2500 in the 768x512 schedule) */
@@ -283,8 +292,10 @@ int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream);
  * probing capped at 8, compare-and-swap insert) with one global atomic per
  * (site, parameter, tile); overflow goes straight to global atomics
  * ([P1] section 5 and B.4).  Writes the bound image when one is bound and
- * the loss into the statistics block.  flags: 0 or SAD_STATS (needs the stats
- * buffer; accumulates into it). */
+ * the loss into the statistics block.  flags: 0, SAD_STATS (needs the stats
+ * buffer; accumulates into it) or SAD_DETERMINISTIC (fixed-point
+ * accumulation, order-independent).  SAD_ERR_UNSUPPORTED for other flags or
+ * both together. */
 int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream);
 
 /* One budget-control event, on the device ([P1] B.5: split by the score

@@ -10,9 +10,9 @@ from __future__ import annotations
 import numpy as np
 
 from . import _lib
-from ._lib import SAD_STATS, SadError, adam_cfg, densify_cfg  # noqa: F401
+from ._lib import SAD_DETERMINISTIC, SAD_STATS, SadError, adam_cfg, densify_cfg  # noqa: F401
 
-__all__ = ["Sad", "SadError", "adam_cfg", "densify_cfg", "SAD_STATS", "load"]
+__all__ = ["Sad", "SadError", "adam_cfg", "densify_cfg", "SAD_STATS", "SAD_DETERMINISTIC", "load"]
 
 
 def load():

@@ -46,6 +46,7 @@ class sad_densify_cfg(ctypes.Structure):
 
 
 SAD_STATS = 1
+SAD_DETERMINISTIC = 2
 
 
 def densify_cfg(grow=2500, prune_frac=0.005, alpha=0.5, eps=1e-6, r_scale=0.85, log_tau_shift=0.6931471805599453,

@@ -303,7 +303,12 @@ int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream) {
 int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream) {
     int r = need_bound(ctx);
     if (r) return r;
-    if (flags & ~SAD_STATS) return fail(ctx, SAD_ERR_UNSUPPORTED, "backward flags 0x%x not supported", flags);
+    if (flags & ~(SAD_STATS | SAD_DETERMINISTIC))
+        return fail(ctx, SAD_ERR_UNSUPPORTED, "backward flags 0x%x not supported", flags);
+    if ((flags & SAD_STATS) && (flags & SAD_DETERMINISTIC))
+        return fail(ctx, SAD_ERR_UNSUPPORTED, "SAD_DETERMINISTIC carries the gradients only, not SAD_STATS");
+    if (flags & SAD_DETERMINISTIC)
+        return cuda_status(ctx, sad::launch_render_backward_det(ctx->dev, cs(stream)), "backward (deterministic)");
     if (flags & SAD_STATS) {
         if (!ctx->buf.stats) return fail(ctx, SAD_ERR_NOT_BOUND, "SAD_STATS needs a bound stats buffer");
         return cuda_status(ctx, sad::launch_render_backward_stats(ctx->dev, cs(stream)), "backward (stats)");

@@ -456,13 +456,21 @@ __device__ __forceinline__ int hash_find_or_insert(uint32_t *keys, uint32_t id) 
 // (summary B.4-B.5): mass sum w, energy sum w e, second moments
 // sum w e (dx^2, dx dy, dy^2) and the removal delta
 // sum |(chat - w c) / max(1 - w, 1e-6) - t|^2 - e, with e = |chat - t|^2.
-template <bool STATS>
+// DET (deterministic): every run sum is rounded to a multiple of 2^-40 and
+// added to a 64-bit fixed-point accumulator per (parameter, site) with
+// integer atomics, which are exact and so independent of their order (the
+// pages' integer-atomic gradient accumulation, summary B.4); no tile table.
+constexpr float DET_SCALE = 1099511627776.0f;  // 2^40
+
+template <bool STATS, bool DET = false>
 __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *__restrict__ rec,
                                                                   const uint32_t *__restrict__ table,
                                                                   const float *__restrict__ target, int H, int W,
                                                                   TableGrid tg, int N, float *__restrict__ image,
                                                                   float *__restrict__ grads,
-                                                                  float *__restrict__ stats, void *ws) {
+                                                                  float *__restrict__ stats, void *ws,
+                                                                  unsigned long long *__restrict__ fixed) {
+    static_assert(!(STATS && DET), "the deterministic backward carries the gradients only");
     constexpr int NV = STATS ? NPARAM + NSTAT : NPARAM;
     __shared__ uint32_t keys[HASH_SLOTS];
     __shared__ float acc[NV][HASH_SLOTS];
@@ -597,7 +605,15 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
             }
         }
         const bool tail = warp_run_reduce(key, v, lane);
-        if (tail && key != EMPTY) {
+        if (DET) {
+            if (tail && key != EMPTY) {
+#pragma unroll
+                for (int k = 0; k < NPARAM; ++k) {
+                    const long long qv = __float2ll_rn(v[k] * DET_SCALE);
+                    if (qv) atomicAdd(fixed + (size_t)k * N + key, (unsigned long long)qv);
+                }
+            }
+        } else if (tail && key != EMPTY) {
             const int slot = hash_find_or_insert(keys, key);
             if (slot >= 0) {
 #pragma unroll
@@ -620,6 +636,7 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
     const int nd = __syncthreads_count(dropped != 0);
     const int no = __syncthreads_count(overflow != 0);
     // flush the tile table: one global atomic per (site, parameter)
+    if (!DET)
     for (int q = tid; q < HASH_SLOTS; q += TILE_THREADS) {
         const uint32_t id = keys[q];
         if (id == EMPTY) continue;
@@ -670,6 +687,19 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
             c->ticket_bwd = 0;
             __threadfence();
         }
+    }
+}
+
+// the deterministic backward's fixed-point sums, added to the gradients and
+// cleared for the next call
+__global__ void __launch_bounds__(SITE_THREADS) fixed_to_grads_kernel(unsigned long long *__restrict__ fixed,
+                                                                      float *__restrict__ grads, long long n) {
+    const long long q = (long long)blockIdx.x * SITE_THREADS + threadIdx.x;
+    if (q >= n) return;
+    const long long v = (long long)fixed[q];
+    if (v) {
+        grads[q] += (float)((double)v * 0x1p-40);
+        fixed[q] = 0ull;
     }
 }
 
@@ -802,10 +832,15 @@ size_t densify_offset(int H, int W) {
     return (COUNTERS_BYTES + tiles * sizeof(double) + 255) / 256 * 256;
 }
 
+size_t fixed_offset(int H, int W, int N) {
+    return (densify_offset(H, W) + 256 + 3 * sizeof(uint32_t) * (size_t)N + 255) / 256 * 256;
+}
+
 size_t workspace_bytes(int H, int W, int N) {
     // densify scratch: a 256-byte header, then the parent and free-slot lists;
-    // then one float per site for tau diffusion
-    return densify_offset(H, W) + 256 + 3 * sizeof(uint32_t) * (size_t)N;
+    // then one float per site for tau diffusion; then the deterministic
+    // backward's 64-bit sums, one per (parameter, site)
+    return fixed_offset(H, W, N) + NPARAM * sizeof(unsigned long long) * (size_t)N;
 }
 
 cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st) {
@@ -882,13 +917,25 @@ cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st) {
 
 cudaError_t launch_render_backward(const Dev &d, cudaStream_t st) {
     render_bwd_kernel<false><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, nullptr, d.ws);
+        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, nullptr, d.ws, nullptr);
     return cudaGetLastError();
 }
 
 cudaError_t launch_render_backward_stats(const Dev &d, cudaStream_t st) {
     render_bwd_kernel<true><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, d.stats, d.ws);
+        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, d.stats, d.ws, nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_render_backward_det(const Dev &d, cudaStream_t st) {
+    unsigned long long *fixed =
+        reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(d.ws) + fixed_offset(d.H, d.W, d.N));
+    render_bwd_kernel<false, true><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
+        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, nullptr, d.ws, fixed);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long n = (long long)NPARAM * d.N;
+    fixed_to_grads_kernel<<<site_blocks(n), SITE_THREADS, 0, st>>>(fixed, d.grads, n);
     return cudaGetLastError();
 }
 

@@ -45,6 +45,7 @@ cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st);
 cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st);
 cudaError_t launch_render_backward(const Dev &d, cudaStream_t st);
 cudaError_t launch_render_backward_stats(const Dev &d, cudaStream_t st);
+cudaError_t launch_render_backward_det(const Dev &d, cudaStream_t st);
 cudaError_t launch_densify(const Dev &d, const DensifyArgs &a, cudaStream_t st);
 cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st);
 cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st);

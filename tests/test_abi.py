@@ -82,9 +82,10 @@ def test_bind_checks_alignment_and_sizes_without_touching_memory():
         with pytest.raises(_lib.SadError) as e:
             _lib.sad_set_sites(ctx, 0x90000, 17)
         assert e.value.status == _lib.SAD_ERR_CAPACITY
-        with pytest.raises(_lib.SadError) as e:
-            _lib.sad_backward(ctx, 2)
-        assert e.value.status == _lib.SAD_ERR_UNSUPPORTED
+        for flags in (4, _lib.SAD_STATS | _lib.SAD_DETERMINISTIC):
+            with pytest.raises(_lib.SadError) as e:
+                _lib.sad_backward(ctx, flags)
+            assert e.value.status == _lib.SAD_ERR_UNSUPPORTED
         with pytest.raises(_lib.SadError) as e:
             _lib.sad_backward(ctx, _lib.SAD_STATS)  # no stats buffer bound
         assert e.value.status == _lib.SAD_ERR_NOT_BOUND

@@ -516,3 +516,28 @@ def test_copy_loss_in_stream_order(torch_cuda):
     torch_cuda.cuda.synchronize()
     L = s.loss()
     assert float(host[0]) == L == float(devbuf.cpu()[0]) and L > 0
+
+
+@pytest.mark.parametrize("wl", ["c1", "c2"])
+def test_backward_deterministic(torch_cuda, wl):
+    """SAD_DETERMINISTIC: gradients bit-identical from run to run (fixed-point
+    integer accumulation), within the gradient tolerance of the oracle, and
+    the same loss as the float path."""
+    from soft_voronoi_render_b200 import SAD_DETERMINISTIC
+    tgt, prm, w = synth.make_workload(wl, seed=6)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt, seed=6)
+    t0, _ = oracle.refresh(w.H, w.W, prm, 2, seed=6)
+    s.set_table(t0)
+    runs = []
+    for _ in range(3):
+        s.grads.zero_()
+        s.backward(SAD_DETERMINISTIC)
+        runs.append(s.grads.cpu().numpy().copy())
+    L_det = s.loss()
+    assert all(np.array_equal(r.view(np.uint32), runs[0].view(np.uint32)) for r in runs[1:])
+    L, g = oracle.loss_backward(w.H, w.W, prm, t0, tgt)
+    assert abs(L_det - L) <= LOSS_RTOL * L
+    assert_grads(runs[0], g, "deterministic")
+    s.grads.zero_()
+    s.backward()
+    assert s.loss() == L_det
