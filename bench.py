@@ -58,7 +58,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
-    ap.add_argument("--workload", default="c3", choices=["c3", "c4", "c5"],
+    ap.add_argument("--workload", default="c3", choices=["c3", "c4", "c5", "rows"],
                     help="c3: the fitting-iteration metric (default); c4: full candidate refresh + render at "
                          "4096x4096, N=524,288; c5: end-to-end 768x512 fit with densify/prune (secondary "
                          "measurements)")
@@ -640,8 +640,106 @@ def run_fit(args):
     return 0
 
 
+def run_rows(args):
+    """Every entry point of the path timed on its own at 2048 x 2048,
+    N = 131,072 (exact top-K on the 256 x 256, N = 1,024 workload), with the
+    algorithmic bytes of one call and their fraction of the measured HBM
+    peak.  Secondary measurements; the headline is the default workload."""
+    import torch
+    import synth
+    from soft_voronoi_render_b200 import SAD_DETERMINISTIC, SAD_STATS, Sad, _lib
+
+    hbm, peak_kind = measured_peaks()
+    reps = max(3, min(args.steps, 20))
+    tgt, prm, wl = synth.make_workload("c3", seed=1)
+    H, W, N, G, P = wl.H, wl.W, wl.N, wl.G, wl.H * wl.W
+    s = Sad(H, W, N, seed=1)
+    s.set_sites(prm)
+    s.set_target(tgt)
+    s.refresh(G)
+    cfg = _lib.adam_cfg(lr_color=5e-3)
+    for _ in range(5):
+        s.fit_iteration(G, cfg)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n=reps, before=None):
+        for _ in range(2):
+            if before:
+                before()
+            fn()
+        torch.cuda.synchronize()
+        total = 0.0
+        for _ in range(n):
+            if before:
+                before()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+        return total / n
+
+    rows = {}
+
+    def row(name, ms, alg_bytes, note, **extra):
+        r = {"ms": ms, "alg_bytes": alg_bytes, "hbm_frac": (alg_bytes / (ms * 1e-3) / 1e9 / hbm) if alg_bytes else None,
+             "what": note}
+        r.update(extra)
+        rows[name] = r
+
+    row("a1_records", timed(s.prep_records), 100 * N, "records from params: 36 B read + 64 B written per site")
+    row("a2_propagate_k1", timed(lambda: s.propagate(1, G)), 64 * P, "one Jacobi pass, jump 1, G = 2: lists 32 + 32 B/px")
+    row("a2_propagate_k16", timed(lambda: s.propagate(16, G)), 64 * P, "one Jacobi pass, jump 16, G = 2")
+    row("a4_render", timed(s.render), 44 * P, "softmax blend: list 32 + image 12 B/px")
+    zero = s.grads.zero_
+    row("a5_a6_backward", timed(s.backward, before=zero), 56 * P + 36 * N,
+        "render + loss + backward, tile hash: list 32 + target 12 + image 12 B/px, gradients 36 B/site")
+    row("a6_backward_stats", timed(lambda: s.backward(SAD_STATS), before=zero), 56 * P + 60 * N,
+        "the same with the budget statistics (+24 B/site)")
+    row("a6_backward_deterministic", timed(lambda: s.backward(SAD_DETERMINISTIC), before=zero), 56 * P + 36 * N,
+        "the same with 64-bit fixed-point accumulation")
+    row("a2_a6_fit_pass", timed(lambda: s.fit_pass(G), before=zero), 88 * P + 100 * N,
+        "fused pass: propagation k = 1 + render + loss + backward")
+    row("a4_a6_fit_pass_cached", timed(s.fit_pass_cached, before=zero), 56 * P + 100 * N,
+        "the tile pass on cached lists (no propagation)")
+    row("a7_adam", timed(lambda: s.adam_step(cfg)), 352 * N, "Adam + records: 352 B/site")
+    row("next4_tau_diffuse", timed(lambda: s.tau_diffuse(0.3)), 48 * N, "tau diffusion: list 32 + 16 B/site")
+    packed = torch.empty((N, 4), dtype=torch.int32, device=s.device)
+    rng = torch.empty(6, dtype=torch.float32, device=s.device)
+    row("next3_pack", timed(lambda: _lib.sad_pack_sites(s.ctx, packed, rng, s.stream)), 52 * N,
+        "16-byte records: 36 B read + 16 B written per site")
+    row("next3_unpack", timed(lambda: _lib.sad_unpack_sites(s.ctx, packed, rng, s.stream)), 116 * N,
+        "decode + records: 16 B read + 36 + 64 B written per site")
+    row("a9_refresh", timed(lambda: s.refresh(G), n=3), 32 * P + 11 * 64 * P, "seed + 11 passes (jumps 1024..1)")
+    row("next2_jfa_prepass", timed(s.jfa_prepass, n=3), 32 * P + 11 * 64 * P, "seed + 11 flood passes")
+    s.refresh(G)
+    row("next1_densify_prune", timed(lambda: s.densify_prune(_lib.densify_cfg(grow=2500, prune_frac=0.005)), n=3,
+                                     before=lambda: (s.grads.zero_(), s.backward(SAD_STATS))), 0,
+        "one event (statistics from a backward before each call, untimed): select, prune, split, records",
+        hbm_frac=None)
+    s.close()
+    # a8 on the 256 x 256, N = 1,024 workload: every site scored at every pixel
+    tgt1, prm1, w1 = synth.make_workload("c1", seed=1)
+    s1 = Sad(w1.H, w1.W, w1.N, seed=1)
+    s1.set_sites(prm1)
+    ms = timed(s1.topk_exact)
+    scores = w1.H * w1.W * w1.N
+    row("a8_topk_exact_c1", ms, 0, "brute force over all 1,024 sites at all 65,536 pixels",
+        gscores_per_s=scores / (ms * 1e-3) / 1e9, hbm_frac=None)
+    s1.close()
+    line = {"metric": "per-entry-point device time, 2048x2048 N=131,072 (exact top-K: 256x256 N=1,024)",
+            "unit": "ms", "n_gpus": 1, "reps": reps, "peak_hbm_gbs": hbm, "peak_kind": peak_kind, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": f"c3: {wl.description}", "H": H, "W": W, "N": N, "G": G},
+            "rows": rows}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.workload == "rows":
+        return run_rows(args)
     if args.workload == "c5" and args.impl == "ours":
         return run_fit(args)
     if args.impl == "reference":
