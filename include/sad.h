@@ -341,7 +341,7 @@ int sad_adam_step(sad_ctx *ctx, const sad_adam_cfg *cfg, sad_stream_t stream);
  * (same result as sad_propagate(ctx, 1, G)), then render, loss and backward
  * on the new lists (same result as sad_backward, up to the summation order
  * of the gradients).  Each 32 x 16 tile (32 x 8 where there are fewer than
- * 16 pixels per site) gathers the distinct sites of its and
+ * 4 pixels per site) gathers the distinct sites of its and
  * its halo's lists into a dense local index (at most 128 sites; tiles with
  * more take a slower generic path) that serves both to de-duplicate the
  * candidate union and to accumulate the tile's gradients ([P1] section 5 and

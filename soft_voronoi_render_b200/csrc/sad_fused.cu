@@ -3,7 +3,7 @@
 // summary section 4 "Candidate maintenance") fused with the soft Apollonius
 // render, the MSE loss and the analytic backward (summary B.4).
 //
-// A block owns a 32 x FY pixel tile (FY = 16 where there are at least 16
+// A block owns a 32 x FY pixel tile (FY = 16 where there are at least 4
 // pixels per site, else 8; one warp per row).  It first gathers the distinct
 // site ids that appear in the candidate lists of the tile and of its
 // one-pixel halo (the only lists a jump-1 pass can read) into a tile-local
@@ -764,13 +764,14 @@ cudaError_t prepare_fused() {
 
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st) {
     // taller tiles amortise the halo and the per-tile work, but hold more
-    // distinct sites: use them where sites are sparse (>= 16 pixels per site)
-    if ((long long)d.H * d.W >= 16ll * d.N) return launch_fit_tile_h<16, true>(d, G, st);
+    // distinct sites: use them unless sites are dense (< 4 pixels per site),
+    // where tiles would often exceed the 128-site index
+    if ((long long)d.H * d.W >= 4ll * d.N) return launch_fit_tile_h<16, true>(d, G, st);
     return launch_fit_tile_h<8, true>(d, G, st);
 }
 
 cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st) {
-    if ((long long)d.H * d.W >= 16ll * d.N) return launch_fit_tile_h<16, false>(d, 0, st);
+    if ((long long)d.H * d.W >= 4ll * d.N) return launch_fit_tile_h<16, false>(d, 0, st);
     return launch_fit_tile_h<8, false>(d, 0, st);
 }
 
