@@ -17,6 +17,7 @@ of this method to run) on the same workload and metric.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import math
@@ -428,19 +429,31 @@ def run_ours(args):
     host_u8 = torch.from_numpy(np.ascontiguousarray(
         np.clip(np.rint(tgt * 255.0), 0, 255).astype(np.uint8).transpose(1, 2, 0))).pin_memory()
     bufs8 = [torch.empty(host_u8.shape, dtype=torch.uint8, device=dev) for _ in range(2)]
-    for ev in used:
-        ev.record(stream)
-
-    def issue_copy8(k):
-        b = k % 2
-        copy_stream.wait_event(used[b])
-        with torch.cuda.stream(copy_stream):
-            bufs8[b].copy_(host_u8, non_blocking=True)
-        copied[b].record(copy_stream)
-
     # each step's loss is copied to its own slot of pinned host memory in
     # stream order (one device -> host transfer per step, no host wait)
     host_loss = torch.zeros(E, dtype=torch.float64).pin_memory()
+    # the loop issues its copies and stream dependencies through the CUDA
+    # runtime directly: a few microseconds of host time per step
+    from cuda.bindings import runtime as cudart
+    L = _lib.load()
+    no_timing = cudart.cudaEventDisableTiming
+    ev_copied = [cudart.cudaEventCreateWithFlags(no_timing)[1] for _ in range(2)]
+    ev_used = [cudart.cudaEventCreateWithFlags(no_timing)[1] for _ in range(2)]
+    cs_h, ms_h = copy_stream.cuda_stream, stream.cuda_stream
+    h2d = cudart.cudaMemcpyKind.cudaMemcpyHostToDevice
+    src, nbytes = host_u8.data_ptr(), host_u8.numel()
+    dst = [b.data_ptr() for b in bufs8]
+    loss0 = host_loss.data_ptr()
+    status = []
+    for ev in ev_used:
+        status.append(cudart.cudaEventRecord(ev, ms_h)[0])
+
+    def issue_copy8(k):
+        b = k % 2
+        status.append(cudart.cudaStreamWaitEvent(cs_h, ev_used[b], 0)[0])
+        status.append(cudart.cudaMemcpyAsync(dst[b], src, nbytes, h2d, cs_h)[0])
+        status.append(cudart.cudaEventRecord(ev_copied[b], cs_h)[0])
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -449,13 +462,19 @@ def run_ours(args):
     for k in range(E):
         if k + 1 < E:
             issue_copy8(k + 1)
-        stream.wait_event(copied[k % 2])
-        _lib.sad_set_target_u8(ctx, bufs8[k % 2].data_ptr(), sp)
-        used[k % 2].record(stream)
-        _lib.sad_fit_iteration(ctx, G, cfg, sp)
-        _lib.sad_copy_loss(ctx, host_loss[k].data_ptr(), sp)
+        b = k % 2
+        status.append(cudart.cudaStreamWaitEvent(ms_h, ev_copied[b], 0)[0])
+        status.append(L.sad_set_target_u8(ctx, dst[b], sp))
+        status.append(cudart.cudaEventRecord(ev_used[b], ms_h)[0])
+        status.append(L.sad_fit_iteration(ctx, G, ctypes.byref(cfg), sp))
+        status.append(L.sad_copy_loss(ctx, loss0 + 8 * k, sp))
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    bad = [x for x in status if x not in (0, cudart.cudaError_t.cudaSuccess)]
+    if bad:
+        raise RuntimeError(f"end-to-end loop: {len(bad)} failing calls, first {bad[0]}")
+    for ev in ev_copied + ev_used:
+        cudart.cudaEventDestroy(ev)
     losses = host_loss.tolist()
     assert len(losses) == E and all(math.isfinite(x) and x > 0 for x in losses)
     e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
