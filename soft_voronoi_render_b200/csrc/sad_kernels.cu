@@ -9,8 +9,15 @@
 //   propagate_kernel    a2/a3  one Jacobi candidate pass (+ injection)
 //   render_kernel       a4  softmax blend of the current candidates
 //   render_bwd_kernel   a4-a6  render + MSE + analytic backward with a per-tile
-//                       shared-memory hash reduction of site gradients
+//                       shared-memory hash reduction of site gradients (or,
+//                       deterministic, 64-bit fixed-point integer atomics
+//                       finished by fixed_to_grads_kernel)
 //   adam_kernel         a7  Adam step + a1 for the updated sites
+//   jfa3x3_kernel       optional 3x3 flood prepass (summary B.3)
+//   tau_diffuse_kernel  Jacobi step on the ln tau gradients (summary B.6)
+//   target_u8_kernel    8-bit RGB -> planar float32 target
+// The fused steady-state pass is in sad_fused.cu, budget control in
+// sad_densify.cu, the 16-byte site record in sad_pack.cu.
 #include "sad_device.cuh"
 #include "sad_launch.h"
 
