@@ -397,10 +397,13 @@ const char *sad_last_error(const sad_ctx *ctx);
  *   loss     one device double, receives L
  * Pointers 16-byte aligned (loss 8-byte).  Returns SAD_ERR_CAPACITY when
  * ceil(W/32) * ceil(H/8) exceeds (SAD_NOALLOC_SCRATCH_BYTES - 256) / 8 =
- * 131,040 tiles (4096 x 8192 fits), SAD_ERR_INVALID_ARG for bad sizes or
- * pointers, SAD_ERR_CUDA when a CUDA call fails.  The first call on a device
- * looks up the array's device address (a one-time set-up): make that first
- * call before capturing a stream.  All calls on a device share the one
+ * 131,040 tiles (4096 x 8192 fits) or ceil(H/8) exceeds 65,535 (the launch
+ * limit on tile rows), SAD_ERR_INVALID_ARG for bad sizes or pointers,
+ * SAD_ERR_CUDA when a CUDA call fails.  The first call on a device looks up
+ * the array's device address and keeps it for the process (a one-time
+ * set-up): make that first call before capturing a stream, and do not call
+ * this entry point on a device again after cudaDeviceReset, which leaves the
+ * kept address stale.  All calls on a device share the one
  * array, which keeps the previous call's contents (each call clears what must
  * start at zero): calls that may overlap on the GPU -- on different streams,
  * or from several threads -- race on it and must be serialised by the

@@ -8,6 +8,7 @@
 // keeps the backward pass's scratch (a 256-byte counter block and one double
 // per 32 x 8 tile for the loss partials) in a file-scope device array that the
 // library owns for the life of the process, on every GPU that loads it.
+#include <atomic>
 #include <cstdint>
 
 #include "sad.h"
@@ -19,11 +20,17 @@ namespace {
 constexpr size_t kScratchBytes = SAD_NOALLOC_SCRATCH_BYTES;
 constexpr int kTileX = 32, kTileY = 8;  // the tile of the render + backward kernel
 constexpr int kMaxDevices = 64;
+constexpr int kMaxGridY = 65535;  // launch limit on the tile rows (gridDim.y)
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-// device address of g_noalloc_scratch per device, filled on first use
-void *g_scratch_addr[kMaxDevices] = {};
+// Device address of g_noalloc_scratch per device ordinal, filled on the first
+// call on that device.  Threads that make a first call at the same time look
+// the address up each and store the same value, so a relaxed atomic suffices.
+// The address belongs to the device's primary context: after a
+// cudaDeviceReset it is stale and the process must not call this entry point
+// again on that device.
+std::atomic<void *> g_scratch_addr[kMaxDevices];
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -39,19 +46,22 @@ extern "C" int sad_backward_noalloc(int H, int W, int N_cap, const float *record
         return SAD_ERR_INVALID_ARG;
     const size_t tiles = (size_t)((W + kTileX - 1) / kTileX) * (size_t)((H + kTileY - 1) / kTileY);
     if (sad::COUNTERS_BYTES + tiles * sizeof(double) > kScratchBytes) return SAD_ERR_CAPACITY;
+    if ((H + kTileY - 1) / kTileY > kMaxGridY) return SAD_ERR_CAPACITY;
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SAD_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return SAD_ERR_UNSUPPORTED;
-    if (!g_scratch_addr[dev]) {
+    void *scratch = g_scratch_addr[dev].load(std::memory_order_relaxed);
+    if (!scratch) {
         // host code only sees a stand-in for the array: ask for its address on
         // this device (a one-time set-up; do it before any stream capture)
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SAD_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+        if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || !scratch) return SAD_ERR_CUDA;
+        g_scratch_addr[dev].store(scratch, std::memory_order_relaxed);
     }
-    void *scratch = g_scratch_addr[dev];
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // a launch error read below must be this call's own, not one left pending
+    // by earlier work of the caller
+    (void)cudaGetLastError();
 
     // the array keeps the previous call's contents: the counters (current
     // table 0, last-tile ticket, statistics) must start at zero

@@ -135,3 +135,19 @@ def test_product_path_has_no_oracle_dependency():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "sad_oracle" not in txt and "orc_" not in txt, f
+
+
+def test_backward_noalloc_rejects_sizes_before_any_cuda_call():
+    """The allocation-free backward checks sizes and pointers on the host and
+    returns before touching the GPU: too many tiles for its fixed scratch, or
+    more tile rows than a launch allows, give SAD_ERR_CAPACITY."""
+    fake = [0x10000, 0x20000, 0x30000, None, 0x40000, 0x50000]  # records, table, target, image, grads, loss
+    for H, W, want in ((8200, 4200, _lib.SAD_ERR_CAPACITY),      # 131,200 tiles of 32 x 8
+                       (600_000, 1, _lib.SAD_ERR_CAPACITY),      # 75,000 tiles but 75,000 tile rows
+                       (0, 8, _lib.SAD_ERR_INVALID_ARG)):
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_backward_noalloc(H, W, 16, *fake)
+        assert e.value.status == want, (H, W)
+    with pytest.raises(_lib.SadError) as e:
+        _lib.sad_backward_noalloc(64, 64, 16, 0x10004, *fake[1:])  # misaligned records
+    assert e.value.status == _lib.SAD_ERR_INVALID_ARG
