@@ -68,6 +68,10 @@ def lib():
         L.orc_pack_ranges.argtypes = [c_int, vp, vp]
         L.orc_pack_sites.argtypes = [c_int, c_int, c_int, vp, vp, vp]
         L.orc_unpack_sites.argtypes = [c_int, c_int, c_int, vp, vp, vp]
+        L.orc_to_binary16.argtypes = [ctypes.c_float]
+        L.orc_to_binary16.restype = ctypes.c_float
+        L.orc_cand16_record.argtypes = [c_int, vp, vp]
+        L.orc_rescore_sort_cell.argtypes = [c_int, c_int, c_int, c_int, vp, vp]
         L.orc_num_threads.restype = c_int
         L.orc_set_threads.argtypes = [c_int]
         _lib = L
@@ -160,16 +164,44 @@ def inject_ids(seed: int, pass_index: int, pixel: int, N: int, G: int) -> np.nda
     return out[:G]
 
 
+def to_binary16(x: float) -> float:
+    """x rounded to the nearest IEEE binary16 value (ties to even), as a float."""
+    return float(lib().orc_to_binary16(float(x)))
+
+
+def cand16_record(rec32: np.ndarray) -> np.ndarray:
+    """The candidate-selection record of the packed candidate-site mode:
+    the float32 record with A, B, C and b rounded to binary16."""
+    rec32 = _f32(rec32)
+    out = np.empty_like(rec32)
+    lib().orc_cand16_record(rec32.shape[0], _p(rec32), _p(out))
+    return out
+
+
+def rescore_sort(H: int, W: int, rec32: np.ndarray, table: np.ndarray, cell: int = 1) -> np.ndarray:
+    """Each list re-scored with the float32 record, in (logit desc, id asc) order."""
+    rec32 = _f32(rec32)
+    GH, GW = grid_dims(H, W, cell)
+    t = _u32(table).reshape(GH * GW, K).copy()
+    lib().orc_rescore_sort_cell(GH, GW, cell, rec32.shape[0], _p(rec32), _p(t))
+    return t
+
+
 def propagate(H: int, W: int, rec32: np.ndarray, table: np.ndarray, jump: int, G: int,
-              seed: int, pass_index: int, cell: int = 1) -> np.ndarray:
+              seed: int, pass_index: int, cell: int = 1, cand16: bool = False) -> np.ndarray:
     """One Jacobi propagation pass on the candidate grid of an H x W image;
-    returns the new (cells, 8) table."""
+    returns the new (cells, 8) table.  With cand16 the candidates are ranked
+    on the packed candidate-site record (cand16_record) and the kept 8 are
+    re-scored in float32 (rescore_sort)."""
     rec32 = _f32(rec32)
     GH, GW = grid_dims(H, W, cell)
     tin = _u32(table).reshape(GH * GW, K)
     tout = np.empty_like(tin)
-    lib().orc_propagate_cell(GH, GW, cell, rec32.shape[0], _p(rec32), _p(tin), _p(tout), int(jump), int(G),
+    sel = cand16_record(rec32) if cand16 else rec32
+    lib().orc_propagate_cell(GH, GW, cell, rec32.shape[0], _p(sel), _p(tin), _p(tout), int(jump), int(G),
                              seed & 0xFFFFFFFF, pass_index & 0xFFFFFFFF)
+    if cand16:
+        lib().orc_rescore_sort_cell(GH, GW, cell, rec32.shape[0], _p(rec32), _p(tout))
     return tout
 
 
@@ -194,14 +226,15 @@ def jump_schedule(H: int, W: int) -> list:
     return out
 
 
-def refresh(H: int, W: int, params: np.ndarray, G: int, seed: int, first_pass: int = 0, cell: int = 1):
+def refresh(H: int, W: int, params: np.ndarray, G: int, seed: int, first_pass: int = 0, cell: int = 1,
+            cand16: bool = False):
     """Seed pass then one propagation pass per jump of ``jump_schedule`` of
     the candidate grid.  Returns (table, number of passes run)."""
     rec = records(H, W, params)
     t = seed_table(H, W, params, cell)
     n = 0
     for k in jump_schedule(*grid_dims(H, W, cell)):
-        t = propagate(H, W, rec, t, k, G, seed, first_pass + n, cell)
+        t = propagate(H, W, rec, t, k, G, seed, first_pass + n, cell, cand16=cand16)
         n += 1
     return t, n
 

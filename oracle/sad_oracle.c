@@ -340,6 +340,66 @@ void orc_propagate_cell(int H, int W, int cell, int N, const float *rec32, const
 }
 
 /*
+ * Packed candidate sites ([P1] B.2: candidate-update kernels score from a
+ * compact 16-byte per-site buffer of float16 pairs; the kept lists are then
+ * used by the float32 renderer).  Reading of this build: the record keeps
+ * the position in float32 (a binary16 position steps by 1-2 px between 2048
+ * and 4096 px) and the score coefficients A, B, C and b as binary16 values;
+ * the candidate update ranks candidates by the logit evaluated in the
+ * float32 order above from those rounded coefficients, and the kept 8 are
+ * re-scored with the float32 record and stored in (float32 logit desc, id
+ * asc) order.
+ */
+
+/* x rounded to the nearest IEEE 754 binary16 value (ties to even; overflow
+ * to infinity), returned as the float32 value it equals.  binary16 has an
+ * 11-bit significand and exponents -14..15, with subnormals down to 2^-24:
+ * the spacing of values near |x| is 2^(floor(log2 |x|) - 10), never below
+ * 2^-24; the largest finite value is 65504 and |x| >= 65520 rounds to inf. */
+static float to_binary16(float x)
+{
+    if (x != x) return x;
+    const float ax = fabsf(x);
+    if (ax >= 65520.0f) return copysignf(INFINITY, x);
+    int e;
+    frexpf(ax, &e); /* ax = m 2^e, 0.5 <= m < 1 */
+    int qe = (e - 1) - 10;
+    if (qe < -24) qe = -24;
+    const float quantum = ldexpf(1.0f, qe);
+    const float r = nearbyintf(ax / quantum) * quantum; /* default rounding: to nearest, ties to even */
+    return copysignf(r, x);
+}
+
+float orc_to_binary16(float x) { return to_binary16(x); }
+
+/* the selection record: rec32 with A, B, C and b rounded to binary16 */
+void orc_cand16_record(int N, const float *rec32, float *rec_sel)
+{
+    for (int64_t i = 0; i < (int64_t)N * ORC_REC; ++i) rec_sel[i] = rec32[i];
+    for (int i = 0; i < N; ++i)
+        for (int f = 2; f <= 5; ++f) rec_sel[(size_t)i * ORC_REC + f] = to_binary16(rec32[(size_t)i * ORC_REC + f]);
+}
+
+/* re-score every kept list with the float32 record and store it in
+ * (logit desc, id asc) order; sentinels stay last */
+void orc_rescore_sort_cell(int GH, int GW, int cell, int N, const float *rec32, uint32_t *table)
+{
+    const int64_t P = (int64_t)GH * GW;
+#pragma omp parallel for schedule(dynamic, 256)
+    for (int64_t p = 0; p < P; ++p) {
+        const float fx = cell_centre((int)(p % GW), cell), fy = cell_centre((int)(p / GW), cell);
+        topk_t t;
+        topk_clear(&t);
+        for (int q = 0; q < ORC_K; ++q) {
+            const uint32_t id = table[p * ORC_K + q];
+            if (id == ORC_SENTINEL || id >= (uint32_t)N) continue;
+            topk_insert(&t, score32(rec32 + (size_t)id * ORC_REC, fx, fy), id);
+        }
+        topk_store(&t, table + p * ORC_K);
+    }
+}
+
+/*
  * Seed pass ([P1] B.3: the JFA prepass starts with a seed pass): clear the
  * table to the sentinel, then every active site whose position lies in the
  * image writes its id to slot 0 of the pixel containing it; the smallest id
