@@ -35,6 +35,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "Mpix/s per fit iter (top-K prop+render+bwd+Adam), 2048² N=128K; % HBM roof"
 WORKLOAD = "c3"
+# the workload's own set-up before any timed or warm-up step: a full refresh
+# and 50 fitting iterations, so that the timed iterations are steady-state
+# ones whatever --warmup is
+SETUP_ITERS = 50
 ADAM_LR = dict(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=5e-3, lr_theta=1e-3, lr_a=1e-3)
 
 # Algorithmic DRAM bytes (compulsory traffic) per launch, per pixel and per site.
@@ -59,10 +63,13 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
-    ap.add_argument("--workload", default="c3", choices=["c3", "c4", "c5", "rows"],
-                    help="c3: the fitting-iteration metric (default); c4: full candidate refresh + render at "
-                         "4096x4096, N=524,288; c5: end-to-end 768x512 fit with densify/prune (secondary "
-                         "measurements)")
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5", "rows"],
+                    help="c3: the fitting-iteration metric (default); c1: 256x256 N=1,024 exact top-K + "
+                         "render + backward + Adam; c2: 768x512 N=50,000 refresh + 200 fit iterations timed "
+                         "whole; c4: full candidate refresh + render at 4096x4096, N=524,288; c5: end-to-end "
+                         "768x512 fit with densify/prune (secondary measurements, each with the oracle beside)")
+    ap.add_argument("--oracle-iters", type=int, default=200,
+                    help="c2: fit iterations the oracle runs on all host cores (1 core: a tenth)")
     ap.add_argument("--oracle-fit", action="store_true", help="c5: also run the CPU oracle's fit (minutes)")
     ap.add_argument("--cell", type=int, default=1,
                     help="c4/c5: candidate lists on a grid of cell x cell pixel cells (1: per pixel)")
@@ -339,7 +346,7 @@ def run_ours(args):
         if ev is not None:
             ev[2].record(stream)
 
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(SETUP_ITERS + max(args.warmup, 3)):
         step()
     torch.cuda.synchronize(dev)
 
@@ -371,12 +378,24 @@ def run_ours(args):
     ms_step = ms_max / K
     value = aggregate_mpix(world, P, K, ms_max)
 
-    # end to end through the C ABI: host target copied in, loss read back
+    # end to end through the C ABI: each step's target comes from pinned host
+    # memory and each step's loss goes back to pinned host memory
     E = max(1, min(args.e2e_steps, K))
     host_tgt = torch.from_numpy(np.ascontiguousarray(tgt)).pin_memory()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
+    from cuda.bindings import runtime as cudart
+    L = _lib.load()
+    h2d = cudart.cudaMemcpyKind.cudaMemcpyHostToDevice
+    copy_stream = torch.cuda.Stream(dev)
+    cs_h, ms_h = copy_stream.cuda_stream, stream.cuda_stream
+    status = []
+
+    def sync_all():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # (a) serial: set the target, one iteration, read the loss (host waits)
+    sync_all()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -388,98 +407,87 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_serial_ms = reduce_max(e0.elapsed_time(e1), dev)
 
-    # the same, with each step's target copied into one of two device buffers
-    # on a copy stream while the previous step computes (sad_bind_target)
-    bufs = [torch.empty_like(s.target), torch.empty_like(s.target)]
-    copy_stream = torch.cuda.Stream(dev)
-    copied = [torch.cuda.Event(), torch.cuda.Event()]
-    used = [torch.cuda.Event(), torch.cuda.Event()]
-    for ev in used:
-        ev.record(stream)
+    def pipelined(src, nbytes, bufs, per_step):
+        """Each step's input copied host -> device on a copy stream into one
+        of two device buffers while the previous step computes; per_step(b)
+        issues the step on the compute stream; each step's loss is copied
+        into its own slot of pinned host memory in stream order (no host
+        wait).  Copies and stream dependencies go through the CUDA runtime
+        directly: a few microseconds of host time per step."""
+        no_timing = cudart.cudaEventDisableTiming
+        ev_copied = [cudart.cudaEventCreateWithFlags(no_timing)[1] for _ in range(2)]
+        ev_used = [cudart.cudaEventCreateWithFlags(no_timing)[1] for _ in range(2)]
+        host_loss = torch.zeros(E, dtype=torch.float64).pin_memory()
+        loss0 = host_loss.data_ptr()
+        for ev in ev_used:
+            status.append(cudart.cudaEventRecord(ev, ms_h)[0])
 
-    def issue_copy(k):
-        b = k % 2
-        copy_stream.wait_event(used[b])  # the step that last read this buffer is done
-        with torch.cuda.stream(copy_stream):
-            bufs[b].copy_(host_tgt, non_blocking=True)
-        copied[b].record(copy_stream)
+        def issue_copy(k):
+            b = k % 2
+            status.append(cudart.cudaStreamWaitEvent(cs_h, ev_used[b], 0)[0])
+            status.append(cudart.cudaMemcpyAsync(bufs[b], src, nbytes, h2d, cs_h)[0])
+            status.append(cudart.cudaEventRecord(ev_copied[b], cs_h)[0])
 
-    host_loss32 = torch.zeros(E, dtype=torch.float64).pin_memory()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    issue_copy(0)
-    for k in range(E):
-        if k + 1 < E:
-            issue_copy(k + 1)
-        stream.wait_event(copied[k % 2])
-        _lib.sad_bind_target(ctx, bufs[k % 2].data_ptr())
-        _lib.sad_fit_iteration(ctx, G, cfg, sp)
-        used[k % 2].record(stream)
-        _lib.sad_copy_loss(ctx, host_loss32[k].data_ptr(), sp)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    _lib.sad_bind_target(ctx, s.target.data_ptr())
-    e2e_f32_ms = reduce_max(e0.elapsed_time(e1), dev)
+        sync_all()
+        e0.record(stream)
+        issue_copy(0)
+        for k in range(E):
+            if k + 1 < E:
+                issue_copy(k + 1)
+            b = k % 2
+            status.append(cudart.cudaStreamWaitEvent(ms_h, ev_copied[b], 0)[0])
+            per_step(b, ev_used[b])
+            status.append(L.sad_copy_loss(ctx, loss0 + 8 * k, sp))
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        for ev in ev_copied + ev_used:
+            cudart.cudaEventDestroy(ev)
+        losses = host_loss.tolist()
+        assert len(losses) == E and all(math.isfinite(x) and x > 0 for x in losses)
+        return reduce_max(e0.elapsed_time(e1), dev)
 
-    # the same pipeline with the target streamed as 8-bit RGB, the format of
-    # the photographs the method fits (the same image rounded to 1/255),
-    # converted on the device by sad_set_target_u8
+    # (b) the workload's float32 target, bound in place (sad_bind_target)
+    bufs32 = [torch.empty_like(s.target), torch.empty_like(s.target)]
+    ptr32 = [b.data_ptr() for b in bufs32]
+
+    def step32(b, ev_used):
+        status.append(L.sad_bind_target(ctx, ptr32[b]))
+        status.append(L.sad_fit_iteration(ctx, G, ctypes.byref(cfg), sp))
+        status.append(cudart.cudaEventRecord(ev_used, ms_h)[0])
+
+    e2e_f32_ms = pipelined(host_tgt.data_ptr(), host_tgt.numel() * 4, ptr32, step32)
+    status.append(L.sad_bind_target(ctx, s.target.data_ptr()))
+
+    # (c) the same image streamed as 8-bit RGB (the format of the photographs
+    # the method fits; the image rounded to 1/255), converted on the device
+    # by sad_set_target_u8 into the bound float target
     host_u8 = torch.from_numpy(np.ascontiguousarray(
         np.clip(np.rint(tgt * 255.0), 0, 255).astype(np.uint8).transpose(1, 2, 0))).pin_memory()
     bufs8 = [torch.empty(host_u8.shape, dtype=torch.uint8, device=dev) for _ in range(2)]
-    # each step's loss is copied to its own slot of pinned host memory in
-    # stream order (one device -> host transfer per step, no host wait)
-    host_loss = torch.zeros(E, dtype=torch.float64).pin_memory()
-    # the loop issues its copies and stream dependencies through the CUDA
-    # runtime directly: a few microseconds of host time per step
-    from cuda.bindings import runtime as cudart
-    L = _lib.load()
-    no_timing = cudart.cudaEventDisableTiming
-    ev_copied = [cudart.cudaEventCreateWithFlags(no_timing)[1] for _ in range(2)]
-    ev_used = [cudart.cudaEventCreateWithFlags(no_timing)[1] for _ in range(2)]
-    cs_h, ms_h = copy_stream.cuda_stream, stream.cuda_stream
-    h2d = cudart.cudaMemcpyKind.cudaMemcpyHostToDevice
-    src, nbytes = host_u8.data_ptr(), host_u8.numel()
-    dst = [b.data_ptr() for b in bufs8]
-    loss0 = host_loss.data_ptr()
-    status = []
-    for ev in ev_used:
-        status.append(cudart.cudaEventRecord(ev, ms_h)[0])
+    ptr8 = [b.data_ptr() for b in bufs8]
 
-    def issue_copy8(k):
-        b = k % 2
-        status.append(cudart.cudaStreamWaitEvent(cs_h, ev_used[b], 0)[0])
-        status.append(cudart.cudaMemcpyAsync(dst[b], src, nbytes, h2d, cs_h)[0])
-        status.append(cudart.cudaEventRecord(ev_copied[b], cs_h)[0])
-
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    issue_copy8(0)
-    for k in range(E):
-        if k + 1 < E:
-            issue_copy8(k + 1)
-        b = k % 2
-        status.append(cudart.cudaStreamWaitEvent(ms_h, ev_copied[b], 0)[0])
-        status.append(L.sad_set_target_u8(ctx, dst[b], sp))
-        status.append(cudart.cudaEventRecord(ev_used[b], ms_h)[0])
+    def step8(b, ev_used):
+        status.append(L.sad_set_target_u8(ctx, ptr8[b], sp))
+        status.append(cudart.cudaEventRecord(ev_used, ms_h)[0])
         status.append(L.sad_fit_iteration(ctx, G, ctypes.byref(cfg), sp))
-        status.append(L.sad_copy_loss(ctx, loss0 + 8 * k, sp))
-    e1.record(stream)
+
+    e2e_u8_ms = pipelined(host_u8.data_ptr(), host_u8.numel(), ptr8, step8)
+
+    # the host link alone: the float32 target copied E times on the copy stream
+    sync_all()
+    c0 = torch.cuda.Event(enable_timing=True)
+    c1 = torch.cuda.Event(enable_timing=True)
+    c0.record(copy_stream)
+    for k in range(E):
+        status.append(cudart.cudaMemcpyAsync(ptr32[k % 2], host_tgt.data_ptr(), host_tgt.numel() * 4, h2d, cs_h)[0])
+    c1.record(copy_stream)
     torch.cuda.synchronize(dev)
+    h2d_ms = c0.elapsed_time(c1) / E
     bad = [x for x in status if x not in (0, cudart.cudaError_t.cudaSuccess)]
     if bad:
         raise RuntimeError(f"end-to-end loop: {len(bad)} failing calls, first {bad[0]}")
-    for ev in ev_copied + ev_used:
-        cudart.cudaEventDestroy(ev)
-    losses = host_loss.tolist()
-    assert len(losses) == E and all(math.isfinite(x) and x > 0 for x in losses)
-    e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
-    e2e_value = aggregate_mpix(world, P, E, e2e_ms)
-    e2e_f32 = aggregate_mpix(world, P, E, e2e_f32_ms)
+    e2e_value = aggregate_mpix(world, P, E, e2e_f32_ms)
+    e2e_u8 = aggregate_mpix(world, P, E, e2e_u8_ms)
     e2e_serial = aggregate_mpix(world, P, E, e2e_serial_ms)
     st = s.stats()
 
@@ -494,7 +502,7 @@ def run_ours(args):
         iter_bytes = ITER_BYTES_PX * P + ITER_BYTES_SITE * N
         line = {
             "metric": METRIC, "value": value, "unit": "Mpix/s", "n_gpus": world, "steps": K,
-            "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": max(args.warmup, 3), "setup_iterations": SETUP_ITERS, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(wl, world),
             "hbm_roof_frac_iter": (iter_bytes / (ms_step * 1e-3) / 1e9) / hbm,
@@ -504,14 +512,17 @@ def run_ours(args):
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
                          "algorithmic_bytes": alg_bytes},
             "issue_roofline": issue_roofline(dom, avg[dom], clocks),
-            "e2e": {"value": e2e_value, "unit": "Mpix/s", "h2d_bytes_per_step": int(host_u8.numel()),
+            "e2e": {"value": e2e_value, "unit": "Mpix/s", "h2d_bytes_per_step": int(host_tgt.numel() * 4),
                     "d2h_bytes_per_step": 8, "steps": E,
-                    "how": "per step: the step's 8-bit RGB target, pinned host -> device on a copy stream "
-                           "(double-buffered, overlapping the previous step), sad_set_target_u8, "
-                           "sad_fit_iteration, sad_copy_loss into that step's slot of pinned host memory; "
-                           "the host reads the losses after the last step",
-                    "f32_value": e2e_f32, "f32_h2d_bytes_per_step": int(host_tgt.numel() * 4),
-                    "f32_serial_value": e2e_serial},
+                    "how": "per step: the step's float32 target (the workload's own), pinned host -> device on a "
+                           "copy stream (double-buffered, overlapping the previous step), sad_bind_target, "
+                           "sad_fit_iteration, sad_copy_loss into that step's slot of pinned host memory; the "
+                           "host reads the losses after the last step",
+                    "h2d_ms_per_step": h2d_ms,
+                    "h2d_gbs": host_tgt.numel() * 4 / (h2d_ms * 1e-3) / 1e9,
+                    "bound_by": "host link" if h2d_ms > ms_step else "device",
+                    "serial_value": e2e_serial,
+                    "u8_value": e2e_u8, "u8_h2d_bytes_per_step": int(host_u8.numel())},
             "gpu_launches": 2 * K,  # timed region: one fused pass + one Adam launch per step
             "clocks": clocks,
             "device_stats": {k: st[k] for k in ("hash_overflow", "empty_pixels", "dropped_ids")},
@@ -653,6 +664,154 @@ def run_fit(args):
     return 0
 
 
+def time_oracle_c2(prm, tgt, wl, iters: int, threads: int | None):
+    """The oracle's c2 pipeline (refresh, then iterations of propagate k = 1,
+    render + backward in double, Adam, records) on `threads` host threads
+    (None: all); returns (seconds, iterations, threads used)."""
+    import oracle
+    all_threads = oracle.num_threads()
+    if threads is not None:
+        oracle.set_threads(threads)
+    try:
+        lr = dict(pos=1e-3, log_tau=1e-3, r=1e-3, color=5e-3, theta=1e-3, a=1e-3)
+        t0 = time.perf_counter()
+        oracle.refresh(wl.H, wl.W, prm, wl.G, 1, 0)
+        t_ref = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        oracle.fit(wl.H, wl.W, prm, tgt, wl.N, iters, (), 0, 0.0, lr, wl.G, 1)
+        t_fit = time.perf_counter() - t0 - t_ref  # oracle.fit refreshes first
+        return t_ref, max(t_fit, 0.0), iters, oracle.num_threads()
+    finally:
+        oracle.set_threads(all_threads)
+
+
+def run_c2(args):
+    """768 x 512, N = 50,000 (the Kodak-shaped workload): seed + refresh at
+    jumps 256..1 with G = 2, then 200 fitting iterations (propagation k = 1,
+    G = 2, render, backward, Adam), timed whole on the GPU; the oracle runs
+    the same pipeline on all host cores and on one core."""
+    import torch
+    import synth
+    from soft_voronoi_render_b200 import Sad, _lib
+
+    tgt, prm, wl = synth.make_workload("c2", seed=1)
+    P, ITER = wl.H * wl.W, 200
+    cfg = _lib.adam_cfg(**ADAM_LR)
+    runs = []
+    for rep in range(max(args.warmup, 1) + 3):
+        s = Sad(wl.H, wl.W, wl.N, seed=1)
+        s.set_sites(prm)
+        s.set_target(tgt)
+        stream = torch.cuda.current_stream()
+        sp = stream.cuda_stream
+        torch.cuda.synchronize()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        _lib.sad_refresh(s.ctx, wl.G, sp)
+        e[1].record(stream)
+        for _ in range(ITER):
+            _lib.sad_fit_iteration(s.ctx, wl.G, cfg, sp)
+        e[2].record(stream)
+        torch.cuda.synchronize()
+        runs.append((e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), s.loss()))
+        s.close()
+    timed = runs[max(args.warmup, 1):]
+    ref_ms = statistics.median(r[0] for r in timed)
+    fit_ms = statistics.median(r[1] for r in timed)
+    line = {"metric": "768x512 N=50,000: refresh + 200 fit iterations, timed whole", "value": ref_ms + fit_ms,
+            "unit": "ms", "higher_is_better": False, "n_gpus": 1, "repeats": len(timed), "refresh_ms": ref_ms,
+            "fit_200_ms": fit_ms, "mpix_per_s_per_iter": P * ITER / (fit_ms * 1e-3) / 1e6,
+            "final_loss": timed[-1][2], "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"c2: {wl.description}", "H": wl.H, "W": wl.W, "N": wl.N, "G": wl.G,
+                       "l2": "working set (~60 MB) is L2-resident; HBM fractions are not meaningful here"}}
+    if not args.no_cpu_baseline:
+        oracle_runs = {}
+        for label, threads, iters in (("all_cores", None, args.oracle_iters),
+                                      ("one_core", 1, max(1, args.oracle_iters // 10))):
+            t_ref, t_fit, n, used = time_oracle_c2(prm, tgt, wl, iters, threads)
+            oracle_runs[label] = {"cores": used, "refresh_s": t_ref, "iterations": n, "fit_s": t_fit,
+                                  "s_per_iter": t_fit / n, "mpix_per_s_per_iter": P * n / t_fit / 1e6,
+                                  "whole_200_s_extrapolated": t_ref + t_fit / n * ITER}
+        line["cpu_baseline"] = {"kind": "oracle", **oracle_runs}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_c1(args):
+    """256 x 256, N = 1,024: exact brute-force top-K, render, MSE backward and
+    one Adam step (lr 1e-3), each timed on the GPU with CUDA events (the
+    exact top-K lists become the context's lists through sad_set_table,
+    untimed); the oracle times the same four steps on all host cores and on
+    one core."""
+    import torch
+    import synth
+    from soft_voronoi_render_b200 import Sad, _lib
+
+    tgt, prm, wl = synth.make_workload("c1", seed=1)
+    P = wl.H * wl.W
+    s = Sad(wl.H, wl.W, wl.N, seed=1)
+    s.set_sites(prm)
+    s.set_target(tgt)
+    cfg = _lib.adam_cfg()
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    out = torch.empty((P, 8), dtype=torch.int32, device=s.device)
+    reps = max(5, min(args.steps, 50))
+    acc = {"topk_exact": [], "render": [], "backward": [], "adam": []}
+    for rep in range(reps + 2):
+        s.set_sites(prm)
+        torch.cuda.synchronize()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        _lib.sad_topk_exact(s.ctx, None, P, out, sp)
+        e[1].record(stream)
+        torch.cuda.synchronize()
+        s.set_table(out.cpu().numpy().view(np.uint32))
+        f = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        f[0].record(stream)
+        _lib.sad_render(s.ctx, None, sp)
+        f[1].record(stream)
+        _lib.sad_backward(s.ctx, 0, sp)
+        f[2].record(stream)
+        _lib.sad_adam_step(s.ctx, cfg, sp)
+        f[3].record(stream)
+        torch.cuda.synchronize()
+        if rep >= 2:
+            acc["topk_exact"].append(e[0].elapsed_time(e[1]))
+            for k, (a, b) in zip(("render", "backward", "adam"), ((0, 1), (1, 2), (2, 3))):
+                acc[k].append(f[a].elapsed_time(f[b]))
+    ms = {k: statistics.median(v) for k, v in acc.items()}
+    total = sum(ms.values())
+    line = {"metric": "256x256 N=1,024: exact top-K + render + backward + one Adam step", "value": total,
+            "unit": "ms", "higher_is_better": False, "n_gpus": 1, "repeats": reps, "kernels_ms": ms,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"c1: {wl.description}", "H": wl.H, "W": wl.W, "N": wl.N}}
+    s.close()
+    if not args.no_cpu_baseline:
+        import oracle
+        all_threads = oracle.num_threads()
+        runs = {}
+        for label, threads in (("all_cores", all_threads), ("one_core", 1)):
+            oracle.set_threads(threads)
+            t0 = time.perf_counter()
+            rec = oracle.records(wl.H, wl.W, prm)
+            table = oracle.topk_exact(wl.H, wl.W, rec)
+            t1 = time.perf_counter()
+            oracle.render(wl.H, wl.W, prm, table)
+            t2 = time.perf_counter()
+            L, g = oracle.loss_backward(wl.H, wl.W, prm, table, tgt)
+            t3 = time.perf_counter()
+            oracle.adam(wl.H, wl.W, prm.astype(np.float64), np.zeros((9, wl.N)), np.zeros((9, wl.N)), g,
+                        dict(pos=1e-3, log_tau=1e-3, r=1e-3, color=1e-3, theta=1e-3, a=1e-3), 1)
+            t4 = time.perf_counter()
+            runs[label] = {"cores": oracle.num_threads(), "topk_exact_s": t1 - t0, "render_s": t2 - t1,
+                           "backward_s": t3 - t2, "adam_s": t4 - t3, "total_s": t4 - t0}
+        oracle.set_threads(all_threads)
+        line["cpu_baseline"] = {"kind": "oracle", **runs}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_rows(args):
     """Every entry point of the path timed on its own at 2048 x 2048,
     N = 131,072 (exact top-K on the 256 x 256, N = 1,024 workload), with the
@@ -753,6 +912,8 @@ def main():
     args = parse()
     if args.workload == "rows":
         return run_rows(args)
+    if args.workload in ("c1", "c2") and args.impl == "ours":
+        return run_c1(args) if args.workload == "c1" else run_c2(args)
     if args.workload == "c5" and args.impl == "ours":
         return run_fit(args)
     if args.impl == "reference":

@@ -93,6 +93,8 @@ typedef struct sad_buffers {
     float *stats; /* optional [6][N_cap]: budget-control statistics (SAD_STATS, sad_densify_prune) */
     const uint8_t *frozen; /* optional [N_cap]: non-zero = frozen site, left untouched by Adam
                               ([P1] section 7: boundary sites excluded from gradient updates) */
+    void *cand16;          /* optional [N_cap] x 16 bytes, 16-byte aligned: packed candidate-site
+                              records (sad_set_candidate_precision) */
 } sad_buffers;
 
 /* sad_backward flag: also accumulate the budget-control statistics into
@@ -145,7 +147,7 @@ typedef struct sad_stats {
     uint32_t n_active;         /* active sites before the last densify event */
     uint32_t n_split;          /* sites split by the last densify event */
     uint32_t n_pruned;         /* sites pruned by the last densify event */
-    uint32_t reserved2;
+    uint32_t check_failures;   /* debug build (libsad_checks): accesses a bounds check refused */
 } sad_stats;
 
 /* Bytes of workspace the caller must bind for an H x W image and N_cap sites. */
@@ -368,6 +370,49 @@ int sad_set_table(sad_ctx *ctx, const uint32_t *src, sad_stream_t stream);
 
 /* Read the statistics block (synchronises the stream). */
 int sad_get_stats(sad_ctx *ctx, sad_stats *out, sad_stream_t stream);
+
+/* Candidate precision ([P1] B.2: candidate-update kernels score from a
+ * compact 16-byte per-site buffer of float16 pairs).  bits = 32 (the
+ * default): candidates are ranked by the float32 logit of the score record.
+ * bits = 16: every candidate update (sad_refresh, sad_propagate and the
+ * propagation of sad_fit_pass / sad_fit_iteration, which then runs as a
+ * propagation pass followed by the tile pass on the new lists) first packs
+ * each site into the bound cand16 buffer -- x and y as float32, then the
+ * binary16 pairs (A, B) and (C, b) (round to nearest even) -- ranks the
+ * candidates by the float32 logit evaluated from those rounded coefficients
+ * (the operation order of the score record), and re-scores the kept 8 with
+ * the float32 record, storing them in (float32 logit desc, id asc) order.
+ * The position stays float32 because binary16 steps by 1-2 px between 2048
+ * and 4096 px.  The JFA prepass and the exact top-K stay float32.  Errors:
+ * SAD_ERR_INVALID_ARG for other bits, SAD_ERR_NOT_BOUND for 16 without a
+ * bound cand16 buffer. */
+int sad_set_candidate_precision(sad_ctx *ctx, int bits, sad_stream_t stream);
+
+/* The fitting state that lives in the library's counter block: the pass
+ * counter that keys the injection randomness ([P1] B.3: xorshift state from
+ * the step index and pixel id), Adam's step count (bias correction) and the
+ * injection seed.  Everything else a fit needs is in caller-owned buffers:
+ * the sites (sad_get_sites / sad_set_sites), the Adam moments (the bound
+ * adam_m / adam_v) and the current candidate lists (sad_get_table /
+ * sad_set_table).  Saved together, they are a checkpoint from which a fit
+ * resumes as if it had not stopped (the pages keep the whole fit on the GPU
+ * and move only site data across the host boundary, [P1] B.7/B.8). */
+typedef struct sad_fit_state {
+    uint32_t pass_counter; /* propagation passes run so far */
+    uint32_t adam_step;    /* Adam steps taken so far */
+    uint32_t seed;         /* injection seed (as given to sad_reset) */
+    uint32_t reserved;     /* 0 */
+} sad_fit_state;
+
+/* Read the fit state (synchronises the stream).  SAD_ERR_INVALID_ARG for a
+ * NULL destination, SAD_ERR_NOT_BOUND before sad_bind. */
+int sad_get_fit_state(sad_ctx *ctx, sad_fit_state *out, sad_stream_t stream);
+
+/* Write the fit state, in stream order (the values travel by value, so
+ * *state may be released when the call returns).  Which table of the double
+ * buffer is current is not part of the state: sad_set_table writes the
+ * current one.  SAD_ERR_INVALID_ARG for NULL or a non-zero reserved field. */
+int sad_set_fit_state(sad_ctx *ctx, const sad_fit_state *state, sad_stream_t stream);
 
 /* Loss of the last backward pass, copied to host memory (synchronises). */
 int sad_get_loss(sad_ctx *ctx, double *loss, sad_stream_t stream);

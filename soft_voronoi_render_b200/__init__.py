@@ -52,13 +52,14 @@ class Sad:
         self.image = torch.zeros((3, self.H, self.W), **f32) if with_image else None
         self.site_stats = torch.zeros((6, self.N), **f32) if with_stats else None
         self.frozen = torch.zeros((self.N,), dtype=torch.uint8, device=self.device)
+        self.cand16 = torch.zeros((self.N, 4), dtype=torch.int32, device=self.device)
         self.ws_bytes = _lib.sad_workspace_bytes(self.H, self.W, self.N)
         self.workspace = torch.zeros(((self.ws_bytes + 255) // 256 * 256,), dtype=torch.uint8, device=self.device)
         self.ctx = _lib.sad_create(self.H, self.W, self.N, _lib.SAD_K)
         _lib.sad_bind(self.ctx, params=self.params, grads=self.grads, adam_m=self.adam_m, adam_v=self.adam_v,
                       records=self.records, table=self.table, target=self.target, image=self.image,
                       workspace=self.workspace, workspace_bytes=self.workspace.numel(), stats=self.site_stats,
-                      frozen=self.frozen)
+                      frozen=self.frozen, cand16=self.cand16)
         _lib.sad_reset(self.ctx, seed, self.stream)
 
     # the stream every call is issued on: torch's current stream
@@ -130,6 +131,12 @@ class Sad:
         _lib.sad_unpack_sites(self.ctx, src, r, self.stream)
         self.torch.cuda.current_stream(self.device).synchronize()
 
+    def set_candidate_precision(self, bits: int):
+        """32: candidates ranked by the float32 logit; 16: ranked on the
+        packed candidate-site records (binary16 coefficients), the kept 8
+        re-scored in float32."""
+        _lib.sad_set_candidate_precision(self.ctx, bits, self.stream)
+
     def set_candidate_grid(self, cell: int):
         """Lists on a ceil(H/cell) x ceil(W/cell) grid; the table starts empty."""
         _lib.sad_set_candidate_grid(self.ctx, cell, self.stream)
@@ -144,6 +151,28 @@ class Sad:
     def set_table(self, table: np.ndarray):
         src = np.ascontiguousarray(table, dtype=np.uint32).reshape(self.PT, 8)
         _lib.sad_set_table(self.ctx, src, self.stream)
+
+    def checkpoint(self) -> dict:
+        """Everything a fit needs to resume: site parameters, Adam moments,
+        the current candidate lists and the fit state (pass counter, Adam
+        step, injection seed), as host arrays."""
+        t = self.torch
+        t.cuda.current_stream(self.device).synchronize()
+        return {"params": self.params.cpu().numpy().copy(), "adam_m": self.adam_m.cpu().numpy().copy(),
+                "adam_v": self.adam_v.cpu().numpy().copy(), "table": self.get_table(),
+                "state": _lib.sad_get_fit_state(self.ctx, self.stream)}
+
+    def restore(self, ck: dict):
+        """Resume from a checkpoint() of a context of the same sizes; the
+        score records are rebuilt from the parameters."""
+        t = self.torch
+        for name in ("params", "adam_m", "adam_v"):
+            getattr(self, name).copy_(t.from_numpy(np.ascontiguousarray(ck[name])).to(self.device))
+        st = ck["state"]
+        _lib.sad_set_fit_state(self.ctx, st["pass_counter"], st["adam_step"], st["seed"], self.stream)
+        self.set_table(ck["table"])
+        self.grads.zero_()
+        self.prep_records()
 
     def stats(self) -> dict:
         return _lib.sad_get_stats(self.ctx, self.stream)

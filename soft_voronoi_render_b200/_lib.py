@@ -36,7 +36,8 @@ class sad_buffers(ctypes.Structure):
     _fields_ = [("params", ctypes.c_void_p), ("grads", ctypes.c_void_p), ("adam_m", ctypes.c_void_p),
                 ("adam_v", ctypes.c_void_p), ("records", ctypes.c_void_p), ("table", ctypes.c_void_p),
                 ("target", ctypes.c_void_p), ("image", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t), ("stats", ctypes.c_void_p), ("frozen", ctypes.c_void_p)]
+                ("workspace_bytes", ctypes.c_size_t), ("stats", ctypes.c_void_p), ("frozen", ctypes.c_void_p),
+                ("cand16", ctypes.c_void_p)]
 
 
 class sad_densify_cfg(ctypes.Structure):
@@ -65,10 +66,15 @@ class sad_stats(ctypes.Structure):
                 ("pass_counter", ctypes.c_uint32), ("adam_step", ctypes.c_uint32),
                 ("current_table", ctypes.c_uint32), ("reserved", ctypes.c_uint32), ("loss", ctypes.c_double),
                 ("n_active", ctypes.c_uint32), ("n_split", ctypes.c_uint32), ("n_pruned", ctypes.c_uint32),
-                ("reserved2", ctypes.c_uint32)]
+                ("check_failures", ctypes.c_uint32)]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_ if not n.startswith("reserved")}
+
+
+class sad_fit_state(ctypes.Structure):
+    _fields_ = [("pass_counter", ctypes.c_uint32), ("adam_step", ctypes.c_uint32), ("seed", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32)]
 
 
 EXPORTED = (
@@ -77,22 +83,25 @@ EXPORTED = (
     "sad_propagate", "sad_fit_pass_cached", "sad_set_candidate_grid", "sad_pack_sites", "sad_unpack_sites", "sad_bind_target", "sad_set_target_u8",
     "sad_render", "sad_backward", "sad_densify_prune", "sad_tau_diffuse", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
     "sad_get_stats", "sad_get_loss", "sad_copy_loss", "sad_last_error", "sad_backward_noalloc",
+    "sad_get_fit_state", "sad_set_fit_state", "sad_set_candidate_precision",
 )
 
 _lib = None
 
 
 def library_path() -> str:
-    return _build.LIB
+    """libsad.so, or with SAD_CHECKS=1 in the environment the debug build
+    libsad_checks.so (device-side bounds checks counted in sad_stats)."""
+    return _build.LIB_CHECKS if os.environ.get("SAD_CHECKS") == "1" else _build.LIB
 
 
 def load(build_if_missing: bool = True) -> ctypes.CDLL:
-    """Load libsad.so from the package's build folder (building it first if
-    it is absent and nvcc is available).  Raises if it cannot be loaded."""
+    """Load the library from the package's build folder (building it first
+    if it is absent and nvcc is available).  Raises if it cannot be loaded."""
     global _lib
     if _lib is not None:
         return _lib
-    path = _build.LIB
+    path = library_path()
     if build_if_missing:
         _build.build()
     if not os.path.exists(path):
@@ -133,6 +142,9 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "sad_copy_loss": [vp, vp, vp],
         "sad_last_error": [vp],
         "sad_backward_noalloc": [ci, ci, ci, vp, vp, vp, vp, vp, vp, vp],
+        "sad_get_fit_state": [vp, ctypes.POINTER(sad_fit_state), vp],
+        "sad_set_fit_state": [vp, ctypes.POINTER(sad_fit_state), vp],
+        "sad_set_candidate_precision": [vp, ci, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -188,9 +200,10 @@ def sad_destroy(ctx: int) -> None:
 
 
 def sad_bind(ctx: int, *, params, grads, adam_m, adam_v, records, table, target, workspace,
-             workspace_bytes: int, image=None, stats=None, frozen=None) -> None:
+             workspace_bytes: int, image=None, stats=None, frozen=None, cand16=None) -> None:
     b = sad_buffers(_ptr(params), _ptr(grads), _ptr(adam_m), _ptr(adam_v), _ptr(records), _ptr(table),
-                    _ptr(target), _ptr(image), _ptr(workspace), workspace_bytes, _ptr(stats), _ptr(frozen))
+                    _ptr(target), _ptr(image), _ptr(workspace), workspace_bytes, _ptr(stats), _ptr(frozen),
+                    _ptr(cand16))
     _check(ctx, load().sad_bind(ctx, ctypes.byref(b)))
 
 
@@ -300,6 +313,21 @@ def sad_get_stats(ctx: int, stream=None) -> dict:
     s = sad_stats()
     _check(ctx, load().sad_get_stats(ctx, ctypes.byref(s), _stream(stream)))
     return s.as_dict()
+
+
+def sad_set_candidate_precision(ctx: int, bits: int, stream=None) -> None:
+    _check(ctx, load().sad_set_candidate_precision(ctx, int(bits), _stream(stream)))
+
+
+def sad_get_fit_state(ctx: int, stream=None) -> dict:
+    s = sad_fit_state()
+    _check(ctx, load().sad_get_fit_state(ctx, ctypes.byref(s), _stream(stream)))
+    return {"pass_counter": s.pass_counter, "adam_step": s.adam_step, "seed": s.seed}
+
+
+def sad_set_fit_state(ctx: int, pass_counter: int, adam_step: int, seed: int, stream=None, reserved: int = 0) -> None:
+    s = sad_fit_state(pass_counter, adam_step, seed, reserved)
+    _check(ctx, load().sad_set_fit_state(ctx, ctypes.byref(s), _stream(stream)))
 
 
 def sad_copy_loss(ctx: int, dst, stream=None) -> None:

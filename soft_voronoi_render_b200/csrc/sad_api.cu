@@ -56,8 +56,17 @@ int read_counters(sad_ctx *ctx, sad::Counters *out, cudaStream_t st) {
     return cuda_status(ctx, e, "read counters");
 }
 
+// the packed candidate-site records follow the current score records: built
+// at the start of every call that updates candidates in the binary16 mode
+int pack_candidates(sad_ctx *ctx, cudaStream_t st) {
+    if (!ctx->dev.f16) return SAD_OK;
+    return cuda_status(ctx, sad::launch_pack_cand16(ctx->dev, st), "pack candidate records");
+}
+
 int run_refresh(sad_ctx *ctx, int G, cudaStream_t st) {
-    int r = cuda_status(ctx, sad::launch_seed(ctx->dev, st), "seed");
+    int r = pack_candidates(ctx, st);
+    if (r) return r;
+    r = cuda_status(ctx, sad::launch_seed(ctx->dev, st), "seed");
     if (r) return r;
     int B = 1;
     const int m = ctx->GH > ctx->GW ? ctx->GH : ctx->GW;
@@ -73,8 +82,12 @@ int run_refresh(sad_ctx *ctx, int G, cudaStream_t st) {
 // grid the propagation runs on the grid, then the tile pass on the cached
 // lists renders and differentiates every pixel from its cell's list
 int run_fit_pass(sad_ctx *ctx, int G, cudaStream_t st) {
-    if (ctx->cell == 1) return cuda_status(ctx, sad::launch_fit_tile(ctx->dev, G, st), "fit pass");
-    int r = cuda_status(ctx, sad::launch_propagate(ctx->dev, 1, G, st), "propagate");
+    if (ctx->cell == 1 && !ctx->dev.f16) return cuda_status(ctx, sad::launch_fit_tile(ctx->dev, G, st), "fit pass");
+    // a coarser candidate grid, or candidates ranked on the packed records:
+    // the propagation pass, then the tile pass on the new lists
+    int r = pack_candidates(ctx, st);
+    if (r) return r;
+    r = cuda_status(ctx, sad::launch_propagate(ctx->dev, 1, G, st), "propagate");
     if (r) return r;
     return cuda_status(ctx, sad::launch_fit_tile_cached(ctx->dev, st), "fit pass (cached lists)");
 }
@@ -145,6 +158,8 @@ int sad_bind(sad_ctx *ctx, const sad_buffers *b) {
     }
     if (b->image && !aligned16(b->image)) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer image is not 16-byte aligned");
     if (b->stats && !aligned16(b->stats)) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer stats is not 16-byte aligned");
+    if (b->cand16 && !aligned16(b->cand16))
+        return fail(ctx, SAD_ERR_INVALID_ARG, "buffer cand16 is not 16-byte aligned");
     const size_t need = sad::workspace_bytes(ctx->H, ctx->W, ctx->N);
     if (b->workspace_bytes < need)
         return fail(ctx, SAD_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", b->workspace_bytes, need);
@@ -168,6 +183,8 @@ int sad_bind(sad_ctx *ctx, const sad_buffers *b) {
     d.image = b->image;
     d.stats = b->stats;
     d.frozen = b->frozen;
+    d.cand16 = reinterpret_cast<uint4 *>(b->cand16);
+    d.f16 = d.f16 && d.cand16;
     d.ws = b->workspace;
     // best effort: the launchers set the attributes themselves when this
     // fails (binding needs no device, only valid pointers)
@@ -288,7 +305,19 @@ int sad_propagate(sad_ctx *ctx, int jump, int G, sad_stream_t stream) {
     if (r) return r;
     if (jump < 1) return fail(ctx, SAD_ERR_INVALID_ARG, "jump must be >= 1");
     if (G < 0 || G > SAD_MAX_INJECT) return fail(ctx, SAD_ERR_CAPACITY, "G=%d outside [0, %d]", G, SAD_MAX_INJECT);
+    r = pack_candidates(ctx, cs(stream));
+    if (r) return r;
     return cuda_status(ctx, sad::launch_propagate(ctx->dev, jump, G, cs(stream)), "propagate");
+}
+
+int sad_set_candidate_precision(sad_ctx *ctx, int bits, sad_stream_t stream) {
+    (void)stream;
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (bits != 32 && bits != 16) return fail(ctx, SAD_ERR_INVALID_ARG, "candidate precision must be 32 or 16 bits");
+    if (bits == 16 && !ctx->dev.cand16) return fail(ctx, SAD_ERR_NOT_BOUND, "16-bit candidates need a bound cand16 buffer");
+    ctx->dev.f16 = bits == 16;
+    return SAD_OK;
 }
 
 int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream) {
@@ -311,7 +340,7 @@ int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream) {
         return cuda_status(ctx, sad::launch_render_backward_det(ctx->dev, cs(stream)), "backward (deterministic)");
     if (flags & SAD_STATS) {
         if (!ctx->buf.stats) return fail(ctx, SAD_ERR_NOT_BOUND, "SAD_STATS needs a bound stats buffer");
-        return cuda_status(ctx, sad::launch_render_backward_stats(ctx->dev, cs(stream)), "backward (stats)");
+        return cuda_status(ctx, sad::launch_fit_tile_cached_stats(ctx->dev, cs(stream)), "backward (stats)");
     }
     return cuda_status(ctx, sad::launch_render_backward(ctx->dev, cs(stream)), "backward");
 }
@@ -481,8 +510,32 @@ int sad_get_stats(sad_ctx *ctx, sad_stats *out, sad_stream_t stream) {
     out->n_split = hdr[0];
     out->n_pruned = hdr[1];
     out->n_active = hdr[2];
-    out->reserved2 = 0;
+    out->check_failures = (uint32_t)(c.check_failures > 0xFFFFFFFFull ? 0xFFFFFFFFull : c.check_failures);
     return SAD_OK;
+}
+
+int sad_get_fit_state(sad_ctx *ctx, sad_fit_state *out, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!out) return fail(ctx, SAD_ERR_INVALID_ARG, "fit state destination is NULL");
+    sad::Counters c;
+    r = read_counters(ctx, &c, cs(stream));
+    if (r) return r;
+    out->pass_counter = c.pass_counter;
+    out->adam_step = c.adam_step;
+    out->seed = c.seed;
+    out->reserved = 0;
+    return SAD_OK;
+}
+
+int sad_set_fit_state(sad_ctx *ctx, const sad_fit_state *state, sad_stream_t stream) {
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (!state) return fail(ctx, SAD_ERR_INVALID_ARG, "fit state is NULL");
+    if (state->reserved != 0) return fail(ctx, SAD_ERR_INVALID_ARG, "fit state: reserved field must be 0");
+    return cuda_status(ctx, sad::launch_set_fit_state(ctx->dev, state->pass_counter, state->adam_step, state->seed,
+                                                      cs(stream)),
+                       "set fit state");
 }
 
 int sad_get_loss(sad_ctx *ctx, double *loss, sad_stream_t stream) {

@@ -39,7 +39,8 @@ struct Counters {
     unsigned long long empty_pixels;
     unsigned long long dropped_ids;
     double loss;
-    double pad1[7];
+    unsigned long long check_failures;  // SAD_CHECKS builds: accesses refused by a bounds check
+    double pad1[6];
     uint32_t pack_ord[6];    // order-preserving encodings of the pack ranges
     float pack_range[6];     // lo ln tau, lo r, lo a, hi ln tau, hi r, hi a
 };
@@ -209,6 +210,22 @@ __device__ __forceinline__ bool warp_run_reduce(uint32_t key, float (&v)[NV], in
 
 
 // workspace views
+__device__ __forceinline__ Counters *ws_counters(void *ws);
+
+// Bounds checks of the debug build (compiled with -DSAD_CHECKS): a failed
+// check is counted in the statistics block and the guarded access is
+// skipped; nothing traps.  In the normal build the checks compile away.
+#ifdef SAD_CHECKS
+__device__ __forceinline__ bool sad_check(bool ok, void *ws) {
+    if (!ok) atomicAdd(&ws_counters(ws)->check_failures, 1ull);
+    return ok;
+}
+#define SAD_CHECK(cond, ws) (::sad::sad_check((cond), (ws)))
+#else
+#define SAD_CHECK(cond, ws) (true)
+#endif
+
+
 __device__ __forceinline__ Counters *ws_counters(void *ws) { return reinterpret_cast<Counters *>(ws); }
 __device__ __forceinline__ double *ws_loss_partials(void *ws) {
     return reinterpret_cast<double *>(reinterpret_cast<char *>(ws) + COUNTERS_BYTES);

@@ -35,6 +35,7 @@ constexpr int UHASH_BITS = 9;
 constexpr int UHASH = 1 << UHASH_BITS;
 constexpr int UPROBES = 8;
 constexpr uint32_t NOLOC = 0xFFFFFFFFu;
+constexpr uint32_t NOSLOT = 0xFFFFu;
 constexpr unsigned FULL = 0xffffffffu;
 
 // top-8 list carrying each entry's tile-local index
@@ -95,30 +96,23 @@ struct Top8L {
     }
 };
 
-// storage slot of sorted entry idx: the low three bits are XORed with bits of
-// the owning thread (idx >> 3), so that the 32 lanes reading entry 8 t + e
-// of their own runs hit distinct banks
-__device__ __forceinline__ uint32_t ent_slot(uint32_t idx) {
-    const uint32_t t = idx >> 3;
-    return idx ^ ((((t >> 3) & 3u) << 1) | ((t >> 1) & 1u));
-}
-
 __device__ __forceinline__ uint32_t uhash(uint32_t id) { return (id * 2654435761u) >> (32 - UHASH_BITS); }
 
 // insert a site id into the tile's key table (linear probing, compare-and-swap)
-__device__ __forceinline__ bool ukey_insert(uint32_t *keys, uint32_t id) {
+// and return the slot that holds it, or NOSLOT when the probes run out
+__device__ __forceinline__ uint32_t ukey_insert(uint32_t *keys, uint32_t id) {
     uint32_t s = uhash(id);
 #pragma unroll 1
     for (int q = 0; q < UPROBES; ++q) {
         const uint32_t k = *reinterpret_cast<volatile uint32_t *>(keys + s);
-        if (k == id) return true;
+        if (k == id) return s;
         if (k == EMPTY) {
             const uint32_t old = atomicCAS(keys + s, EMPTY, id);
-            if (old == EMPTY || old == id) return true;
+            if (old == EMPTY || old == id) return s;
         }
         s = (s + 1) & (UHASH - 1);
     }
-    return false;
+    return NOSLOT;
 }
 
 __device__ __forceinline__ uint32_t ukey_lookup(const uint32_t *keys, const uint32_t *lid, uint32_t id) {
@@ -133,23 +127,37 @@ __device__ __forceinline__ uint32_t ukey_lookup(const uint32_t *keys, const uint
     return NOLOC;
 }
 
-template <int FY>
+// four local indices (< 256) as the bytes of one word, and back
+__device__ __forceinline__ uint32_t pack_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+__device__ __forceinline__ uint32_t byte_of(uint32_t w, int q) { return __byte_perm(w, 0, 0x4440 | (q & 3)); }
+
+template <int FY, bool STATS>
 struct FusedSmem {
-    static constexpr int FT = FX * FY, HN = HX * (FY + 2);
+    static constexpr int FT = FX * FY, HN = HX * (FY + 2), RING = HN - FT;
+    // The tile's (pixel, slot) entries grouped by site, each site's run padded
+    // to a multiple of 8 so that every group of 8 belongs to one site: at most
+    // FT + 7 UCAP / 8 groups.  Entry e of group g is stored at [e][g]; the
+    // plane strides are 4 words modulo 32 so that the scatter's consecutive
+    // entries (consecutive e) fall in distinct banks.
+    static constexpr int NG = FT + 7 * UCAP / 8;
+    static constexpr int NGS = (NG + 15) / 16 * 16 + 2;    // float2 planes
+    static constexpr int NGS16 = (NG + 63) / 64 * 64 + 8;  // uint16 planes
     uint32_t keys[UHASH];
     uint32_t lid[UHASH];
     uint32_t ulist[UCAP];
-    float4 urec[REC_F4][UCAP];   // field-major: conflict-free for distinct sites
-    uint4 masks[HN];             // 128-bit membership of every tile + halo pixel
-    float acc[NPARAM][UCAP];      // the tile's gradient sums per local site
-    uint32_t cnt[UCAP];           // (pixel, slot) entries per local site
-    uint32_t cursor[UCAP];        // scatter cursor of the counting sort
-    float4 pixg[FT];              // per pixel: dL/dchat (3), chat . dL/dchat
-    float2 ent_wl[FT * K];        // entries grouped by site: softmax weight, logit
-    uint16_t ent_pu[FT * K];      //   pixel (low 9 bits) and local site (high 7 bits)
-    uint32_t ring_id[(HN - FT) * K];  // the halo lists, read once from the table
+    float4 urec[REC_F4][UCAP + 1];  // field-major; entry UCAP is all zero
+    uint4 masks[HN];                // 128-bit membership of every tile + halo pixel
+    uint32_t cnt[UCAP];             // (pixel, slot) entries per local site
+    uint32_t cursor[UCAP];          // scatter cursor; afterwards the end of each site's entries
+    float4 pixg[FT];                // per pixel: dL/dchat (3), chat . dL/dchat
+    float2 ent_wl[K][NGS];          // softmax weight, logit
+    uint16_t ent_pu[K][NGS16];      // pixel (low 9 bits), local site (high 7 bits)
+    float ent_rd[STATS ? K : 1][STATS ? NGS : 1];  // removal delta (budget statistics)
     float warp_loss[FY];
-    uint32_t n_ent;
+    uint32_t warp_cnt[3][FY];       // per warp: empty pixels, global-atomic pixels, dropped ids
+    uint32_t n_groups;
     uint32_t ucount;
     int overflow;
     int last;
@@ -173,15 +181,6 @@ __device__ __forceinline__ void ring_coords(int r, int &hx, int &hy) {
     }
 }
 
-__device__ __forceinline__ void set_bit(uint4 &m, uint32_t u) {
-    const uint32_t b = 1u << (u & 31u);
-    const uint32_t w = u >> 5;
-    m.x |= (w == 0) ? b : 0u;
-    m.y |= (w == 1) ? b : 0u;
-    m.z |= (w == 2) ? b : 0u;
-    m.w |= (w == 3) ? b : 0u;
-}
-
 // bounds of the run of equal keys (in lane order) that holds this lane
 __device__ __forceinline__ void run_bounds(uint32_t key, int lane, int &start, int &tail_lane) {
     const uint32_t key_next = __shfl_down_sync(FULL, key, 1);
@@ -199,10 +198,12 @@ __device__ __forceinline__ void run_bounds(uint32_t key, int lane, int &start, i
 //   dL/da = -gamma (k^2 e^a alpha^2 - k^2 e^-a beta^2) / (2 m),
 //   dL/dtheta = -gamma alpha beta (k^2 e^a - k^2 e^-a) / m
 // with m = sqrt(delta^T G' delta) = k n (0 where m = 0).
+template <int NV>
 __device__ __forceinline__ void slot_grad(const float4 r0, const float4 r1, const float4 r2, const float4 r3,
                                           float fx, float fy, float l, float w, float gr, float gg, float gb,
-                                          float cdg, float (&v)[NPARAM]) {
-    const float dx = fx - r0.x, dy = fy - r0.y;
+                                          float cdg, float (&v)[NV], float &dx, float &dy) {
+    dx = fx - r0.x;
+    dy = fy - r0.y;
     const float u1 = fmaf(r0.z, dx, r0.w * dy);
     const float u2 = fmaf(r1.x, dy, r0.w * dx);
     const float qf = fmaf(dx, u1, dy * u2);
@@ -220,6 +221,50 @@ __device__ __forceinline__ void slot_grad(const float4 r0, const float4 r1, cons
     v[PCB] = w * gb;
     v[PTH] = -gi * al * be * (r3.y - r3.z);
     v[PA] = -0.5f * gi * (r3.y * al * al - r3.z * be * be);
+}
+
+// budget-control statistics of one (pixel, slot) (summary B.4-B.5): mass w,
+// energy w e, error-weighted second moments w e (dx^2, dx dy, dy^2) and the
+// removal delta rd, with e = |chat - t|^2 = (P / 2)^2 |g|^2
+template <int NV>
+__device__ __forceinline__ void slot_stats(float w, float ex, float dx, float dy, float rd, float (&v)[NV]) {
+    const float we = w * ex;
+    v[NPARAM + 0] = w;
+    v[NPARAM + 1] = we;
+    v[NPARAM + 2] = we * dx * dx;
+    v[NPARAM + 3] = we * dx * dy;
+    v[NPARAM + 4] = we * dy * dy;
+    v[NPARAM + 5] = rd;
+}
+
+// Removal delta of one slot: |(chat - w c) / (1 - w) - t|^2 - |chat - t|^2,
+// evaluated as (a - b) . (a + b) with b = chat - t (er, eg, eb) and
+// a - b = w (c_rest - c), c_rest the blend of the other slots.  Their
+// unnormalised sums are Z - e_q and Z chat - e_q c, except for the dominant
+// slot, whose are summed directly (zmm, cm*), so that removing a site that
+// holds almost all the weight subtracts no two nearly equal numbers.  Where
+// the other slots hold less than 1e-6 of the weight, 1 - w is clamped to
+// 1e-6.
+__device__ __forceinline__ float removal_delta(float eq, float4 c, bool dominant, float Z, float iz, float chr,
+                                               float chg, float chb, float zmm, float cmr, float cmg, float cmb,
+                                               float er, float eg, float eb) {
+    const float w = eq * iz;
+    const float oz = dominant ? zmm : Z - eq;
+    const float ocr = dominant ? cmr : fmaf(-eq, c.x, chr * Z);
+    const float ocg = dominant ? cmg : fmaf(-eq, c.y, chg * Z);
+    const float ocb = dominant ? cmb : fmaf(-eq, c.z, chb * Z);
+    float dr, dg, db;
+    if (oz * iz >= 1e-6f) {
+        const float ioz = 1.0f / oz;
+        dr = w * (ocr * ioz - c.x);
+        dg = w * (ocg * ioz - c.y);
+        db = w * (ocb * ioz - c.z);
+    } else {
+        dr = ocr * iz * 1e6f - chr;
+        dg = ocg * iz * 1e6f - chg;
+        db = ocb * iz * 1e6f - chb;
+    }
+    return dr * (2.0f * er + dr) + dg * (2.0f * eg + dg) + db * (2.0f * eb + db);
 }
 
 // generic candidate offer (no tile index): dedup against the running list
@@ -257,15 +302,20 @@ __device__ __forceinline__ void generic_pass(Top8L &t, const uint4 *__restrict__
     }
 }
 
-template <int FY, bool PROP>
+template <int FY, bool PROP, bool STATS>
 __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(const float4 *__restrict__ rec,
                                                                             uint32_t *table,
                                                          const float *__restrict__ target, int H, int W, int N,
                                                          int G, float *__restrict__ image,
-                                                         float *__restrict__ grads, void *ws, TableGrid lists) {
-    constexpr int FT = FX * FY, HY = FY + 2, HN = HX * HY, RING = HN - FT;
+                                                         float *__restrict__ grads, float *__restrict__ stats,
+                                                         void *ws, TableGrid lists) {
+    static_assert(!(PROP && STATS), "the statistics come with the cached-list form");
+    using Smem = FusedSmem<FY, STATS>;
+    constexpr int NV = STATS ? NPARAM + NSTAT : NPARAM;
+    constexpr int FT = Smem::FT, HN = Smem::HN, RING = Smem::RING;
+    constexpr int NRE = (RING * K + FT - 1) / FT;  // halo (pixel, slot) entries per thread
     extern __shared__ __align__(16) unsigned char fused_smem_raw[];
-    FusedSmem<FY> &sm = *reinterpret_cast<FusedSmem<FY> *>(fused_smem_raw);
+    Smem &sm = *reinterpret_cast<Smem *>(fused_smem_raw);
     Counters *c = ws_counters(ws);
     const uint32_t cur = c->cur, pass = c->pass_counter, seed = c->seed;
     const int lane = threadIdx.x, ty = threadIdx.y;
@@ -282,30 +332,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     uint4 *out1 = out0 + P;
     const uint32_t Nu = (uint32_t)N;
 
-    for (int q = tid; q < UHASH; q += FT) sm.keys[q] = EMPTY;
-    if (PROP)
-    for (int r = tid; r < RING; r += FT) {
-        int hx, hy;
-        ring_coords<FY>(r, hx, hy);
-        sm.masks[hy * HX + hx] = make_uint4(0, 0, 0, 0);
-    }
-    for (int q = tid; q < NPARAM * UCAP; q += FT) (&sm.acc[0][0])[q] = 0.0f;
-    if (tid < UCAP) sm.cnt[tid] = 0;
-    if (tid == 0) {
-        sm.ucount = 0;
-        sm.overflow = 0;
-    }
-    __syncthreads();
-
-    // the target is needed last; start its loads first
-    float tr = 0.0f, tg = 0.0f, tb = 0.0f;
-    if (inside) {
-        const size_t p = (size_t)j * W + i;
-        tr = __ldg(target + p);
-        tg = __ldg(target + P + p);
-        tb = __ldg(target + 2 * P + p);
-    }
-    // ---- A1: collect the distinct ids of the tile and halo lists ----------
+    // ---- global loads first: the pixel's list, the halo entries, the target
     uint32_t own[K];
     {
         uint4 a = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY), b = a;
@@ -318,27 +345,68 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         own[0] = a.x; own[1] = a.y; own[2] = a.z; own[3] = a.w;
         own[4] = b.x; own[5] = b.y; own[6] = b.z; own[7] = b.w;
     }
+    // halo entry e = tid + x FT is ring pixel e % RING, slot e / RING; rv[x]
+    // holds its id, then its hash slot | mask cell << 16 (NOLOC: none)
+    uint32_t rv[NRE], rcell[NRE];
+    if (PROP) {
+#pragma unroll
+        for (int x = 0; x < NRE; ++x) {
+            const int e = tid + x * FT;
+            uint32_t id = EMPTY, cell = 0;
+            if (e < RING * K) {
+                const int r = e % RING, q = e / RING;
+                int hx, hy;
+                ring_coords<FY>(r, hx, hy);
+                cell = (uint32_t)(hy * HX + hx);
+                const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
+                if (gi >= 0 && gi < W && gj >= 0 && gj < H)
+                    id = table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
+            }
+            rv[x] = id;
+            rcell[x] = cell;
+        }
+    }
+    // the target is read last: bring its lines into L2 now, registers later
+    if (inside && lane == 0) {
+        const size_t p = (size_t)j * W + i;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(target + p));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(target + P + p));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(target + 2 * P + p));
+    }
+
+    for (int q = tid; q < UHASH; q += FT) sm.keys[q] = EMPTY;
+    if (PROP)
+        for (int q = tid; q < HN; q += FT) sm.masks[q] = make_uint4(0, 0, 0, 0);
+    if (tid < UCAP) sm.cnt[tid] = 0;
+    if (tid < REC_F4) sm.urec[tid][UCAP] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid == 0) {
+        sm.ucount = 0;
+        sm.overflow = 0;
+    }
+    __syncthreads();
+
+    // ---- A1: the distinct ids of the tile and halo lists -------------------
+    uint32_t slot[K];  // hash slot of each own entry
     bool ok = true;
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-        // neighbouring pixels mostly hold the same id in the same slot
-        const uint32_t id = own[q];
-        const uint32_t prev = __shfl_up_sync(FULL, id, 1);
-        if (id < Nu && !(lane > 0 && prev == id)) ok &= ukey_insert(sm.keys, id);
+        slot[q] = NOSLOT;
+        if (own[q] < Nu) {
+            slot[q] = ukey_insert(sm.keys, own[q]);
+            ok &= slot[q] != NOSLOT;
+        }
     }
-    // the halo pixels x 8 slots, spread over all threads: entry e is halo
-    // pixel e % RING, slot e / RING
-    if (PROP)
-    for (int e = tid; e < RING * K; e += FT) {
-        const int r = e % RING, q = e / RING;
-        int hx, hy;
-        ring_coords<FY>(r, hx, hy);
-        const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
-        uint32_t id = EMPTY;
-        if (gi >= 0 && gi < W && gj >= 0 && gj < H)
-            id = table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
-        sm.ring_id[e] = id;
-        if (id < Nu) ok &= ukey_insert(sm.keys, id);
+    if (PROP) {
+#pragma unroll
+        for (int x = 0; x < NRE; ++x) {
+            uint32_t v = NOLOC;
+            if (rv[x] < Nu) {
+                const uint32_t s = ukey_insert(sm.keys, rv[x]);
+                ok &= s != NOSLOT;
+                if (s != NOSLOT) v = s | (rcell[x] << 16);
+            }
+            rv[x] = v;
+        }
     }
     if (!ok) sm.overflow = 1;
     __syncthreads();
@@ -356,32 +424,33 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     const bool fast = !sm.overflow && sm.ucount <= UCAP;  // block-uniform
     const uint32_t ucount = fast ? sm.ucount : 0u;
 
-    uint4 own_mask = make_uint4(0, 0, 0, 0);
-    uint32_t own_lx_lo = 0xFFFFFFFFu, own_lx_hi = 0xFFFFFFFFu;  // slot q's local index in byte q (0xFF: none)
+    // slot q's local index in byte q & 3 of own_lx[q >> 2] (0xFF: none)
+    uint32_t own_lx_lo = 0xFFFFFFFFu, own_lx_hi = 0xFFFFFFFFu;
     if (fast) {
-        // ---- A3: per-pixel local indices and membership masks --------------
+        // ---- A3: local indices, membership masks, site records -------------
+        uint32_t ux[K];
 #pragma unroll
-        for (int q = 0; q < K; ++q) {
-            const uint32_t u = own[q] < Nu ? ukey_lookup(sm.keys, sm.lid, own[q]) : NOLOC;
-            if (u != NOLOC) set_bit(own_mask, u);
-            const uint32_t b = (u == NOLOC ? 0xFFu : u) << ((q & 3) * 8);
-            const uint32_t m = ~(0xFFu << ((q & 3) * 8));
-            if (q < 4) own_lx_lo = (own_lx_lo & m) | b;
-            else own_lx_hi = (own_lx_hi & m) | b;
+        for (int q = 0; q < K; ++q)
+            ux[q] = (slot[q] != NOSLOT && SAD_CHECK(slot[q] < UHASH && sm.lid[slot[q]] < UCAP, ws)) ? sm.lid[slot[q]]
+                                                                                                   : 0xFFu;
+        own_lx_lo = pack_bytes(ux[0], ux[1], ux[2], ux[3]);
+        own_lx_hi = pack_bytes(ux[4], ux[5], ux[6], ux[7]);
+        if (PROP) {
+            uint32_t *m = reinterpret_cast<uint32_t *>(&sm.masks[(ty + 1) * HX + lane + 1]);
+#pragma unroll
+            for (int q = 0; q < K; ++q)
+                if (ux[q] != 0xFFu) atomicOr(m + (ux[q] >> 5), 1u << (ux[q] & 31u));
+#pragma unroll
+            for (int x = 0; x < NRE; ++x) {
+                if (rv[x] != NOLOC && SAD_CHECK((rv[x] & 0xFFFFu) < UHASH && (rv[x] >> 16) < (uint32_t)HN, ws)) {
+                    const uint32_t u = sm.lid[rv[x] & 0xFFFFu];
+                    if (SAD_CHECK(u < UCAP, ws))
+                        atomicOr(reinterpret_cast<uint32_t *>(&sm.masks[rv[x] >> 16]) + (u >> 5), 1u << (u & 31u));
+                }
+            }
         }
-        if (PROP) sm.masks[(ty + 1) * HX + lane + 1] = own_mask;
-        if (PROP)
-        for (int e = tid; e < RING * K; e += FT) {
-            const int r = e % RING;
-            const uint32_t id = sm.ring_id[e];
-            if (id >= Nu) continue;  // also the halo pixels outside the image
-            int hx, hy;
-            ring_coords<FY>(r, hx, hy);
-            const uint32_t u = ukey_lookup(sm.keys, sm.lid, id);
-            if (u != NOLOC) atomicOr(reinterpret_cast<uint32_t *>(&sm.masks[hy * HX + hx]) + (u >> 5), 1u << (u & 31u));
-        }
-        // ---- B: stage the tile's site records --------------------------------
         for (uint32_t u = tid; u < ucount; u += FT) {
+            if (!SAD_CHECK(sm.ulist[u] < Nu, ws)) continue;
             const float4 *R = rec + (size_t)sm.ulist[u] * REC_F4;
             sm.urec[0][u] = __ldg(R);
             sm.urec[1][u] = __ldg(R + 1);
@@ -404,10 +473,9 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             const uint32_t id = own[q];
             dropped += (id >= Nu && id != EMPTY);
             if (id >= Nu) continue;
-            uint32_t u = NOLOC;
+            uint32_t u = byte_of(q < 4 ? own_lx_lo : own_lx_hi, q);
             float4 r0;
             float2 r1;
-            if (fast) u = ((q < 4 ? own_lx_lo : own_lx_hi) >> ((q & 3) * 8)) & 0xFFu;
             if (u < UCAP) {
                 r0 = sm.urec[0][u];
                 r1 = make_float2(sm.urec[1][u].x, sm.urec[1][u].y);
@@ -429,7 +497,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             int nslots = 0;
 #pragma unroll
             for (int q = 0; q < K; ++q) {
-                const uint32_t u = ((q < 4 ? own_lx_lo : own_lx_hi) >> ((q & 3) * 8)) & 0xFFu;
+                const uint32_t u = byte_of(q < 4 ? own_lx_lo : own_lx_hi, q);
                 float l = -__int_as_float(0x7f800000);
                 bool v = false;
                 uint32_t gid = EMPTY;
@@ -447,6 +515,8 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
                 t.id[q] = v ? gid : EMPTY;
                 t.lx[q] = v ? u : NOLOC;
             }
+            const int hc = (ty + 1) * HX + lane + 1;
+            const uint4 own_mask = sm.masks[hc];
             // a list holding one id twice keeps it once (the pass works on sets)
             if (nslots != __popc(own_mask.x) + __popc(own_mask.y) + __popc(own_mask.z) + __popc(own_mask.w)) {
 #pragma unroll
@@ -466,26 +536,45 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
                 t.cx(0, 1); t.cx(2, 3); t.cx(4, 5); t.cx(6, 7);
                 t.cx(1, 2); t.cx(3, 4); t.cx(5, 6);
             }
-            // candidates the four neighbours add
-            const int hc = (ty + 1) * HX + lane + 1;
+            // candidates the four neighbours add.  A candidate can only enter
+            // if it scores at least the current 8th, which insertions only
+            // raise: score every candidate once against it, then insert the
+            // few that pass (in the same order, so the same result)
             const uint4 mL = sm.masks[hc - 1], mR = sm.masks[hc + 1], mU = sm.masks[hc - HX],
                         mD = sm.masks[hc + HX];
             const uint32_t nw[UW] = {(mL.x | mR.x | mU.x | mD.x) & ~own_mask.x,
                                      (mL.y | mR.y | mU.y | mD.y) & ~own_mask.y,
                                      (mL.z | mR.z | mU.z | mD.z) & ~own_mask.z,
                                      (mL.w | mR.w | mU.w | mD.w) & ~own_mask.w};
+            const float l8 = t.l[K - 1];
+            uint32_t pass_bits[UW] = {0u, 0u, 0u, 0u};
 #pragma unroll
             for (int w = 0; w < UW; ++w) {
                 uint32_t bits = nw[w];
                 while (bits) {
+                    const int b = __ffs(bits) - 1;
+                    bits &= bits - 1u;
+                    const uint32_t u = (uint32_t)(w * 32 + b);
+                    if (!SAD_CHECK(u < ucount, ws)) continue;
+                    const float4 r0 = sm.urec[0][u];
+                    const float2 r1 = *reinterpret_cast<const float2 *>(&sm.urec[1][u]);
+                    const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+                    // NaN (inactive site or NaN parameters) fails the test
+                    if (r0.x >= 0.0f && l >= l8) pass_bits[w] |= 1u << b;
+                }
+            }
+#pragma unroll
+            for (int w = 0; w < UW; ++w) {
+                uint32_t bits = pass_bits[w];
+                while (bits) {
                     const uint32_t u = (uint32_t)(w * 32 + __ffs(bits) - 1);
                     bits &= bits - 1u;
+                    if (!SAD_CHECK(u < ucount, ws)) continue;
                     const float4 r0 = sm.urec[0][u];
-                    if (!(r0.x >= 0.0f)) continue;
-                    const float4 r1 = sm.urec[1][u];
+                    const float2 r1 = *reinterpret_cast<const float2 *>(&sm.urec[1][u]);
                     const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
                     const uint32_t gid = sm.ulist[u];
-                    if (l == l && t.beats_last(l, gid)) t.insert(l, gid, u);
+                    if (t.beats_last(l, gid)) t.insert(l, gid, u);
                 }
             }
         } else {
@@ -496,7 +585,15 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
 #pragma unroll 1
             for (int g = 0; g < G; ++g) {
                 h = xorshift32(h);
-                offer_global(t, __umulhi(h, Nu), rec, Nu, fx, fy);
+                const uint32_t id = __umulhi(h, Nu);  // < N
+                const float4 r0 = __ldg(rec + (size_t)id * REC_F4);
+                const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
+                const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+                if (r0.x >= 0.0f && l == l && t.beats_last(l, id) && !t.has(id)) {
+                    // a winner the tile index holds keeps its local index
+                    uint32_t u = fast ? ukey_lookup(sm.keys, sm.lid, id) : NOLOC;
+                    t.insert(l, id, u < ucount ? u : NOLOC);
+                }
             }
         }
         const size_t p = (size_t)j * W + i;
@@ -505,37 +602,35 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     }
 
     // ---- D: render, loss and backward on the new lists ---------------------
+    // A slot is valid iff its logit is finite: every list form above leaves
+    // -inf in the slots it does not fill.
     unsigned vmask = 0;
     float M = -__int_as_float(0x7f800000);
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-        if (inside && t.id[q] != EMPTY && isfinite(t.l[q])) {
-            vmask |= 1u << q;
-            M = fmaxf(M, t.l[q]);
-        }
+        const bool v = inside && isfinite(t.l[q]);
+        vmask |= (unsigned)v << q;
+        M = v ? fmaxf(M, t.l[q]) : M;
     }
+    const float Mf = vmask ? M : 0.0f;
     float Z = 0.0f, cr = 0.0f, cg = 0.0f, cb = 0.0f;
     bool far_slot = false;  // a slot whose site has no tile-local index
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-        if (vmask >> q & 1u) {
-            const float e = __expf(t.l[q] - M);
-            Z += e;
-            if (t.lx[q] != NOLOC) {
-                const float4 r2 = sm.urec[2][t.lx[q]];
-                cr = fmaf(e, r2.x, cr);
-                cg = fmaf(e, r2.y, cg);
-                cb = fmaf(e, r2.z, cb);
-            } else {
-                far_slot = true;
-            }
-        }
+        const bool v = vmask >> q & 1u;
+        const float e = v ? __expf(t.l[q] - Mf) : 0.0f;
+        Z += e;
+        const float4 r2 = sm.urec[2][t.lx[q] < UCAP ? t.lx[q] : UCAP];  // NOLOC: the zero entry
+        cr = fmaf(e, r2.x, cr);
+        cg = fmaf(e, r2.y, cg);
+        cb = fmaf(e, r2.z, cb);
+        far_slot |= v && t.lx[q] == NOLOC;
     }
     if (__any_sync(FULL, far_slot)) {
 #pragma unroll
         for (int q = 0; q < K; ++q) {
             if ((vmask >> q & 1u) && t.lx[q] == NOLOC) {
-                const float e = __expf(t.l[q] - M);
+                const float e = __expf(t.l[q] - Mf);
                 const float4 r2 = __ldg(rec + (size_t)t.id[q] * REC_F4 + 2);
                 cr = fmaf(e, r2.x, cr);
                 cg = fmaf(e, r2.y, cg);
@@ -548,10 +643,14 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     cg *= iz;
     cb *= iz;
     float lsum = 0.0f, gr = 0.0f, gg = 0.0f, gb = 0.0f;
+    float er = 0.0f, eg = 0.0f, eb = 0.0f;
     if (inside) {
         const size_t p = (size_t)j * W + i;
+        const float tr = __ldg(target + p), tg = __ldg(target + P + p), tb = __ldg(target + 2 * P + p);
         const float two_over_P = 2.0f / (float)P;
-        const float er = cr - tr, eg = cg - tg, eb = cb - tb;
+        er = cr - tr;
+        eg = cg - tg;
+        eb = cb - tb;
         lsum = er * er + eg * eg + eb * eb;
         gr = er * two_over_P;
         gg = eg * two_over_P;
@@ -562,10 +661,35 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             image[2 * P + p] = cb;
         }
     }
+    // STATS: the dominant slot (largest weight, first in slot order) and the
+    // weight and colour sums of the other slots
+    int qstar = -1;
+    float zmm = 0.0f, cmr = 0.0f, cmg = 0.0f, cmb = 0.0f;
+    if constexpr (STATS) {
+        float emax = -1.0f;
+#pragma unroll
+        for (int q = 0; q < K; ++q) {
+            const float e = (vmask >> q & 1u) ? __expf(t.l[q] - Mf) : -1.0f;
+            if (e > emax) {
+                emax = e;
+                qstar = q;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < K; ++q) {
+            if (!(vmask >> q & 1u) || q == qstar) continue;
+            const float e = __expf(t.l[q] - Mf);
+            const float4 c2 = t.lx[q] != NOLOC ? sm.urec[2][t.lx[q]] : __ldg(rec + (size_t)t.id[q] * REC_F4 + 2);
+            zmm += e;
+            cmr = fmaf(e, c2.x, cmr);
+            cmg = fmaf(e, c2.y, cmg);
+            cmb = fmaf(e, c2.z, cmb);
+        }
+    }
     // ---- D2: group the tile's (pixel, slot) entries by site ----------------
     // Entries whose site has a tile-local index are counted here and summed
-    // site by site below; the rare rest (injected winners, crowded tiles) go
-    // straight to global atomics.
+    // site by site below; the rare rest (injected winners from outside the
+    // tile index, crowded tiles) go straight to global atomics.
     unsigned global_adds = 0;
     const float cdg = fmaf(cr, gr, fmaf(cg, gg, cb * gb));
     sm.pixg[tid] = make_float4(gr, gg, gb, cdg);
@@ -576,24 +700,34 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         const uint32_t key = (vq && t.lx[q] != NOLOC) ? t.lx[q] : EMPTY;
         int start, tail_lane;
         run_bounds(key, lane, start, tail_lane);
-        if (lane == tail_lane && key != EMPTY) atomicAdd(&sm.cnt[key], (uint32_t)(tail_lane - start + 1));
+        if (lane == tail_lane && key != EMPTY && SAD_CHECK(key < UCAP, ws))
+            atomicAdd(&sm.cnt[key], (uint32_t)(tail_lane - start + 1));
         if (vq && t.lx[q] == NOLOC) {
             const float4 *R = rec + (size_t)t.id[q] * REC_F4;
-            float v[NPARAM];
-            slot_grad(__ldg(R), __ldg(R + 1), __ldg(R + 2), __ldg(R + 3), fx, fy, t.l[q], __expf(t.l[q] - M) * iz,
-                      gr, gg, gb, cdg, v);
+            const float4 r2 = __ldg(R + 2);
+            const float eq = __expf(t.l[q] - Mf);
+            float v[NV], dx, dy;
+            slot_grad(__ldg(R), __ldg(R + 1), r2, __ldg(R + 3), fx, fy, t.l[q], eq * iz, gr, gg, gb, cdg, v, dx, dy);
+            if constexpr (STATS)
+                slot_stats(eq * iz, er * er + eg * eg + eb * eb, dx, dy,
+                           removal_delta(eq, r2, q == qstar, Z, iz, cr, cg, cb, zmm, cmr, cmg, cmb, er, eg, eb), v);
             ++global_adds;
 #pragma unroll
             for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + t.id[q], v[k]);
+            if constexpr (STATS) {
+#pragma unroll
+                for (int k = 0; k < NSTAT; ++k) atomicAdd(stats + (size_t)k * N + t.id[q], v[NPARAM + k]);
+            }
         }
     }
     __syncthreads();
     if (ty == 0) {
-        // exclusive scan of the 128 counts by one warp, 4 per lane
+        // exclusive scan of the 128 counts, each rounded up to a multiple of
+        // 8, by one warp (4 per lane)
         uint32_t c4[4], run = 0;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            c4[e] = sm.cnt[lane * 4 + e];
+            c4[e] = (sm.cnt[lane * 4 + e] + 7u) & ~7u;
             run += c4[e];
         }
         uint32_t incl = run;
@@ -608,7 +742,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             sm.cursor[lane * 4 + e] = base;
             base += c4[e];
         }
-        if (lane == 31) sm.n_ent = incl;
+        if (lane == 31) sm.n_groups = incl >> 3;
     }
     __syncthreads();
 #pragma unroll
@@ -618,78 +752,91 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         int start, tail_lane;
         run_bounds(key, lane, start, tail_lane);
         uint32_t pos0 = 0;
-        if (lane == tail_lane && key != EMPTY) pos0 = atomicAdd(&sm.cursor[key], (uint32_t)(tail_lane - start + 1));
+        if (lane == tail_lane && key != EMPTY && SAD_CHECK(key < UCAP, ws))
+            pos0 = atomicAdd(&sm.cursor[key], (uint32_t)(tail_lane - start + 1));
         pos0 = __shfl_sync(FULL, pos0, tail_lane);
-        if (vq) {
+        if (vq && SAD_CHECK(((pos0 + (uint32_t)(lane - start)) >> 3) < (uint32_t)Smem::NG, ws)) {
             const uint32_t pos = pos0 + (uint32_t)(lane - start);
-            const uint32_t slot = ent_slot(pos);
-            sm.ent_wl[slot] = make_float2(__expf(t.l[q] - M) * iz, t.l[q]);
-            sm.ent_pu[slot] = (uint16_t)(tid | (key << 9));
+            const float eq = __expf(t.l[q] - Mf);
+            sm.ent_wl[pos & 7u][pos >> 3] = make_float2(eq * iz, t.l[q]);
+            sm.ent_pu[pos & 7u][pos >> 3] = (uint16_t)(tid | (key << 9));
+            if constexpr (STATS)
+                sm.ent_rd[pos & 7u][pos >> 3] = removal_delta(eq, sm.urec[2][key], q == qstar, Z, iz, cr, cg, cb, zmm,
+                                                              cmr, cmg, cmb, er, eg, eb);
         }
     }
     __syncthreads();
-    // ---- D3: every thread sums a run of 8 consecutive entries -------------
+    // ---- D3: every thread sums one group of 8 entries of one site ----------
     {
-        const uint32_t n_ent = sm.n_ent;
+        const uint32_t ng = sm.n_groups;
         const float fx0 = (float)i0 + 0.5f, fy0 = (float)j0 + 0.5f;
-        uint32_t cur = NOLOC;
-        float4 r0 = make_float4(0.f, 0.f, 0.f, 0.f), r1 = r0, r2 = r0, r3 = r0;
-        float a[NPARAM];
+        const float half_P = 0.5f * (float)P, ex_scale = half_P * half_P;  // |chat - t|^2 = ex_scale |g|^2
+#pragma unroll 1
+        for (uint32_t g0 = 0; g0 < ng; g0 += FT) {
+            if (g0 + (uint32_t)ty * 32u >= ng) break;  // warp-uniform
+            const uint32_t g = g0 + (uint32_t)tid;
+            uint32_t u = EMPTY;
+            float a[NV];
 #pragma unroll
-        for (int k = 0; k < NPARAM; ++k) a[k] = 0.0f;
-        const uint32_t e0 = (uint32_t)tid * K;
+            for (int k = 0; k < NV; ++k) a[k] = 0.0f;
+            if (g < ng && SAD_CHECK(g < (uint32_t)Smem::NG && (sm.ent_pu[0][g] >> 9) < ucount, ws)) {
+                u = sm.ent_pu[0][g] >> 9;
+                const uint32_t rem = sm.cursor[u] - 8u * g;  // entries of the group (>= 1)
+                const float4 r0 = sm.urec[0][u], r1 = sm.urec[1][u], r2 = sm.urec[2][u], r3 = sm.urec[3][u];
 #pragma unroll
-        for (int e = 0; e < K; ++e) {
-            const uint32_t idx = e0 + e;
-            if (idx >= n_ent) break;
-            const uint32_t pu = sm.ent_pu[ent_slot(idx)];
-            const uint32_t u = pu >> 9, px = pu & 0x1FFu;
-            if (u != cur) {
-                if (cur != NOLOC) {
+                for (int e = 0; e < K; ++e) {
+                    const bool ve = (uint32_t)e < rem && SAD_CHECK((sm.ent_pu[e][g] & 0x1FFu) < (uint32_t)FT, ws);
+                    const uint32_t px = ve ? (uint32_t)(sm.ent_pu[e][g] & 0x1FFu) : 0u;
+                    const float2 wl = sm.ent_wl[e][g];
+                    const float4 pa = sm.pixg[px];
+                    float v[NV], dx, dy;
+                    slot_grad(r0, r1, r2, r3, fx0 + (float)(px & (FX - 1)), fy0 + (float)(px / FX), wl.y, wl.x, pa.x,
+                              pa.y, pa.z, pa.w, v, dx, dy);
+                    if constexpr (STATS)
+                        slot_stats(wl.x, ex_scale * (pa.x * pa.x + pa.y * pa.y + pa.z * pa.z), dx, dy,
+                                   sm.ent_rd[e][g], v);
+                    if (ve) {
 #pragma unroll
-                    for (int k = 0; k < NPARAM; ++k) {
-                        atomicAdd(&sm.acc[k][cur], a[k]);
-                        a[k] = 0.0f;
+                        for (int k = 0; k < NV; ++k) a[k] += v[k];
                     }
                 }
-                cur = u;
-                r0 = sm.urec[0][u];
-                r1 = sm.urec[1][u];
-                r2 = sm.urec[2][u];
-                r3 = sm.urec[3][u];
             }
-            const float2 wl = sm.ent_wl[ent_slot(idx)];
-            const float4 pa = sm.pixg[px];
-            float v[NPARAM];
-            slot_grad(r0, r1, r2, r3, fx0 + (float)(px & (FX - 1)), fy0 + (float)(px / FX), wl.y, wl.x, pa.x,
-                      pa.y, pa.z, pa.w, v);
+            // groups of one site sit on consecutive lanes: sum each run across
+            // lanes, then one global update per run
+            const bool tail = warp_run_reduce(u, a, lane);
+            if (tail && u != EMPTY) {
+                const uint32_t gid = sm.ulist[u];
 #pragma unroll
-            for (int k = 0; k < NPARAM; ++k) a[k] += v[k];
-        }
-        // the last sites of consecutive lanes repeat (entries are sorted):
-        // sum each run across lanes first, then one update per run
-        const uint32_t key = cur == NOLOC ? EMPTY : cur;
-        const bool tail = warp_run_reduce(key, a, lane);
-        if (tail && key != EMPTY) {
+                for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + gid, a[k]);
+                if constexpr (STATS) {
 #pragma unroll
-            for (int k = 0; k < NPARAM; ++k) atomicAdd(&sm.acc[k][key], a[k]);
+                    for (int k = 0; k < NSTAT; ++k) atomicAdd(stats + (size_t)k * N + gid, a[NPARAM + k]);
+                }
+            }
         }
     }
 
-    // ---- E: flush the tile accumulators, loss partial, last-block epilogue
+    // ---- E: loss partial, statistics, last-block epilogue ------------------
     for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(FULL, lsum, o);
-    if (lane == 0) sm.warp_loss[ty] = lsum;
-    const int n_empty = __syncthreads_count(inside && !vmask);
-    const int n_global = __syncthreads_count(global_adds != 0);
-    const int n_dropped = PROP ? 0 : __syncthreads_count(dropped != 0);
-    for (uint32_t e = tid; e < ucount * NPARAM; e += FT) {
-        const uint32_t u = e % ucount, k = e / ucount;
-        const float a = sm.acc[k][u];
-        if (a != 0.0f) atomicAdd(grads + (size_t)k * N + sm.ulist[u], a);
+    const unsigned b_empty = __ballot_sync(FULL, inside && !vmask);
+    const unsigned b_global = __ballot_sync(FULL, global_adds != 0);
+    const unsigned b_drop = __ballot_sync(FULL, dropped != 0);
+    if (lane == 0) {
+        sm.warp_loss[ty] = lsum;
+        sm.warp_cnt[0][ty] = __popc(b_empty);
+        sm.warp_cnt[1][ty] = __popc(b_global);
+        sm.warp_cnt[2][ty] = __popc(b_drop);
     }
+    __syncthreads();
     if (tid == 0) {
         float tl = 0.0f;
-        for (int q = 0; q < FY; ++q) tl += sm.warp_loss[q];
+        unsigned n_empty = 0, n_global = 0, n_dropped = 0;
+        for (int q = 0; q < FY; ++q) {
+            tl += sm.warp_loss[q];
+            n_empty += sm.warp_cnt[0][q];
+            n_global += sm.warp_cnt[1][q];
+            n_dropped += sm.warp_cnt[2][q];
+        }
         ws_loss_partials(ws)[blockIdx.y * gridDim.x + blockIdx.x] = (double)tl;
         if (n_empty) atomicAdd(&c->empty_pixels, (unsigned long long)n_empty);
         if (n_global) atomicAdd(&c->hash_overflow, (unsigned long long)n_global);
@@ -724,55 +871,61 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
 
 // the tile state exceeds the 48 KB default: opt in once per device (done
 // when buffers are bound, so that a stream capture sees launches only)
-template <int FY, bool PROP>
+template <int FY, bool PROP, bool STATS>
 cudaError_t ensure_smem_attr() {
     static bool attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(fit_tile_kernel<FY, PROP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(FusedSmem<FY>));
+        e = cudaFuncSetAttribute(fit_tile_kernel<FY, PROP, STATS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(FusedSmem<FY, STATS>));
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
     return cudaSuccess;
 }
 
-template <int FY, bool PROP>
+template <int FY, bool PROP, bool STATS>
 cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
     // the propagating form works on the pixel grid only
     if (PROP && d.cell != 1) return cudaErrorInvalidValue;
     const TableGrid lists{d.cell, d.GW, (size_t)d.PT};
-    cudaError_t e = ensure_smem_attr<FY, PROP>();
+    cudaError_t e = ensure_smem_attr<FY, PROP, STATS>();
     if (e != cudaSuccess) return e;
     const dim3 grid((d.W + FX - 1) / FX, (d.H + FY - 1) / FY);
-    fit_tile_kernel<FY, PROP><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY>), st>>>(d.records, d.table, d.target, d.H, d.W,
-                                                                           d.N, G, d.image, d.grads, d.ws, lists);
+    fit_tile_kernel<FY, PROP, STATS><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY, STATS>), st>>>(
+        d.records, d.table, d.target, d.H, d.W, d.N, G, d.image, d.grads, d.stats, d.ws, lists);
     return cudaGetLastError();
 }
+
+// taller tiles amortise the halo and the per-tile work, but hold more
+// distinct sites: use them unless sites are dense (< 4 pixels per site),
+// where tiles would often exceed the 128-site index
+bool tall_tiles(const Dev &d) { return (long long)d.H * d.W >= 4ll * d.N; }
 
 }  // namespace
 
 cudaError_t prepare_fused() {
-    cudaError_t e = ensure_smem_attr<8, true>();
-    if (e == cudaSuccess) e = ensure_smem_attr<16, true>();
-    if (e == cudaSuccess) e = ensure_smem_attr<8, false>();
-    if (e == cudaSuccess) e = ensure_smem_attr<16, false>();
+    cudaError_t e = ensure_smem_attr<8, true, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, true, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<8, false, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, false, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<8, false, true>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, false, true>();
     return e;
 }
 
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st) {
-    // taller tiles amortise the halo and the per-tile work, but hold more
-    // distinct sites: use them unless sites are dense (< 4 pixels per site),
-    // where tiles would often exceed the 128-site index
-    if ((long long)d.H * d.W >= 4ll * d.N) return launch_fit_tile_h<16, true>(d, G, st);
-    return launch_fit_tile_h<8, true>(d, G, st);
+    return tall_tiles(d) ? launch_fit_tile_h<16, true, false>(d, G, st) : launch_fit_tile_h<8, true, false>(d, G, st);
 }
 
 cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st) {
-    if ((long long)d.H * d.W >= 4ll * d.N) return launch_fit_tile_h<16, false>(d, 0, st);
-    return launch_fit_tile_h<8, false>(d, 0, st);
+    return tall_tiles(d) ? launch_fit_tile_h<16, false, false>(d, 0, st) : launch_fit_tile_h<8, false, false>(d, 0, st);
+}
+
+cudaError_t launch_fit_tile_cached_stats(const Dev &d, cudaStream_t st) {
+    return tall_tiles(d) ? launch_fit_tile_h<16, false, true>(d, 0, st) : launch_fit_tile_h<8, false, true>(d, 0, st);
 }
 
 }  // namespace sad

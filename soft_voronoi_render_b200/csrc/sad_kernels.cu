@@ -18,6 +18,8 @@
 //   target_u8_kernel    8-bit RGB -> planar float32 target
 // The fused steady-state pass is in sad_fused.cu, budget control in
 // sad_densify.cu, the 16-byte site record in sad_pack.cu.
+#include <cuda_fp16.h>
+
 #include "sad_device.cuh"
 #include "sad_launch.h"
 
@@ -86,7 +88,14 @@ __global__ void init_counters_kernel(Counters *c, uint32_t seed) {
     c->seed = seed;
     c->ticket_prop = c->ticket_bwd = c->ticket_adam = 0;
     c->hash_overflow = c->nonfinite_pixels = c->empty_pixels = c->dropped_ids = 0;
+    c->check_failures = 0;
     c->loss = 0.0;
+}
+
+__global__ void set_fit_state_kernel(Counters *c, uint32_t pass_counter, uint32_t adam_step, uint32_t seed) {
+    c->pass_counter = pass_counter;
+    c->adam_step = adam_step;
+    c->seed = seed;
 }
 
 __global__ void mark_inactive_kernel(float *prm, int N, int from) {
@@ -174,77 +183,160 @@ __global__ void seed_scatter_kernel(const float *__restrict__ prm, int N, int H,
 // ---------------------------------------------------------------------------
 // a2/a3: one Jacobi propagation pass.
 // ---------------------------------------------------------------------------
-// Offer a batch of up to 8 candidate ids.  Their records are fetched
-// together (independent loads in flight), then the candidates are offered in
-// order; the duplicate check runs at insertion time, so the result is the
-// same as offering them one by one.
-template <int NB>
-__device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], const float4 *__restrict__ rec,
-                                            uint32_t N, float fx, float fy) {
-    float l[NB];
+// A pass offers every pixel the 8 ids of each neighbour list (and the
+// injections).  In a refresh most of them are new to the pixel and about 6
+// of its 8 entries are replaced per pass, so the candidates are merged a
+// batch of 8 at a time without branches: the batch is scored, ids the pixel
+// already holds (or that repeat within the batch) are dropped, the batch is
+// sorted by Batcher's odd-even merge network and merged into the running
+// top-8 by a bitonic merge.  The top-8 of a set under the strict order
+// (logit desc, id asc) does not depend on how the set is assembled, so this
+// equals offering the ids one by one.
+
+// compare-exchange: afterwards (la, ia) ranks above (lb, ib)
+__device__ __forceinline__ void cx(float &la, uint32_t &ia, float &lb, uint32_t &ib) {
+    const bool s = ranks_above(lb, ib, la, ia);
+    const float tl = la;
+    const uint32_t ti = ia;
+    la = s ? lb : la;
+    ia = s ? ib : ia;
+    lb = s ? tl : lb;
+    ib = s ? ti : ib;
+}
+
+// sort 8 entries best first: Batcher's odd-even merge sort (19 comparators)
+__device__ __forceinline__ void sort8(float (&l)[K], uint32_t (&id)[K]) {
+    cx(l[0], id[0], l[1], id[1]); cx(l[2], id[2], l[3], id[3]); cx(l[4], id[4], l[5], id[5]); cx(l[6], id[6], l[7], id[7]);
+    cx(l[0], id[0], l[2], id[2]); cx(l[1], id[1], l[3], id[3]); cx(l[4], id[4], l[6], id[6]); cx(l[5], id[5], l[7], id[7]);
+    cx(l[1], id[1], l[2], id[2]); cx(l[5], id[5], l[6], id[6]);
+    cx(l[0], id[0], l[4], id[4]); cx(l[1], id[1], l[5], id[5]); cx(l[2], id[2], l[6], id[6]); cx(l[3], id[3], l[7], id[7]);
+    cx(l[2], id[2], l[4], id[4]); cx(l[3], id[3], l[5], id[5]);
+    cx(l[1], id[1], l[2], id[2]); cx(l[3], id[3], l[4], id[4]); cx(l[5], id[5], l[6], id[6]);
+}
+
+// keep the best 8 of the running list and a sorted batch: the better of
+// t[i] and batch[7 - i] for every i are the 8 best, as a bitonic sequence,
+// which half-cleaners at distances 4, 2 and 1 put in order
+__device__ __forceinline__ void merge8(Top8 &t, const float (&l)[K], const uint32_t (&id)[K]) {
 #pragma unroll
-    for (int q = 0; q < NB; ++q) {
-        l[q] = __int_as_float(0x7fc00000);  // NaN: not a candidate
-        const uint32_t id = ids[q];
-        if (id < N && !t.has(id)) {
-            const float4 r0 = __ldg(rec + (size_t)id * REC_F4);
-            const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
-            if (r0.x >= 0.0f) l[q] = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
-        }
+    for (int q = 0; q < K; ++q) {
+        const bool b = ranks_above(l[K - 1 - q], id[K - 1 - q], t.l[q], t.id[q]);
+        t.l[q] = b ? l[K - 1 - q] : t.l[q];
+        t.id[q] = b ? id[K - 1 - q] : t.id[q];
     }
 #pragma unroll
-    for (int q = 0; q < NB; ++q) {
-        if (l[q] == l[q] && t.beats_last(l[q], ids[q]) && !t.has(ids[q])) t.insert(l[q], ids[q]);
+    for (int d = 4; d >= 1; d >>= 1)
+#pragma unroll
+        for (int q = 0; q < K; ++q)
+            if ((q & d) == 0) cx(t.l[q], t.id[q], t.l[q + d], t.id[q + d]);
+}
+
+// Logit of site x at (fx, fy) for ranking candidates: from the float32 score
+// record, or (F16) from the packed candidate-site record -- x, y as float32,
+// (A, B) and (C, b) as binary16 pairs -- with the same operation order.
+template <bool F16>
+__device__ __forceinline__ float cand_logit(const float4 *__restrict__ rec, const uint4 *__restrict__ c16,
+                                            uint32_t x, float fx, float fy, bool &active) {
+    if constexpr (F16) {
+        const uint4 v = __ldg(c16 + x);
+        const float px = __uint_as_float(v.x), py = __uint_as_float(v.y);
+        const float2 ab = __half22float2(*reinterpret_cast<const __half2 *>(&v.z));
+        const float2 cb = __half22float2(*reinterpret_cast<const __half2 *>(&v.w));
+        active = px >= 0.0f;
+        return sad_logit(px, py, ab.x, ab.y, cb.x, cb.y, fx, fy);
+    } else {
+        const float4 r0 = __ldg(rec + (size_t)x * REC_F4);
+        const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)x * REC_F4 + 1));
+        active = r0.x >= 0.0f;
+        return sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+    }
+}
+
+// Offer up to 8 candidate ids as one batch.  Their records are fetched
+// together (independent loads in flight).  Invalid entries (id >= N,
+// inactive site, NaN logit, an id already held or repeated earlier in the
+// batch) become (-inf, EMPTY), which ranks below every candidate.  When no
+// active lane has a candidate that beats its 8th, the network is skipped.
+template <int NB, bool F16 = false>
+__device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], const float4 *__restrict__ rec,
+                                            const uint4 *__restrict__ c16, uint32_t N, float fx, float fy) {
+    float l[K];
+    uint32_t id[K];
+    bool enters = false;
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+        l[q] = -__int_as_float(0x7f800000);
+        id[q] = EMPTY;
+        if (q < NB) {
+            const uint32_t x = ids[q];
+            bool fresh = x < N && !t.has(x);
+#pragma unroll
+            for (int r = 0; r < q; ++r) fresh &= x != ids[r];
+            if (fresh) {
+                bool active;
+                const float lv = cand_logit<F16>(rec, c16, x, fx, fy, active);
+                if (active && lv == lv) {
+                    l[q] = lv;
+                    id[q] = x;
+                    enters |= t.beats_last(lv, x);
+                }
+            }
+        }
+    }
+    if (__any_sync(__activemask(), enters)) {
+        sort8(l, id);
+        merge8(t, l, id);
     }
 }
 
 // The pixel's own list as the first candidates of a pass into an empty list:
 // re-scored in its previous order it is usually still sorted and free of
 // repeats (the records do not change between refresh passes), and then it is
-// the top-8 of its own candidates as it stands; otherwise its ids are offered
-// one by one like any other list.  Same result either way.
+// the top-8 of its own candidates as it stands; otherwise its repeats are
+// dropped and it is sorted.  Same result either way.
+template <bool F16>
 __device__ __forceinline__ void take_own_list(Top8 &t, const uint4 a, const uint4 b, const float4 *__restrict__ rec,
-                                              uint32_t N, float fx, float fy) {
+                                              const uint4 *__restrict__ c16, uint32_t N, float fx, float fy) {
     const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    float l[8];
-    uint32_t id[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-        l[q] = -__int_as_float(0x7f800000);
-        id[q] = EMPTY;
+        t.l[q] = -__int_as_float(0x7f800000);
+        t.id[q] = EMPTY;
         if (ids[q] < N) {
-            const float4 r0 = __ldg(rec + (size_t)ids[q] * REC_F4);
-            const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)ids[q] * REC_F4 + 1));
-            if (r0.x >= 0.0f) {
-                const float lv = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
-                if (lv == lv) {
-                    l[q] = lv;
-                    id[q] = ids[q];
-                }
+            bool active;
+            const float lv = cand_logit<F16>(rec, c16, ids[q], fx, fy, active);
+            if (active && lv == lv) {
+                t.l[q] = lv;
+                t.id[q] = ids[q];
             }
         }
     }
     bool clean = true;
 #pragma unroll
     for (int q = 1; q < 8; ++q) {
-        clean &= !ranks_above(l[q], id[q], l[q - 1], id[q - 1]);
+        clean &= !ranks_above(t.l[q], t.id[q], t.l[q - 1], t.id[q - 1]);
 #pragma unroll
-        for (int r = 0; r < q; ++r) clean &= (id[q] == EMPTY) || (id[q] != id[r]);
+        for (int r = 0; r < q; ++r) clean &= (t.id[q] == EMPTY) || (t.id[q] != t.id[r]);
     }
-    if (clean) {
+    if (__any_sync(__activemask(), !clean)) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            t.l[q] = l[q];
-            t.id[q] = id[q];
-        }
-    } else {
-        offer_batch<8>(t, ids, rec, N, fx, fy);
+        for (int q = 1; q < 8; ++q)
+#pragma unroll
+            for (int r = 0; r < q; ++r)
+                if (t.id[q] != EMPTY && t.id[q] == t.id[r]) {
+                    t.l[q] = -__int_as_float(0x7f800000);
+                    t.id[q] = EMPTY;
+                }
+        sort8(t.l, t.id);
     }
 }
 
 // H x W is the candidate grid; a cell is scored at its centre, (i + 0.5) cs
-// (cs = 1: the pixel grid)
-__global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *__restrict__ rec, uint32_t *table,
+// (cs = 1: the pixel grid).  F16: candidates are ranked on the packed
+// records c16 and the kept 8 re-scored with the float32 records.
+template <bool F16>
+__global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *__restrict__ rec,
+                                                                 const uint4 *__restrict__ c16, uint32_t *table,
                                                                  int H, int W, float cs, int N, int jump, int G,
                                                                  Counters *c) {
     const uint32_t cur = c->cur, pass = c->pass_counter, seed = c->seed;
@@ -259,26 +351,29 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
         const size_t p = (size_t)j * W + i;
         const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
         Top8 t;
-        t.clear();
-        take_own_list(t, in0[p], in1[p], rec, (uint32_t)N, fx, fy);
-        // the neighbours at (-k, 0), (+k, 0), (0, -k), (0, +k)
+        take_own_list<F16>(t, in0[p], in1[p], rec, c16, (uint32_t)N, fx, fy);
+        // the neighbours at (-k, 0), (+k, 0), (0, -k), (0, +k); one outside
+        // the image offers nothing
 #pragma unroll 1
         for (int d = 1; d < 5; ++d) {
             const int ni = i + (d == 1 ? -jump : (d == 2 ? jump : 0));
             const int nj = j + (d == 3 ? -jump : (d == 4 ? jump : 0));
-            if (ni < 0 || ni >= W || nj < 0 || nj >= H) continue;
-            const size_t pn = (size_t)nj * W + ni;
-            const uint4 a = in0[pn], b = in1[pn];
+            uint4 a = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY), b = a;
+            if (ni >= 0 && ni < W && nj >= 0 && nj < H) {
+                const size_t pn = (size_t)nj * W + ni;
+                a = in0[pn];
+                b = in1[pn];
+            }
             const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            offer_batch<8>(t, ids, rec, (uint32_t)N, fx, fy);
+            offer_batch<8, F16>(t, ids, rec, c16, (uint32_t)N, fx, fy);
         }
         if (G > 0) {
             uint32_t h = inject_state(seed, pass, (uint32_t)p);
 #pragma unroll 1
-            for (int g0 = 0; g0 < G; g0 += 4) {
-                uint32_t ids[4];
+            for (int g0 = 0; g0 < G; g0 += 8) {
+                uint32_t ids[8];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 8; ++q) {
                     if (g0 + q < G) {
                         h = xorshift32(h);
                         ids[q] = __umulhi(h, (uint32_t)N);
@@ -286,8 +381,18 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
                         ids[q] = EMPTY;
                     }
                 }
-                offer_batch<4>(t, ids, rec, (uint32_t)N, fx, fy);
+                offer_batch<8, F16>(t, ids, rec, c16, (uint32_t)N, fx, fy);
             }
+        }
+        if constexpr (F16) {
+            // the kept 8 in float32 logit order
+#pragma unroll
+            for (int q = 0; q < K; ++q) {
+                if (t.id[q] == EMPTY) continue;
+                bool active;
+                t.l[q] = cand_logit<false>(rec, nullptr, t.id[q], fx, fy, active);
+            }
+            sort8(t.l, t.id);
         }
         out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
         out1[p] = make_uint4(t.id[4], t.id[5], t.id[6], t.id[7]);
@@ -305,6 +410,21 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
             __threadfence();
         }
     }
+}
+
+// Packed candidate-site record of every site (summary B.2): x and y as
+// float32, then (A, B) and (C, b) rounded to binary16 pairs (round to
+// nearest even, overflow to infinity).
+__global__ void __launch_bounds__(SITE_THREADS) pack_cand16_kernel(const float4 *__restrict__ rec, int N,
+                                                                   uint4 *__restrict__ c16) {
+    const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
+    if (i >= N) return;
+    const float4 r0 = rec[(size_t)i * REC_F4];
+    const float4 r1 = rec[(size_t)i * REC_F4 + 1];
+    const __half2 ab = __floats2half2_rn(r0.z, r0.w);
+    const __half2 cb = __floats2half2_rn(r1.x, r1.y);
+    c16[i] = make_uint4(__float_as_uint(r0.x), __float_as_uint(r0.y), *reinterpret_cast<const uint32_t *>(&ab),
+                        *reinterpret_cast<const uint32_t *>(&cb));
 }
 
 // One 3x3 flood pass of the optional JFA prepass (summary B.3): the 4 best
@@ -332,7 +452,7 @@ __global__ void __launch_bounds__(TILE_THREADS) jfa3x3_kernel(const float4 *__re
             const size_t pn = (size_t)nj * W + ni;
             const uint4 a = in0[pn], b = in1[pn];
             const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            offer_batch<8>(t, ids, rec, (uint32_t)N, fx, fy);
+            offer_batch<8>(t, ids, rec, nullptr, (uint32_t)N, fx, fy);
         }
         out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
         out1[p] = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY);
@@ -459,26 +579,20 @@ __device__ __forceinline__ int hash_find_or_insert(uint32_t *keys, uint32_t id) 
     return -1;
 }
 
-// STATS additionally accumulates the budget-control statistics per site
-// (summary B.4-B.5): mass sum w, energy sum w e, second moments
-// sum w e (dx^2, dx dy, dy^2) and the removal delta
-// sum |(chat - w c) / max(1 - w, 1e-6) - t|^2 - e, with e = |chat - t|^2.
 // DET (deterministic): every run sum is rounded to a multiple of 2^-40 and
 // added to a 64-bit fixed-point accumulator per (parameter, site) with
 // integer atomics, which are exact and so independent of their order (the
 // pages' integer-atomic gradient accumulation, summary B.4); no tile table.
 constexpr float DET_SCALE = 1099511627776.0f;  // 2^40
 
-template <bool STATS, bool DET = false>
+template <bool DET>
 __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *__restrict__ rec,
                                                                   const uint32_t *__restrict__ table,
                                                                   const float *__restrict__ target, int H, int W,
                                                                   TableGrid tg, int N, float *__restrict__ image,
-                                                                  float *__restrict__ grads,
-                                                                  float *__restrict__ stats, void *ws,
+                                                                  float *__restrict__ grads, void *ws,
                                                                   unsigned long long *__restrict__ fixed) {
-    static_assert(!(STATS && DET), "the deterministic backward carries the gradients only");
-    constexpr int NV = STATS ? NPARAM + NSTAT : NPARAM;
+    constexpr int NV = NPARAM;
     __shared__ uint32_t keys[HASH_SLOTS];
     __shared__ float acc[NV][HASH_SLOTS];
     __shared__ float warp_loss[TILE_THREADS / 32];
@@ -527,29 +641,6 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
         gb = 2.0f * eb * invP;
         iz = nv ? 1.0f / s.Z : 0.0f;
     }
-    // STATS: the weight and colour sums over all slots but the dominant one,
-    // summed directly (the removal of the dominant site must not subtract
-    // two nearly equal numbers)
-    int qstar = -1;
-    float zmm = 0.0f, cmr = 0.0f, cmg = 0.0f, cmb = 0.0f;
-    if constexpr (STATS) {
-        float emax = -1.0f;
-#pragma unroll
-        for (int q = 0; q < K; ++q)
-            if ((s.valid >> q & 1u) && s.l[q] > emax) {
-                emax = s.l[q];
-                qstar = q;
-            }
-#pragma unroll
-        for (int q = 0; q < K; ++q) {
-            if (!(s.valid >> q & 1u) || q == qstar) continue;
-            const float4 r2 = __ldg(rec + (size_t)s.id[q] * REC_F4 + 2);
-            zmm += s.l[q];
-            cmr = fmaf(s.l[q], r2.x, cmr);
-            cmg = fmaf(s.l[q], r2.y, cmg);
-            cmb = fmaf(s.l[q], r2.z, cmb);
-        }
-    }
     // every lane runs the slot loop (the run reduction needs the whole warp)
 #pragma unroll
     for (int q = 0; q < K; ++q) {
@@ -578,38 +669,6 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
             v[PCB] = w * gb;
             v[PTH] = -gi * al * be * (r3.y - r3.z);
             v[PA] = -0.5f * gi * (r3.y * al * al - r3.z * be * be);
-            if constexpr (STATS) {
-                const float ex = er * er + eg * eg + eb * eb;  // e = |chat - t|^2
-                // removal delta |a|^2 - |b|^2 = (a - b) . (a + b) with b = chat - t,
-                // a = (chat - w c) / max(1 - w, 1e-6) - t; the sums over the other
-                // slots come in unnormalised form: sum_{j != q} e_j (and e_j c_j)
-                const float Z = s.Z, eq = s.l[q];
-                const float oz = q == qstar ? zmm : Z - eq;
-                const float ocr = q == qstar ? cmr : fmaf(-eq, r2.x, s.cr * Z);
-                const float ocg = q == qstar ? cmg : fmaf(-eq, r2.y, s.cg * Z);
-                const float ocb = q == qstar ? cmb : fmaf(-eq, r2.z, s.cb * Z);
-                const float rest = oz * iz;  // 1 - w, without cancellation
-                float dr, dg, db;
-                if (rest >= 1e-6f) {
-                    // a - b = w (chat - c) / (1 - w) = w (c_rest - c), with c_rest the
-                    // blend of the other slots (chat - c itself cancels when w -> 1)
-                    const float ioz = 1.0f / oz;
-                    dr = w * (ocr * ioz - r2.x);
-                    dg = w * (ocg * ioz - r2.y);
-                    db = w * (ocb * ioz - r2.z);
-                } else {
-                    dr = ocr * iz * 1e6f - s.cr;
-                    dg = ocg * iz * 1e6f - s.cg;
-                    db = ocb * iz * 1e6f - s.cb;
-                }
-                const float we = w * ex;
-                v[NPARAM + 0] = w;
-                v[NPARAM + 1] = we;
-                v[NPARAM + 2] = we * dx * dx;
-                v[NPARAM + 3] = we * dx * dy;
-                v[NPARAM + 4] = we * dy * dy;
-                v[NPARAM + 5] = dr * (2.0f * er + dr) + dg * (2.0f * eg + dg) + db * (2.0f * eb + db);
-            }
         }
         const bool tail = warp_run_reduce(key, v, lane);
         if (DET) {
@@ -629,10 +688,6 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
                 ++overflow;
 #pragma unroll
                 for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + key, v[k]);
-                if constexpr (STATS) {
-#pragma unroll
-                    for (int k = 0; k < NSTAT; ++k) atomicAdd(stats + (size_t)k * N + key, v[NPARAM + k]);
-                }
             }
         }
     }
@@ -651,13 +706,6 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
         for (int k = 0; k < NPARAM; ++k) {
             const float a = acc[k][q];
             if (a != 0.0f) atomicAdd(grads + (size_t)k * N + id, a);
-        }
-        if constexpr (STATS) {
-#pragma unroll
-            for (int k = 0; k < NSTAT; ++k) {
-                const float a = acc[NPARAM + k][q];
-                if (a != 0.0f) atomicAdd(stats + (size_t)k * N + id, a);
-            }
         }
     }
     if (tid == 0) {
@@ -866,6 +914,12 @@ cudaError_t launch_init_counters(const Dev &d, uint32_t seed, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+cudaError_t launch_set_fit_state(const Dev &d, uint32_t pass_counter, uint32_t adam_step, uint32_t seed,
+                                 cudaStream_t st) {
+    set_fit_state_kernel<<<1, 1, 0, st>>>(host_counters(d), pass_counter, adam_step, seed);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_mark_inactive(const Dev &d, int from, cudaStream_t st) {
     if (from >= d.N) return cudaSuccess;
     mark_inactive_kernel<<<site_blocks(d.N - from), SITE_THREADS, 0, st>>>(d.params, d.N, from);
@@ -905,8 +959,17 @@ cudaError_t launch_seed(const Dev &d, cudaStream_t st) {
 }
 
 cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st) {
-    propagate_kernel<<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d));
+    if (d.f16)
+        propagate_kernel<true><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
+            d.records, d.cand16, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d));
+    else
+        propagate_kernel<false><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
+            d.records, nullptr, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_cand16(const Dev &d, cudaStream_t st) {
+    pack_cand16_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.records, d.N, d.cand16);
     return cudaGetLastError();
 }
 
@@ -924,21 +987,15 @@ cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st) {
 
 cudaError_t launch_render_backward(const Dev &d, cudaStream_t st) {
     render_bwd_kernel<false><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, nullptr, d.ws, nullptr);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_render_backward_stats(const Dev &d, cudaStream_t st) {
-    render_bwd_kernel<true><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, d.stats, d.ws, nullptr);
+        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, d.ws, nullptr);
     return cudaGetLastError();
 }
 
 cudaError_t launch_render_backward_det(const Dev &d, cudaStream_t st) {
     unsigned long long *fixed =
         reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(d.ws) + fixed_offset(d.H, d.W, d.N));
-    render_bwd_kernel<false, true><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, nullptr, d.ws, fixed);
+    render_bwd_kernel<true><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
+        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, d.ws, fixed);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long n = (long long)NPARAM * d.N;

@@ -18,6 +18,8 @@ struct Dev {
     float *target, *image;
     float *stats;  // [6][N] budget-control statistics (optional)
     const uint8_t *frozen;  // [N] sites Adam leaves untouched (optional)
+    uint4 *cand16;          // [N] packed candidate-site records (optional)
+    bool f16;               // candidate updates rank on cand16
     void *ws;
 };
 
@@ -35,6 +37,8 @@ size_t workspace_bytes(int H, int W, int N);
 size_t densify_offset(int H, int W);
 
 cudaError_t launch_init_counters(const Dev &d, uint32_t seed, cudaStream_t st);
+cudaError_t launch_set_fit_state(const Dev &d, uint32_t pass_counter, uint32_t adam_step, uint32_t seed,
+                                 cudaStream_t st);
 cudaError_t launch_mark_inactive(const Dev &d, int from, cudaStream_t st);
 cudaError_t launch_records(const Dev &d, cudaStream_t st);
 cudaError_t launch_target_u8(const Dev &d, const uint8_t *src, cudaStream_t st);
@@ -42,14 +46,15 @@ cudaError_t launch_topk_exact(const Dev &d, const int64_t *pix, int64_t n, uint3
 cudaError_t launch_seed(const Dev &d, cudaStream_t st);
 cudaError_t launch_clear_table(const Dev &d, cudaStream_t st);
 cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st);
+cudaError_t launch_pack_cand16(const Dev &d, cudaStream_t st);
 cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st);
 cudaError_t launch_render_backward(const Dev &d, cudaStream_t st);
-cudaError_t launch_render_backward_stats(const Dev &d, cudaStream_t st);
 cudaError_t launch_render_backward_det(const Dev &d, cudaStream_t st);
 cudaError_t launch_densify(const Dev &d, const DensifyArgs &a, cudaStream_t st);
 cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st);
 cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st);
 cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st);
+cudaError_t launch_fit_tile_cached_stats(const Dev &d, cudaStream_t st);
 cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st);
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st);
 cudaError_t prepare_fused();

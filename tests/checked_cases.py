@@ -1,0 +1,61 @@
+"""Cases run against the bounds-checked debug build (libsad_checks.so).
+
+Run as a script in a process of its own with SAD_CHECKS=1 in the
+environment (the library is chosen when it is first loaded).  Each case runs
+the kernels whose indices rest on invariants rather than explicit guards --
+the fused pass (tile index, masks, grouped entries), the cached-list pass,
+the statistics backward, the standalone propagation and refresh -- on tiny
+and ragged sizes, checks the result against the CPU oracle, and reads the
+number of accesses the device-side checks refused.  Prints one JSON line."""
+import json
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import oracle  # noqa: E402
+import synth  # noqa: E402
+
+
+def main():
+    assert os.environ.get("SAD_CHECKS") == "1"
+    from soft_voronoi_render_b200 import SAD_STATS, Sad, _lib
+    assert _lib.library_path().endswith("libsad_checks.so")
+    out = {"cases": 0, "check_failures": 0}
+    for (H, W, N, seed) in ((1, 1, 3, 1), (9, 33, 40, 2), (37, 53, 300, 3), (16, 40, 200, 4), (24, 72, 6000, 5)):
+        prm = synth.uniform_sites(H, W, N, seed)
+        tgt = synth.make_image(H, W, 4, 0, seed)
+        t0 = oracle.topk_exact(H, W, oracle.records(H, W, prm))
+        if N == 200:
+            t0[::3, 5] = t0[::3, 1]
+            t0[::7, 7] = N + 11
+        s = Sad(H, W, N, seed=seed)
+        s.set_sites(prm)
+        s.set_target(tgt)
+        s.set_table(t0)
+        s.fit_pass(2)
+        t1 = oracle.propagate(H, W, oracle.records(H, W, prm), t0, 1, 2, seed=seed, pass_index=0)
+        assert np.array_equal(s.get_table(), t1), (H, W, N)
+        L, g = oracle.loss_backward(H, W, prm, t1, tgt)
+        assert abs(s.loss() - L) <= 1e-5 * L
+        gg = s.grads.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(gg - g) <= np.maximum(1e-4 * np.abs(g), 1e-6))
+        s.grads.zero_()
+        s.fit_pass_cached()
+        s.grads.zero_()
+        s.backward(SAD_STATS)
+        s.refresh(2)
+        ref, _ = oracle.refresh(H, W, prm, 2, seed=seed, first_pass=1)
+        assert np.array_equal(s.get_table(), ref), (H, W, N)
+        st = s.stats()
+        out["cases"] += 1
+        out["check_failures"] += st["check_failures"]
+        s.close()
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

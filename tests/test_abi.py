@@ -25,6 +25,11 @@ def test_library_exports_every_declared_symbol():
     L = _lib.load()
     for name in _declared():
         assert hasattr(L, name), name
+    # the bounds-checked debug build exports the same ABI
+    from soft_voronoi_render_b200 import build as _build
+    Lc = ctypes.CDLL(_build.LIB_CHECKS)
+    for name in _declared():
+        assert hasattr(Lc, name), name
 
 
 def test_create_validates_arguments():
@@ -58,6 +63,9 @@ def test_bind_checks_alignment_and_sizes_without_touching_memory():
         # calls that need bound buffers fail before binding
         with pytest.raises(_lib.SadError) as e:
             _lib.sad_render(ctx)
+        assert e.value.status == _lib.SAD_ERR_NOT_BOUND
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_set_fit_state(ctx, 0, 0, 1)
         assert e.value.status == _lib.SAD_ERR_NOT_BOUND
         with pytest.raises(_lib.SadError) as e:
             _lib.sad_bind(ctx, **{**fake, "records": 0x50004})
@@ -122,6 +130,21 @@ def test_bind_checks_alignment_and_sizes_without_touching_memory():
         with pytest.raises(_lib.SadError) as e:
             _lib.sad_unpack_sites(ctx, 0xC0000, None)
         assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        # packed candidates need a bound cand16 buffer; only 32 and 16 bits
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_set_candidate_precision(ctx, 16)
+        assert e.value.status == _lib.SAD_ERR_NOT_BOUND
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_set_candidate_precision(ctx, 8)
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        _lib.sad_set_candidate_precision(ctx, 32)
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_bind(ctx, **fake, cand16=0xD0008)
+        assert "cand16" in str(e.value)
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_set_fit_state(ctx, 1, 1, 1, reserved=3)
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        assert _lib.load().sad_get_fit_state(ctx, None, None) == _lib.SAD_ERR_INVALID_ARG
     finally:
         _lib.sad_destroy(ctx)
 

@@ -55,6 +55,42 @@ def test_backward_stats(torch_cuda, wl):
     assert np.all(np.abs(sg - st) <= tol), [float((np.abs(sg - st) / tol)[r].max()) for r in range(6)]
 
 
+@pytest.mark.parametrize("case", ["crowded", "repeated"])
+def test_backward_stats_edge_cases(torch_cuda, case):
+    """Statistics where tiles hold more sites than the tile index (every
+    entry takes the global-atomic path) and where lists repeat an id or hold
+    one beyond capacity (each slot counts on its own, the stray id is
+    dropped)."""
+    from soft_voronoi_render_b200 import SAD_STATS
+    if case == "crowded":
+        H, W, N = 24, 72, 6000
+    else:
+        H, W, N = 40, 70, 300
+    prm = synth.uniform_sites(H, W, N, 31)
+    tgt = synth.make_image(H, W, 8, 0, 31)
+    table = oracle.topk_exact(H, W, oracle.records(H, W, prm))
+    if case == "repeated":
+        table[::5, 6] = table[::5, 2]
+        table[::11, 7] = N + 3
+    s = _ctx(H, W, N, prm, tgt)
+    s.set_table(table)
+    s.backward(SAD_STATS)
+    clean = table.copy()
+    clean[clean >= N] = 0xFFFFFFFF
+    L, g, st, sa = oracle.loss_backward_stats(H, W, prm, clean, tgt, want_abs=True)
+    assert abs(s.loss() - L) <= 1e-5 * L
+    gg = s.grads.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(gg - g) <= np.maximum(GRAD_RTOL * np.abs(g), GRAD_ATOL))
+    sg = s.site_stats.cpu().numpy().astype(np.float64)
+    tol = 1e-4 * np.abs(st) + 3e-5 * sa + 1e-9
+    assert np.all(np.abs(sg - st) <= tol), [float((np.abs(sg - st) / tol)[r].max()) for r in range(6)]
+    info = s.stats()
+    if case == "crowded":
+        assert info["hash_overflow"] > 0
+    else:
+        assert info["dropped_ids"] > 0
+
+
 def test_densify_prune_matches_oracle(torch_cuda):
     H, W, N = 96, 128, 3000
     tgt = synth.make_image(H, W, 20, 0, 21)

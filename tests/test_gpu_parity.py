@@ -407,6 +407,46 @@ def test_full_size_c3_iteration_pieces(torch_cuda):
 
 
 @pytest.mark.slow
+def test_full_size_c3_benchmark_state(torch_cuda):
+    """2048 x 2048, N = 131,072 in the state the benchmark times: a refresh
+    and 50 fitting iterations (fused pass + Adam) on the GPU.  From the GPU's
+    own sites and current lists, one more fused pass is bit-exact against the
+    oracle's propagation (run on the device records' bits, which first agree
+    with the oracle's own records within 4 ulps) and agrees with the oracle's
+    render and backward."""
+    from soft_voronoi_render_b200 import adam_cfg
+    tgt, prm, w = synth.make_workload("c3", seed=1)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt, seed=1)
+    s.refresh(w.G)
+    cfg = adam_cfg(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=5e-3, lr_theta=1e-3, lr_a=1e-3)
+    for _ in range(50):
+        s.fit_iteration(w.G, cfg)
+    prm_now = s.get_sites()
+    table = s.get_table()
+    rec_dev = s.records.cpu().numpy()
+    pass_index = s.stats()["pass_counter"]
+    rec_orc = oracle.records(w.H, w.W, prm_now)
+    ulps = np.abs(rec_dev.view(np.int32).astype(np.int64) - rec_orc.view(np.int32).astype(np.int64))
+    assert ulps.max() <= 4, int(ulps.max())
+    assert not np.array_equal(prm_now, prm)  # the sites did move
+    s.grads.zero_()
+    before = s.stats()["hash_overflow"]
+    s.fit_pass(w.G)
+    ref = oracle.propagate(w.H, w.W, rec_dev, table, 1, w.G, seed=1, pass_index=pass_index)
+    got = s.get_table()
+    np.testing.assert_array_equal(got, ref)
+    assert (got != table).any(axis=1).mean() > 0.01  # lists still change in this state
+    L, g, img = oracle.loss_backward(w.H, w.W, prm_now, ref, tgt, want_image=True)
+    assert abs(s.loss() - L) <= LOSS_RTOL * L
+    assert np.abs(s.image.cpu().numpy() - img).max() <= RENDER_ATOL
+    assert_grads(s.grads.cpu().numpy(), g, "c3 benchmark state")
+    st = s.stats()
+    assert st["empty_pixels"] == 0
+    # report how often entries took the global-atomic path in this pass
+    print("global-atomic pixels in the pass:", st["hash_overflow"] - before)
+
+
+@pytest.mark.slow
 def test_full_size_c4_refresh_and_render(torch_cuda):
     """4096 x 4096, N = 524,288: the full refresh (seed + jumps 2048..1, G = 4)
     is bit-exact against the oracle's, the render of it agrees, and the
