@@ -686,8 +686,12 @@ double orc_loss_backward_stats(int H, int W, int N, const float *params, const u
  *   m <- b1 m + (1 - b1) ghat;   v <- b2 v + (1 - b2) ghat^2
  *   param <- param - lr_j sigma_j (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
  * then the position is clamped into [0, W^-] x [0, H^-] (W^- the largest
- * float below W).  Inactive sites are left untouched.  All arrays 9 x N
- * doubles, in place.
+ * float below W).  The clamp is a reading of this build, not a step of the
+ * pages: they mark a pruned site with x < 0 ([P1] B.2, B.5), which an
+ * optimiser step must not produce, and they say nothing about the upper
+ * edges or y; clamping every coordinate into the image is the plainest way
+ * to keep an active site active and inside the image it fits.  Inactive
+ * sites are left untouched.  All arrays 9 x N doubles, in place.
  */
 void orc_adam_frozen(int H, int W, int N, double *params, double *m, double *v, const double *grads,
                      const double *lr, double b1, double b2, double eps, int t, const uint8_t *frozen);
