@@ -264,12 +264,22 @@ def time_oracle_steps(tgt, prm, H, W, G, rows, n_steps, budget_s):
 
 
 def cpu_baseline(tgt, prm, wl, budget_s=15.0, rows=256):
+    """The oracle on all host cores (the reported baseline), and the same
+    sample on one core beside it."""
     import oracle
     done, dt, px = time_oracle_steps(tgt, prm, wl.H, wl.W, wl.G, rows, 10 ** 6, budget_s)
-    return {"value": px * done / dt / 1e6, "unit": "Mpix/s", "cores": oracle.num_threads(), "kind": "oracle",
+    all_threads = oracle.num_threads()
+    oracle.set_threads(1)
+    try:
+        done1, dt1, px1 = time_oracle_steps(tgt, prm, wl.H, wl.W, wl.G, rows // 4, 10 ** 6, budget_s / 3)
+    finally:
+        oracle.set_threads(all_threads)
+    return {"value": px * done / dt / 1e6, "unit": "Mpix/s", "cores": all_threads, "kind": "oracle",
             "sample": f"{done} oracle fit iterations (propagate k=1 G={wl.G}, fp64 render+backward, Adam on the "
                       f"band's share of {int(round(wl.N * rows / wl.H))} sites, record rebuild) on a {rows}-row x "
-                      f"{wl.W} band of the {wl.H}x{wl.W} N={wl.N} workload, {dt:.1f} s"}
+                      f"{wl.W} band of the {wl.H}x{wl.W} N={wl.N} workload, {dt:.1f} s",
+            "one_core": {"value": px1 * done1 / dt1 / 1e6, "cores": 1,
+                         "sample": f"{done1} iterations on a {rows // 4}-row band, {dt1:.1f} s"}}
 
 
 def workload_config(wl, world: int) -> dict:

@@ -115,6 +115,20 @@ __device__ __forceinline__ uint32_t ukey_insert(uint32_t *keys, uint32_t id) {
     return NOSLOT;
 }
 
+// insert once per run of equal ids on consecutive lanes: the first lane of
+// the run inserts, the others take its slot (neighbouring pixels mostly hold
+// the same id in the same slot, which would otherwise contend for one key).
+// An id >= N inserts nothing and gets NOSLOT.
+__device__ __forceinline__ uint32_t warp_insert(uint32_t *keys, uint32_t id, uint32_t N, int lane) {
+    const uint32_t prev = __shfl_up_sync(FULL, id, 1);
+    const bool head = lane == 0 || prev != id;
+    const uint32_t heads = __ballot_sync(FULL, head);
+    const int start = 31 - __clz(heads & (0xFFFFFFFFu >> (31 - lane)));
+    uint32_t s = NOSLOT;
+    if (head && id < N) s = ukey_insert(keys, id);
+    return __shfl_sync(FULL, s, start);
+}
+
 __device__ __forceinline__ uint32_t ukey_lookup(const uint32_t *keys, const uint32_t *lid, uint32_t id) {
     uint32_t s = uhash(id);
 #pragma unroll 1
@@ -137,10 +151,12 @@ template <int FY, bool STATS>
 struct FusedSmem {
     static constexpr int FT = FX * FY, HN = HX * (FY + 2), RING = HN - FT;
     // The tile's (pixel, slot) entries grouped by site, each site's run padded
-    // to a multiple of 8 so that every group of 8 belongs to one site: at most
+    // to a multiple of the group size gs (8, or 9 where that makes the groups
+    // fit one per thread) so that every group belongs to one site: at most
     // FT + 7 UCAP / 8 groups.  Entry e of group g is stored at [e][g]; the
     // plane strides are 4 words modulo 32 so that the scatter's consecutive
     // entries (consecutive e) fall in distinct banks.
+    static constexpr int GMAX = FY == 16 ? 9 : 8;
     static constexpr int NG = FT + 7 * UCAP / 8;
     static constexpr int NGS = (NG + 15) / 16 * 16 + 2;    // float2 planes
     static constexpr int NGS16 = (NG + 63) / 64 * 64 + 8;  // uint16 planes
@@ -152,15 +168,15 @@ struct FusedSmem {
     uint32_t cnt[UCAP];             // (pixel, slot) entries per local site
     uint32_t cursor[UCAP];          // scatter cursor; afterwards the end of each site's entries
     float4 pixg[FT];                // per pixel: dL/dchat (3), chat . dL/dchat
-    float2 ent_wl[K][NGS];          // softmax weight, logit
-    uint16_t ent_pu[K][NGS16];      // pixel (low 9 bits), local site (high 7 bits)
-    float ent_rd[STATS ? K : 1][STATS ? NGS : 1];  // removal delta (budget statistics)
+    float2 ent_wl[GMAX][NGS];       // softmax weight, logit
+    uint16_t ent_pu[GMAX][NGS16];   // pixel (low 9 bits), local site (high 7 bits)
+    float ent_rd[STATS ? GMAX : 1][STATS ? NGS : 1];  // removal delta (budget statistics)
     float warp_loss[FY];
     uint32_t warp_cnt[3][FY];       // per warp: empty pixels, global-atomic pixels, dropped ids
     uint32_t n_groups;
+    uint32_t gs;                    // entries per group
     uint32_t ucount;
     int overflow;
-    int last;
 };
 
 // halo ring pixel r -> halo coordinates: top row, bottom row, then the left
@@ -390,22 +406,15 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     bool ok = true;
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-        slot[q] = NOSLOT;
-        if (own[q] < Nu) {
-            slot[q] = ukey_insert(sm.keys, own[q]);
-            ok &= slot[q] != NOSLOT;
-        }
+        slot[q] = warp_insert(sm.keys, own[q], Nu, lane);
+        ok &= own[q] >= Nu || slot[q] != NOSLOT;
     }
     if (PROP) {
 #pragma unroll
         for (int x = 0; x < NRE; ++x) {
-            uint32_t v = NOLOC;
-            if (rv[x] < Nu) {
-                const uint32_t s = ukey_insert(sm.keys, rv[x]);
-                ok &= s != NOSLOT;
-                if (s != NOSLOT) v = s | (rcell[x] << 16);
-            }
-            rv[x] = v;
+            const uint32_t s = warp_insert(sm.keys, rv[x], Nu, lane);
+            ok &= rv[x] >= Nu || s != NOSLOT;
+            rv[x] = s != NOSLOT ? (s | (rcell[x] << 16)) : NOLOC;
         }
     }
     if (!ok) sm.overflow = 1;
@@ -427,7 +436,15 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     // slot q's local index in byte q & 3 of own_lx[q >> 2] (0xFF: none)
     uint32_t own_lx_lo = 0xFFFFFFFFu, own_lx_hi = 0xFFFFFFFFu;
     if (fast) {
-        // ---- A3: local indices, membership masks, site records -------------
+        // ---- A3: site records (loads in flight first), local indices, masks
+        for (uint32_t u = tid; u < ucount; u += FT) {
+            if (!SAD_CHECK(sm.ulist[u] < Nu, ws)) continue;
+            const float4 *R = rec + (size_t)sm.ulist[u] * REC_F4;
+            sm.urec[0][u] = __ldg(R);
+            sm.urec[1][u] = __ldg(R + 1);
+            sm.urec[2][u] = __ldg(R + 2);
+            sm.urec[3][u] = __ldg(R + 3);
+        }
         uint32_t ux[K];
 #pragma unroll
         for (int q = 0; q < K; ++q)
@@ -448,14 +465,6 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
                         atomicOr(reinterpret_cast<uint32_t *>(&sm.masks[rv[x] >> 16]) + (u >> 5), 1u << (u & 31u));
                 }
             }
-        }
-        for (uint32_t u = tid; u < ucount; u += FT) {
-            if (!SAD_CHECK(sm.ulist[u] < Nu, ws)) continue;
-            const float4 *R = rec + (size_t)sm.ulist[u] * REC_F4;
-            sm.urec[0][u] = __ldg(R);
-            sm.urec[1][u] = __ldg(R + 1);
-            sm.urec[2][u] = __ldg(R + 2);
-            sm.urec[3][u] = __ldg(R + 3);
         }
     }
     __syncthreads();
@@ -723,11 +732,20 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     __syncthreads();
     if (ty == 0) {
         // exclusive scan of the 128 counts, each rounded up to a multiple of
-        // 8, by one warp (4 per lane)
-        uint32_t c4[4], run = 0;
+        // the group size, by one warp (4 per lane).  Groups of 9 where they
+        // then fit one per thread (the padding of groups of 8 pushes a full
+        // tile just past one group per thread).
+        uint32_t c4[4], run = 0, n9 = 0;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            c4[e] = (sm.cnt[lane * 4 + e] + 7u) & ~7u;
+            c4[e] = sm.cnt[lane * 4 + e];
+            n9 += (c4[e] + 8u) / 9u;
+        }
+        n9 = __reduce_add_sync(FULL, n9);
+        const uint32_t gs = (Smem::GMAX == 9 && n9 <= (uint32_t)FT) ? 9u : 8u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            c4[e] = gs == 9u ? (c4[e] + 8u) / 9u * 9u : (c4[e] + 7u) & ~7u;
             run += c4[e];
         }
         uint32_t incl = run;
@@ -742,9 +760,13 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             sm.cursor[lane * 4 + e] = base;
             base += c4[e];
         }
-        if (lane == 31) sm.n_groups = incl >> 3;
+        if (lane == 31) {
+            sm.n_groups = incl / gs;
+            sm.gs = gs;
+        }
     }
     __syncthreads();
+    const uint32_t gs = sm.gs;
 #pragma unroll
     for (int q = 0; q < K; ++q) {
         const bool vq = (vmask >> q & 1u) && t.lx[q] != NOLOC;
@@ -755,18 +777,20 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         if (lane == tail_lane && key != EMPTY && SAD_CHECK(key < UCAP, ws))
             pos0 = atomicAdd(&sm.cursor[key], (uint32_t)(tail_lane - start + 1));
         pos0 = __shfl_sync(FULL, pos0, tail_lane);
-        if (vq && SAD_CHECK(((pos0 + (uint32_t)(lane - start)) >> 3) < (uint32_t)Smem::NG, ws)) {
-            const uint32_t pos = pos0 + (uint32_t)(lane - start);
+        const uint32_t pos = pos0 + (uint32_t)(lane - start);
+        const uint32_t g = gs == 9u ? __umulhi(pos, 477218590u) : pos >> 3;  // pos / 9 exactly for pos < 2^16
+        const uint32_t e = pos - g * gs;
+        if (vq && SAD_CHECK(g < (uint32_t)Smem::NG && e < (uint32_t)Smem::GMAX, ws)) {
             const float eq = __expf(t.l[q] - Mf);
-            sm.ent_wl[pos & 7u][pos >> 3] = make_float2(eq * iz, t.l[q]);
-            sm.ent_pu[pos & 7u][pos >> 3] = (uint16_t)(tid | (key << 9));
+            sm.ent_wl[e][g] = make_float2(eq * iz, t.l[q]);
+            sm.ent_pu[e][g] = (uint16_t)(tid | (key << 9));
             if constexpr (STATS)
-                sm.ent_rd[pos & 7u][pos >> 3] = removal_delta(eq, sm.urec[2][key], q == qstar, Z, iz, cr, cg, cb, zmm,
-                                                              cmr, cmg, cmb, er, eg, eb);
+                sm.ent_rd[e][g] = removal_delta(eq, sm.urec[2][key], q == qstar, Z, iz, cr, cg, cb, zmm, cmr, cmg,
+                                                cmb, er, eg, eb);
         }
     }
     __syncthreads();
-    // ---- D3: every thread sums one group of 8 entries of one site ----------
+    // ---- D3: every thread sums one group of entries of one site ------------
     {
         const uint32_t ng = sm.n_groups;
         const float fx0 = (float)i0 + 0.5f, fy0 = (float)j0 + 0.5f;
@@ -781,10 +805,10 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             for (int k = 0; k < NV; ++k) a[k] = 0.0f;
             if (g < ng && SAD_CHECK(g < (uint32_t)Smem::NG && (sm.ent_pu[0][g] >> 9) < ucount, ws)) {
                 u = sm.ent_pu[0][g] >> 9;
-                const uint32_t rem = sm.cursor[u] - 8u * g;  // entries of the group (>= 1)
+                const uint32_t rem = min(sm.cursor[u] - gs * g, gs);  // entries of the group (>= 1)
                 const float4 r0 = sm.urec[0][u], r1 = sm.urec[1][u], r2 = sm.urec[2][u], r3 = sm.urec[3][u];
 #pragma unroll
-                for (int e = 0; e < K; ++e) {
+                for (int e = 0; e < Smem::GMAX; ++e) {
                     const bool ve = (uint32_t)e < rem && SAD_CHECK((sm.ent_pu[e][g] & 0x1FFu) < (uint32_t)FT, ws);
                     const uint32_t px = ve ? (uint32_t)(sm.ent_pu[e][g] & 0x1FFu) : 0u;
                     const float2 wl = sm.ent_wl[e][g];
@@ -837,34 +861,36 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             n_global += sm.warp_cnt[1][q];
             n_dropped += sm.warp_cnt[2][q];
         }
+        // finish_pass_kernel, launched next, sums the partials
         ws_loss_partials(ws)[blockIdx.y * gridDim.x + blockIdx.x] = (double)tl;
         if (n_empty) atomicAdd(&c->empty_pixels, (unsigned long long)n_empty);
         if (n_global) atomicAdd(&c->hash_overflow, (unsigned long long)n_global);
         if (n_dropped) atomicAdd(&c->dropped_ids, (unsigned long long)n_dropped);
-        __threadfence();
-        sm.last = atomicAdd(&c->ticket_bwd, 1u) == gridDim.x * gridDim.y - 1;
     }
+}
+
+// The end of a fitting pass, once every tile is done: the loss from the
+// tiles' partials (summed in double) and, for the propagating form, the
+// other table made current and the pass counter advanced.  A separate launch
+// instead of a last-tile ticket: no tile waits on a global round trip.
+__global__ void __launch_bounds__(1024) finish_pass_kernel(void *ws, unsigned n_tiles, double P, int prop) {
+    Counters *c = ws_counters(ws);
+    const double *lp = ws_loss_partials(ws);
+    double s = 0.0;
+    for (unsigned q = threadIdx.x; q < n_tiles; q += 1024) s += lp[q];
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
+    __shared__ double red[32];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
     __syncthreads();
-    if (sm.last) {
-        // every block has read cur/pass and written its partial: finish the pass
-        const unsigned total = gridDim.x * gridDim.y;
-        const volatile double *lp = ws_loss_partials(ws);
-        double s = 0.0;
-        for (unsigned q = tid; q < total; q += FT) s += lp[q];
+    if (threadIdx.x < 32) {
+        s = red[threadIdx.x];
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
-        __shared__ double red[FT / 32];
-        if (lane == 0) red[ty] = s;
-        __syncthreads();
-        if (tid == 0) {
-            double tsum = 0.0;
-            for (int q = 0; q < FY; ++q) tsum += red[q];
-            c->loss = tsum / (double)P;
-            if (PROP) {
-                c->cur = cur ^ 1u;
-                c->pass_counter = pass + 1u;
+        if (threadIdx.x == 0) {
+            c->loss = s / P;
+            if (prop) {
+                c->cur ^= 1u;
+                c->pass_counter += 1u;
             }
-            c->ticket_bwd = 0;
-            __threadfence();
         }
     }
 }
@@ -896,6 +922,9 @@ cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
     const dim3 grid((d.W + FX - 1) / FX, (d.H + FY - 1) / FY);
     fit_tile_kernel<FY, PROP, STATS><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY, STATS>), st>>>(
         d.records, d.table, d.target, d.H, d.W, d.N, G, d.image, d.grads, d.stats, d.ws, lists);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    finish_pass_kernel<<<1, 1024, 0, st>>>(d.ws, grid.x * grid.y, (double)d.P, PROP ? 1 : 0);
     return cudaGetLastError();
 }
 
