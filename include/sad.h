@@ -296,8 +296,11 @@ int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream);
  * ([P1] section 5 and B.4).  Writes the bound image when one is bound and
  * the loss into the statistics block.  flags: 0, SAD_STATS (needs the stats
  * buffer; accumulates into it) or SAD_DETERMINISTIC (fixed-point
- * accumulation, order-independent).  SAD_ERR_UNSUPPORTED for other flags or
- * both together. */
+ * accumulation, order-independent).  With SAD_STATS the pass runs as the
+ * fused tile pass on the current lists (the work of sad_fit_pass_cached),
+ * whose per-tile accumulation groups the tile's entries by site and carries
+ * the six statistics beside the nine gradients.  SAD_ERR_UNSUPPORTED for
+ * other flags or both together. */
 int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream);
 
 /* One budget-control event, on the device ([P1] B.5: split by the score

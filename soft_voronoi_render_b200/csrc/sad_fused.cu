@@ -239,6 +239,44 @@ __device__ __forceinline__ void slot_grad(const float4 r0, const float4 r1, cons
     v[PA] = -0.5f * gi * (r3.y * al * al - r3.z * be * be);
 }
 
+// The same contributions added into the sums a of one site, with the factors
+// that are the site's own left for the end (group_finish): a[PR] collects
+// gamma (times k), a[PTH] gi al be (times -(k^2 e^a - k^2 e^-a)) and a[PA]
+// gi (k^2 e^a al^2 - k^2 e^-a be^2) (times -1/2), where gi = gamma / m.
+template <int NV>
+__device__ __forceinline__ void slot_accumulate(const float4 r0, const float4 r1, const float4 r2, const float4 r3,
+                                                float fx, float fy, float l, float w, float gr, float gg, float gb,
+                                                float cdg, float (&a)[NV], float &dx, float &dy) {
+    dx = fx - r0.x;
+    dy = fy - r0.y;
+    const float u1 = fmaf(r0.z, dx, r0.w * dy);
+    const float u2 = fmaf(r1.x, dy, r0.w * dx);
+    const float qf = fmaf(dx, u1, dy * u2);
+    const float im = qf > 0.0f ? rsqrtf(qf) : 0.0f;
+    const float gamma = w * (fmaf(r2.x, gr, fmaf(r2.y, gg, r2.z * gb)) - cdg);
+    const float gi = gamma * im;
+    const float al = fmaf(r2.w, dx, r3.x * dy);   // u . delta
+    const float be = fmaf(r2.w, dy, -r3.x * dx);  // v . delta
+    a[PX] = fmaf(gi, u1, a[PX]);
+    a[PY] = fmaf(gi, u2, a[PY]);
+    a[PLT] = fmaf(gamma, l, a[PLT]);
+    a[PR] += gamma;
+    a[PCR] = fmaf(w, gr, a[PCR]);
+    a[PCG] = fmaf(w, gg, a[PCG]);
+    a[PCB] = fmaf(w, gb, a[PCB]);
+    const float gal = gi * al, gbe = gi * be;
+    a[PTH] = fmaf(gal, be, a[PTH]);
+    a[PA] = fmaf(gal, r3.y * al, a[PA]);
+    a[PA] = fmaf(-gbe, r3.z * be, a[PA]);
+}
+
+template <int NV>
+__device__ __forceinline__ void group_finish(const float4 r1, const float4 r3, float (&a)[NV]) {
+    a[PR] *= r1.z;
+    a[PTH] *= -(r3.y - r3.z);
+    a[PA] *= -0.5f;
+}
+
 // budget-control statistics of one (pixel, slot) (summary B.4-B.5): mass w,
 // energy w e, error-weighted second moments w e (dx^2, dx dy, dy^2) and the
 // removal delta rd, with e = |chat - t|^2 = (P / 2)^2 |g|^2
@@ -499,6 +537,8 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             t.lx[q] = u;
         }
     }
+    uint32_t nw[UW] = {0u, 0u, 0u, 0u};  // candidates the neighbours add (tile-local bits)
+    float l8 = -__int_as_float(0x7f800000);
     if (inside && PROP) {
         if (fast) {
             // the pixel's own list re-scored in its previous order, which the
@@ -545,33 +585,40 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
                 t.cx(0, 1); t.cx(2, 3); t.cx(4, 5); t.cx(6, 7);
                 t.cx(1, 2); t.cx(3, 4); t.cx(5, 6);
             }
-            // candidates the four neighbours add.  A candidate can only enter
-            // if it scores at least the current 8th, which insertions only
-            // raise: score every candidate once against it, then insert the
-            // few that pass (in the same order, so the same result)
+            // the candidates the four neighbours add
             const uint4 mL = sm.masks[hc - 1], mR = sm.masks[hc + 1], mU = sm.masks[hc - HX],
                         mD = sm.masks[hc + HX];
-            const uint32_t nw[UW] = {(mL.x | mR.x | mU.x | mD.x) & ~own_mask.x,
-                                     (mL.y | mR.y | mU.y | mD.y) & ~own_mask.y,
-                                     (mL.z | mR.z | mU.z | mD.z) & ~own_mask.z,
-                                     (mL.w | mR.w | mU.w | mD.w) & ~own_mask.w};
-            const float l8 = t.l[K - 1];
-            uint32_t pass_bits[UW] = {0u, 0u, 0u, 0u};
+            nw[0] = (mL.x | mR.x | mU.x | mD.x) & ~own_mask.x;
+            nw[1] = (mL.y | mR.y | mU.y | mD.y) & ~own_mask.y;
+            nw[2] = (mL.z | mR.z | mU.z | mD.z) & ~own_mask.z;
+            nw[3] = (mL.w | mR.w | mU.w | mD.w) & ~own_mask.w;
+            l8 = t.l[K - 1];
+        }
+    }
+    // A neighbour's candidate can only enter if it scores at least the
+    // pixel's current 8th, which insertions only raise: every candidate is
+    // scored once against it, then the few that pass are inserted (in the
+    // same order as scoring them one by one, so the same result).
+    uint32_t pass_bits[UW] = {0u, 0u, 0u, 0u};
+    if (inside && PROP && fast) {
 #pragma unroll
-            for (int w = 0; w < UW; ++w) {
-                uint32_t bits = nw[w];
-                while (bits) {
-                    const int b = __ffs(bits) - 1;
-                    bits &= bits - 1u;
-                    const uint32_t u = (uint32_t)(w * 32 + b);
-                    if (!SAD_CHECK(u < ucount, ws)) continue;
-                    const float4 r0 = sm.urec[0][u];
-                    const float2 r1 = *reinterpret_cast<const float2 *>(&sm.urec[1][u]);
-                    const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
-                    // NaN (inactive site or NaN parameters) fails the test
-                    if (r0.x >= 0.0f && l >= l8) pass_bits[w] |= 1u << b;
-                }
+        for (int w = 0; w < UW; ++w) {
+            uint32_t bits = nw[w];
+            while (bits) {
+                const int b = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                const uint32_t u = (uint32_t)(w * 32 + b);
+                if (!SAD_CHECK(u < ucount, ws)) continue;
+                const float4 r0 = sm.urec[0][u];
+                const float2 r1 = *reinterpret_cast<const float2 *>(&sm.urec[1][u]);
+                const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+                // NaN (inactive site or NaN parameters) fails the test
+                if (r0.x >= 0.0f && l >= l8) pass_bits[w] |= 1u << b;
             }
+        }
+    }
+    if (inside && PROP) {
+        if (fast) {
 #pragma unroll
             for (int w = 0; w < UW; ++w) {
                 uint32_t bits = pass_bits[w];
@@ -590,18 +637,29 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             generic_pass(t, in0, in1, rec, Nu, H, W, i, j, fx, fy);
         }
         if (G > 0) {
+            // two injections per round: both records in flight together
             uint32_t h = inject_state(seed, pass, (uint32_t)((size_t)j * W + i));
 #pragma unroll 1
-            for (int g = 0; g < G; ++g) {
-                h = xorshift32(h);
-                const uint32_t id = __umulhi(h, Nu);  // < N
-                const float4 r0 = __ldg(rec + (size_t)id * REC_F4);
-                const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
-                const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
-                if (r0.x >= 0.0f && l == l && t.beats_last(l, id) && !t.has(id)) {
-                    // a winner the tile index holds keeps its local index
-                    uint32_t u = fast ? ukey_lookup(sm.keys, sm.lid, id) : NOLOC;
-                    t.insert(l, id, u < ucount ? u : NOLOC);
+            for (int g = 0; g < G; g += 2) {
+                uint32_t id[2];
+                float4 r0[2];
+                float2 r1[2];
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    if (g + x < G) h = xorshift32(h);
+                    id[x] = g + x < G ? __umulhi(h, Nu) : EMPTY;  // < N when drawn
+                    const size_t rr = (size_t)(id[x] < Nu ? id[x] : 0u) * REC_F4;
+                    r0[x] = __ldg(rec + rr);
+                    r1[x] = __ldg(reinterpret_cast<const float2 *>(rec + rr + 1));
+                }
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    const float l = sad_logit(r0[x].x, r0[x].y, r0[x].z, r0[x].w, r1[x].x, r1[x].y, fx, fy);
+                    if (id[x] < Nu && r0[x].x >= 0.0f && l == l && t.beats_last(l, id[x]) && !t.has(id[x])) {
+                        // a winner the tile index holds keeps its local index
+                        const uint32_t u = fast ? ukey_lookup(sm.keys, sm.lid, id[x]) : NOLOC;
+                        t.insert(l, id[x], u < ucount ? u : NOLOC);
+                    }
                 }
             }
         }
@@ -813,17 +871,20 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
                     const uint32_t px = ve ? (uint32_t)(sm.ent_pu[e][g] & 0x1FFu) : 0u;
                     const float2 wl = sm.ent_wl[e][g];
                     const float4 pa = sm.pixg[px];
-                    float v[NV], dx, dy;
-                    slot_grad(r0, r1, r2, r3, fx0 + (float)(px & (FX - 1)), fy0 + (float)(px / FX), wl.y, wl.x, pa.x,
-                              pa.y, pa.z, pa.w, v, dx, dy);
-                    if constexpr (STATS)
-                        slot_stats(wl.x, ex_scale * (pa.x * pa.x + pa.y * pa.y + pa.z * pa.z), dx, dy,
-                                   sm.ent_rd[e][g], v);
                     if (ve) {
+                        float dx, dy;
+                        slot_accumulate(r0, r1, r2, r3, fx0 + (float)(px & (FX - 1)), fy0 + (float)(px / FX), wl.y,
+                                        wl.x, pa.x, pa.y, pa.z, pa.w, a, dx, dy);
+                        if constexpr (STATS) {
+                            float v[NV];
+                            slot_stats(wl.x, ex_scale * (pa.x * pa.x + pa.y * pa.y + pa.z * pa.z), dx, dy,
+                                       sm.ent_rd[e][g], v);
 #pragma unroll
-                        for (int k = 0; k < NV; ++k) a[k] += v[k];
+                            for (int k = NPARAM; k < NV; ++k) a[k] += v[k];
+                        }
                     }
                 }
+                group_finish(r1, r3, a);
             }
             // groups of one site sit on consecutive lanes: sum each run across
             // lanes, then one global update per run
