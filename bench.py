@@ -78,6 +78,8 @@ def parse():
     ap.add_argument("--update-every", type=int, default=1,
                     help="c5: propagate the candidate lists every U iterations (cached lists between)")
     ap.add_argument("--passes-per-update", type=int, default=1, help="c5: propagation passes per update")
+    ap.add_argument("--candidates", type=int, default=32, choices=[32, 16],
+                    help="c4/c5: rank candidates on the float32 record (32) or the packed binary16 one (16)")
     return ap.parse_args()
 
 
@@ -565,6 +567,8 @@ def run_refresh(args):
     s.set_target(tgt)
     if args.cell != 1:
         s.set_candidate_grid(args.cell)
+    if args.candidates == 16:
+        s.set_candidate_precision(16)
     GH, GW = (H + args.cell - 1) // args.cell, (W + args.cell - 1) // args.cell
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
@@ -612,7 +616,7 @@ def run_refresh(args):
             "mpix_per_s_per_pass": PT * passes / (t_ref * 1e-3) / 1e6 if passes else None,
             "owner_right_sampled": owner_right, "dtype": "f32", "data": "synthetic",
             "config": {"workload": f"c4: {wl.description}", "H": H, "W": W, "N": N, "G": G, "cell": args.cell,
-                       "refresh": args.refresh},
+                       "refresh": args.refresh, "candidate_bits": args.candidates},
             "hbm_roof_frac": alg / ((t_ref + t_ren) * 1e-3) / 1e9 / hbm, "peak_kind": peak_kind,
             "device_stats": s.stats()}
     print(json.dumps(line), flush=True)
@@ -637,6 +641,8 @@ def run_fit(args):
     s.set_target(tgt)
     if args.cell != 1:
         s.set_candidate_grid(args.cell)
+    if args.candidates == 16:
+        s.set_candidate_precision(16)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -652,7 +658,8 @@ def run_fit(args):
             "iterations": sched.iterations, "events": len(sched.events), "schedule_run": info,
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": f"c5: {wl.description}", "H": H, "W": W, "N_start": prm.shape[1],
-                       "N_cap": N_cap, "G": sched.G, "cell": args.cell, "update_every": sched.update_every,
+                       "N_cap": N_cap, "G": sched.G, "cell": args.cell, "candidate_bits": args.candidates,
+                       "update_every": sched.update_every,
                        "passes_per_update": sched.passes_per_update}}
     if args.oracle_fit:
         import oracle
