@@ -253,13 +253,44 @@ __device__ __forceinline__ float cand_logit(const float4 *__restrict__ rec, cons
 }
 
 // Offer up to 8 candidate ids as one batch.  Their records are fetched
-// together (independent loads in flight).  Invalid entries (id >= N,
-// inactive site, NaN logit, an id already held or repeated earlier in the
-// batch) become (-inf, EMPTY), which ranks below every candidate.  When no
-// active lane has a candidate that beats its 8th, the network is skipped.
-template <int NB, bool F16 = false>
+// together (independent loads in flight).  With merge, invalid entries (id
+// >= N, inactive site, NaN logit, an id already held or repeated earlier in
+// the batch) become (-inf, EMPTY), which ranks below every candidate, and the
+// batch is sorted and merged; the network is skipped when no active lane has
+// a candidate that beats its 8th.  Without merge the candidates that beat
+// the 8th are inserted one by one: the JFA prepass keeps 4 entries and takes
+// few new ones per pass, and its kernel stays at 48 registers (5 blocks per
+// SM) without the network.
+template <int NB, bool F16, bool MERGE>
 __device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], const float4 *__restrict__ rec,
                                             const uint4 *__restrict__ c16, uint32_t N, float fx, float fy) {
+    if constexpr (!MERGE) {
+        float li[NB];
+#pragma unroll
+        for (int q = 0; q < NB; ++q) {
+            li[q] = __int_as_float(0x7fc00000);  // NaN: not a candidate
+            const uint32_t x = ids[q];
+            if (x < N && !t.has(x)) {
+                // the score only for an active site (keeps fewer values live)
+                if constexpr (F16) {
+                    const uint4 v = __ldg(c16 + x);
+                    if (__uint_as_float(v.x) >= 0.0f) {
+                        const float2 ab = __half22float2(*reinterpret_cast<const __half2 *>(&v.z));
+                        const float2 cb = __half22float2(*reinterpret_cast<const __half2 *>(&v.w));
+                        li[q] = sad_logit(__uint_as_float(v.x), __uint_as_float(v.y), ab.x, ab.y, cb.x, cb.y, fx, fy);
+                    }
+                } else {
+                    const float4 r0 = __ldg(rec + (size_t)x * REC_F4);
+                    const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)x * REC_F4 + 1));
+                    if (r0.x >= 0.0f) li[q] = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < NB; ++q)
+            if (li[q] == li[q] && t.beats_last(li[q], ids[q]) && !t.has(ids[q])) t.insert(li[q], ids[q]);
+        return;
+    } else {
     float l[K];
     uint32_t id[K];
     bool enters = false;
@@ -287,6 +318,7 @@ __device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], 
         sort8(l, id);
         merge8(t, l, id);
     }
+    }
 }
 
 // The pixel's own list as the first candidates of a pass into an empty list:
@@ -294,7 +326,7 @@ __device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], 
 // repeats (the records do not change between refresh passes), and then it is
 // the top-8 of its own candidates as it stands; otherwise its repeats are
 // dropped and it is sorted.  Same result either way.
-template <bool F16>
+template <bool F16, bool MERGE>
 __device__ __forceinline__ void take_own_list(Top8 &t, const uint4 a, const uint4 b, const float4 *__restrict__ rec,
                                               const uint4 *__restrict__ c16, uint32_t N, float fx, float fy) {
     const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -318,23 +350,29 @@ __device__ __forceinline__ void take_own_list(Top8 &t, const uint4 a, const uint
 #pragma unroll
         for (int r = 0; r < q; ++r) clean &= (t.id[q] == EMPTY) || (t.id[q] != t.id[r]);
     }
-    if (__any_sync(__activemask(), !clean)) {
+    if constexpr (MERGE) {
+        if (__any_sync(__activemask(), !clean)) {
 #pragma unroll
-        for (int q = 1; q < 8; ++q)
+            for (int q = 1; q < 8; ++q)
 #pragma unroll
-            for (int r = 0; r < q; ++r)
-                if (t.id[q] != EMPTY && t.id[q] == t.id[r]) {
-                    t.l[q] = -__int_as_float(0x7f800000);
-                    t.id[q] = EMPTY;
-                }
-        sort8(t.l, t.id);
+                for (int r = 0; r < q; ++r)
+                    if (t.id[q] != EMPTY && t.id[q] == t.id[r]) {
+                        t.l[q] = -__int_as_float(0x7f800000);
+                        t.id[q] = EMPTY;
+                    }
+            sort8(t.l, t.id);
+        }
+    } else if (!clean) {
+        // the ids one by one into an empty list
+        t.clear();
+        offer_batch<8, F16, false>(t, ids, rec, c16, N, fx, fy);
     }
 }
 
 // H x W is the candidate grid; a cell is scored at its centre, (i + 0.5) cs
 // (cs = 1: the pixel grid).  F16: candidates are ranked on the packed
 // records c16 and the kept 8 re-scored with the float32 records.
-template <bool F16>
+template <bool F16, bool MERGE>
 __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *__restrict__ rec,
                                                                  const uint4 *__restrict__ c16, uint32_t *table,
                                                                  int H, int W, float cs, int N, int jump, int G,
@@ -351,7 +389,7 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
         const size_t p = (size_t)j * W + i;
         const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
         Top8 t;
-        take_own_list<F16>(t, in0[p], in1[p], rec, c16, (uint32_t)N, fx, fy);
+        take_own_list<F16, MERGE>(t, in0[p], in1[p], rec, c16, (uint32_t)N, fx, fy);
         // the neighbours at (-k, 0), (+k, 0), (0, -k), (0, +k); one outside
         // the image offers nothing
 #pragma unroll 1
@@ -365,7 +403,7 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
                 b = in1[pn];
             }
             const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            offer_batch<8, F16>(t, ids, rec, c16, (uint32_t)N, fx, fy);
+            offer_batch<8, F16, MERGE>(t, ids, rec, c16, (uint32_t)N, fx, fy);
         }
         if (G > 0) {
             uint32_t h = inject_state(seed, pass, (uint32_t)p);
@@ -381,7 +419,7 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
                         ids[q] = EMPTY;
                     }
                 }
-                offer_batch<8, F16>(t, ids, rec, c16, (uint32_t)N, fx, fy);
+                offer_batch<8, F16, MERGE>(t, ids, rec, c16, (uint32_t)N, fx, fy);
             }
         }
         if constexpr (F16) {
@@ -452,7 +490,7 @@ __global__ void __launch_bounds__(TILE_THREADS) jfa3x3_kernel(const float4 *__re
             const size_t pn = (size_t)nj * W + ni;
             const uint4 a = in0[pn], b = in1[pn];
             const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            offer_batch<8>(t, ids, rec, nullptr, (uint32_t)N, fx, fy);
+            offer_batch<8, false, false>(t, ids, rec, nullptr, (uint32_t)N, fx, fy);
         }
         out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
         out1[p] = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY);
@@ -958,13 +996,21 @@ cudaError_t launch_seed(const Dev &d, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// propagation passes merge their candidates as batches (measured faster than
+// one-by-one insertion at every jump of the refresh, and within 15 % of it
+// for a lone jump-1 pass); the JFA prepass inserts
+template <bool F16>
+void launch_propagate_f(const Dev &d, int jump, int G, cudaStream_t st) {
+    const uint4 *c16 = F16 ? d.cand16 : nullptr;
+    propagate_kernel<F16, true><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
+        d.records, c16, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d));
+}
+
 cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st) {
     if (d.f16)
-        propagate_kernel<true><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
-            d.records, d.cand16, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d));
+        launch_propagate_f<true>(d, jump, G, st);
     else
-        propagate_kernel<false><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
-            d.records, nullptr, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d));
+        launch_propagate_f<false>(d, jump, G, st);
     return cudaGetLastError();
 }
 
