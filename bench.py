@@ -80,6 +80,9 @@ def parse():
     ap.add_argument("--passes-per-update", type=int, default=1, help="c5: propagation passes per update")
     ap.add_argument("--candidates", type=int, default=32, choices=[32, 16],
                     help="c4/c5: rank candidates on the float32 record (32) or the packed binary16 one (16)")
+    ap.add_argument("--staging", default="loads", choices=["loads", "tma"],
+                    help="c3: the fit pass loads each tile's lists per thread (default) or stages them by TMA "
+                         "copies in persistent blocks")
     return ap.parse_args()
 
 
@@ -342,6 +345,8 @@ def run_ours(args):
     s = Sad(H, W, N, device=dev, seed=1 + rank)
     s.set_sites(prm)
     s.set_target(tgt)
+    if args.staging == "tma":
+        s.set_list_staging(_lib.SAD_STAGING_TMA)
     s.refresh(G)
     cfg = _lib.adam_cfg(**ADAM_LR)
     ctx = s.ctx
@@ -516,7 +521,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "Mpix/s", "n_gpus": world, "steps": K,
             "warmup": max(args.warmup, 3), "setup_iterations": SETUP_ITERS, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(wl, world),
+            "config": dict(workload_config(wl, world), list_staging=args.staging),
             "hbm_roof_frac_iter": (iter_bytes / (ms_step * 1e-3) / 1e9) / hbm,
             "iter_algorithmic_bytes": iter_bytes,
             "kernels_ms": {k: round(v, 5) for k, v in avg.items()},
@@ -883,7 +888,7 @@ def run_rows(args):
     row("a4_render", timed(s.render), 44 * P, "softmax blend: list 32 + image 12 B/px")
     zero = s.grads.zero_
     row("a5_a6_backward", timed(s.backward, before=zero), 56 * P + 36 * N,
-        "render + loss + backward, tile hash: list 32 + target 12 + image 12 B/px, gradients 36 B/site")
+        "render + loss + backward (tile pass on the current lists): list 32 + target 12 + image 12 B/px, gradients 36 B/site")
     row("a6_backward_stats", timed(lambda: s.backward(SAD_STATS), before=zero), 56 * P + 60 * N,
         "the same with the budget statistics (+24 B/site)")
     row("a6_backward_deterministic", timed(lambda: s.backward(SAD_DETERMINISTIC), before=zero), 56 * P + 36 * N,

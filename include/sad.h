@@ -142,7 +142,9 @@ typedef struct sad_stats {
     uint32_t pass_counter;     /* propagation passes run (drives injection randomness) */
     uint32_t adam_step;        /* Adam steps taken (bias-correction t of the next step is +1) */
     uint32_t current_table;    /* 0 or 1: which table of the double buffer is current */
-    uint32_t reserved;
+    uint32_t staging_fallbacks; /* fit passes: tile-list copies into shared memory that did not
+                                   arrive within the wait bound, after which the block read the
+                                   lists from global memory instead (expected 0) */
     double loss;               /* loss of the last sad_backward / sad_fit_iteration */
     uint32_t n_active;         /* active sites before the last densify event */
     uint32_t n_split;          /* sites split by the last densify event */
@@ -390,6 +392,27 @@ int sad_get_stats(sad_ctx *ctx, sad_stats *out, sad_stream_t stream);
  * SAD_ERR_INVALID_ARG for other bits, SAD_ERR_NOT_BOUND for 16 without a
  * bound cand16 buffer. */
 int sad_set_candidate_precision(sad_ctx *ctx, int bits, sad_stream_t stream);
+
+/* How the propagating fit pass (sad_fit_pass, sad_fit_iteration) brings each
+ * tile's candidate lists and their one-pixel halo on chip ([P1] section 5:
+ * per-tile staging in shared memory).
+ *   SAD_STAGING_LOADS (default): one block per 32 x 16 tile; every thread
+ *     loads its own list and a share of the halo.
+ *   SAD_STAGING_TMA: as many persistent blocks as fit the device take tiles
+ *     from a ticket; while a block works on one tile, a TMA tensor copy
+ *     brings the next tile's list block (both planes with the halo, 19.6 KB)
+ *     into shared memory, signalled on a shared-memory barrier whose wait is
+ *     bounded: a copy that does not arrive in time switches the block to
+ *     plain loads and is counted in sad_stats.staging_fallbacks.
+ * Both give the same lists bit for bit and the same sums.  The default is
+ * the faster on B200: the co-resident block already hides the list loads'
+ * latency, and a persistent block cannot begin its next tile before its
+ * slowest warp has finished the current one.  The TMA form applies where
+ * the pass uses 32 x 16 tiles (at least 4 pixels per site) on the pixel
+ * grid; elsewhere the default runs.  SAD_ERR_INVALID_ARG for other modes. */
+#define SAD_STAGING_LOADS 0
+#define SAD_STAGING_TMA 1
+int sad_set_list_staging(sad_ctx *ctx, int mode, sad_stream_t stream);
 
 /* The fitting state that lives in the library's counter block: the pass
  * counter that keys the injection randomness ([P1] B.3: xorshift state from

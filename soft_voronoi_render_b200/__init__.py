@@ -10,9 +10,11 @@ from __future__ import annotations
 import numpy as np
 
 from . import _lib
-from ._lib import SAD_DETERMINISTIC, SAD_STATS, SadError, adam_cfg, densify_cfg  # noqa: F401
+from ._lib import (SAD_DETERMINISTIC, SAD_STAGING_LOADS, SAD_STAGING_TMA, SAD_STATS, SadError,  # noqa: F401
+                   adam_cfg, densify_cfg)
 
-__all__ = ["Sad", "SadError", "adam_cfg", "densify_cfg", "SAD_STATS", "SAD_DETERMINISTIC", "load"]
+__all__ = ["Sad", "SadError", "adam_cfg", "densify_cfg", "SAD_STATS", "SAD_DETERMINISTIC", "SAD_STAGING_LOADS",
+           "SAD_STAGING_TMA", "load"]
 
 
 def load():
@@ -136,6 +138,11 @@ class Sad:
         packed candidate-site records (binary16 coefficients), the kept 8
         re-scored in float32."""
         _lib.sad_set_candidate_precision(self.ctx, bits, self.stream)
+
+    def set_list_staging(self, mode: int):
+        """SAD_STAGING_LOADS (default) or SAD_STAGING_TMA: how the fit pass
+        brings each tile's lists on chip (see sad_set_list_staging)."""
+        _lib.sad_set_list_staging(self.ctx, mode, self.stream)
 
     def set_candidate_grid(self, cell: int):
         """Lists on a ceil(H/cell) x ceil(W/cell) grid; the table starts empty."""

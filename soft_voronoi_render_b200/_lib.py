@@ -48,6 +48,8 @@ class sad_densify_cfg(ctypes.Structure):
 
 SAD_STATS = 1
 SAD_DETERMINISTIC = 2
+SAD_STAGING_LOADS = 0
+SAD_STAGING_TMA = 1
 
 
 def densify_cfg(grow=2500, prune_frac=0.005, alpha=0.5, eps=1e-6, r_scale=0.85, log_tau_shift=0.6931471805599453,
@@ -64,7 +66,7 @@ class sad_stats(ctypes.Structure):
     _fields_ = [("hash_overflow", ctypes.c_uint64), ("nonfinite_pixels", ctypes.c_uint64),
                 ("empty_pixels", ctypes.c_uint64), ("dropped_ids", ctypes.c_uint64),
                 ("pass_counter", ctypes.c_uint32), ("adam_step", ctypes.c_uint32),
-                ("current_table", ctypes.c_uint32), ("reserved", ctypes.c_uint32), ("loss", ctypes.c_double),
+                ("current_table", ctypes.c_uint32), ("staging_fallbacks", ctypes.c_uint32), ("loss", ctypes.c_double),
                 ("n_active", ctypes.c_uint32), ("n_split", ctypes.c_uint32), ("n_pruned", ctypes.c_uint32),
                 ("check_failures", ctypes.c_uint32)]
 
@@ -83,7 +85,7 @@ EXPORTED = (
     "sad_propagate", "sad_fit_pass_cached", "sad_set_candidate_grid", "sad_pack_sites", "sad_unpack_sites", "sad_bind_target", "sad_set_target_u8",
     "sad_render", "sad_backward", "sad_densify_prune", "sad_tau_diffuse", "sad_adam_step", "sad_fit_pass", "sad_fit_iteration", "sad_get_table", "sad_set_table",
     "sad_get_stats", "sad_get_loss", "sad_copy_loss", "sad_last_error", "sad_backward_noalloc",
-    "sad_get_fit_state", "sad_set_fit_state", "sad_set_candidate_precision",
+    "sad_get_fit_state", "sad_set_fit_state", "sad_set_candidate_precision", "sad_set_list_staging",
 )
 
 _lib = None
@@ -145,6 +147,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "sad_get_fit_state": [vp, ctypes.POINTER(sad_fit_state), vp],
         "sad_set_fit_state": [vp, ctypes.POINTER(sad_fit_state), vp],
         "sad_set_candidate_precision": [vp, ci, vp],
+        "sad_set_list_staging": [vp, ci, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -317,6 +320,10 @@ def sad_get_stats(ctx: int, stream=None) -> dict:
 
 def sad_set_candidate_precision(ctx: int, bits: int, stream=None) -> None:
     _check(ctx, load().sad_set_candidate_precision(ctx, int(bits), _stream(stream)))
+
+
+def sad_set_list_staging(ctx: int, mode: int, stream=None) -> None:
+    _check(ctx, load().sad_set_list_staging(ctx, int(mode), _stream(stream)))
 
 
 def sad_get_fit_state(ctx: int, stream=None) -> dict:

@@ -320,6 +320,16 @@ int sad_set_candidate_precision(sad_ctx *ctx, int bits, sad_stream_t stream) {
     return SAD_OK;
 }
 
+int sad_set_list_staging(sad_ctx *ctx, int mode, sad_stream_t stream) {
+    (void)stream;
+    int r = need_bound(ctx);
+    if (r) return r;
+    if (mode != SAD_STAGING_LOADS && mode != SAD_STAGING_TMA)
+        return fail(ctx, SAD_ERR_INVALID_ARG, "list staging mode must be SAD_STAGING_LOADS or SAD_STAGING_TMA");
+    ctx->dev.tma_staging = mode == SAD_STAGING_TMA;
+    return SAD_OK;
+}
+
 int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream) {
     int r = need_bound(ctx);
     if (r) return r;
@@ -342,7 +352,7 @@ int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream) {
         if (!ctx->buf.stats) return fail(ctx, SAD_ERR_NOT_BOUND, "SAD_STATS needs a bound stats buffer");
         return cuda_status(ctx, sad::launch_fit_tile_cached_stats(ctx->dev, cs(stream)), "backward (stats)");
     }
-    return cuda_status(ctx, sad::launch_render_backward(ctx->dev, cs(stream)), "backward");
+    return cuda_status(ctx, sad::launch_fit_tile_cached(ctx->dev, cs(stream)), "backward");
 }
 
 int sad_densify_prune(sad_ctx *ctx, const sad_densify_cfg *cfg, sad_stream_t stream) {
@@ -501,7 +511,7 @@ int sad_get_stats(sad_ctx *ctx, sad_stats *out, sad_stream_t stream) {
     out->pass_counter = c.pass_counter;
     out->adam_step = c.adam_step;
     out->current_table = c.cur;
-    out->reserved = 0;
+    out->staging_fallbacks = c.staging_fallbacks;
     out->loss = c.loss;
     uint32_t hdr[4] = {0, 0, 0, 0};
     cudaError_t e = cudaMemcpy(hdr, reinterpret_cast<char *>(ctx->buf.workspace) + sad::densify_offset(ctx->H, ctx->W),

@@ -33,14 +33,16 @@ struct Counters {
     uint32_t ticket_prop;    // last-block tickets (reset by the last block)
     uint32_t ticket_bwd;
     uint32_t ticket_adam;
-    uint32_t pad0;
+    uint32_t staging_fallbacks;  // list-staging copies that did not arrive in time (tiles read from global)
     unsigned long long hash_overflow;
     unsigned long long nonfinite_pixels;
     unsigned long long empty_pixels;
     unsigned long long dropped_ids;
     double loss;
     unsigned long long check_failures;  // SAD_CHECKS builds: accesses refused by a bounds check
-    double pad1[6];
+    uint32_t tile_ticket;    // persistent fit pass: tiles handed out beyond the first wave (reset by its finish)
+    uint32_t pad2;
+    double pad1[5];
     uint32_t pack_ord[6];    // order-preserving encodings of the pack ranges
     float pack_range[6];     // lo ln tau, lo r, lo a, hi ln tau, hi r, hi a
 };

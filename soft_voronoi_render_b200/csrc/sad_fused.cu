@@ -20,6 +20,11 @@
 // differentiates the cached lists as they stand, for the iterations between
 // candidate updates (summary B.3): no halo, no new lists, the pass counter
 // and the current table are left alone.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
 #include "sad_device.cuh"
 #include "sad_launch.h"
 
@@ -147,9 +152,57 @@ __device__ __forceinline__ uint32_t pack_bytes(uint32_t a, uint32_t b, uint32_t 
 }
 __device__ __forceinline__ uint32_t byte_of(uint32_t w, int q) { return __byte_perm(w, 0, 0x4440 | (q & 3)); }
 
-template <int FY, bool STATS>
+// ---- TMA staging of the list block (shared-memory barrier + bulk tensor copy)
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// one arrival that also announces the bytes the copy will deliver
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// wait until the barrier's phase with the given parity has completed, giving
+// up after a bounded number of polls (false: the copy did not arrive)
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    constexpr int POLLS = 1 << 22;
+    const uint32_t a = smem_u32(bar);
+#pragma unroll 1
+    for (int n = 0; n < POLLS; ++n) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+// 3-D tile copy global -> shared (no multicast), completion counted in bytes
+// on the barrier.  x (words) must be a multiple of 4: 16-byte boundaries.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+template <int FY, bool STATS, bool TMA = false>
 struct FusedSmem {
     static constexpr int FT = FX * FY, HN = HX * (FY + 2), RING = HN - FT;
+    // TMA form: a tile's two list planes with the one-pixel halo, as the copy
+    // lands them: [plane][halo row][4 words per halo column]
+    static constexpr int LBZ = TMA ? 2 : 1, LBY = TMA ? FY + 2 : 1, LBX = TMA ? 4 * HX : 4;
+    static constexpr uint32_t LBYTES = LBZ * LBY * LBX * 4;
     // The tile's (pixel, slot) entries grouped by site, each site's run padded
     // to a multiple of the group size gs (8, or 9 where that makes the groups
     // fit one per thread) so that every group belongs to one site: at most
@@ -160,6 +213,8 @@ struct FusedSmem {
     static constexpr int NG = FT + 7 * UCAP / 8;
     static constexpr int NGS = (NG + 15) / 16 * 16 + 2;    // float2 planes
     static constexpr int NGS16 = (NG + 63) / 64 * 64 + 8;  // uint16 planes
+    alignas(128) uint32_t lbuf[LBZ][LBY][LBX];
+    uint64_t bar;                   // completion of the staging copy
     uint32_t keys[UHASH];
     uint32_t lid[UHASH];
     uint32_t ulist[UCAP];
@@ -174,6 +229,7 @@ struct FusedSmem {
     float warp_loss[FY];
     uint32_t warp_cnt[3][FY];       // per warp: empty pixels, global-atomic pixels, dropped ids
     uint32_t n_groups;
+    uint32_t next_tile;             // persistent form: the tile after this one
     uint32_t gs;                    // entries per group
     uint32_t ucount;
     int overflow;
@@ -356,27 +412,24 @@ __device__ __forceinline__ void generic_pass(Top8L &t, const uint4 *__restrict__
     }
 }
 
-template <int FY, bool PROP, bool STATS>
-__global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(const float4 *__restrict__ rec,
-                                                                            uint32_t *table,
-                                                         const float *__restrict__ target, int H, int W, int N,
-                                                         int G, float *__restrict__ image,
-                                                         float *__restrict__ grads, float *__restrict__ stats,
-                                                         void *ws, TableGrid lists) {
+template <int FY, bool PROP, bool STATS, bool TMA>
+__global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
+    fit_tile_kernel(const float4 *__restrict__ rec, uint32_t *table, const float *__restrict__ target, int H, int W,
+                    int N, int G, float *__restrict__ image, float *__restrict__ grads, float *__restrict__ stats,
+                    void *ws, TableGrid lists, const __grid_constant__ CUtensorMap lmap, int tiles_x,
+                    uint32_t n_tiles) {
     static_assert(!(PROP && STATS), "the statistics come with the cached-list form");
-    using Smem = FusedSmem<FY, STATS>;
+    static_assert(!TMA || (PROP && !STATS), "list staging serves the propagating form");
+    using Smem = FusedSmem<FY, STATS, TMA>;
     constexpr int NV = STATS ? NPARAM + NSTAT : NPARAM;
     constexpr int FT = Smem::FT, HN = Smem::HN, RING = Smem::RING;
     constexpr int NRE = (RING * K + FT - 1) / FT;  // halo (pixel, slot) entries per thread
-    extern __shared__ __align__(16) unsigned char fused_smem_raw[];
+    extern __shared__ __align__(128) unsigned char fused_smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(fused_smem_raw);
     Counters *c = ws_counters(ws);
     const uint32_t cur = c->cur, pass = c->pass_counter, seed = c->seed;
     const int lane = threadIdx.x, ty = threadIdx.y;
     const int tid = ty * FX + lane;
-    const int i0 = blockIdx.x * FX, j0 = blockIdx.y * FY;
-    const int i = i0 + lane, j = j0 + ty;
-    const bool inside = i < W && j < H;
     const size_t P = (size_t)H * W;
     // the cached-list form also reads lists kept per cell of a coarser grid
     const size_t PT = PROP ? P : lists.PT;
@@ -386,9 +439,72 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
     uint4 *out1 = out0 + P;
     const uint32_t Nu = (uint32_t)N;
 
-    // ---- global loads first: the pixel's list, the halo entries, the target
+    // TMA form: a persistent block starts on tile blockIdx.x and takes its
+    // next tile from a ticket as soon as it starts the current one, so that
+    // the next tile's list block (tile + halo, both planes) is copied into
+    // shared memory while it works on the current one.  A copy that does
+    // not arrive within the wait's bound switches the block to global loads
+    // (block-uniform, counted in staging_fallbacks).
+    uint32_t tile = TMA ? blockIdx.x : blockIdx.y * gridDim.x + blockIdx.x;
+    uint32_t phase = 0, lost_phase = 0;
+    bool staged = TMA, lost = false;
+    if constexpr (TMA) {
+        staged = (smem_u32(&sm.lbuf[0][0][0]) & 127u) == 0u;
+        if (tid == 0 && staged) {
+            mbar_init(&sm.bar, 1u);
+            if (tile < n_tiles) {
+                mbar_arrive_expect_tx(&sm.bar, Smem::LBYTES);
+                tma_load_3d(&sm.lbuf[0][0][0], &lmap, &sm.bar, 4 * ((int)(tile % (uint32_t)tiles_x) * FX - 1),
+                            (int)(tile / (uint32_t)tiles_x) * FY - 1, 2 * (int)cur);
+            }
+        }
+        if (tid == 0 && !staged) atomicAdd(&c->staging_fallbacks, 1u);
+        __syncthreads();
+    }
+#pragma unroll 1
+    for (;;) {
+    if (TMA && tile >= n_tiles) break;
+    const int bx = TMA ? (int)(tile % (uint32_t)tiles_x) : (int)blockIdx.x;
+    const int by = TMA ? (int)(tile / (uint32_t)tiles_x) : (int)blockIdx.y;
+    const int i0 = bx * FX, j0 = by * FY;
+    const int i = i0 + lane, j = j0 + ty;
+    const bool inside = i < W && j < H;
+
+    // ---- the lists first (staged copy, else global loads), then the target
+    // halo entry e = tid + x FT is ring pixel e % RING, slot e / RING; rv[x]
+    // holds its id, then its hash slot | mask cell << 16 (NOLOC: none)
     uint32_t own[K];
-    {
+    uint32_t rv[NRE], rcell[NRE];
+    bool got = false;
+    if constexpr (TMA) {
+        if (staged) got = mbar_wait_bounded(&sm.bar, phase);
+        if (got) {
+            // halo row hy, halo column hx of plane z is lbuf[z][hy][4 hx ...]
+            uint4 a = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY), b = a;
+            if (inside) {
+                a = *reinterpret_cast<const uint4 *>(&sm.lbuf[0][ty + 1][4 * (lane + 1)]);
+                b = *reinterpret_cast<const uint4 *>(&sm.lbuf[1][ty + 1][4 * (lane + 1)]);
+            }
+            own[0] = a.x; own[1] = a.y; own[2] = a.z; own[3] = a.w;
+            own[4] = b.x; own[5] = b.y; own[6] = b.z; own[7] = b.w;
+#pragma unroll
+            for (int x = 0; x < NRE; ++x) {
+                const int e = tid + x * FT;
+                uint32_t id = EMPTY, cell = 0;
+                if (e < RING * K) {
+                    const int r = e % RING, q = e / RING;
+                    int hx, hy;
+                    ring_coords<FY>(r, hx, hy);
+                    cell = (uint32_t)(hy * HX + hx);
+                    const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
+                    if (gi >= 0 && gi < W && gj >= 0 && gj < H) id = sm.lbuf[q >> 2][hy][4 * hx + (q & 3)];
+                }
+                rv[x] = id;
+                rcell[x] = cell;
+            }
+        }
+    }
+    if (!got) {
         uint4 a = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY), b = a;
         if (inside) {
             const size_t p = (size_t)j * W + i;
@@ -398,26 +514,23 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         }
         own[0] = a.x; own[1] = a.y; own[2] = a.z; own[3] = a.w;
         own[4] = b.x; own[5] = b.y; own[6] = b.z; own[7] = b.w;
-    }
-    // halo entry e = tid + x FT is ring pixel e % RING, slot e / RING; rv[x]
-    // holds its id, then its hash slot | mask cell << 16 (NOLOC: none)
-    uint32_t rv[NRE], rcell[NRE];
-    if (PROP) {
+        if (PROP) {
 #pragma unroll
-        for (int x = 0; x < NRE; ++x) {
-            const int e = tid + x * FT;
-            uint32_t id = EMPTY, cell = 0;
-            if (e < RING * K) {
-                const int r = e % RING, q = e / RING;
-                int hx, hy;
-                ring_coords<FY>(r, hx, hy);
-                cell = (uint32_t)(hy * HX + hx);
-                const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
-                if (gi >= 0 && gi < W && gj >= 0 && gj < H)
-                    id = table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
+            for (int x = 0; x < NRE; ++x) {
+                const int e = tid + x * FT;
+                uint32_t id = EMPTY, cell = 0;
+                if (e < RING * K) {
+                    const int r = e % RING, q = e / RING;
+                    int hx, hy;
+                    ring_coords<FY>(r, hx, hy);
+                    cell = (uint32_t)(hy * HX + hx);
+                    const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
+                    if (gi >= 0 && gi < W && gj >= 0 && gj < H)
+                        id = table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
+                }
+                rv[x] = id;
+                rcell[x] = cell;
             }
-            rv[x] = id;
-            rcell[x] = cell;
         }
     }
     // the target is read last: bring its lines into L2 now, registers later
@@ -437,7 +550,29 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
         sm.ucount = 0;
         sm.overflow = 0;
     }
-    __syncthreads();
+    if constexpr (TMA) {
+        // every thread is done with the staging buffer: refill it with the
+        // next tile's lists, unless a copy failed to arrive
+        const bool all_got = __syncthreads_and(got || !staged) != 0;
+        if (staged && !all_got) {
+            staged = false;
+            lost = true;
+            lost_phase = phase;
+            if (tid == 0) atomicAdd(&c->staging_fallbacks, 1u);
+        }
+        if (tid == 0) {
+            const uint32_t next = gridDim.x + atomicAdd(&c->tile_ticket, 1u);
+            sm.next_tile = next;
+            if (staged && next < n_tiles) {
+                mbar_arrive_expect_tx(&sm.bar, Smem::LBYTES);
+                tma_load_3d(&sm.lbuf[0][0][0], &lmap, &sm.bar, 4 * ((int)(next % (uint32_t)tiles_x) * FX - 1),
+                            (int)(next / (uint32_t)tiles_x) * FY - 1, 2 * (int)cur);
+            }
+        }
+        phase ^= 1u;
+    } else {
+        __syncthreads();
+    }
 
     // ---- A1: the distinct ids of the tile and halo lists -------------------
     uint32_t slot[K];  // hash slot of each own entry
@@ -923,11 +1058,17 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY)) fit_tile_kernel(con
             n_dropped += sm.warp_cnt[2][q];
         }
         // finish_pass_kernel, launched next, sums the partials
-        ws_loss_partials(ws)[blockIdx.y * gridDim.x + blockIdx.x] = (double)tl;
+        ws_loss_partials(ws)[tile] = (double)tl;
         if (n_empty) atomicAdd(&c->empty_pixels, (unsigned long long)n_empty);
         if (n_global) atomicAdd(&c->hash_overflow, (unsigned long long)n_global);
         if (n_dropped) atomicAdd(&c->dropped_ids, (unsigned long long)n_dropped);
     }
+    if (!TMA) break;
+    tile = sm.next_tile;  // written before this tile's later barriers, rewritten after the next tile's first
+    }
+    // a copy that timed out may still land: let it finish (bounded) before
+    // the block's shared memory is released
+    if (TMA && lost && tid == 0) (void)mbar_wait_bounded(&sm.bar, lost_phase);
 }
 
 // The end of a fitting pass, once every tile is done: the loss from the
@@ -948,6 +1089,7 @@ __global__ void __launch_bounds__(1024) finish_pass_kernel(void *ws, unsigned n_
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
         if (threadIdx.x == 0) {
             c->loss = s / P;
+            c->tile_ticket = 0u;
             if (prop) {
                 c->cur ^= 1u;
                 c->pass_counter += 1u;
@@ -957,20 +1099,70 @@ __global__ void __launch_bounds__(1024) finish_pass_kernel(void *ws, unsigned n_
 }
 
 // the tile state exceeds the 48 KB default: opt in once per device (done
-// when buffers are bound, so that a stream capture sees launches only)
-template <int FY, bool PROP, bool STATS>
-cudaError_t ensure_smem_attr() {
-    static bool attr_set[64] = {};
+// when buffers are bound, so that a stream capture sees launches only); the
+// persistent form also records how many blocks fill the device
+constexpr int MAX_DEV = 64;
+
+template <int FY, bool PROP, bool STATS, bool TMA>
+cudaError_t ensure_smem_attr(int *grid_blocks = nullptr) {
+    static bool attr_set[MAX_DEV] = {};
+    static int blocks[MAX_DEV] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(fit_tile_kernel<FY, PROP, STATS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(FusedSmem<FY, STATS>));
+    const bool cached = dev >= 0 && dev < MAX_DEV && attr_set[dev];
+    if (!cached) {
+        const int bytes = (int)sizeof(FusedSmem<FY, STATS, TMA>);
+        e = cudaFuncSetAttribute(fit_tile_kernel<FY, PROP, STATS, TMA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 bytes);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+        int per_sm = 0, sms = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fit_tile_kernel<FY, PROP, STATS, TMA>, FX * FY,
+                                                          (size_t)bytes);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < MAX_DEV) {
+            blocks[dev] = per_sm * sms;
+            attr_set[dev] = true;
+        }
+        if (grid_blocks) *grid_blocks = per_sm * sms;
+        return cudaSuccess;
     }
+    if (grid_blocks) *grid_blocks = blocks[dev];
     return cudaSuccess;
+}
+
+// cuTensorMapEncodeTiled, looked up through the runtime (no link against the
+// driver library); null where the driver does not offer it
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// The pixel-grid table as a 3-D array of 32-bit words for the staging copy:
+// x = the 4 W words of an image row of one plane, y = the H rows, z = table
+// * 2 + plane (plane stride P * 16 bytes).  The box is one tile's list block
+// with its halo: 4 (FX + 2) words x (FY + 2) rows x both planes; positions
+// outside the image read as zero, which the kernel masks by coordinates.
+bool encode_list_map(const Dev &d, int FY, CUtensorMap *map) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode || (reinterpret_cast<uintptr_t>(d.table) & 15u) || d.cell != 1) return false;
+    const cuuint64_t dims[3] = {4ull * (cuuint64_t)d.W, (cuuint64_t)d.H, 4ull};
+    const cuuint64_t strides[2] = {16ull * (cuuint64_t)d.W, 16ull * (cuuint64_t)d.P};
+    const cuuint32_t box[3] = {4u * HX, (cuuint32_t)FY + 2u, 2u};
+    const cuuint32_t elem[3] = {1u, 1u, 1u};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, d.table, dims, strides, box, elem,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int FY, bool PROP, bool STATS>
@@ -978,14 +1170,36 @@ cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
     // the propagating form works on the pixel grid only
     if (PROP && d.cell != 1) return cudaErrorInvalidValue;
     const TableGrid lists{d.cell, d.GW, (size_t)d.PT};
-    cudaError_t e = ensure_smem_attr<FY, PROP, STATS>();
-    if (e != cudaSuccess) return e;
     const dim3 grid((d.W + FX - 1) / FX, (d.H + FY - 1) / FY);
-    fit_tile_kernel<FY, PROP, STATS><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY, STATS>), st>>>(
-        d.records, d.table, d.target, d.H, d.W, d.N, G, d.image, d.grads, d.stats, d.ws, lists);
+    const uint32_t n_tiles = grid.x * grid.y;
+    CUtensorMap map;
+    std::memset(&map, 0, sizeof(map));
+    cudaError_t e;
+    bool staged = false;
+    if constexpr (PROP && !STATS && FY == 16) {
+        if (d.tma_staging && encode_list_map(d, FY, &map)) {
+            // persistent blocks with the list block staged by TMA
+            int blocks = 0;
+            e = ensure_smem_attr<FY, true, false, true>(&blocks);
+            if (e != cudaSuccess) return e;
+            if (blocks < 1) return cudaErrorInvalidConfiguration;
+            const unsigned nb = n_tiles < (uint32_t)blocks ? n_tiles : (unsigned)blocks;
+            fit_tile_kernel<FY, true, false, true><<<nb, dim3(FX, FY), sizeof(FusedSmem<FY, false, true>), st>>>(
+                d.records, d.table, d.target, d.H, d.W, d.N, G, d.image, d.grads, d.stats, d.ws, lists, map,
+                (int)grid.x, n_tiles);
+            staged = true;
+        }
+    }
+    if (!staged) {
+        e = ensure_smem_attr<FY, PROP, STATS, false>();
+        if (e != cudaSuccess) return e;
+        fit_tile_kernel<FY, PROP, STATS, false><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY, STATS>), st>>>(
+            d.records, d.table, d.target, d.H, d.W, d.N, G, d.image, d.grads, d.stats, d.ws, lists, map,
+            (int)grid.x, n_tiles);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    finish_pass_kernel<<<1, 1024, 0, st>>>(d.ws, grid.x * grid.y, (double)d.P, PROP ? 1 : 0);
+    finish_pass_kernel<<<1, 1024, 0, st>>>(d.ws, n_tiles, (double)d.P, PROP ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -997,12 +1211,13 @@ bool tall_tiles(const Dev &d) { return (long long)d.H * d.W >= 4ll * d.N; }
 }  // namespace
 
 cudaError_t prepare_fused() {
-    cudaError_t e = ensure_smem_attr<8, true, false>();
-    if (e == cudaSuccess) e = ensure_smem_attr<16, true, false>();
-    if (e == cudaSuccess) e = ensure_smem_attr<8, false, false>();
-    if (e == cudaSuccess) e = ensure_smem_attr<16, false, false>();
-    if (e == cudaSuccess) e = ensure_smem_attr<8, false, true>();
-    if (e == cudaSuccess) e = ensure_smem_attr<16, false, true>();
+    cudaError_t e = ensure_smem_attr<8, true, false, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, true, false, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, true, false, true>();
+    if (e == cudaSuccess) e = ensure_smem_attr<8, false, false, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, false, false, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<8, false, true, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, false, true, false>();
     return e;
 }
 

@@ -8,15 +8,16 @@
 //   seed_*_kernel       a9  seed pass of a refresh
 //   propagate_kernel    a2/a3  one Jacobi candidate pass (+ injection)
 //   render_kernel       a4  softmax blend of the current candidates
-//   render_bwd_kernel   a4-a6  render + MSE + analytic backward with a per-tile
-//                       shared-memory hash reduction of site gradients (or,
-//                       deterministic, 64-bit fixed-point integer atomics
-//                       finished by fixed_to_grads_kernel)
+//   render_bwd_det_kernel  a4-a6  render + MSE + analytic backward whose
+//                       gradients are summed in 64-bit fixed point with
+//                       integer atomics (order-independent), finished by
+//                       fixed_to_grads_kernel; the float backward is the
+//                       cached-list form of fit_tile_kernel
 //   adam_kernel         a7  Adam step + a1 for the updated sites
 //   jfa3x3_kernel       optional 3x3 flood prepass (summary B.3)
 //   tau_diffuse_kernel  Jacobi step on the ln tau gradients (summary B.6)
 //   target_u8_kernel    8-bit RGB -> planar float32 target
-// The fused steady-state pass is in sad_fused.cu, budget control in
+// The fused steady-state pass (also the float backward) is in sad_fused.cu, budget control in
 // sad_densify.cu, the 16-byte site record in sad_pack.cu.
 #include <cuda_fp16.h>
 
@@ -89,6 +90,8 @@ __global__ void init_counters_kernel(Counters *c, uint32_t seed) {
     c->ticket_prop = c->ticket_bwd = c->ticket_adam = 0;
     c->hash_overflow = c->nonfinite_pixels = c->empty_pixels = c->dropped_ids = 0;
     c->check_failures = 0;
+    c->staging_fallbacks = 0;
+    c->tile_ticket = 0;
     c->loss = 0.0;
 }
 
@@ -596,53 +599,26 @@ __global__ void __launch_bounds__(TILE_THREADS) render_kernel(const float4 *__re
 }
 
 // ---------------------------------------------------------------------------
-// a4-a6: render + MSE + backward, per-tile hash reduction of site gradients.
+// a4-a6, order-independent: render + MSE + backward whose gradients do not
+// depend on the order of the atomic additions.  Every warp-run sum is rounded
+// to a multiple of 2^-40 and added to a 64-bit fixed-point accumulator per
+// (parameter, site) with integer atomics, which are exact and so independent
+// of their order (the pages' integer-atomic gradient accumulation, summary
+// B.4).  The float form of this pass is fit_tile_kernel's cached-list form.
 // ---------------------------------------------------------------------------
-constexpr int HASH_BITS = 9;
-constexpr int HASH_SLOTS = 1 << HASH_BITS;
-constexpr int HASH_PROBES = 8;  // "linear probing capped at 8 probes"
-
-__device__ __forceinline__ int hash_find_or_insert(uint32_t *keys, uint32_t id) {
-    uint32_t s = (id * 2654435761u) >> (32 - HASH_BITS);
-#pragma unroll 1
-    for (int q = 0; q < HASH_PROBES; ++q) {
-        const uint32_t k = *reinterpret_cast<volatile uint32_t *>(keys + s);
-        if (k == id) return (int)s;
-        if (k == EMPTY) {
-            const uint32_t old = atomicCAS(keys + s, EMPTY, id);
-            if (old == EMPTY || old == id) return (int)s;
-        }
-        s = (s + 1) & (HASH_SLOTS - 1);
-    }
-    return -1;
-}
-
-// DET (deterministic): every run sum is rounded to a multiple of 2^-40 and
-// added to a 64-bit fixed-point accumulator per (parameter, site) with
-// integer atomics, which are exact and so independent of their order (the
-// pages' integer-atomic gradient accumulation, summary B.4); no tile table.
 constexpr float DET_SCALE = 1099511627776.0f;  // 2^40
 
-template <bool DET>
-__global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *__restrict__ rec,
-                                                                  const uint32_t *__restrict__ table,
-                                                                  const float *__restrict__ target, int H, int W,
-                                                                  TableGrid tg, int N, float *__restrict__ image,
-                                                                  float *__restrict__ grads, void *ws,
-                                                                  unsigned long long *__restrict__ fixed) {
+__global__ void __launch_bounds__(TILE_THREADS) render_bwd_det_kernel(const float4 *__restrict__ rec,
+                                                                      const uint32_t *__restrict__ table,
+                                                                      const float *__restrict__ target, int H,
+                                                                      int W, TableGrid tg, int N,
+                                                                      float *__restrict__ image, void *ws,
+                                                                      unsigned long long *__restrict__ fixed) {
     constexpr int NV = NPARAM;
-    __shared__ uint32_t keys[HASH_SLOTS];
-    __shared__ float acc[NV][HASH_SLOTS];
     __shared__ float warp_loss[TILE_THREADS / 32];
     Counters *c = counters(ws);
     const int lane = threadIdx.x;  // blockDim.x == 32: one warp per row segment
     const int tid = threadIdx.y * TILE_X + threadIdx.x;
-    for (int q = tid; q < HASH_SLOTS; q += TILE_THREADS) {
-        keys[q] = EMPTY;
-#pragma unroll
-        for (int j = 0; j < NV; ++j) acc[j][q] = 0.0f;
-    }
-    __syncthreads();
 
     const size_t P = (size_t)H * W;
     const uint4 *in0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * tg.PT * K);
@@ -653,7 +629,7 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
     const float invP = 1.0f / (float)P;
     const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
     float lsum = 0.0f;
-    unsigned dropped = 0, overflow = 0;
+    unsigned dropped = 0;
     bool empty = false;
     PixelSoftmax s;
     s.valid = 0;
@@ -709,23 +685,11 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
             v[PA] = -0.5f * gi * (r3.y * al * al - r3.z * be * be);
         }
         const bool tail = warp_run_reduce(key, v, lane);
-        if (DET) {
-            if (tail && key != EMPTY) {
+        if (tail && key != EMPTY) {
 #pragma unroll
-                for (int k = 0; k < NPARAM; ++k) {
-                    const long long qv = __float2ll_rn(v[k] * DET_SCALE);
-                    if (qv) atomicAdd(fixed + (size_t)k * N + key, (unsigned long long)qv);
-                }
-            }
-        } else if (tail && key != EMPTY) {
-            const int slot = hash_find_or_insert(keys, key);
-            if (slot >= 0) {
-#pragma unroll
-                for (int k = 0; k < NV; ++k) atomicAdd(&acc[k][slot], v[k]);
-            } else {
-                ++overflow;
-#pragma unroll
-                for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + key, v[k]);
+            for (int k = 0; k < NPARAM; ++k) {
+                const long long qv = __float2ll_rn(v[k] * DET_SCALE);
+                if (qv) atomicAdd(fixed + (size_t)k * N + key, (unsigned long long)qv);
             }
         }
     }
@@ -734,18 +698,6 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
     if ((tid & 31) == 0) warp_loss[tid >> 5] = lsum;
     const int ne = __syncthreads_count(empty);
     const int nd = __syncthreads_count(dropped != 0);
-    const int no = __syncthreads_count(overflow != 0);
-    // flush the tile table: one global atomic per (site, parameter)
-    if (!DET)
-    for (int q = tid; q < HASH_SLOTS; q += TILE_THREADS) {
-        const uint32_t id = keys[q];
-        if (id == EMPTY) continue;
-#pragma unroll
-        for (int k = 0; k < NPARAM; ++k) {
-            const float a = acc[k][q];
-            if (a != 0.0f) atomicAdd(grads + (size_t)k * N + id, a);
-        }
-    }
     if (tid == 0) {
         float t = 0.0f;
         for (int q = 0; q < TILE_THREADS / 32; ++q) t += warp_loss[q];
@@ -753,7 +705,6 @@ __global__ void __launch_bounds__(TILE_THREADS) render_bwd_kernel(const float4 *
         loss_partials(ws)[b] = (double)t;
         if (ne) atomicAdd(&c->empty_pixels, (unsigned long long)ne);
         if (nd) atomicAdd(&c->dropped_ids, (unsigned long long)nd);
-        if (no) atomicAdd(&c->hash_overflow, (unsigned long long)no);
         __threadfence();
     }
     // the last tile sums the loss partials in double
@@ -1031,17 +982,11 @@ cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_render_backward(const Dev &d, cudaStream_t st) {
-    render_bwd_kernel<false><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, d.ws, nullptr);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_render_backward_det(const Dev &d, cudaStream_t st) {
     unsigned long long *fixed =
         reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(d.ws) + fixed_offset(d.H, d.W, d.N));
-    render_bwd_kernel<true><<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.grads, d.ws, fixed);
+    render_bwd_det_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
+        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.ws, fixed);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long n = (long long)NPARAM * d.N;

@@ -20,6 +20,7 @@ struct Dev {
     const uint8_t *frozen;  // [N] sites Adam leaves untouched (optional)
     uint4 *cand16;          // [N] packed candidate-site records (optional)
     bool f16;               // candidate updates rank on cand16
+    bool tma_staging;       // propagating fit pass: persistent blocks, TMA-staged list blocks
     void *ws;
 };
 
@@ -48,7 +49,6 @@ cudaError_t launch_clear_table(const Dev &d, cudaStream_t st);
 cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st);
 cudaError_t launch_pack_cand16(const Dev &d, cudaStream_t st);
 cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st);
-cudaError_t launch_render_backward(const Dev &d, cudaStream_t st);
 cudaError_t launch_render_backward_det(const Dev &d, cudaStream_t st);
 cudaError_t launch_densify(const Dev &d, const DensifyArgs &a, cudaStream_t st);
 cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st);

@@ -6,7 +6,7 @@
 // over only input and output pointers, or latency-critical paths that must
 // not call cudaMalloc (it can synchronise the device).  For them this file
 // keeps the backward pass's scratch (a 256-byte counter block and one double
-// per 32 x 8 tile for the loss partials) in a file-scope device array that the
+// per tile of at least 32 x 8 pixels for the loss partials) in a file-scope device array that the
 // library owns for the life of the process, on every GPU that loads it.
 #include <atomic>
 #include <cstdint>
@@ -18,7 +18,7 @@
 namespace {
 
 constexpr size_t kScratchBytes = SAD_NOALLOC_SCRATCH_BYTES;
-constexpr int kTileX = 32, kTileY = 8;  // the tile of the render + backward kernel
+constexpr int kTileX = 32, kTileY = 8;  // the smallest tile of the render + backward kernel
 constexpr int kMaxDevices = 64;
 constexpr int kMaxGridY = 65535;  // launch limit on the tile rows (gridDim.y)
 
@@ -82,7 +82,7 @@ extern "C" int sad_backward_noalloc(int H, int W, int N_cap, const float *record
     d.image = image;
     d.grads = grads;
     d.ws = scratch;
-    if (sad::launch_render_backward(d, st) != cudaSuccess) return SAD_ERR_CUDA;
+    if (sad::launch_fit_tile_cached(d, st) != cudaSuccess) return SAD_ERR_CUDA;
     const double *src = &reinterpret_cast<const sad::Counters *>(scratch)->loss;
     if (cudaMemcpyAsync(loss, src, sizeof(double), cudaMemcpyDeviceToDevice, st) != cudaSuccess) return SAD_ERR_CUDA;
     return SAD_OK;

@@ -138,6 +138,12 @@ def test_bind_checks_alignment_and_sizes_without_touching_memory():
             _lib.sad_set_candidate_precision(ctx, 8)
         assert e.value.status == _lib.SAD_ERR_INVALID_ARG
         _lib.sad_set_candidate_precision(ctx, 32)
+        for bad in (-1, 2):
+            with pytest.raises(_lib.SadError) as e:
+                _lib.sad_set_list_staging(ctx, bad)
+            assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+        _lib.sad_set_list_staging(ctx, _lib.SAD_STAGING_TMA)
+        _lib.sad_set_list_staging(ctx, _lib.SAD_STAGING_LOADS)
         with pytest.raises(_lib.SadError) as e:
             _lib.sad_bind(ctx, **fake, cand16=0xD0008)
         assert "cand16" in str(e.value)

@@ -315,17 +315,23 @@ def test_fit_iteration_c1(torch_cuda):
     assert s.stats()["adam_step"] == 1 and s.stats()["pass_counter"] == 1
 
 
+@pytest.mark.parametrize("staging", ["loads", "tma"])
 @pytest.mark.parametrize("wl,H,W,N", [("c1", None, None, None), ("c2", None, None, None),
                                       ("c1", 37, 70, 400), ("c1", 8, 33, 50)])
-def test_fit_pass_matches_oracle(torch_cuda, wl, H, W, N):
+def test_fit_pass_matches_oracle(torch_cuda, wl, H, W, N, staging):
     """The fused pass (propagation at jump 1 + render + loss + backward) gives
-    the oracle's propagated table bit for bit and the oracle's gradients on it."""
+    the oracle's propagated table bit for bit and the oracle's gradients on it,
+    with the tiles' lists loaded per thread or staged by TMA copies (ragged
+    sizes: the copies' boxes reach past the image edges)."""
+    from soft_voronoi_render_b200 import SAD_STAGING_TMA
     tgt, prm, w = synth.make_workload(wl, seed=4, H=H, W=W, N=N)
     H, W, N = tgt.shape[1], tgt.shape[2], prm.shape[1]
     prm = prm.copy()
     prm[0, 3] = -1.0
     t0, npass = oracle.refresh(H, W, prm, 2, seed=21)
     s = make_ctx(torch_cuda, H, W, N, prm, tgt, seed=21)
+    if staging == "tma":
+        s.set_list_staging(SAD_STAGING_TMA)
     s.set_table(t0)
     s.fit_pass(2)
     rec = oracle.records(H, W, prm)
@@ -337,6 +343,38 @@ def test_fit_pass_matches_oracle(torch_cuda, wl, H, W, N):
     assert_grads(s.grads.cpu().numpy(), g, "fit_pass")
     st = s.stats()
     assert st["pass_counter"] == 1 and st["current_table"] == 1
+    assert st["staging_fallbacks"] == 0
+
+
+def test_full_size_c3_tma_staging(torch_cuda):
+    """2048 x 2048, N = 131,072, a few fitting iterations after a refresh:
+    the TMA-staged persistent form of the fit pass gives the per-tile form's
+    lists bit for bit over three passes (each pass hands out its tiles by a
+    ticket that the pass's finishing kernel resets), the same loss, and the
+    same gradients within the gradient tolerance (their float sums run in
+    another order)."""
+    from soft_voronoi_render_b200 import SAD_STAGING_LOADS, SAD_STAGING_TMA, adam_cfg
+    tgt, prm, w = synth.make_workload("c3", seed=2)
+    s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt, seed=2)
+    s.refresh(w.G)
+    cfg = adam_cfg(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=5e-3, lr_theta=1e-3, lr_a=1e-3)
+    for _ in range(5):
+        s.fit_iteration(w.G, cfg)
+    ck = s.checkpoint()
+    out = {}
+    for mode in (SAD_STAGING_LOADS, SAD_STAGING_TMA):
+        s.restore(ck)
+        s.set_list_staging(mode)
+        for _ in range(3):
+            s.grads.zero_()
+            s.fit_pass(w.G)
+        out[mode] = (s.get_table(), s.loss(), s.grads.cpu().numpy().astype(np.float64), s.stats())
+    (ta, la, ga, sa), (tb, lb, gb, sb) = out[SAD_STAGING_LOADS], out[SAD_STAGING_TMA]
+    np.testing.assert_array_equal(tb, ta)
+    assert (ta != ck["table"]).any(axis=1).mean() > 0.01  # the passes did change lists
+    assert abs(lb - la) <= 1e-6 * la
+    assert_grads(gb, ga, "tma staging")
+    assert sb["staging_fallbacks"] == 0 and sb["pass_counter"] == sa["pass_counter"] == ck["state"]["pass_counter"] + 3
 
 
 def test_fit_pass_generic_path_for_crowded_tiles(torch_cuda):
@@ -442,8 +480,9 @@ def test_full_size_c3_benchmark_state(torch_cuda):
     assert_grads(s.grads.cpu().numpy(), g, "c3 benchmark state")
     st = s.stats()
     assert st["empty_pixels"] == 0
-    # report how often entries took the global-atomic path in this pass
-    print("global-atomic pixels in the pass:", st["hash_overflow"] - before)
+    # in this state some injected winners come from outside their tile's
+    # index, so the global-atomic path of the pass is exercised too
+    assert st["hash_overflow"] - before > 0
 
 
 @pytest.mark.slow
@@ -562,7 +601,8 @@ def test_copy_loss_in_stream_order(torch_cuda):
 def test_backward_deterministic(torch_cuda, wl):
     """SAD_DETERMINISTIC: gradients bit-identical from run to run (fixed-point
     integer accumulation), within the gradient tolerance of the oracle, and
-    the same loss as the float path."""
+    the loss of the float path up to float32 rounding (the two kernels
+    blend and square in a different order)."""
     from soft_voronoi_render_b200 import SAD_DETERMINISTIC
     tgt, prm, w = synth.make_workload(wl, seed=6)
     s = make_ctx(torch_cuda, w.H, w.W, w.N, prm, tgt, seed=6)
@@ -580,4 +620,4 @@ def test_backward_deterministic(torch_cuda, wl):
     assert_grads(runs[0], g, "deterministic")
     s.grads.zero_()
     s.backward()
-    assert s.loss() == L_det
+    assert abs(s.loss() - L_det) <= 1e-6 * L_det
