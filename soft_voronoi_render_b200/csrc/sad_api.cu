@@ -404,6 +404,13 @@ int sad_fit_iteration(sad_ctx *ctx, int G, const sad_adam_cfg *cfg, sad_stream_t
     r = check_adam(ctx, cfg, h);
     if (r) return r;
     cudaStream_t st = cs(stream);
+    if (ctx->cell == 1 && !ctx->dev.f16) {
+        // the fused pass, then Adam, whose first block also finishes the pass
+        unsigned tiles = 0;
+        r = cuda_status(ctx, sad::launch_fit_tile(ctx->dev, G, st, &tiles), "fit pass");
+        if (r) return r;
+        return cuda_status(ctx, sad::launch_adam(ctx->dev, h, st, tiles), "adam");
+    }
     r = run_fit_pass(ctx, G, st);
     if (r) return r;
     return cuda_status(ctx, sad::launch_adam(ctx->dev, h, st), "adam");

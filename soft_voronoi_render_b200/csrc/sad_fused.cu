@@ -1071,31 +1071,10 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     if (TMA && lost && tid == 0) (void)mbar_wait_bounded(&sm.bar, lost_phase);
 }
 
-// The end of a fitting pass, once every tile is done: the loss from the
-// tiles' partials (summed in double) and, for the propagating form, the
-// other table made current and the pass counter advanced.  A separate launch
-// instead of a last-tile ticket: no tile waits on a global round trip.
-__global__ void __launch_bounds__(1024) finish_pass_kernel(void *ws, unsigned n_tiles, double P, int prop) {
-    Counters *c = ws_counters(ws);
-    const double *lp = ws_loss_partials(ws);
-    double s = 0.0;
-    for (unsigned q = threadIdx.x; q < n_tiles; q += 1024) s += lp[q];
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
-    __shared__ double red[32];
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        s = red[threadIdx.x];
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
-        if (threadIdx.x == 0) {
-            c->loss = s / P;
-            c->tile_ticket = 0u;
-            if (prop) {
-                c->cur ^= 1u;
-                c->pass_counter += 1u;
-            }
-        }
-    }
+// The end of a fitting pass as a launch of its own (sad_fit_iteration folds
+// it into the Adam launch instead): no tile waits on a global round trip.
+__global__ void __launch_bounds__(FINISH_THREADS) finish_pass_kernel(void *ws, unsigned n_tiles, double P, int prop) {
+    finish_pass_block(ws, n_tiles, P, prop);
 }
 
 // the tile state exceeds the 48 KB default: opt in once per device (done
@@ -1165,8 +1144,10 @@ bool encode_list_map(const Dev &d, int FY, CUtensorMap *map) {
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// finish_tiles: where given, the finishing step is left to the caller (it
+// gets the number of tile partials to sum); otherwise it is launched here
 template <int FY, bool PROP, bool STATS>
-cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
+cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st, unsigned *finish_tiles = nullptr) {
     // the propagating form works on the pixel grid only
     if (PROP && d.cell != 1) return cudaErrorInvalidValue;
     const TableGrid lists{d.cell, d.GW, (size_t)d.PT};
@@ -1199,7 +1180,11 @@ cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st) {
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    finish_pass_kernel<<<1, 1024, 0, st>>>(d.ws, n_tiles, (double)d.P, PROP ? 1 : 0);
+    if (finish_tiles) {
+        *finish_tiles = n_tiles;
+        return cudaSuccess;
+    }
+    finish_pass_kernel<<<1, FINISH_THREADS, 0, st>>>(d.ws, n_tiles, (double)d.P, PROP ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -1221,8 +1206,9 @@ cudaError_t prepare_fused() {
     return e;
 }
 
-cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st) {
-    return tall_tiles(d) ? launch_fit_tile_h<16, true, false>(d, G, st) : launch_fit_tile_h<8, true, false>(d, G, st);
+cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st, unsigned *finish_tiles) {
+    return tall_tiles(d) ? launch_fit_tile_h<16, true, false>(d, G, st, finish_tiles)
+                         : launch_fit_tile_h<8, true, false>(d, G, st, finish_tiles);
 }
 
 cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st) {

@@ -32,6 +32,7 @@ constexpr int TILE_X = 32;  // image-space blocks: one warp per 32-pixel row seg
 constexpr int TILE_Y = 8;
 constexpr int TILE_THREADS = TILE_X * TILE_Y;
 constexpr int SITE_THREADS = 256;
+static_assert(SITE_THREADS == FINISH_THREADS, "Adam's first block runs a pass's finishing step");
 
 
 __device__ __forceinline__ Counters *counters(void *ws) { return reinterpret_cast<Counters *>(ws); }
@@ -760,7 +761,11 @@ __global__ void __launch_bounds__(SITE_THREADS, 4) adam_kernel(float *__restrict
                                                             float *__restrict__ m1, float *__restrict__ m2,
                                                             float4 *__restrict__ rec, int N, int maxHW,
                                                             float xmax, float ymax, AdamArgs a,
-                                                            const uint8_t *__restrict__ frozen, Counters *c) {
+                                                            const uint8_t *__restrict__ frozen, Counters *c,
+                                                            unsigned finish_tiles, double P) {
+    // the preceding propagating fit pass's finishing step (its own launch
+    // otherwise): block 0 first
+    if (finish_tiles && blockIdx.x == 0) finish_pass_block(c, finish_tiles, P, 1);
     const uint32_t t = c->adam_step + 1u;
     const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
     // bias corrections 1 - beta^t, once per block
@@ -994,7 +999,7 @@ cudaError_t launch_render_backward_det(const Dev &d, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st) {
+cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st, unsigned finish_tiles) {
     AdamArgs a;
     for (int k = 0; k < NPARAM; ++k) a.lr[k] = h.lr[k];
     a.beta1 = h.beta1;
@@ -1002,7 +1007,8 @@ cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st) {
     a.eps = h.eps;
     adam_kernel<<<site_blocks(d.N), SITE_THREADS, 0, st>>>(d.params, d.grads, d.adam_m, d.adam_v, d.records, d.N,
                                                           d.H > d.W ? d.H : d.W, nextafterf((float)d.W, 0.0f),
-                                                          nextafterf((float)d.H, 0.0f), a, d.frozen, host_counters(d));
+                                                          nextafterf((float)d.H, 0.0f), a, d.frozen, host_counters(d),
+                                                          finish_tiles, (double)d.P);
     return cudaGetLastError();
 }
 

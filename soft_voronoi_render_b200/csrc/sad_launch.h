@@ -55,8 +55,11 @@ cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st);
 cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st);
 cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st);
 cudaError_t launch_fit_tile_cached_stats(const Dev &d, cudaStream_t st);
-cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st);
-cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st);
+// finish_tiles > 0: block 0 also finishes the fitting pass that wrote that
+// many tile partials (the propagating form), saving that pass its own launch
+cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st, unsigned finish_tiles = 0);
+// finish_tiles: where given, the pass's finishing step is left to the caller
+cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st, unsigned *finish_tiles = nullptr);
 cudaError_t prepare_fused();
 float *pack_range_device(const Dev &d);
 cudaError_t launch_pack(const Dev &d, uint32_t *packed, cudaStream_t st);
