@@ -173,12 +173,13 @@ class ClockSampler:
 # committed ncu traffic for the dominant kernel (null when the source changed)
 # ---------------------------------------------------------------------------
 def kernel_source_digest() -> str:
-    """Digest of the code the fused-pass kernel is compiled from (its own
-    file and the two headers it includes), comments and blank lines removed,
-    so that only a change of code makes committed counters stale."""
+    """Digest of the device code the fused-pass kernel is compiled from (the
+    kernel's header and the device header it includes), comments and blank
+    lines removed, so that only a change of device code makes committed
+    counters stale."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "soft_voronoi_render_b200", "csrc")
-    for f in ("sad_device.cuh", "sad_fused.cu", "sad_launch.h"):
+    for f in ("sad_device.cuh", "sad_fused_kernel.cuh"):
         txt = open(os.path.join(csrc, f)).read()
         txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
         lines = (re.sub(r"//.*", "", ln).rstrip() for ln in txt.splitlines())
