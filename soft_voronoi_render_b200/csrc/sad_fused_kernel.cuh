@@ -223,7 +223,7 @@ struct FusedSmem {
     float4 urec[REC_F4][UCAP + 1];  // field-major; entry UCAP is all zero
     uint4 masks[HN];                // 128-bit membership of every tile + halo pixel
     uint32_t cnt[UCAP];             // (pixel, slot) entries per local site
-    uint32_t cursor[UCAP];          // scatter cursor; afterwards the end of each site's entries
+    uint32_t cursor[UCAP];          // where each site's entries start
     float4 pixg[FT];                // per pixel: dL/dchat (3), chat . dL/dchat
     float2 ent_wl[GMAX][NGS];       // softmax weight, logit
     uint16_t ent_pu[GMAX][NGS16];   // pixel (low 9 bits), local site (high 7 bits)
@@ -897,6 +897,9 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     unsigned global_adds = 0;
     const float cdg = fmaf(cr, gr, fmaf(cg, gg, cb * gb));
     sm.pixg[tid] = make_float4(gr, gg, gb, cdg);
+    // slot q's place among its site's entries (16 bits, two slots a word):
+    // the count's atomic returns where the run starts
+    uint32_t offw[K / 2];
 #pragma unroll
     for (int q = 0; q < K; ++q) {
         const bool vq = vmask >> q & 1u;
@@ -904,8 +907,12 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
         const uint32_t key = (vq && t.lx[q] != NOLOC) ? t.lx[q] : EMPTY;
         int start, tail_lane;
         run_bounds(key, lane, start, tail_lane);
+        uint32_t first = 0;
         if (lane == tail_lane && key != EMPTY && SAD_CHECK(key < UCAP, ws))
-            atomicAdd(&sm.cnt[key], (uint32_t)(tail_lane - start + 1));
+            first = atomicAdd(&sm.cnt[key], (uint32_t)(tail_lane - start + 1));
+        first = __shfl_sync(FULL, first, tail_lane);
+        const uint32_t off = (first + (uint32_t)(lane - start)) & 0xFFFFu;
+        offw[q >> 1] = (q & 1) ? (offw[q >> 1] | off << 16) : off;
         if (vq && t.lx[q] == NOLOC) {
             const float4 *R = rec + (size_t)t.id[q] * REC_F4;
             const float4 r2 = __ldg(R + 2);
@@ -952,7 +959,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
         uint32_t base = incl - run;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            sm.cursor[lane * 4 + e] = base;
+            sm.cursor[lane * 4 + e] = base;  // where the site's entries start
             base += c4[e];
         }
         if (lane == 31) {
@@ -964,15 +971,9 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     const uint32_t gs = sm.gs;
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-        const bool vq = (vmask >> q & 1u) && t.lx[q] != NOLOC;
-        const uint32_t key = vq ? t.lx[q] : EMPTY;
-        int start, tail_lane;
-        run_bounds(key, lane, start, tail_lane);
-        uint32_t pos0 = 0;
-        if (lane == tail_lane && key != EMPTY && SAD_CHECK(key < UCAP, ws))
-            pos0 = atomicAdd(&sm.cursor[key], (uint32_t)(tail_lane - start + 1));
-        pos0 = __shfl_sync(FULL, pos0, tail_lane);
-        const uint32_t pos = pos0 + (uint32_t)(lane - start);
+        const bool vq = (vmask >> q & 1u) && t.lx[q] != NOLOC && SAD_CHECK(t.lx[q] < UCAP, ws);
+        const uint32_t key = vq ? t.lx[q] : 0u;
+        const uint32_t pos = sm.cursor[key] + (offw[q >> 1] >> ((q & 1) * 16) & 0xFFFFu);
         const uint32_t g = gs == 9u ? __umulhi(pos, 477218590u) : pos >> 3;  // pos / 9 exactly for pos < 2^16
         const uint32_t e = pos - g * gs;
         if (vq && SAD_CHECK(g < (uint32_t)Smem::NG && e < (uint32_t)Smem::GMAX, ws)) {
@@ -1000,7 +1001,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
             for (int k = 0; k < NV; ++k) a[k] = 0.0f;
             if (g < ng && SAD_CHECK(g < (uint32_t)Smem::NG && (sm.ent_pu[0][g] >> 9) < ucount, ws)) {
                 u = sm.ent_pu[0][g] >> 9;
-                const uint32_t rem = min(sm.cursor[u] - gs * g, gs);  // entries of the group (>= 1)
+                const uint32_t rem = min(sm.cursor[u] + sm.cnt[u] - gs * g, gs);  // entries of the group (>= 1)
                 const float4 r0 = sm.urec[0][u], r1 = sm.urec[1][u], r2 = sm.urec[2][u], r3 = sm.urec[3][u];
 #pragma unroll
                 for (int e = 0; e < Smem::GMAX; ++e) {
