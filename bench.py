@@ -524,6 +524,8 @@ def run_ours(args):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": dict(workload_config(wl, world), list_staging=args.staging),
             "hbm_roof_frac_iter": (iter_bytes / (ms_step * 1e-3) / 1e9) / hbm,
+            # the same bytes over the nominal 8 TB/s of B200's HBM3e
+            "hbm_roof_frac_iter_nominal_8tbs": (iter_bytes / (ms_step * 1e-3) / 1e9) / 8000.0,
             "iter_algorithmic_bytes": iter_bytes,
             "kernels_ms": {k: round(v, 5) for k, v in avg.items()},
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm,

@@ -233,33 +233,4 @@ __device__ __forceinline__ double *ws_loss_partials(void *ws) {
     return reinterpret_cast<double *>(reinterpret_cast<char *>(ws) + COUNTERS_BYTES);
 }
 
-// The end of a fitting pass, once every tile is done, run by one block of
-// FINISH_THREADS threads: the loss from the tiles' partials (summed in
-// double, always in the same order) and, for the propagating form, the other
-// table made current and the pass counter advanced.
-constexpr int FINISH_THREADS = 256;
-
-__device__ __forceinline__ void finish_pass_block(void *ws, unsigned n_tiles, double P, int prop) {
-    Counters *c = ws_counters(ws);
-    const double *lp = ws_loss_partials(ws);
-    double s = 0.0;
-    for (unsigned q = threadIdx.x; q < n_tiles; q += FINISH_THREADS) s += lp[q];
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    __shared__ double red[FINISH_THREADS / 32];
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        s = threadIdx.x < FINISH_THREADS / 32 ? red[threadIdx.x] : 0.0;
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (threadIdx.x == 0) {
-            c->loss = s / P;
-            c->tile_ticket = 0u;
-            if (prop) {
-                c->cur ^= 1u;
-                c->pass_counter += 1u;
-            }
-        }
-    }
-}
-
 }  // namespace sad

@@ -1,18 +1,26 @@
 // sad_fused.cu -- host launchers of the fused fitting pass (the kernel and
-// its tile state are in sad_fused_kernel.cuh): shared-memory opt-in, the
-// persistent grid of the TMA-staged form, the list block's tensor map.
+// its tile state are in sad_fused_kernel.cuh): the one-block finishing
+// kernel, shared-memory opt-in, the persistent grid of the TMA-staged form,
+// the list block's tensor map.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <atomic>
 #include <cstring>
 
+#include "sad_finish.cuh"
 #include "sad_fused_kernel.cuh"
 #include "sad_launch.h"
 
 namespace sad {
 
 namespace {
+
+// The end of a fitting pass as a launch of its own (sad_fit_iteration folds
+// it into the Adam launch instead): no tile waits on a global round trip.
+__global__ void __launch_bounds__(FINISH_THREADS) finish_pass_kernel(void *ws, unsigned n_tiles, double P, int prop) {
+    finish_pass_block(ws, n_tiles, P, prop);
+}
 
 // the tile state exceeds the 48 KB default: opt in once per device (done
 // when buffers are bound, so that a stream capture sees launches only); the

@@ -1,5 +1,5 @@
 // sad_fused_kernel.cuh -- device code of the fused fitting pass: the tile
-// state, the kernel and the one-block finishing kernel (host launchers in
+// state and the kernel (host launchers and the one-block finishing kernel in
 // sad_fused.cu, the only file that includes this one).
 //
 // One steady-state fitting pass over the image in a single kernel: the
@@ -1074,11 +1074,6 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     if (TMA && lost && tid == 0) (void)mbar_wait_bounded(&sm.bar, lost_phase);
 }
 
-// The end of a fitting pass as a launch of its own (sad_fit_iteration folds
-// it into the Adam launch instead): no tile waits on a global round trip.
-__global__ void __launch_bounds__(FINISH_THREADS) finish_pass_kernel(void *ws, unsigned n_tiles, double P, int prop) {
-    finish_pass_block(ws, n_tiles, P, prop);
-}
 
 }  // namespace
 

@@ -22,6 +22,7 @@
 #include <cuda_fp16.h>
 
 #include "sad_device.cuh"
+#include "sad_finish.cuh"
 #include "sad_launch.h"
 
 namespace sad {

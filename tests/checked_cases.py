@@ -6,7 +6,9 @@ the kernels whose indices rest on invariants rather than explicit guards --
 the fused pass (tile index, masks, grouped entries), the cached-list pass,
 the statistics backward, the standalone propagation and refresh -- on tiny
 and ragged sizes, checks the result against the CPU oracle, and reads the
-number of accesses the device-side checks refused.  Prints one JSON line."""
+number of accesses the device-side checks refused; the fused pass runs
+again with the TMA-staged list blocks (where its 32 x 16 tiles apply; the
+other cases take the default form).  Prints one JSON line."""
 import json
 import os
 import sys
@@ -22,7 +24,7 @@ import synth  # noqa: E402
 
 def main():
     assert os.environ.get("SAD_CHECKS") == "1"
-    from soft_voronoi_render_b200 import SAD_STATS, Sad, _lib
+    from soft_voronoi_render_b200 import SAD_STAGING_LOADS, SAD_STAGING_TMA, SAD_STATS, Sad, _lib
     assert _lib.library_path().endswith("libsad_checks.so")
     out = {"cases": 0, "check_failures": 0}
     for (H, W, N, seed) in ((1, 1, 3, 1), (9, 33, 40, 2), (37, 53, 300, 3), (16, 40, 200, 4), (24, 72, 6000, 5)):
@@ -43,6 +45,18 @@ def main():
         assert abs(s.loss() - L) <= 1e-5 * L
         gg = s.grads.cpu().numpy().astype(np.float64)
         assert np.all(np.abs(gg - g) <= np.maximum(1e-4 * np.abs(g), 1e-6))
+        # the same pass with the lists staged by TMA copies, from the same state
+        _lib.sad_set_fit_state(s.ctx, 0, 0, seed, s.stream)
+        s.set_table(t0)
+        s.set_list_staging(SAD_STAGING_TMA)
+        s.grads.zero_()
+        s.fit_pass(2)
+        assert np.array_equal(s.get_table(), t1), ("tma", H, W, N)
+        assert abs(s.loss() - L) <= 1e-5 * L
+        gg = s.grads.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(gg - g) <= np.maximum(1e-4 * np.abs(g), 1e-6))
+        assert s.stats()["staging_fallbacks"] == 0
+        s.set_list_staging(SAD_STAGING_LOADS)
         s.grads.zero_()
         s.fit_pass_cached()
         s.grads.zero_()

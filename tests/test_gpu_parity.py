@@ -317,12 +317,13 @@ def test_fit_iteration_c1(torch_cuda):
 
 @pytest.mark.parametrize("staging", ["loads", "tma"])
 @pytest.mark.parametrize("wl,H,W,N", [("c1", None, None, None), ("c2", None, None, None),
-                                      ("c1", 37, 70, 400), ("c1", 8, 33, 50)])
+                                      ("c1", 37, 70, 400), ("c1", 8, 33, 50), ("c1", 40, 48, 1000)])
 def test_fit_pass_matches_oracle(torch_cuda, wl, H, W, N, staging):
     """The fused pass (propagation at jump 1 + render + loss + backward) gives
     the oracle's propagated table bit for bit and the oracle's gradients on it,
     with the tiles' lists loaded per thread or staged by TMA copies (ragged
-    sizes: the copies' boxes reach past the image edges)."""
+    sizes: the copies' boxes reach past the image edges; 40 x 48 with 1,000
+    sites is dense enough for 32 x 8 tiles, where the default form runs)."""
     from soft_voronoi_render_b200 import SAD_STAGING_TMA
     tgt, prm, w = synth.make_workload(wl, seed=4, H=H, W=W, N=N)
     H, W, N = tgt.shape[1], tgt.shape[2], prm.shape[1]
