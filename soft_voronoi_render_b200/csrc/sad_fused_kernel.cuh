@@ -106,8 +106,11 @@ struct Top8L {
 __device__ __forceinline__ uint32_t uhash(uint32_t id) { return (id * 2654435761u) >> (32 - UHASH_BITS); }
 
 // insert a site id into the tile's key table (linear probing, compare-and-swap)
-// and return the slot that holds it, or NOSLOT when the probes run out
-__device__ __forceinline__ uint32_t ukey_insert(uint32_t *keys, uint32_t id) {
+// and return the slot that holds it, or NOSLOT when the probes run out.  The
+// lane that adds a new key also gives it the next dense tile-local index
+// (lid, and ulist for the first UCAP of them).
+__device__ __forceinline__ uint32_t ukey_insert(uint32_t *keys, uint32_t *lid, uint32_t *ulist, uint32_t *ucount,
+                                                uint32_t id) {
     uint32_t s = uhash(id);
 #pragma unroll 1
     for (int q = 0; q < UPROBES; ++q) {
@@ -115,7 +118,13 @@ __device__ __forceinline__ uint32_t ukey_insert(uint32_t *keys, uint32_t id) {
         if (k == id) return s;
         if (k == EMPTY) {
             const uint32_t old = atomicCAS(keys + s, EMPTY, id);
-            if (old == EMPTY || old == id) return s;
+            if (old == EMPTY) {
+                const uint32_t u = atomicAdd(ucount, 1u);
+                lid[s] = u;
+                if (u < UCAP) ulist[u] = id;
+                return s;
+            }
+            if (old == id) return s;
         }
         s = (s + 1) & (UHASH - 1);
     }
@@ -126,13 +135,14 @@ __device__ __forceinline__ uint32_t ukey_insert(uint32_t *keys, uint32_t id) {
 // the run inserts, the others take its slot (neighbouring pixels mostly hold
 // the same id in the same slot, which would otherwise contend for one key).
 // An id >= N inserts nothing and gets NOSLOT.
-__device__ __forceinline__ uint32_t warp_insert(uint32_t *keys, uint32_t id, uint32_t N, int lane) {
+__device__ __forceinline__ uint32_t warp_insert(uint32_t *keys, uint32_t *lid, uint32_t *ulist, uint32_t *ucount,
+                                                uint32_t id, uint32_t N, int lane) {
     const uint32_t prev = __shfl_up_sync(FULL, id, 1);
     const bool head = lane == 0 || prev != id;
     const uint32_t heads = __ballot_sync(FULL, head);
     const int start = 31 - __clz(heads & (0xFFFFFFFFu >> (31 - lane)));
     uint32_t s = NOSLOT;
-    if (head && id < N) s = ukey_insert(keys, id);
+    if (head && id < N) s = ukey_insert(keys, lid, ulist, ucount, id);
     return __shfl_sync(FULL, s, start);
 }
 
@@ -581,29 +591,18 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     bool ok = true;
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-        slot[q] = warp_insert(sm.keys, own[q], Nu, lane);
+        slot[q] = warp_insert(sm.keys, sm.lid, sm.ulist, &sm.ucount, own[q], Nu, lane);
         ok &= own[q] >= Nu || slot[q] != NOSLOT;
     }
     if (PROP) {
 #pragma unroll
         for (int x = 0; x < NRE; ++x) {
-            const uint32_t s = warp_insert(sm.keys, rv[x], Nu, lane);
+            const uint32_t s = warp_insert(sm.keys, sm.lid, sm.ulist, &sm.ucount, rv[x], Nu, lane);
             ok &= rv[x] >= Nu || s != NOSLOT;
             rv[x] = s != NOSLOT ? (s | (rcell[x] << 16)) : NOLOC;
         }
     }
     if (!ok) sm.overflow = 1;
-    __syncthreads();
-
-    // ---- A2: dense tile-local indices ------------------------------------
-    for (int s = tid; s < UHASH; s += FT) {
-        const uint32_t k = sm.keys[s];
-        if (k != EMPTY) {
-            const uint32_t u = atomicAdd(&sm.ucount, 1u);
-            sm.lid[s] = u;
-            if (u < UCAP) sm.ulist[u] = k;
-        }
-    }
     __syncthreads();
     const bool fast = !sm.overflow && sm.ucount <= UCAP;  // block-uniform
     const uint32_t ucount = fast ? sm.ucount : 0u;
