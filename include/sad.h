@@ -39,7 +39,9 @@
  *                                K = 8, 0xffffffff = empty).
  *   target   float32 [3][P]      planar linear RGB.
  *   image    float32 [3][P]      planar rendered image (may be NULL).
- *   workspace bytes >= sad_workspace_bytes(); counters, statistics, loss.
+ *   workspace bytes >= sad_workspace_bytes(); counters, statistics, loss,
+ *                                scratch, and the refresh's score cache
+ *                                (32 bytes per pixel).
  * Every pointer must be 16-byte aligned; target and image must not overlap
  * other buffers.  Which of the two tables is current is kept in device
  * memory, so a captured CUDA graph of the calls below keeps alternating.
@@ -214,7 +216,10 @@ int sad_topk_exact(sad_ctx *ctx, const int64_t *pixels, int64_t n_pix, uint32_t 
  * passes).  Clears the current table, writes each active site's id into slot
  * 0 of the pixel containing it (smallest id wins), then runs propagation
  * passes at jumps B/2, B/4, ..., 1 with B the largest power of two
- * <= max(H, W), each with G injections.  0 <= G <= 64. */
+ * <= max(H, W), each with G injections.  0 <= G <= 64.  The records do not
+ * change during a refresh, so with float32 candidates each pass keeps its
+ * lists' scores in the workspace and the next pass takes the pixel's own
+ * list's scores from there instead of recomputing them (the same bits). */
 int sad_refresh(sad_ctx *ctx, int G, sad_stream_t stream);
 
 /* Rebind the target image to another caller-owned device buffer (float32

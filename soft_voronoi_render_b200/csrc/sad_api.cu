@@ -71,8 +71,10 @@ int run_refresh(sad_ctx *ctx, int G, cudaStream_t st) {
     int B = 1;
     const int m = ctx->GH > ctx->GW ? ctx->GH : ctx->GW;
     while (B * 2 <= m) B *= 2;
+    // the records stay as they are during the refresh: the first pass stores
+    // each new list's scores, every later pass takes its own list's from there
     for (int k = B / 2; k >= 1; k /= 2) {
-        r = cuda_status(ctx, sad::launch_propagate(ctx->dev, k, G, st), "propagate");
+        r = cuda_status(ctx, sad::launch_propagate(ctx->dev, k, G, st, k == B / 2 ? 1 : 2), "propagate");
         if (r) return r;
     }
     return SAD_OK;

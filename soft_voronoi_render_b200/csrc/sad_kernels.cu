@@ -330,21 +330,36 @@ __device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], 
 // re-scored in its previous order it is usually still sorted and free of
 // repeats (the records do not change between refresh passes), and then it is
 // the top-8 of its own candidates as it stands; otherwise its repeats are
-// dropped and it is sorted.  Same result either way.
-template <bool F16, bool MERGE>
+// dropped and it is sorted.  Same result either way.  CACHED: the scores are
+// the ones the previous pass of the same refresh stored beside the list (the
+// same records, the same pixel: the same bits), so no record is fetched.
+template <bool F16, bool MERGE, bool CACHED = false>
 __device__ __forceinline__ void take_own_list(Top8 &t, const uint4 a, const uint4 b, const float4 *__restrict__ rec,
-                                              const uint4 *__restrict__ c16, uint32_t N, float fx, float fy) {
+                                              const uint4 *__restrict__ c16, uint32_t N, float fx, float fy,
+                                              const float4 *__restrict__ lc = nullptr) {
     const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    if constexpr (CACHED) {
+        const float4 l0 = lc[0], l1 = lc[1];
+        const float ls[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        t.l[q] = -__int_as_float(0x7f800000);
-        t.id[q] = EMPTY;
-        if (ids[q] < N) {
-            bool active;
-            const float lv = cand_logit<F16>(rec, c16, ids[q], fx, fy, active);
-            if (active && lv == lv) {
-                t.l[q] = lv;
-                t.id[q] = ids[q];
+        for (int q = 0; q < 8; ++q) {
+            // an empty slot was stored as -inf
+            const bool v = ids[q] < N && ls[q] == ls[q] && ls[q] != -__int_as_float(0x7f800000);
+            t.l[q] = v ? ls[q] : -__int_as_float(0x7f800000);
+            t.id[q] = v ? ids[q] : EMPTY;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            t.l[q] = -__int_as_float(0x7f800000);
+            t.id[q] = EMPTY;
+            if (ids[q] < N) {
+                bool active;
+                const float lv = cand_logit<F16>(rec, c16, ids[q], fx, fy, active);
+                if (active && lv == lv) {
+                    t.l[q] = lv;
+                    t.id[q] = ids[q];
+                }
             }
         }
     }
@@ -377,11 +392,16 @@ __device__ __forceinline__ void take_own_list(Top8 &t, const uint4 a, const uint
 // H x W is the candidate grid; a cell is scored at its centre, (i + 0.5) cs
 // (cs = 1: the pixel grid).  F16: candidates are ranked on the packed
 // records c16 and the kept 8 re-scored with the float32 records.
-template <bool F16, bool MERGE>
+// LC (score cache, float32 ranking only): 1 = store each list's scores in
+// lcache (two float4 per list, -inf for an empty slot), 2 = also take the
+// own list's scores from there; valid while the records stay unchanged,
+// which holds between the passes of one refresh.
+template <bool F16, bool MERGE, int LC = 0>
 __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *__restrict__ rec,
                                                                  const uint4 *__restrict__ c16, uint32_t *table,
                                                                  int H, int W, float cs, int N, int jump, int G,
-                                                                 Counters *c) {
+                                                                 Counters *c, float4 *__restrict__ lcache) {
+    static_assert(!(F16 && LC), "cached scores are float32 scores");
     const uint32_t cur = c->cur, pass = c->pass_counter, seed = c->seed;
     const size_t P = (size_t)H * W;
     const uint4 *in0 = reinterpret_cast<const uint4 *>(table + cur * P * K);
@@ -394,7 +414,8 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
         const size_t p = (size_t)j * W + i;
         const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
         Top8 t;
-        take_own_list<F16, MERGE>(t, in0[p], in1[p], rec, c16, (uint32_t)N, fx, fy);
+        take_own_list<F16, MERGE, LC == 2>(t, in0[p], in1[p], rec, c16, (uint32_t)N, fx, fy,
+                                           LC == 2 ? lcache + 2 * p : nullptr);
         // the neighbours at (-k, 0), (+k, 0), (0, -k), (0, +k); one outside
         // the image offers nothing
 #pragma unroll 1
@@ -439,6 +460,10 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
         }
         out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
         out1[p] = make_uint4(t.id[4], t.id[5], t.id[6], t.id[7]);
+        if constexpr (LC > 0) {
+            lcache[2 * p] = make_float4(t.l[0], t.l[1], t.l[2], t.l[3]);
+            lcache[2 * p + 1] = make_float4(t.l[4], t.l[5], t.l[6], t.l[7]);
+        }
     }
     // the last block to finish flips the double buffer and advances the pass
     // counter; every block has read both before taking its ticket
@@ -886,11 +911,17 @@ size_t fixed_offset(int H, int W, int N) {
     return (densify_offset(H, W) + 256 + 3 * sizeof(uint32_t) * (size_t)N + 255) / 256 * 256;
 }
 
+// the refresh's score cache: 8 float32 scores per list (32 bytes a pixel)
+size_t lcache_offset(int H, int W, int N) {
+    return (fixed_offset(H, W, N) + NPARAM * sizeof(unsigned long long) * (size_t)N + 255) / 256 * 256;
+}
+
 size_t workspace_bytes(int H, int W, int N) {
     // densify scratch: a 256-byte header, then the parent and free-slot lists;
     // then one float per site for tau diffusion; then the deterministic
-    // backward's 64-bit sums, one per (parameter, site)
-    return fixed_offset(H, W, N) + NPARAM * sizeof(unsigned long long) * (size_t)N;
+    // backward's 64-bit sums, one per (parameter, site); then the refresh's
+    // score cache
+    return lcache_offset(H, W, N) + 8 * sizeof(float) * (size_t)H * (size_t)W;
 }
 
 cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st) {
@@ -960,14 +991,24 @@ template <bool F16>
 void launch_propagate_f(const Dev &d, int jump, int G, cudaStream_t st) {
     const uint4 *c16 = F16 ? d.cand16 : nullptr;
     propagate_kernel<F16, true><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, c16, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d));
+        d.records, c16, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d), nullptr);
 }
 
-cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st) {
-    if (d.f16)
-        launch_propagate_f<true>(d, jump, G, st);
+cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st, int score_cache) {
+    if (d.f16 || score_cache == 0) {
+        if (d.f16)
+            launch_propagate_f<true>(d, jump, G, st);
+        else
+            launch_propagate_f<false>(d, jump, G, st);
+        return cudaGetLastError();
+    }
+    float4 *lc = reinterpret_cast<float4 *>(reinterpret_cast<char *>(d.ws) + lcache_offset(d.H, d.W, d.N));
+    if (score_cache == 1)
+        propagate_kernel<false, true, 1><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
+            d.records, nullptr, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d), lc);
     else
-        launch_propagate_f<false>(d, jump, G, st);
+        propagate_kernel<false, true, 2><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
+            d.records, nullptr, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d), lc);
     return cudaGetLastError();
 }
 

@@ -46,7 +46,10 @@ cudaError_t launch_target_u8(const Dev &d, const uint8_t *src, cudaStream_t st);
 cudaError_t launch_topk_exact(const Dev &d, const int64_t *pix, int64_t n, uint32_t *out, cudaStream_t st);
 cudaError_t launch_seed(const Dev &d, cudaStream_t st);
 cudaError_t launch_clear_table(const Dev &d, cudaStream_t st);
-cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st);
+// score_cache (float32 ranking only): 0 = none, 1 = store the new lists'
+// scores in the workspace, 2 = also take the own lists' scores from there
+// (only between passes over unchanged records, i.e. within one refresh)
+cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st, int score_cache = 0);
 cudaError_t launch_pack_cand16(const Dev &d, cudaStream_t st);
 cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st);
 cudaError_t launch_render_backward_det(const Dev &d, cudaStream_t st);
