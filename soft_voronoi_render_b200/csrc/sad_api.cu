@@ -295,8 +295,10 @@ int sad_jfa_prepass(sad_ctx *ctx, sad_stream_t stream) {
     const int m = ctx->GH > ctx->GW ? ctx->GH : ctx->GW;
     while ((1 << n) < m) ++n;
     if (n == 0) n = 1;
+    // the records stay as they are: each pass after the first starts from its
+    // own list's stored scores
     for (int q = n - 1; q >= 0; --q) {
-        r = cuda_status(ctx, sad::launch_jfa3x3(ctx->dev, 1 << q, st), "jfa pass");
+        r = cuda_status(ctx, sad::launch_jfa3x3(ctx->dev, 1 << q, st, q == n - 1 ? 1 : 2), "jfa pass");
         if (r) return r;
     }
     return SAD_OK;

@@ -497,9 +497,13 @@ __global__ void __launch_bounds__(SITE_THREADS) pack_cand16_kernel(const float4 
 
 // One 3x3 flood pass of the optional JFA prepass (summary B.3): the 4 best
 // distinct candidates of the lists at (i + a k, j + b k), a, b in {-1, 0, 1},
-// go to slots 0-3; slots 4-7 are emptied.
-__global__ void __launch_bounds__(TILE_THREADS) jfa3x3_kernel(const float4 *__restrict__ rec, uint32_t *table,
-                                                              int H, int W, float cs, int N, int jump, Counters *c) {
+// go to slots 0-3; slots 4-7 are emptied.  LC as in propagate_kernel: 1 =
+// store the new lists' scores in lcache, 2 = also start from the own list's
+// stored scores (its 4 entries, in order) and offer only the 8 neighbours.
+template <int LC = 0>
+__global__ void __launch_bounds__(TILE_THREADS, 5) jfa3x3_kernel(const float4 *__restrict__ rec, uint32_t *table,
+                                                              int H, int W, float cs, int N, int jump, Counters *c,
+                                                              float4 *__restrict__ lcache) {
     const uint32_t cur = c->cur, pass = c->pass_counter;
     const size_t P = (size_t)H * W;
     const uint4 *in0 = reinterpret_cast<const uint4 *>(table + cur * P * K);
@@ -513,8 +517,22 @@ __global__ void __launch_bounds__(TILE_THREADS) jfa3x3_kernel(const float4 *__re
         const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
         Top8 t;
         t.clear();
+        if constexpr (LC == 2) {
+            // the own list is the previous pass's top 4, sorted and distinct
+            const uint4 a = in0[p];
+            const float4 l0 = lcache[2 * p];
+            const uint32_t ids[4] = {a.x, a.y, a.z, a.w};
+            const float ls[4] = {l0.x, l0.y, l0.z, l0.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const bool v = ids[q] < (uint32_t)N && ls[q] == ls[q] && ls[q] != -__int_as_float(0x7f800000);
+                t.l[q] = v ? ls[q] : -__int_as_float(0x7f800000);
+                t.id[q] = v ? ids[q] : EMPTY;
+            }
+        }
 #pragma unroll 1
         for (int d = 0; d < 9; ++d) {
+            if (LC == 2 && d == 4) continue;
             const int ni = i + (d % 3 - 1) * jump, nj = j + (d / 3 - 1) * jump;
             if (ni < 0 || ni >= W || nj < 0 || nj >= H) continue;
             const size_t pn = (size_t)nj * W + ni;
@@ -524,6 +542,7 @@ __global__ void __launch_bounds__(TILE_THREADS) jfa3x3_kernel(const float4 *__re
         }
         out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
         out1[p] = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY);
+        if constexpr (LC > 0) lcache[2 * p] = make_float4(t.l[0], t.l[1], t.l[2], t.l[3]);
     }
     __syncthreads();
     if (threadIdx.x == 0 && threadIdx.y == 0) {
@@ -1017,9 +1036,17 @@ cudaError_t launch_pack_cand16(const Dev &d, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st) {
-    jfa3x3_kernel<<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(d.records, d.table, d.GH, d.GW,
-                                                                          (float)d.cell, d.N, jump, host_counters(d));
+cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st, int score_cache) {
+    float4 *lc = reinterpret_cast<float4 *>(reinterpret_cast<char *>(d.ws) + lcache_offset(d.H, d.W, d.N));
+    if (score_cache == 1)
+        jfa3x3_kernel<1><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
+            d.records, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, host_counters(d), lc);
+    else if (score_cache == 2)
+        jfa3x3_kernel<2><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
+            d.records, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, host_counters(d), lc);
+    else
+        jfa3x3_kernel<0><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
+            d.records, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, host_counters(d), nullptr);
     return cudaGetLastError();
 }
 

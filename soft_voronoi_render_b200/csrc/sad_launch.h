@@ -55,7 +55,7 @@ cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st);
 cudaError_t launch_render_backward_det(const Dev &d, cudaStream_t st);
 cudaError_t launch_densify(const Dev &d, const DensifyArgs &a, cudaStream_t st);
 cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st);
-cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st);
+cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st, int score_cache = 0);
 cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st);
 cudaError_t launch_fit_tile_cached_stats(const Dev &d, cudaStream_t st);
 // finish_tiles > 0: block 0 also finishes the fitting pass that wrote that
