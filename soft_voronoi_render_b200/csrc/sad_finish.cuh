@@ -35,7 +35,7 @@ __device__ __forceinline__ void finish_pass_block(void *ws, unsigned n_tiles, do
         s = threadIdx.x < FINISH_THREADS / 32 ? red[threadIdx.x] : 0.0;
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
         if (threadIdx.x == 0) {
-            c->loss = s / P;
+            if (n_tiles) c->loss = s / P;  // a pass without render leaves the loss alone
             c->tile_ticket = 0u;
             if (prop) {
                 c->cur ^= 1u;

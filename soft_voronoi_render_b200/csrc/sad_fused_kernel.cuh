@@ -23,7 +23,8 @@
 // The same kernel without the propagation (PROP = false) renders and
 // differentiates the cached lists as they stand, for the iterations between
 // candidate updates (summary B.3): no halo, no new lists, the pass counter
-// and the current table are left alone.
+// and the current table are left alone.  Without the render and backward
+// (BWD = false) it is a jump-1 propagation pass on its own.
 #pragma once
 
 #include <cuda.h>
@@ -424,7 +425,7 @@ __device__ __forceinline__ void generic_pass(Top8L &t, const uint4 *__restrict__
     }
 }
 
-template <int FY, bool PROP, bool STATS, bool TMA>
+template <int FY, bool PROP, bool STATS, bool TMA, bool BWD = true>
 __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     fit_tile_kernel(const float4 *__restrict__ rec, uint32_t *table, const float *__restrict__ target, int H, int W,
                     int N, int G, float *__restrict__ image, float *__restrict__ grads, float *__restrict__ stats,
@@ -432,6 +433,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
                     uint32_t n_tiles) {
     static_assert(!(PROP && STATS), "the statistics come with the cached-list form");
     static_assert(!TMA || (PROP && !STATS), "list staging serves the propagating form");
+    static_assert(BWD || (PROP && !STATS && !TMA), "the propagation alone is a form of the propagating pass");
     using Smem = FusedSmem<FY, STATS, TMA>;
     constexpr int NV = STATS ? NPARAM + NSTAT : NPARAM;
     constexpr int FT = Smem::FT, HN = Smem::HN, RING = Smem::RING;
@@ -546,7 +548,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
         }
     }
     // the target is read last: bring its lines into L2 now, registers later
-    if (inside && lane == 0) {
+    if (BWD && inside && lane == 0) {
         const size_t p = (size_t)j * W + i;
         asm volatile("prefetch.global.L2 [%0];" ::"l"(target + p));
         asm volatile("prefetch.global.L2 [%0];" ::"l"(target + P + p));
@@ -803,6 +805,8 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
         out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
         out1[p] = make_uint4(t.id[4], t.id[5], t.id[6], t.id[7]);
     }
+    // !BWD: a jump-1 propagation pass on its own (the whole block leaves here)
+    if constexpr (!BWD) return;
 
     // ---- D: render, loss and backward on the new lists ---------------------
     // A slot is valid iff its logit is finite: every list form above leaves
