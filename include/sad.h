@@ -217,9 +217,9 @@ int sad_topk_exact(sad_ctx *ctx, const int64_t *pixels, int64_t n_pix, uint32_t 
  * 0 of the pixel containing it (smallest id wins), then runs propagation
  * passes at jumps B/2, B/4, ..., 1 with B the largest power of two
  * <= max(H, W), each with G injections.  0 <= G <= 64.  The records do not
- * change during a refresh, so with float32 candidates each pass keeps its
- * lists' scores in the workspace and the next pass takes the pixel's own
- * list's scores from there instead of recomputing them (the same bits). */
+ * change during a refresh, so each pass keeps its lists' ranking scores in
+ * the workspace and the next pass takes the pixel's own list's scores from
+ * there instead of recomputing them (the same bits). */
 int sad_refresh(sad_ctx *ctx, int G, sad_stream_t stream);
 
 /* Rebind the target image to another caller-owned device buffer (float32
@@ -259,7 +259,7 @@ int sad_unpack_sites(sad_ctx *ctx, const uint32_t *packed, const float *range, s
  * one list per pixel.  Cell (i, j) holds the pixels with floor(x/cell) = i,
  * floor(y/cell) = j (integer mapping, no interpolation); propagation, seed,
  * exact top-K and the JFA prepass work on the grid and score candidates at
- * the cell centre ((i + 0.5) cell, (j + 0.5) cell) ("centred cell UVs");
+ * the cell centre ((i + 0.5) cell, (j + 0.5) cell), as the pages score cells;
  * render and backward score each pixel's cell list at the pixel centre.
  * Injections are keyed on the cell index.  cell = 1 (the default) is the
  * pixel grid.  On a coarser grid sad_fit_pass runs a propagation pass on the
@@ -276,7 +276,7 @@ int sad_set_candidate_grid(sad_ctx *ctx, int cell, sad_stream_t stream);
  * edits): the seed pass, then ceil(log2 max(H, W)) flood passes at jumps
  * 2^(n-1), ..., 1, each taking for every pixel the 4 best distinct candidates
  * of the 9 lists at (i + a k, j + b k), a, b in {-1, 0, 1}, into slots 0-3
- * ("four closest sites into the first candidate texture"; slots 4-7 empty).
+ * (the first of the two four-id planes; slots 4-7 empty).
  * Propagation passes then fill the lists. */
 int sad_jfa_prepass(sad_ctx *ctx, sad_stream_t stream);
 
@@ -284,7 +284,7 @@ int sad_jfa_prepass(sad_ctx *ctx, sad_stream_t stream);
  * for every pixel the new list is the top 8 by (logit desc, id asc) of the
  * distinct valid ids among its own list, the lists of the four pixels at
  * (+-jump, 0) and (0, +-jump) that lie inside the image, and G injected ids.
- * Injection ([P1] B.3: xorshift state from the step index and pixel id):
+ * Injection ([P1] B.3: an xorshift generator seeded per pass and pixel):
  * h = fmix32(p ^ fmix32(seed ^ pass * 0x9E3779B9)), 1 if zero, then G times
  * h = xorshift32(h) (13, 17, 5), id = (h * N_cap) >> 32.  Reads the current
  * table, writes the other one, makes it current, advances the pass counter. */
@@ -296,18 +296,20 @@ int sad_propagate(sad_ctx *ctx, int jump, int G, sad_stream_t stream);
 int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream);
 
 /* Steps a4-a6: render, MSE loss L = (1/P) sum_x sum_ch (chat - t)^2 and the
- * analytic gradient ([P1] B.4), accumulated into grads through a per-tile
- * shared-memory hash table keyed by site id (multiplicative hash, linear
- * probing capped at 8, compare-and-swap insert) with one global atomic per
- * (site, parameter, tile); overflow goes straight to global atomics
- * ([P1] section 5 and B.4).  Writes the bound image when one is bound and
+ * analytic gradient ([P1] B.4), accumulated into grads per tile before the
+ * global atomics ([P1] section 5 and B.4).  The pass is the tile pass on the
+ * current lists (the work of sad_fit_pass_cached): the tile's site ids go
+ * into a shared-memory hash keyed by site id (multiplicative hash, linear
+ * probing capped at 8, compare-and-swap insert) that gives each a dense
+ * tile-local index; the tile's (pixel, slot) entries are grouped by site and
+ * summed in registers, with one global atomic per (site, parameter, run of
+ * groups); entries of sites outside the index (more than 128 in a tile) go
+ * straight to global atomics.  Writes the bound image when one is bound and
  * the loss into the statistics block.  flags: 0, SAD_STATS (needs the stats
- * buffer; accumulates into it) or SAD_DETERMINISTIC (fixed-point
- * accumulation, order-independent).  With SAD_STATS the pass runs as the
- * fused tile pass on the current lists (the work of sad_fit_pass_cached),
- * whose per-tile accumulation groups the tile's entries by site and carries
- * the six statistics beside the nine gradients.  SAD_ERR_UNSUPPORTED for
- * other flags or both together. */
+ * buffer; carries the six statistics beside the nine gradients) or
+ * SAD_DETERMINISTIC (a pixel-per-thread pass whose warp sums are added in
+ * 64-bit fixed point: order-independent).  SAD_ERR_UNSUPPORTED for other
+ * flags or both together. */
 int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream);
 
 /* One budget-control event, on the device ([P1] B.5: split by the score
@@ -420,8 +422,8 @@ int sad_set_candidate_precision(sad_ctx *ctx, int bits, sad_stream_t stream);
 int sad_set_list_staging(sad_ctx *ctx, int mode, sad_stream_t stream);
 
 /* The fitting state that lives in the library's counter block: the pass
- * counter that keys the injection randomness ([P1] B.3: xorshift state from
- * the step index and pixel id), Adam's step count (bias correction) and the
+ * counter that keys the injection randomness ([P1] B.3: an xorshift
+ * generator seeded per pass and pixel), Adam's step count (bias correction) and the
  * injection seed.  Everything else a fit needs is in caller-owned buffers:
  * the sites (sad_get_sites / sad_set_sites), the Adam moments (the bound
  * adam_m / adam_v) and the current candidate lists (sad_get_table /

@@ -274,7 +274,7 @@ uint32_t orc_xorshift32(uint32_t h) { return xorshift32(h); }
 
 /*
  * The G injected site ids of pixel p in propagation pass number `pass`
- * ([P1] B.3: xorshift state from the step index and pixel id).  State
+ * ([P1] B.3: an xorshift generator seeded per pass and pixel).  State
  * h = fmix32(p ^ fmix32(seed ^ pass * 0x9E3779B9)), replaced by 1 if zero;
  * then h <- xorshift32(h) and id = floor(h * N / 2^32) (Lemire's
  * multiply-high range reduction) for each injection.
@@ -959,7 +959,7 @@ void orc_tau_diffuse(int H, int W, int N, const float *params, const uint32_t *t
  * One 3x3 flood pass at jump k: for each pixel, the distinct valid ids of the
  * lists at (i + a k, j + b k), a, b in {-1, 0, 1}, inside the image, re-scored
  * at the pixel; the 4 best by (logit desc, id asc) go to slots 0-3 and slots
- * 4-7 are emptied ("four closest sites into the first candidate texture").
+ * 4-7 are emptied (the prepass fills only the first of the two four-id planes).
  */
 void orc_jfa3x3_cell(int H, int W, int cell, int N, const float *rec32, const uint32_t *tin, uint32_t *tout,
                      int jump)

@@ -101,7 +101,7 @@ __device__ __forceinline__ float sad_logit_parts(float px, float py, float A, fl
 }
 
 // ---------------------------------------------------------------------------
-// injection randomness ("xorshift state from the step index and pixel ID")
+// injection randomness (an xorshift generator seeded per pass and pixel)
 // ---------------------------------------------------------------------------
 // MurmurHash3 32-bit finaliser (Austin Appleby, public domain).
 __device__ __forceinline__ uint32_t fmix32(uint32_t h) {

@@ -219,6 +219,29 @@ __device__ __forceinline__ void sort8(float (&l)[K], uint32_t (&id)[K]) {
     cx(l[1], id[1], l[2], id[2]); cx(l[3], id[3], l[4], id[4]); cx(l[5], id[5], l[6], id[6]);
 }
 
+// the same network carrying a payload with each entry
+__device__ __forceinline__ void cxp(float &la, uint32_t &ia, float &pa, float &lb, uint32_t &ib, float &pb) {
+    const bool s = ranks_above(lb, ib, la, ia);
+    const float tl = la, tp = pa;
+    const uint32_t ti = ia;
+    la = s ? lb : la;
+    ia = s ? ib : ia;
+    pa = s ? pb : pa;
+    lb = s ? tl : lb;
+    ib = s ? ti : ib;
+    pb = s ? tp : pb;
+}
+__device__ __forceinline__ void sort8p(float (&l)[K], uint32_t (&id)[K], float (&p)[K]) {
+#define SAD_CXP(a, b) cxp(l[a], id[a], p[a], l[b], id[b], p[b])
+    SAD_CXP(0, 1); SAD_CXP(2, 3); SAD_CXP(4, 5); SAD_CXP(6, 7);
+    SAD_CXP(0, 2); SAD_CXP(1, 3); SAD_CXP(4, 6); SAD_CXP(5, 7);
+    SAD_CXP(1, 2); SAD_CXP(5, 6);
+    SAD_CXP(0, 4); SAD_CXP(1, 5); SAD_CXP(2, 6); SAD_CXP(3, 7);
+    SAD_CXP(2, 4); SAD_CXP(3, 5);
+    SAD_CXP(1, 2); SAD_CXP(3, 4); SAD_CXP(5, 6);
+#undef SAD_CXP
+}
+
 // keep the best 8 of the running list and a sorted batch: the better of
 // t[i] and batch[7 - i] for every i are the 8 best, as a bitonic sequence,
 // which half-cleaners at distances 4, 2 and 1 put in order
@@ -392,16 +415,16 @@ __device__ __forceinline__ void take_own_list(Top8 &t, const uint4 a, const uint
 // H x W is the candidate grid; a cell is scored at its centre, (i + 0.5) cs
 // (cs = 1: the pixel grid).  F16: candidates are ranked on the packed
 // records c16 and the kept 8 re-scored with the float32 records.
-// LC (score cache, float32 ranking only): 1 = store each list's scores in
-// lcache (two float4 per list, -inf for an empty slot), 2 = also take the
-// own list's scores from there; valid while the records stay unchanged,
-// which holds between the passes of one refresh.
+// LC (score cache): 1 = store each list's ranking scores in lcache (two
+// float4 per list, -inf for an empty slot; with F16 the packed-record scores,
+// carried through the final float32 re-sort), 2 = also take the own list's
+// scores from there; valid while the records stay unchanged, which holds
+// between the passes of one refresh.
 template <bool F16, bool MERGE, int LC = 0>
 __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *__restrict__ rec,
                                                                  const uint4 *__restrict__ c16, uint32_t *table,
                                                                  int H, int W, float cs, int N, int jump, int G,
                                                                  Counters *c, float4 *__restrict__ lcache) {
-    static_assert(!(F16 && LC), "cached scores are float32 scores");
     const uint32_t cur = c->cur, pass = c->pass_counter, seed = c->seed;
     const size_t P = (size_t)H * W;
     const uint4 *in0 = reinterpret_cast<const uint4 *>(table + cur * P * K);
@@ -448,21 +471,27 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
                 offer_batch<8, F16, MERGE>(t, ids, rec, c16, (uint32_t)N, fx, fy);
             }
         }
+        float lrank[K];  // F16 with LC: each kept entry's packed-record score
         if constexpr (F16) {
             // the kept 8 in float32 logit order
 #pragma unroll
             for (int q = 0; q < K; ++q) {
+                lrank[q] = t.l[q];
                 if (t.id[q] == EMPTY) continue;
                 bool active;
                 t.l[q] = cand_logit<false>(rec, nullptr, t.id[q], fx, fy, active);
             }
-            sort8(t.l, t.id);
+            if constexpr (LC > 0)
+                sort8p(t.l, t.id, lrank);
+            else
+                sort8(t.l, t.id);
         }
         out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
         out1[p] = make_uint4(t.id[4], t.id[5], t.id[6], t.id[7]);
         if constexpr (LC > 0) {
-            lcache[2 * p] = make_float4(t.l[0], t.l[1], t.l[2], t.l[3]);
-            lcache[2 * p + 1] = make_float4(t.l[4], t.l[5], t.l[6], t.l[7]);
+            const float *ls = F16 ? lrank : t.l;
+            lcache[2 * p] = make_float4(ls[0], ls[1], ls[2], ls[3]);
+            lcache[2 * p + 1] = make_float4(ls[4], ls[5], ls[6], ls[7]);
         }
     }
     // the last block to finish flips the double buffer and advances the pass
@@ -1018,7 +1047,7 @@ cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st, int
     // every distinct candidate of a tile once from shared memory (no later
     // pass reads a score cache after a jump-1 pass)
     if (jump == 1 && d.cell == 1 && !d.f16) return launch_propagate_tile(d, G, st);
-    if (d.f16 || score_cache == 0) {
+    if (score_cache == 0) {
         if (d.f16)
             launch_propagate_f<true>(d, jump, G, st);
         else
@@ -1026,12 +1055,19 @@ cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st, int
         return cudaGetLastError();
     }
     float4 *lc = reinterpret_cast<float4 *>(reinterpret_cast<char *>(d.ws) + lcache_offset(d.H, d.W, d.N));
-    if (score_cache == 1)
-        propagate_kernel<false, true, 1><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
-            d.records, nullptr, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d), lc);
+    const dim3 grid = tile_grid(d.GH, d.GW), block(TILE_X, TILE_Y);
+    if (d.f16 && score_cache == 1)
+        propagate_kernel<true, true, 1><<<grid, block, 0, st>>>(d.records, d.cand16, d.table, d.GH, d.GW,
+                                                                (float)d.cell, d.N, jump, G, host_counters(d), lc);
+    else if (d.f16)
+        propagate_kernel<true, true, 2><<<grid, block, 0, st>>>(d.records, d.cand16, d.table, d.GH, d.GW,
+                                                                (float)d.cell, d.N, jump, G, host_counters(d), lc);
+    else if (score_cache == 1)
+        propagate_kernel<false, true, 1><<<grid, block, 0, st>>>(d.records, nullptr, d.table, d.GH, d.GW,
+                                                                 (float)d.cell, d.N, jump, G, host_counters(d), lc);
     else
-        propagate_kernel<false, true, 2><<<tile_grid(d.GH, d.GW), dim3(TILE_X, TILE_Y), 0, st>>>(
-            d.records, nullptr, d.table, d.GH, d.GW, (float)d.cell, d.N, jump, G, host_counters(d), lc);
+        propagate_kernel<false, true, 2><<<grid, block, 0, st>>>(d.records, nullptr, d.table, d.GH, d.GW,
+                                                                 (float)d.cell, d.N, jump, G, host_counters(d), lc);
     return cudaGetLastError();
 }
 

@@ -1,7 +1,7 @@
 """Pins of the oracle's downscaled candidate grid ("Soft Anisotropic Diagrams
 for Differentiable Image Representation", summary B.3 "Candidate field"):
 lists on a ceil(W/s) x ceil(H/s) grid, integer cell mapping, candidates
-scored at centred cell UVs.
+scored at the centres of their cells.
 
 Independent checks: exact top-K at the cell centres against scipy's k-d
 tree; one propagation pass against a numpy restatement scored at the cell
