@@ -830,6 +830,19 @@ struct AdamArgs {
     float beta1, beta2, eps;
 };
 
+// beta^t for an integer t by repeated squaring in double (at most 2 log2 t
+// roundings of relative size 2^-53: far below the float32 it is used in)
+__device__ __forceinline__ double pow_uint(double b, uint32_t t) {
+    double r = 1.0;
+#pragma unroll 1
+    while (t) {
+        if (t & 1u) r *= b;
+        b *= b;
+        t >>= 1;
+    }
+    return r;
+}
+
 // 4 blocks/SM (64 registers): the kernel is latency-bound, more warps hide it
 __global__ void __launch_bounds__(SITE_THREADS, 4) adam_kernel(float *__restrict__ prm, float *__restrict__ grads,
                                                             float *__restrict__ m1, float *__restrict__ m2,
@@ -842,13 +855,6 @@ __global__ void __launch_bounds__(SITE_THREADS, 4) adam_kernel(float *__restrict
     if (finish_tiles && blockIdx.x == 0) finish_pass_block(c, finish_tiles, P, 1);
     const uint32_t t = c->adam_step + 1u;
     const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
-    // bias corrections 1 - beta^t, once per block
-    __shared__ float bc[2];
-    if (threadIdx.x == 0) {
-        bc[0] = (float)(1.0 - pow((double)a.beta1, (double)t));
-        bc[1] = (float)(1.0 - pow((double)a.beta2, (double)t));
-    }
-    __syncthreads();
     if (i < N) {
         const size_t n = (size_t)N;
         float v[NPARAM];
@@ -856,7 +862,10 @@ __global__ void __launch_bounds__(SITE_THREADS, 4) adam_kernel(float *__restrict
         for (int k = 0; k < NPARAM; ++k) v[k] = prm[k * n + i];
         // frozen sites keep their parameters (summary section 7)
         if (v[PX] >= 0.0f && !(frozen && frozen[i])) {
-            const float bc1 = bc[0], bc2 = bc[1];
+            // bias corrections 1 - beta^t, every thread its own (no barrier),
+            // applied as multiplications by their reciprocals
+            const float ibc1 = (float)(1.0 / (1.0 - pow_uint((double)a.beta1, t)));
+            const float ibc2 = (float)(1.0 / (1.0 - pow_uint((double)a.beta2, t)));
             const float sig_pos = (float)maxHW;
 #pragma unroll
             for (int k = 0; k < NPARAM; ++k) {
@@ -866,7 +875,7 @@ __global__ void __launch_bounds__(SITE_THREADS, 4) adam_kernel(float *__restrict
                 const float vk = a.beta2 * m2[k * n + i] + (1.0f - a.beta2) * gh * gh;
                 m1[k * n + i] = mk;
                 m2[k * n + i] = vk;
-                const float mh = mk / bc1, vh = vk / bc2;
+                const float mh = mk * ibc1, vh = vk * ibc2;
                 v[k] -= a.lr[k] * sig * mh / (sqrtf(vh) + a.eps);
             }
             // the step keeps the position inside the image (x < 0 marks a pruned site)
