@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(FINISH_THREADS) finish_pass_kernel(void *ws, u
 // values, so relaxed atomics suffice.
 constexpr int MAX_DEV = 64;
 
-template <int FY, bool PROP, bool STATS, bool TMA, bool BWD = true>
+template <int FY, bool PROP, bool STATS, bool TMA, bool BWD = true, int JK = 1>
 cudaError_t ensure_smem_attr(int *grid_blocks = nullptr) {
     static std::atomic<int> blocks[MAX_DEV];  // 0: not yet set up on that device; -1: no block fits
     int dev = 0;
@@ -38,12 +38,12 @@ cudaError_t ensure_smem_attr(int *grid_blocks = nullptr) {
     const bool known = dev >= 0 && dev < MAX_DEV;
     int b = known ? blocks[dev].load(std::memory_order_relaxed) : 0;
     if (b == 0) {
-        const int bytes = (int)sizeof(FusedSmem<FY, STATS, TMA>);
-        e = cudaFuncSetAttribute(fit_tile_kernel<FY, PROP, STATS, TMA, BWD>,
+        const int bytes = (int)sizeof(FusedSmem<FY, STATS, TMA, JK>);
+        e = cudaFuncSetAttribute(fit_tile_kernel<FY, PROP, STATS, TMA, BWD, JK>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess) return e;
         int per_sm = 0, sms = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fit_tile_kernel<FY, PROP, STATS, TMA, BWD>,
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fit_tile_kernel<FY, PROP, STATS, TMA, BWD, JK>,
                                                           FX * FY, (size_t)bytes);
         if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -131,17 +131,19 @@ cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st, unsigned *fi
     return cudaGetLastError();
 }
 
-// a jump-1 propagation pass by the tile kernel without its render and
-// backward: the table flips and the pass counter advances, the loss stays
-template <int FY>
+// a jump-JK propagation pass (JK = 1, 2) by the tile kernel without its
+// render and backward: the table flips and the pass counter advances, the
+// loss stays
+template <int FY, int JK>
 cudaError_t launch_propagate_tile_h(const Dev &d, int G, cudaStream_t st) {
     const TableGrid lists{1, d.W, (size_t)d.P};
-    cudaError_t e = ensure_smem_attr<FY, true, false, false, false>();
+    cudaError_t e = ensure_smem_attr<FY, true, false, false, false, JK>();
     if (e != cudaSuccess) return e;
     const dim3 grid((d.W + FX - 1) / FX, (d.H + FY - 1) / FY);
     CUtensorMap map;
     std::memset(&map, 0, sizeof(map));
-    fit_tile_kernel<FY, true, false, false, false><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY, false>), st>>>(
+    fit_tile_kernel<FY, true, false, false, false, JK>
+        <<<grid, dim3(FX, FY), sizeof(FusedSmem<FY, false, false, JK>), st>>>(
         d.records, d.table, d.target, d.H, d.W, d.N, G, nullptr, nullptr, nullptr, d.ws, lists, map, (int)grid.x,
         grid.x * grid.y);
     e = cudaGetLastError();
@@ -165,14 +167,18 @@ cudaError_t prepare_fused() {
     if (e == cudaSuccess) e = ensure_smem_attr<16, false, false, false>();
     if (e == cudaSuccess) e = ensure_smem_attr<8, false, true, false>();
     if (e == cudaSuccess) e = ensure_smem_attr<16, false, true, false>();
-    if (e == cudaSuccess) e = ensure_smem_attr<8, true, false, false, false>();
-    if (e == cudaSuccess) e = ensure_smem_attr<16, true, false, false, false>();
+    if (e == cudaSuccess) e = ensure_smem_attr<8, true, false, false, false, 1>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, true, false, false, false, 1>();
+    if (e == cudaSuccess) e = ensure_smem_attr<8, true, false, false, false, 2>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, true, false, false, false, 2>();
     return e;
 }
 
-cudaError_t launch_propagate_tile(const Dev &d, int G, cudaStream_t st) {
-    if (d.cell != 1 || d.f16) return cudaErrorInvalidValue;
-    return tall_tiles(d) ? launch_propagate_tile_h<16>(d, G, st) : launch_propagate_tile_h<8>(d, G, st);
+cudaError_t launch_propagate_tile(const Dev &d, int jump, int G, cudaStream_t st) {
+    if (d.cell != 1 || d.f16 || (jump != 1 && jump != 2)) return cudaErrorInvalidValue;
+    if (jump == 2)
+        return tall_tiles(d) ? launch_propagate_tile_h<16, 2>(d, G, st) : launch_propagate_tile_h<8, 2>(d, G, st);
+    return tall_tiles(d) ? launch_propagate_tile_h<16, 1>(d, G, st) : launch_propagate_tile_h<8, 1>(d, G, st);
 }
 
 cudaError_t launch_fit_tile(const Dev &d, int G, cudaStream_t st, unsigned *finish_tiles) {

@@ -24,7 +24,9 @@
 // differentiates the cached lists as they stand, for the iterations between
 // candidate updates (summary B.3): no halo, no new lists, the pass counter
 // and the current table are left alone.  Without the render and backward
-// (BWD = false) it is a jump-1 propagation pass on its own.
+// (BWD = false) it is a propagation pass on its own, at jump JK = 1 or 2
+// (with a halo of width JK; at jump 2 the tile and its halo still hold at
+// most about 120 distinct sites during a refresh, within the index).
 #pragma once
 
 #include <cuda.h>
@@ -36,7 +38,7 @@ namespace sad {
 namespace {
 
 constexpr int FX = 32;                                 // tile width: one warp per row
-constexpr int HX = FX + 2;                             // halo row length
+constexpr int HX = FX + 2;                             // halo row length (halo width 1)
 constexpr int UCAP = 128;                              // tile-local site capacity
 constexpr int UW = UCAP / 32;                          // mask words
 constexpr int UHASH_BITS = 9;
@@ -209,9 +211,12 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
-template <int FY, bool STATS, bool TMA = false>
+// JK: the jump of the propagation and the width of the halo (1, or 2 for
+// the propagation alone)
+template <int FY, bool STATS, bool TMA = false, int JK = 1>
 struct FusedSmem {
-    static constexpr int FT = FX * FY, HN = HX * (FY + 2), RING = HN - FT;
+    static constexpr int HXJ = FX + 2 * JK;  // halo row length
+    static constexpr int FT = FX * FY, HN = HXJ * (FY + 2 * JK), RING = HN - FT;
     // TMA form: a tile's two list planes with the one-pixel halo, as the copy
     // lands them: [plane][halo row][4 words per halo column]
     static constexpr int LBZ = TMA ? 2 : 1, LBY = TMA ? FY + 2 : 1, LBX = TMA ? 4 * HX : 4;
@@ -248,21 +253,24 @@ struct FusedSmem {
     int overflow;
 };
 
-// halo ring pixel r -> halo coordinates: top row, bottom row, then the left
-// and right columns of the FY inner rows
-template <int FY>
+// halo ring pixel r -> halo coordinates for a halo of width JK: the JK top
+// rows, the JK bottom rows, then the JK left and JK right columns of each of
+// the FY inner rows
+template <int FY, int JK = 1>
 __device__ __forceinline__ void ring_coords(int r, int &hx, int &hy) {
-    constexpr int HY = FY + 2;
-    if (r < HX) {
-        hx = r;
-        hy = 0;
-    } else if (r < 2 * HX) {
-        hx = r - HX;
-        hy = HY - 1;
+    constexpr int HXJ = FX + 2 * JK, HY = FY + 2 * JK;
+    if (r < JK * HXJ) {
+        hy = r / HXJ;
+        hx = r - hy * HXJ;
+    } else if (r < 2 * JK * HXJ) {
+        const int q = r - JK * HXJ;
+        hy = HY - JK + q / HXJ;
+        hx = q - (q / HXJ) * HXJ;
     } else {
-        const int q = r - 2 * HX;
-        hy = 1 + (q >> 1);
-        hx = (q & 1) ? HX - 1 : 0;
+        const int q = r - 2 * JK * HXJ;
+        const int c = q % (2 * JK);
+        hy = JK + q / (2 * JK);
+        hx = c < JK ? c : FX + c;
     }
 }
 
@@ -405,12 +413,12 @@ __device__ __forceinline__ void offer_global(Top8L &t, uint32_t id, const float4
 
 __device__ __forceinline__ void generic_pass(Top8L &t, const uint4 *__restrict__ in0, const uint4 *__restrict__ in1,
                                              const float4 *__restrict__ rec, uint32_t N, int H, int W, int i, int j,
-                                             float fx, float fy) {
-    // own list, then the neighbours at (-1, 0), (+1, 0), (0, -1), (0, +1)
+                                             float fx, float fy, int jump) {
+    // own list, then the neighbours at (-k, 0), (+k, 0), (0, -k), (0, +k)
 #pragma unroll 1
     for (int d = 0; d < 5; ++d) {
-        const int ni = i + (d == 1 ? -1 : (d == 2 ? 1 : 0));
-        const int nj = j + (d == 3 ? -1 : (d == 4 ? 1 : 0));
+        const int ni = i + (d == 1 ? -jump : (d == 2 ? jump : 0));
+        const int nj = j + (d == 3 ? -jump : (d == 4 ? jump : 0));
         if (ni < 0 || ni >= W || nj < 0 || nj >= H) continue;
         const size_t pn = (size_t)nj * W + ni;
         const uint4 a = in0[pn], b = in1[pn];
@@ -425,7 +433,7 @@ __device__ __forceinline__ void generic_pass(Top8L &t, const uint4 *__restrict__
     }
 }
 
-template <int FY, bool PROP, bool STATS, bool TMA, bool BWD = true>
+template <int FY, bool PROP, bool STATS, bool TMA, bool BWD = true, int JK = 1>
 __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     fit_tile_kernel(const float4 *__restrict__ rec, uint32_t *table, const float *__restrict__ target, int H, int W,
                     int N, int G, float *__restrict__ image, float *__restrict__ grads, float *__restrict__ stats,
@@ -434,7 +442,10 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     static_assert(!(PROP && STATS), "the statistics come with the cached-list form");
     static_assert(!TMA || (PROP && !STATS), "list staging serves the propagating form");
     static_assert(BWD || (PROP && !STATS && !TMA), "the propagation alone is a form of the propagating pass");
-    using Smem = FusedSmem<FY, STATS, TMA>;
+    static_assert(JK == 1 || !BWD, "a wider halo serves the propagation alone");
+    static_assert(JK == 1 || !TMA, "the staged list block has a one-pixel halo");
+    using Smem = FusedSmem<FY, STATS, TMA, JK>;
+    constexpr int HXJ = Smem::HXJ;
     constexpr int NV = STATS ? NPARAM + NSTAT : NPARAM;
     constexpr int FT = Smem::FT, HN = Smem::HN, RING = Smem::RING;
     constexpr int NRE = (RING * K + FT - 1) / FT;  // halo (pixel, slot) entries per thread
@@ -508,9 +519,9 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
                 if (e < RING * K) {
                     const int r = e % RING, q = e / RING;
                     int hx, hy;
-                    ring_coords<FY>(r, hx, hy);
-                    cell = (uint32_t)(hy * HX + hx);
-                    const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
+                    ring_coords<FY, JK>(r, hx, hy);
+                    cell = (uint32_t)(hy * HXJ + hx);
+                    const int gi = i0 - JK + hx, gj = j0 - JK + hy;
                     if (gi >= 0 && gi < W && gj >= 0 && gj < H) id = sm.lbuf[q >> 2][hy][4 * hx + (q & 3)];
                 }
                 rv[x] = id;
@@ -536,9 +547,9 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
                 if (e < RING * K) {
                     const int r = e % RING, q = e / RING;
                     int hx, hy;
-                    ring_coords<FY>(r, hx, hy);
-                    cell = (uint32_t)(hy * HX + hx);
-                    const int gi = i0 - 1 + hx, gj = j0 - 1 + hy;
+                    ring_coords<FY, JK>(r, hx, hy);
+                    cell = (uint32_t)(hy * HXJ + hx);
+                    const int gi = i0 - JK + hx, gj = j0 - JK + hy;
                     if (gi >= 0 && gi < W && gj >= 0 && gj < H)
                         id = table[cur * P * K + (size_t)(q >> 2) * P * 4 + ((size_t)gj * W + gi) * 4 + (q & 3)];
                 }
@@ -629,7 +640,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
         own_lx_lo = pack_bytes(ux[0], ux[1], ux[2], ux[3]);
         own_lx_hi = pack_bytes(ux[4], ux[5], ux[6], ux[7]);
         if (PROP) {
-            uint32_t *m = reinterpret_cast<uint32_t *>(&sm.masks[(ty + 1) * HX + lane + 1]);
+            uint32_t *m = reinterpret_cast<uint32_t *>(&sm.masks[(ty + JK) * HXJ + lane + JK]);
 #pragma unroll
             for (int q = 0; q < K; ++q)
                 if (ux[q] != 0xFFu) atomicOr(m + (ux[q] >> 5), 1u << (ux[q] & 31u));
@@ -702,7 +713,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
                 t.id[q] = v ? gid : EMPTY;
                 t.lx[q] = v ? u : NOLOC;
             }
-            const int hc = (ty + 1) * HX + lane + 1;
+            const int hc = (ty + JK) * HXJ + lane + JK;
             const uint4 own_mask = sm.masks[hc];
             // a list holding one id twice keeps it once (the pass works on sets)
             if (nslots != __popc(own_mask.x) + __popc(own_mask.y) + __popc(own_mask.z) + __popc(own_mask.w)) {
@@ -724,8 +735,8 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
                 t.cx(1, 2); t.cx(3, 4); t.cx(5, 6);
             }
             // the candidates the four neighbours add
-            const uint4 mL = sm.masks[hc - 1], mR = sm.masks[hc + 1], mU = sm.masks[hc - HX],
-                        mD = sm.masks[hc + HX];
+            const uint4 mL = sm.masks[hc - JK], mR = sm.masks[hc + JK], mU = sm.masks[hc - JK * HXJ],
+                        mD = sm.masks[hc + JK * HXJ];
             nw[0] = (mL.x | mR.x | mU.x | mD.x) & ~own_mask.x;
             nw[1] = (mL.y | mR.y | mU.y | mD.y) & ~own_mask.y;
             nw[2] = (mL.z | mR.z | mU.z | mD.z) & ~own_mask.z;
@@ -772,7 +783,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
                 }
             }
         } else {
-            generic_pass(t, in0, in1, rec, Nu, H, W, i, j, fx, fy);
+            generic_pass(t, in0, in1, rec, Nu, H, W, i, j, fx, fy, JK);
         }
         if (G > 0) {
             // two injections per round: both records in flight together

@@ -1052,10 +1052,10 @@ void launch_propagate_f(const Dev &d, int jump, int G, cudaStream_t st) {
 }
 
 cudaError_t launch_propagate(const Dev &d, int jump, int G, cudaStream_t st, int score_cache) {
-    // jump 1 on the pixel grid: the tile kernel, whose tile index scores
-    // every distinct candidate of a tile once from shared memory (no later
-    // pass reads a score cache after a jump-1 pass)
-    if (jump == 1 && d.cell == 1 && !d.f16) return launch_propagate_tile(d, G, st);
+    // jumps 1 and 2 on the pixel grid: the tile kernel, whose tile index
+    // scores every distinct candidate of a tile once from shared memory (a
+    // refresh's passes after jump 4 read no score cache)
+    if ((jump == 1 || jump == 2) && d.cell == 1 && !d.f16) return launch_propagate_tile(d, jump, G, st);
     if (score_cache == 0) {
         if (d.f16)
             launch_propagate_f<true>(d, jump, G, st);

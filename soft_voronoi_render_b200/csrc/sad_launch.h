@@ -57,8 +57,9 @@ cudaError_t launch_densify(const Dev &d, const DensifyArgs &a, cudaStream_t st);
 cudaError_t launch_tau_diffuse(const Dev &d, float lambda, cudaStream_t st);
 cudaError_t launch_jfa3x3(const Dev &d, int jump, cudaStream_t st, int score_cache = 0);
 cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st);
-// a jump-1 propagation pass by the tile kernel (pixel grid, float32 ranking)
-cudaError_t launch_propagate_tile(const Dev &d, int G, cudaStream_t st);
+// a jump-1 or jump-2 propagation pass by the tile kernel (pixel grid,
+// float32 ranking)
+cudaError_t launch_propagate_tile(const Dev &d, int jump, int G, cudaStream_t st);
 cudaError_t launch_fit_tile_cached_stats(const Dev &d, cudaStream_t st);
 // finish_tiles > 0: block 0 also finishes the fitting pass that wrote that
 // many tile partials (the propagating form), saving that pass its own launch

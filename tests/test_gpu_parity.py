@@ -236,7 +236,9 @@ def test_adam_step_parity(torch_cuda):
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("H,W,N,jump,G", [(37, 53, 300, 1, 2), (37, 53, 300, 4, 0), (64, 40, 500, 16, 5),
-                                          (20, 17, 60, 64, 64), (1, 1, 1, 1, 3), (256, 256, 1024, 1, 2)])
+                                          (20, 17, 60, 64, 64), (1, 1, 1, 1, 3), (256, 256, 1024, 1, 2),
+                                          (37, 53, 300, 2, 2), (256, 256, 1024, 2, 2), (9, 33, 40, 2, 64),
+                                          (40, 48, 1000, 2, 3)])
 def test_propagate_bit_exact(torch_cuda, H, W, N, jump, G):
     prm = synth.uniform_sites(H, W, N, 6)
     prm[0, ::11] = -1.0
