@@ -107,12 +107,12 @@ typedef struct sad_buffers {
 #define SAD_STATS 1u
 
 /* sad_backward flag: gradients that do not depend on the order of the
- * atomic additions (bit-identical from run to run).  Every per-warp run sum
- * is rounded to a multiple of 2^-40 and accumulated in 64-bit fixed point
- * with integer atomics (exact, hence order-free), then added to grads; the
- * pages accumulate scaled integer gradients the same way on WebGPU
- * ([P1] B.4).  Magnitudes up to 2^23 per site and parameter; terms below
- * 2^-41 vanish.  Not combinable with SAD_STATS. */
+ * atomic additions (bit-identical from run to run).  Every (pixel, slot)
+ * contribution is rounded to a multiple of 2^-40 and summed in 64-bit fixed
+ * point, per tile and then with integer atomics (exact, hence order-free),
+ * then added to grads; the pages accumulate scaled integer gradients the
+ * same way on WebGPU ([P1] B.4).  Magnitudes up to 2^23 per site and
+ * parameter; terms below 2^-41 vanish.  Not combinable with SAD_STATS. */
 #define SAD_DETERMINISTIC 2u
 
 /* Densify / prune configuration ([P1] B.5, [P2] design 4). */
@@ -307,9 +307,9 @@ int sad_render(sad_ctx *ctx, float *image, sad_stream_t stream);
  * straight to global atomics.  Writes the bound image when one is bound and
  * the loss into the statistics block.  flags: 0, SAD_STATS (needs the stats
  * buffer; carries the six statistics beside the nine gradients) or
- * SAD_DETERMINISTIC (a pixel-per-thread pass whose warp sums are added in
- * 64-bit fixed point: order-independent).  SAD_ERR_UNSUPPORTED for other
- * flags or both together. */
+ * SAD_DETERMINISTIC (the same pass with its sums in 64-bit fixed point:
+ * order-independent).  SAD_ERR_UNSUPPORTED for other flags or both
+ * together. */
 int sad_backward(sad_ctx *ctx, uint32_t flags, sad_stream_t stream);
 
 /* One budget-control event, on the device ([P1] B.5: split by the score

@@ -168,8 +168,8 @@ struct Top8 {
 // lane order; a warp covers 32 consecutive pixels of a row, and neighbouring
 // pixels usually hold the same site in the same slot).  Afterwards the last
 // lane of every run holds the run's total.  Returns true on those lanes.
-template <int NV>
-__device__ __forceinline__ bool warp_run_reduce(uint32_t key, float (&v)[NV], int lane) {
+template <int NV, typename T>
+__device__ __forceinline__ bool warp_run_reduce(uint32_t key, T (&v)[NV], int lane) {
     constexpr unsigned FULL = 0xffffffffu;
     const uint32_t key_next = __shfl_down_sync(FULL, key, 1);
     const bool tail = lane == 31 || key_next != key;
@@ -201,7 +201,7 @@ __device__ __forceinline__ bool warp_run_reduce(uint32_t key, float (&v)[NV], in
                 const bool take = lane - off >= start;
 #pragma unroll
                 for (int k = 0; k < NV; ++k) {
-                    const float x = __shfl_up_sync(FULL, v[k], off);
+                    const T x = __shfl_up_sync(FULL, v[k], off);
                     if (take) v[k] += x;
                 }
             }
@@ -213,6 +213,11 @@ __device__ __forceinline__ bool warp_run_reduce(uint32_t key, float (&v)[NV], in
 
 // workspace views
 __device__ __forceinline__ Counters *ws_counters(void *ws);
+
+// Order-independent gradients: every contribution is rounded to a multiple
+// of 2^-40 and summed in 64-bit fixed point (integer sums are exact, so
+// their order does not matter); magnitudes up to 2^23 per sum.
+constexpr float FIXED_SCALE = 1099511627776.0f;  // 2^40
 
 // Bounds checks of the debug build (compiled with -DSAD_CHECKS): a failed
 // check is counted in the statistics block and the guarded access is

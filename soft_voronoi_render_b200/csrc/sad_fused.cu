@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(FINISH_THREADS) finish_pass_kernel(void *ws, u
 // values, so relaxed atomics suffice.
 constexpr int MAX_DEV = 64;
 
-template <int FY, bool PROP, bool STATS, bool TMA, bool BWD = true, int JK = 1>
+template <int FY, bool PROP, bool STATS, bool TMA, bool BWD = true, int JK = 1, bool DET = false>
 cudaError_t ensure_smem_attr(int *grid_blocks = nullptr) {
     static std::atomic<int> blocks[MAX_DEV];  // 0: not yet set up on that device; -1: no block fits
     int dev = 0;
@@ -39,12 +39,12 @@ cudaError_t ensure_smem_attr(int *grid_blocks = nullptr) {
     int b = known ? blocks[dev].load(std::memory_order_relaxed) : 0;
     if (b == 0) {
         const int bytes = (int)sizeof(FusedSmem<FY, STATS, TMA, JK>);
-        e = cudaFuncSetAttribute(fit_tile_kernel<FY, PROP, STATS, TMA, BWD, JK>,
+        e = cudaFuncSetAttribute(fit_tile_kernel<FY, PROP, STATS, TMA, BWD, JK, DET>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess) return e;
         int per_sm = 0, sms = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fit_tile_kernel<FY, PROP, STATS, TMA, BWD, JK>,
-                                                          FX * FY, (size_t)bytes);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &per_sm, fit_tile_kernel<FY, PROP, STATS, TMA, BWD, JK, DET>, FX * FY, (size_t)bytes);
         if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
@@ -152,6 +152,25 @@ cudaError_t launch_propagate_tile_h(const Dev &d, int G, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// the order-independent backward: the tile pass on the cached lists with
+// its sums in 64-bit fixed point (added to grads by the caller's next step)
+template <int FY>
+cudaError_t launch_fit_tile_cached_det_h(const Dev &d, unsigned long long *fixed, cudaStream_t st) {
+    const TableGrid lists{d.cell, d.GW, (size_t)d.PT};
+    cudaError_t e = ensure_smem_attr<FY, false, false, false, true, 1, true>();
+    if (e != cudaSuccess) return e;
+    const dim3 grid((d.W + FX - 1) / FX, (d.H + FY - 1) / FY);
+    CUtensorMap map;
+    std::memset(&map, 0, sizeof(map));
+    fit_tile_kernel<FY, false, false, false, true, 1, true><<<grid, dim3(FX, FY), sizeof(FusedSmem<FY, false>), st>>>(
+        d.records, d.table, d.target, d.H, d.W, d.N, 0, d.image, d.grads, d.stats, d.ws, lists, map, (int)grid.x,
+        grid.x * grid.y, fixed);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    finish_pass_kernel<<<1, FINISH_THREADS, 0, st>>>(d.ws, grid.x * grid.y, (double)d.P, 0);
+    return cudaGetLastError();
+}
+
 // taller tiles amortise the halo and the per-tile work, but hold more
 // distinct sites: use them unless sites are dense (< 4 pixels per site),
 // where tiles would often exceed the 128-site index
@@ -171,7 +190,14 @@ cudaError_t prepare_fused() {
     if (e == cudaSuccess) e = ensure_smem_attr<16, true, false, false, false, 1>();
     if (e == cudaSuccess) e = ensure_smem_attr<8, true, false, false, false, 2>();
     if (e == cudaSuccess) e = ensure_smem_attr<16, true, false, false, false, 2>();
+    if (e == cudaSuccess) e = ensure_smem_attr<8, false, false, false, true, 1, true>();
+    if (e == cudaSuccess) e = ensure_smem_attr<16, false, false, false, true, 1, true>();
     return e;
+}
+
+cudaError_t launch_fit_tile_cached_det(const Dev &d, unsigned long long *fixed, cudaStream_t st) {
+    return tall_tiles(d) ? launch_fit_tile_cached_det_h<16>(d, fixed, st)
+                         : launch_fit_tile_cached_det_h<8>(d, fixed, st);
 }
 
 cudaError_t launch_propagate_tile(const Dev &d, int jump, int G, cudaStream_t st) {

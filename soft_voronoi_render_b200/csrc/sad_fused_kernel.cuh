@@ -433,17 +433,18 @@ __device__ __forceinline__ void generic_pass(Top8L &t, const uint4 *__restrict__
     }
 }
 
-template <int FY, bool PROP, bool STATS, bool TMA, bool BWD = true, int JK = 1>
+template <int FY, bool PROP, bool STATS, bool TMA, bool BWD = true, int JK = 1, bool DET = false>
 __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     fit_tile_kernel(const float4 *__restrict__ rec, uint32_t *table, const float *__restrict__ target, int H, int W,
                     int N, int G, float *__restrict__ image, float *__restrict__ grads, float *__restrict__ stats,
                     void *ws, TableGrid lists, const __grid_constant__ CUtensorMap lmap, int tiles_x,
-                    uint32_t n_tiles) {
+                    uint32_t n_tiles, unsigned long long *__restrict__ fixed = nullptr) {
     static_assert(!(PROP && STATS), "the statistics come with the cached-list form");
     static_assert(!TMA || (PROP && !STATS), "list staging serves the propagating form");
     static_assert(BWD || (PROP && !STATS && !TMA), "the propagation alone is a form of the propagating pass");
     static_assert(JK == 1 || !BWD, "a wider halo serves the propagation alone");
     static_assert(JK == 1 || !TMA, "the staged list block has a one-pixel halo");
+    static_assert(!DET || (!PROP && !STATS && BWD), "the order-independent sums serve the cached-list backward");
     using Smem = FusedSmem<FY, STATS, TMA, JK>;
     constexpr int HXJ = Smem::HXJ;
     constexpr int NV = STATS ? NPARAM + NSTAT : NPARAM;
@@ -937,8 +938,14 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
                 slot_stats(eq * iz, er * er + eg * eg + eb * eb, dx, dy,
                            removal_delta(eq, r2, q == qstar, Z, iz, cr, cg, cb, zmm, cmr, cmg, cmb, er, eg, eb), v);
             ++global_adds;
+            if constexpr (DET) {
 #pragma unroll
-            for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + t.id[q], v[k]);
+                for (int k = 0; k < NPARAM; ++k)
+                    atomicAdd(fixed + (size_t)k * N + t.id[q], (unsigned long long)__float2ll_rn(v[k] * FIXED_SCALE));
+            } else {
+#pragma unroll
+                for (int k = 0; k < NPARAM; ++k) atomicAdd(grads + (size_t)k * N + t.id[q], v[k]);
+            }
             if constexpr (STATS) {
 #pragma unroll
                 for (int k = 0; k < NSTAT; ++k) atomicAdd(stats + (size_t)k * N + t.id[q], v[NPARAM + k]);
@@ -1001,7 +1008,46 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     }
     __syncthreads();
     // ---- D3: every thread sums one group of entries of one site ------------
-    {
+    if constexpr (DET) {
+        // order-independent: each entry's full contribution in fixed point,
+        // the group and run sums in 64-bit integers
+        const uint32_t ng = sm.n_groups;
+        const float fx0 = (float)i0 + 0.5f, fy0 = (float)j0 + 0.5f;
+#pragma unroll 1
+        for (uint32_t g0 = 0; g0 < ng; g0 += FT) {
+            if (g0 + (uint32_t)ty * 32u >= ng) break;  // warp-uniform
+            const uint32_t g = g0 + (uint32_t)tid;
+            uint32_t u = EMPTY;
+            long long a[NPARAM];
+#pragma unroll
+            for (int k = 0; k < NPARAM; ++k) a[k] = 0;
+            if (g < ng && SAD_CHECK(g < (uint32_t)Smem::NG && (sm.ent_pu[0][g] >> 9) < ucount, ws)) {
+                u = sm.ent_pu[0][g] >> 9;
+                const uint32_t rem = min(sm.cursor[u] + sm.cnt[u] - gs * g, gs);
+                const float4 r0 = sm.urec[0][u], r1 = sm.urec[1][u], r2 = sm.urec[2][u], r3 = sm.urec[3][u];
+#pragma unroll 1
+                for (int e = 0; e < Smem::GMAX; ++e) {
+                    if ((uint32_t)e >= rem) break;
+                    if (!SAD_CHECK((sm.ent_pu[e][g] & 0x1FFu) < (uint32_t)FT, ws)) continue;
+                    const uint32_t px = sm.ent_pu[e][g] & 0x1FFu;
+                    const float2 wl = sm.ent_wl[e][g];
+                    const float4 pa = sm.pixg[px];
+                    float v[NPARAM], dx, dy;
+                    slot_grad(r0, r1, r2, r3, fx0 + (float)(px & (FX - 1)), fy0 + (float)(px / FX), wl.y, wl.x, pa.x,
+                              pa.y, pa.z, pa.w, v, dx, dy);
+#pragma unroll
+                    for (int k = 0; k < NPARAM; ++k) a[k] += __float2ll_rn(v[k] * FIXED_SCALE);
+                }
+            }
+            const bool tail = warp_run_reduce(u, a, lane);
+            if (tail && u != EMPTY) {
+                const uint32_t gid = sm.ulist[u];
+#pragma unroll
+                for (int k = 0; k < NPARAM; ++k)
+                    if (a[k]) atomicAdd(fixed + (size_t)k * N + gid, (unsigned long long)a[k]);
+            }
+        }
+    } else {
         const uint32_t ng = sm.n_groups;
         const float fx0 = (float)i0 + 0.5f, fy0 = (float)j0 + 0.5f;
         const float half_P = 0.5f * (float)P, ex_scale = half_P * half_P;  // |chat - t|^2 = ex_scale |g|^2

@@ -8,11 +8,9 @@
 //   seed_*_kernel       a9  seed pass of a refresh
 //   propagate_kernel    a2/a3  one Jacobi candidate pass (+ injection)
 //   render_kernel       a4  softmax blend of the current candidates
-//   render_bwd_det_kernel  a4-a6  render + MSE + analytic backward whose
-//                       gradients are summed in 64-bit fixed point with
-//                       integer atomics (order-independent), finished by
-//                       fixed_to_grads_kernel; the float backward is the
-//                       cached-list form of fit_tile_kernel
+//   fixed_to_grads_kernel  adds the order-independent backward's 64-bit
+//                       fixed-point sums (the tile pass, sad_fused.cu) to
+//                       the gradients
 //   adam_kernel         a7  Adam step + a1 for the updated sites
 //   jfa3x3_kernel       optional 3x3 flood prepass (summary B.3)
 //   tau_diffuse_kernel  Jacobi step on the ln tau gradients (summary B.6)
@@ -673,142 +671,6 @@ __global__ void __launch_bounds__(TILE_THREADS) render_kernel(const float4 *__re
     }
 }
 
-// ---------------------------------------------------------------------------
-// a4-a6, order-independent: render + MSE + backward whose gradients do not
-// depend on the order of the atomic additions.  Every warp-run sum is rounded
-// to a multiple of 2^-40 and added to a 64-bit fixed-point accumulator per
-// (parameter, site) with integer atomics, which are exact and so independent
-// of their order (the pages' integer-atomic gradient accumulation, summary
-// B.4).  The float form of this pass is fit_tile_kernel's cached-list form.
-// ---------------------------------------------------------------------------
-constexpr float DET_SCALE = 1099511627776.0f;  // 2^40
-
-__global__ void __launch_bounds__(TILE_THREADS) render_bwd_det_kernel(const float4 *__restrict__ rec,
-                                                                      const uint32_t *__restrict__ table,
-                                                                      const float *__restrict__ target, int H,
-                                                                      int W, TableGrid tg, int N,
-                                                                      float *__restrict__ image, void *ws,
-                                                                      unsigned long long *__restrict__ fixed) {
-    constexpr int NV = NPARAM;
-    __shared__ float warp_loss[TILE_THREADS / 32];
-    Counters *c = counters(ws);
-    const int lane = threadIdx.x;  // blockDim.x == 32: one warp per row segment
-    const int tid = threadIdx.y * TILE_X + threadIdx.x;
-
-    const size_t P = (size_t)H * W;
-    const uint4 *in0 = reinterpret_cast<const uint4 *>(table + (size_t)c->cur * tg.PT * K);
-    const uint4 *in1 = in0 + tg.PT;
-    const int i = blockIdx.x * TILE_X + threadIdx.x;
-    const int j = blockIdx.y * TILE_Y + threadIdx.y;
-    const bool inside = i < W && j < H;
-    const float invP = 1.0f / (float)P;
-    const float fx = (float)i + 0.5f, fy = (float)j + 0.5f;
-    float lsum = 0.0f;
-    unsigned dropped = 0;
-    bool empty = false;
-    PixelSoftmax s;
-    s.valid = 0;
-    s.cr = s.cg = s.cb = 0.0f;
-    float gr = 0.0f, gg = 0.0f, gb = 0.0f, iz = 0.0f;
-    float er = 0.0f, eg = 0.0f, eb = 0.0f;
-    if (inside) {
-        const size_t p = (size_t)j * W + i;
-        const size_t pt = tg.cell_of(i, j, p);
-        const int nv = pixel_softmax(in0[pt], in1[pt], rec, (uint32_t)N, fx, fy, s, dropped);
-        empty = nv == 0;
-        er = s.cr - target[p];
-        eg = s.cg - target[P + p];
-        eb = s.cb - target[2 * P + p];
-        lsum = er * er + eg * eg + eb * eb;
-        if (image) {
-            image[p] = s.cr;
-            image[P + p] = s.cg;
-            image[2 * P + p] = s.cb;
-        }
-        gr = 2.0f * er * invP;
-        gg = 2.0f * eg * invP;
-        gb = 2.0f * eb * invP;
-        iz = nv ? 1.0f / s.Z : 0.0f;
-    }
-    // every lane runs the slot loop (the run reduction needs the whole warp)
-#pragma unroll
-    for (int q = 0; q < K; ++q) {
-        const bool vq = (s.valid >> q) & 1u;
-        const uint32_t key = vq ? s.id[q] : EMPTY;
-        float v[NV];
-#pragma unroll
-        for (int k = 0; k < NV; ++k) v[k] = 0.0f;
-        if (vq) {
-            const float4 *R = rec + (size_t)key * REC_F4;
-            const float4 r0 = __ldg(R), r1 = __ldg(R + 1), r2 = __ldg(R + 2), r3 = __ldg(R + 3);
-            float dx, dy, u1, u2, m;
-            const float l = sad_logit_parts(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy, dx, dy, u1, u2, m);
-            const float w = s.l[q] * iz;
-            const float gamma = w * ((r2.x - s.cr) * gr + (r2.y - s.cg) * gg + (r2.z - s.cb) * gb);
-            const float im = m > 0.0f ? 1.0f / m : 0.0f;
-            const float gi = gamma * im;
-            const float al = r2.w * dx + r3.x * dy;   // u . delta
-            const float be = -r3.x * dx + r2.w * dy;  // v . delta
-            v[PX] = gi * u1;
-            v[PY] = gi * u2;
-            v[PLT] = gamma * l;
-            v[PR] = gamma * r1.z;
-            v[PCR] = w * gr;
-            v[PCG] = w * gg;
-            v[PCB] = w * gb;
-            v[PTH] = -gi * al * be * (r3.y - r3.z);
-            v[PA] = -0.5f * gi * (r3.y * al * al - r3.z * be * be);
-        }
-        const bool tail = warp_run_reduce(key, v, lane);
-        if (tail && key != EMPTY) {
-#pragma unroll
-            for (int k = 0; k < NPARAM; ++k) {
-                const long long qv = __float2ll_rn(v[k] * DET_SCALE);
-                if (qv) atomicAdd(fixed + (size_t)k * N + key, (unsigned long long)qv);
-            }
-        }
-    }
-    // loss partial of this tile
-    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    if ((tid & 31) == 0) warp_loss[tid >> 5] = lsum;
-    const int ne = __syncthreads_count(empty);
-    const int nd = __syncthreads_count(dropped != 0);
-    if (tid == 0) {
-        float t = 0.0f;
-        for (int q = 0; q < TILE_THREADS / 32; ++q) t += warp_loss[q];
-        const unsigned b = blockIdx.y * gridDim.x + blockIdx.x;
-        loss_partials(ws)[b] = (double)t;
-        if (ne) atomicAdd(&c->empty_pixels, (unsigned long long)ne);
-        if (nd) atomicAdd(&c->dropped_ids, (unsigned long long)nd);
-        __threadfence();
-    }
-    // the last tile sums the loss partials in double
-    __shared__ bool last;
-    if (tid == 0) {
-        const unsigned total = gridDim.x * gridDim.y;
-        last = atomicAdd(&c->ticket_bwd, 1u) == total - 1;
-    }
-    __syncthreads();
-    if (last) {
-        __shared__ double red[TILE_THREADS];
-        const unsigned total = gridDim.x * gridDim.y;
-        const volatile double *lp = loss_partials(ws);
-        double t = 0.0;
-        for (unsigned q = tid; q < total; q += TILE_THREADS) t += lp[q];
-        red[tid] = t;
-        __syncthreads();
-        for (int o = TILE_THREADS / 2; o > 0; o >>= 1) {
-            if (tid < o) red[tid] += red[tid + o];
-            __syncthreads();
-        }
-        if (tid == 0) {
-            c->loss = red[0] / (double)P;
-            c->ticket_bwd = 0;
-            __threadfence();
-        }
-    }
-}
-
 // the deterministic backward's fixed-point sums, added to the gradients and
 // cleared for the next call
 __global__ void __launch_bounds__(SITE_THREADS) fixed_to_grads_kernel(unsigned long long *__restrict__ fixed,
@@ -1108,9 +970,7 @@ cudaError_t launch_render(const Dev &d, float *image, cudaStream_t st) {
 cudaError_t launch_render_backward_det(const Dev &d, cudaStream_t st) {
     unsigned long long *fixed =
         reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(d.ws) + fixed_offset(d.H, d.W, d.N));
-    render_bwd_det_kernel<<<tile_grid(d.H, d.W), dim3(TILE_X, TILE_Y), 0, st>>>(
-        d.records, d.table, d.target, d.H, d.W, grid_of(d), d.N, d.image, d.ws, fixed);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_fit_tile_cached_det(d, fixed, st);
     if (e != cudaSuccess) return e;
     const long long n = (long long)NPARAM * d.N;
     fixed_to_grads_kernel<<<site_blocks(n), SITE_THREADS, 0, st>>>(fixed, d.grads, n);

@@ -61,6 +61,9 @@ cudaError_t launch_fit_tile_cached(const Dev &d, cudaStream_t st);
 // float32 ranking)
 cudaError_t launch_propagate_tile(const Dev &d, int jump, int G, cudaStream_t st);
 cudaError_t launch_fit_tile_cached_stats(const Dev &d, cudaStream_t st);
+// the cached-list tile pass with order-independent sums into fixed ([NPARAM][N]
+// 64-bit fixed point, 2^-40 units)
+cudaError_t launch_fit_tile_cached_det(const Dev &d, unsigned long long *fixed, cudaStream_t st);
 // finish_tiles > 0: block 0 also finishes the fitting pass that wrote that
 // many tile partials (the propagating form), saving that pass its own launch
 cudaError_t launch_adam(const Dev &d, const AdamHyper &h, cudaStream_t st, unsigned finish_tiles = 0);
