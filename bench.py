@@ -396,6 +396,30 @@ def run_ours(args):
     ms_step = ms_max / K
     value = aggregate_mpix(world, P, K, ms_max)
 
+    # Cross-check with a CUDA graph: one sad_fit_iteration (the fused pass
+    # and Adam, two launches) captured once, 20 warm-up replays, then 5
+    # repeats of 200 timed replays; the median repeat is reported.
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        _lib.sad_fit_iteration(ctx, G, cfg, torch.cuda.current_stream(dev).cuda_stream)
+    for _ in range(20):
+        graph.replay()
+    g_reps = []
+    g0 = torch.cuda.Event(enable_timing=True)
+    g1 = torch.cuda.Event(enable_timing=True)
+    for _ in range(5):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        g0.record(stream)
+        for _ in range(200):
+            graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        g_reps.append(reduce_max(g0.elapsed_time(g1), dev) / 200)
+    del graph
+    graph_ms = statistics.median(g_reps)
+
     # end to end through the C ABI: each step's target comes from pinned host
     # memory and each step's loss goes back to pinned host memory
     E = max(1, min(args.e2e_steps, K))
@@ -554,6 +578,10 @@ def run_ours(args):
                     "serial_value": e2e_serial,
                     "u8_value": e2e_u8, "u8_h2d_bytes_per_step": int(host_u8.numel())},
             "gpu_launches": 3 * K,  # timed region: the fused pass, its finishing launch and Adam, per step
+            "graph": {"ms_per_step": graph_ms, "value": aggregate_mpix(world, P, 1, graph_ms), "unit": "Mpix/s",
+                      "repeats_ms": [round(x, 5) for x in g_reps],
+                      "how": "sad_fit_iteration captured once in a CUDA graph; 20 warm-up replays, 5 repeats of "
+                             "200 timed replays, median"},
             "clocks": clocks,
             "device_stats": {k: st[k] for k in ("hash_overflow", "empty_pixels", "dropped_ids")},
             "loss": st["loss"],
