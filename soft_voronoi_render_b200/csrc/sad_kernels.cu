@@ -34,10 +34,6 @@ constexpr int SITE_THREADS = 256;
 static_assert(SITE_THREADS == FINISH_THREADS, "Adam's first block runs a pass's finishing step");
 
 
-__device__ __forceinline__ Counters *counters(void *ws) { return reinterpret_cast<Counters *>(ws); }
-__device__ __forceinline__ double *loss_partials(void *ws) {
-    return reinterpret_cast<double *>(reinterpret_cast<char *>(ws) + COUNTERS_BYTES);
-}
 
 // ---------------------------------------------------------------------------
 // a1: per-site record, evaluated in double with the operation order of the
