@@ -137,8 +137,11 @@ typedef struct sad_adam_cfg {
 } sad_adam_cfg;
 
 typedef struct sad_stats {
-    uint64_t hash_overflow;    /* backward contributions that bypassed the tile table */
-    uint64_t nonfinite_pixels; /* pixels skipped by render/backward: sum of weights not finite */
+    uint64_t hash_overflow;    /* pixels with a backward contribution that bypassed the tile
+                                  index (a site outside it: crowded tiles, injected winners) */
+    uint64_t nonfinite_pixels; /* always 0: a slot whose logit is not finite (NaN parameters)
+                                  is not a candidate, so such a pixel renders from its other
+                                  slots or counts in empty_pixels */
     uint64_t empty_pixels;     /* pixels without any valid candidate (render writes 0) */
     uint64_t dropped_ids;      /* table entries >= N_cap met by render/backward */
     uint32_t pass_counter;     /* propagation passes run (drives injection randomness) */
