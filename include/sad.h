@@ -419,7 +419,12 @@ int sad_set_candidate_precision(sad_ctx *ctx, int bits, sad_stream_t stream);
  * latency, and a persistent block cannot begin its next tile before its
  * slowest warp has finished the current one.  The TMA form applies where
  * the pass uses 32 x 16 tiles (at least 4 pixels per site) on the pixel
- * grid; elsewhere the default runs.  SAD_ERR_INVALID_ARG for other modes. */
+ * grid; elsewhere the default runs.  The bounds-checked build of the
+ * library (compiled with SAD_CHECKS) withholds every persistent block's
+ * first copy when SAD_TEST_WITHHOLD_STAGING=1 is in the environment at the
+ * launch, and bounds that wait at 1,024 polls, so that a test can run the
+ * fallback; the normal build ignores the variable.  SAD_ERR_INVALID_ARG for
+ * other modes. */
 #define SAD_STAGING_LOADS 0
 #define SAD_STAGING_TMA 1
 int sad_set_list_staging(sad_ctx *ctx, int mode, sad_stream_t stream);

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstdlib>
 #include <cstring>
 
 #include "sad_finish.cuh"
@@ -87,6 +88,19 @@ bool encode_list_map(const Dev &d, int FY, CUtensorMap *map) {
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The bounds-checked build reads SAD_TEST_WITHHOLD_STAGING=1 from the
+// environment and then withholds the first staging copy of every persistent
+// block, so that a test can run the bounded wait's fallback to plain loads.
+// The normal build never withholds a copy.
+static uint32_t staging_test_flags() {
+#ifdef SAD_CHECKS
+    const char *v = std::getenv("SAD_TEST_WITHHOLD_STAGING");
+    return (v && v[0] == '1') ? 1u : 0u;
+#else
+    return 0u;
+#endif
+}
+
 // finish_tiles: where given, the finishing step is left to the caller (it
 // gets the number of tile partials to sum); otherwise it is launched here
 template <int FY, bool PROP, bool STATS>
@@ -110,7 +124,7 @@ cudaError_t launch_fit_tile_h(const Dev &d, int G, cudaStream_t st, unsigned *fi
             const unsigned nb = n_tiles < (uint32_t)blocks ? n_tiles : (unsigned)blocks;
             fit_tile_kernel<FY, true, false, true><<<nb, dim3(FX, FY), sizeof(FusedSmem<FY, false, true>), st>>>(
                 d.records, d.table, d.target, d.H, d.W, d.N, G, d.image, d.grads, d.stats, d.ws, lists, map,
-                (int)grid.x, n_tiles);
+                (int)grid.x, n_tiles, nullptr, staging_test_flags());
             staged = true;
         }
     }

@@ -183,11 +183,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 
 // wait until the barrier's phase with the given parity has completed, giving
 // up after a bounded number of polls (false: the copy did not arrive)
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
-    constexpr int POLLS = 1 << 22;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int polls) {
     const uint32_t a = smem_u32(bar);
 #pragma unroll 1
-    for (int n = 0; n < POLLS; ++n) {
+    for (int n = 0; n < polls; ++n) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -438,7 +437,8 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     fit_tile_kernel(const float4 *__restrict__ rec, uint32_t *table, const float *__restrict__ target, int H, int W,
                     int N, int G, float *__restrict__ image, float *__restrict__ grads, float *__restrict__ stats,
                     void *ws, TableGrid lists, const __grid_constant__ CUtensorMap lmap, int tiles_x,
-                    uint32_t n_tiles, unsigned long long *__restrict__ fixed = nullptr) {
+                    uint32_t n_tiles, unsigned long long *__restrict__ fixed = nullptr,
+                    uint32_t test_flags = 0) {
     static_assert(!(PROP && STATS), "the statistics come with the cached-list form");
     static_assert(!TMA || (PROP && !STATS), "list staging serves the propagating form");
     static_assert(BWD || (PROP && !STATS && !TMA), "the propagation alone is a form of the propagating pass");
@@ -472,13 +472,18 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     // not arrive within the wait's bound switches the block to global loads
     // (block-uniform, counted in staging_fallbacks).
     uint32_t tile = TMA ? blockIdx.x : blockIdx.y * gridDim.x + blockIdx.x;
+    // test_flags bit 0 (set only by the bounds-checked build's tests): the
+    // first staging copy is withheld, so the first wait runs out (after a
+    // short bound) and the block falls back to plain loads
+    const bool withhold = (test_flags & 1u) != 0;
+    const int polls = withhold ? 1024 : (1 << 22);
     uint32_t phase = 0, lost_phase = 0;
     bool staged = TMA, lost = false;
     if constexpr (TMA) {
         staged = (smem_u32(&sm.lbuf[0][0][0]) & 127u) == 0u;
         if (tid == 0 && staged) {
             mbar_init(&sm.bar, 1u);
-            if (tile < n_tiles) {
+            if (tile < n_tiles && !withhold) {
                 mbar_arrive_expect_tx(&sm.bar, Smem::LBYTES);
                 tma_load_3d(&sm.lbuf[0][0][0], &lmap, &sm.bar, 4 * ((int)(tile % (uint32_t)tiles_x) * FX - 1),
                             (int)(tile / (uint32_t)tiles_x) * FY - 1, 2 * (int)cur);
@@ -503,7 +508,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     uint32_t rv[NRE], rcell[NRE];
     bool got = false;
     if constexpr (TMA) {
-        if (staged) got = mbar_wait_bounded(&sm.bar, phase);
+        if (staged) got = mbar_wait_bounded(&sm.bar, phase, polls);
         if (got) {
             // halo row hy, halo column hx of plane z is lbuf[z][hy][4 hx ...]
             uint4 a = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY), b = a;
@@ -1131,7 +1136,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
     }
     // a copy that timed out may still land: let it finish (bounded) before
     // the block's shared memory is released
-    if (TMA && lost && tid == 0) (void)mbar_wait_bounded(&sm.bar, lost_phase);
+    if (TMA && lost && tid == 0) (void)mbar_wait_bounded(&sm.bar, lost_phase, polls);
 }
 
 

@@ -8,7 +8,11 @@ the statistics backward, the standalone propagation and refresh -- on tiny
 and ragged sizes, checks the result against the CPU oracle, and reads the
 number of accesses the device-side checks refused; the fused pass runs
 again with the TMA-staged list blocks (where its 32 x 16 tiles apply; the
-other cases take the default form).  Prints one JSON line."""
+other cases take the default form), and once more with every block's first
+staging copy withheld (SAD_TEST_WITHHOLD_STAGING=1, read only by this
+build): each block's bounded wait for the copy runs out, the block reads its
+lists from global memory, the result is the same and staging_fallbacks
+counts one fallback per block.  Prints one JSON line."""
 import json
 import os
 import sys
@@ -26,7 +30,7 @@ def main():
     assert os.environ.get("SAD_CHECKS") == "1"
     from soft_voronoi_render_b200 import SAD_STAGING_LOADS, SAD_STAGING_TMA, SAD_STATS, Sad, _lib
     assert _lib.library_path().endswith("libsad_checks.so")
-    out = {"cases": 0, "check_failures": 0}
+    out = {"cases": 0, "check_failures": 0, "withheld_fallbacks": 0}
     for (H, W, N, seed) in ((1, 1, 3, 1), (9, 33, 40, 2), (37, 53, 300, 3), (16, 40, 200, 4), (24, 72, 6000, 5)):
         prm = synth.uniform_sites(H, W, N, seed)
         tgt = synth.make_image(H, W, 4, 0, seed)
@@ -56,6 +60,25 @@ def main():
         gg = s.grads.cpu().numpy().astype(np.float64)
         assert np.all(np.abs(gg - g) <= np.maximum(1e-4 * np.abs(g), 1e-6))
         assert s.stats()["staging_fallbacks"] == 0
+        # the first copy of every persistent block withheld: one persistent
+        # block per tile at these sizes, each falling back once
+        tall = H * W >= 4 * N
+        n_tiles = ((W + 31) // 32) * ((H + 15) // 16)
+        _lib.sad_set_fit_state(s.ctx, 0, 0, seed, s.stream)
+        s.set_table(t0)
+        s.grads.zero_()
+        os.environ["SAD_TEST_WITHHOLD_STAGING"] = "1"
+        try:
+            s.fit_pass(2)  # the variable is read when the pass is launched
+        finally:
+            del os.environ["SAD_TEST_WITHHOLD_STAGING"]
+        assert np.array_equal(s.get_table(), t1), ("withheld", H, W, N)
+        assert abs(s.loss() - L) <= 1e-5 * L
+        gg = s.grads.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(gg - g) <= np.maximum(1e-4 * np.abs(g), 1e-6))
+        fb = s.stats()["staging_fallbacks"]
+        assert fb == (n_tiles if tall else 0), (H, W, N, fb, n_tiles)
+        out["withheld_fallbacks"] += fb
         s.set_list_staging(SAD_STAGING_LOADS)
         s.grads.zero_()
         s.fit_pass_cached()

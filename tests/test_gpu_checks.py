@@ -24,3 +24,6 @@ def test_checked_build_refuses_no_access():
     assert r.returncode == 0, r.stderr[-3000:]
     res = json.loads(r.stdout.strip().splitlines()[-1])
     assert res["cases"] == 5 and res["check_failures"] == 0, res
+    # two of the cases take the TMA-staged form (2 and 6 tiles); with their
+    # first copies withheld every block fell back to plain loads
+    assert res["withheld_fallbacks"] == 8, res
