@@ -42,8 +42,9 @@
  *   workspace bytes >= sad_workspace_bytes(); counters, statistics, loss,
  *                                scratch, and the refresh's score cache
  *                                (32 bytes per pixel).
- * Every pointer must be 16-byte aligned; target and image must not overlap
- * other buffers.  Which of the two tables is current is kept in device
+ * Every pointer must be 16-byte aligned and records 32-byte aligned (the
+ * kernels read a record's ranking fields in one 32-byte load); target and
+ * image must not overlap other buffers.  Which of the two tables is current is kept in device
  * memory, so a captured CUDA graph of the calls below keeps alternating.
  *
  * Calls.  Every call except sad_get_stats, sad_get_loss, sad_get_table and
@@ -481,7 +482,8 @@ const char *sad_last_error(const sad_ctx *ctx);
  *   target   float32 [3][P];  image float32 [3][P] or NULL
  *   grads    float32 [9][N_cap], accumulated into (zero it first)
  *   loss     one device double, receives L
- * Pointers 16-byte aligned (loss 8-byte).  Returns SAD_ERR_CAPACITY when
+ * Pointers 16-byte aligned, records 32-byte (loss 8-byte).  Returns
+ * SAD_ERR_CAPACITY when
  * ceil(W/32) * ceil(H/8) exceeds (SAD_NOALLOC_SCRATCH_BYTES - 256) / 8 =
  * 131,040 tiles (4096 x 8192 fits) or ceil(H/8) exceeds 65,535 (the launch
  * limit on tile rows), SAD_ERR_INVALID_ARG for bad sizes or pointers,

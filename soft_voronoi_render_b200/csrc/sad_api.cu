@@ -158,6 +158,9 @@ int sad_bind(sad_ctx *ctx, const sad_buffers *b) {
         if (!req[q]) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer %s is NULL", names[q]);
         if (!aligned16(req[q])) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer %s is not 16-byte aligned", names[q]);
     }
+    // the kernels read a record's ranking fields in one 32-byte load
+    if ((reinterpret_cast<uintptr_t>(b->records) & 31u) != 0)
+        return fail(ctx, SAD_ERR_INVALID_ARG, "buffer records is not 32-byte aligned");
     if (b->image && !aligned16(b->image)) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer image is not 16-byte aligned");
     if (b->stats && !aligned16(b->stats)) return fail(ctx, SAD_ERR_INVALID_ARG, "buffer stats is not 16-byte aligned");
     if (b->cand16 && !aligned16(b->cand16))

@@ -60,6 +60,17 @@ struct TableGrid {
     }
 };
 
+// The ranking fields of site x's record -- x, y, A, B, C, b, the first 24 of
+// its 64 bytes -- in one 256-bit load (the last two words of the 32 are not
+// kept).  The records buffer is 32-byte aligned (sad_bind and the
+// allocation-free entry point refuse one that is not).
+__device__ __forceinline__ void load_rank_fields(const float4 *__restrict__ rec, uint32_t x, float &px, float &py,
+                                                 float &A, float &B, float &C, float &b) {
+    asm("ld.global.nc.v8.f32 {%0, %1, %2, %3, %4, %5, _, _}, [%6];"
+        : "=f"(px), "=f"(py), "=f"(A), "=f"(B), "=f"(C), "=f"(b)
+        : "l"(rec + (size_t)x * REC_F4));
+}
+
 // ---------------------------------------------------------------------------
 // ranking: (logit desc, id asc)
 // ---------------------------------------------------------------------------

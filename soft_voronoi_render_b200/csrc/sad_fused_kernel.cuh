@@ -402,10 +402,10 @@ __device__ __forceinline__ void offer_global(Top8L &t, uint32_t id, const float4
                                              float fx, float fy) {
     if (id >= N) return;
     if (t.has(id)) return;
-    const float4 r0 = __ldg(rec + (size_t)id * REC_F4);
-    if (!(r0.x >= 0.0f)) return;
-    const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
-    const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+    float px, py, A, B, C, b;
+    load_rank_fields(rec, id, px, py, A, B, C, b);
+    if (!(px >= 0.0f)) return;
+    const float l = sad_logit(px, py, A, B, C, b, fx, fy);
     if (l != l) return;
     if (t.beats_last(l, id)) t.insert(l, id, NOLOC);
 }
@@ -683,8 +683,7 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
                 r1 = make_float2(sm.urec[1][u].x, sm.urec[1][u].y);
             } else {
                 u = NOLOC;
-                r0 = __ldg(rec + (size_t)id * REC_F4);
-                r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
+                load_rank_fields(rec, id, r0.x, r0.y, r0.z, r0.w, r1.x, r1.y);
             }
             if (!(r0.x >= 0.0f)) continue;
             t.l[q] = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
@@ -797,20 +796,17 @@ __global__ void __launch_bounds__(FX * FY, 1024 / (FX * FY))
 #pragma unroll 1
             for (int g = 0; g < G; g += 2) {
                 uint32_t id[2];
-                float4 r0[2];
-                float2 r1[2];
+                float px[2], py[2], A[2], B[2], C[2], b[2];
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     if (g + x < G) h = xorshift32(h);
                     id[x] = g + x < G ? __umulhi(h, Nu) : EMPTY;  // < N when drawn
-                    const size_t rr = (size_t)(id[x] < Nu ? id[x] : 0u) * REC_F4;
-                    r0[x] = __ldg(rec + rr);
-                    r1[x] = __ldg(reinterpret_cast<const float2 *>(rec + rr + 1));
+                    load_rank_fields(rec, id[x] < Nu ? id[x] : 0u, px[x], py[x], A[x], B[x], C[x], b[x]);
                 }
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    const float l = sad_logit(r0[x].x, r0[x].y, r0[x].z, r0[x].w, r1[x].x, r1[x].y, fx, fy);
-                    if (id[x] < Nu && r0[x].x >= 0.0f && l == l && t.beats_last(l, id[x]) && !t.has(id[x])) {
+                    const float l = sad_logit(px[x], py[x], A[x], B[x], C[x], b[x], fx, fy);
+                    if (id[x] < Nu && px[x] >= 0.0f && l == l && t.beats_last(l, id[x]) && !t.has(id[x])) {
                         // a winner the tile index holds keeps its local index
                         const uint32_t u = fast ? ukey_lookup(sm.keys, sm.lid, id[x]) : NOLOC;
                         t.insert(l, id[x], u < ucount ? u : NOLOC);

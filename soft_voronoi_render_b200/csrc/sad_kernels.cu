@@ -267,10 +267,10 @@ __device__ __forceinline__ float cand_logit(const float4 *__restrict__ rec, cons
         active = px >= 0.0f;
         return sad_logit(px, py, ab.x, ab.y, cb.x, cb.y, fx, fy);
     } else {
-        const float4 r0 = __ldg(rec + (size_t)x * REC_F4);
-        const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)x * REC_F4 + 1));
-        active = r0.x >= 0.0f;
-        return sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+        float px, py, A, B, C, b;
+        load_rank_fields(rec, x, px, py, A, B, C, b);
+        active = px >= 0.0f;
+        return sad_logit(px, py, A, B, C, b, fx, fy);
     }
 }
 
@@ -302,9 +302,9 @@ __device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], 
                         li[q] = sad_logit(__uint_as_float(v.x), __uint_as_float(v.y), ab.x, ab.y, cb.x, cb.y, fx, fy);
                     }
                 } else {
-                    const float4 r0 = __ldg(rec + (size_t)x * REC_F4);
-                    const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)x * REC_F4 + 1));
-                    if (r0.x >= 0.0f) li[q] = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+                    float px, py, A, B, C, b;
+                    load_rank_fields(rec, x, px, py, A, B, C, b);
+                    if (px >= 0.0f) li[q] = sad_logit(px, py, A, B, C, b, fx, fy);
                 }
             }
         }
@@ -607,10 +607,10 @@ __device__ __forceinline__ int pixel_softmax(const uint4 a, const uint4 b, const
             dropped += (id != EMPTY);
             continue;
         }
-        const float4 r0 = __ldg(rec + (size_t)id * REC_F4);
-        if (!(r0.x >= 0.0f)) continue;
-        const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
-        const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
+        float px, py, A, B, C, b;
+        load_rank_fields(rec, id, px, py, A, B, C, b);
+        if (!(px >= 0.0f)) continue;
+        const float l = sad_logit(px, py, A, B, C, b, fx, fy);
         if (!isfinite(l)) continue;
         s.l[q] = l;
         s.valid |= 1u << q;

@@ -41,7 +41,7 @@ extern "C" int sad_backward_noalloc(int H, int W, int N_cap, const float *record
                                     sad_stream_t stream) {
     if (H < 1 || W < 1 || N_cap < 1 || (long long)H * W >= (1ll << 31)) return SAD_ERR_INVALID_ARG;
     if (!records || !table || !target || !grads || !loss) return SAD_ERR_INVALID_ARG;
-    if (!aligned(records, 16) || !aligned(table, 16) || !aligned(target, 16) || !aligned(grads, 16) ||
+    if (!aligned(records, 32) || !aligned(table, 16) || !aligned(target, 16) || !aligned(grads, 16) ||
         (image && !aligned(image, 16)) || !aligned(loss, 8))
         return SAD_ERR_INVALID_ARG;
     const size_t tiles = (size_t)((W + kTileX - 1) / kTileX) * (size_t)((H + kTileY - 1) / kTileY);

@@ -70,6 +70,10 @@ def test_bind_checks_alignment_and_sizes_without_touching_memory():
         with pytest.raises(_lib.SadError) as e:
             _lib.sad_bind(ctx, **{**fake, "records": 0x50004})
         assert e.value.status == _lib.SAD_ERR_INVALID_ARG and "aligned" in str(e.value)
+        # records are read in 32-byte loads: 16-byte alignment is not enough
+        with pytest.raises(_lib.SadError) as e:
+            _lib.sad_bind(ctx, **{**fake, "records": 0x50010})
+        assert e.value.status == _lib.SAD_ERR_INVALID_ARG and "32-byte" in str(e.value)
         with pytest.raises(_lib.SadError) as e:
             _lib.sad_bind(ctx, **{**fake, "target": None})
         assert e.value.status == _lib.SAD_ERR_INVALID_ARG
@@ -179,4 +183,7 @@ def test_backward_noalloc_rejects_sizes_before_any_cuda_call():
         assert e.value.status == want, (H, W)
     with pytest.raises(_lib.SadError) as e:
         _lib.sad_backward_noalloc(64, 64, 16, 0x10004, *fake[1:])  # misaligned records
+    assert e.value.status == _lib.SAD_ERR_INVALID_ARG
+    with pytest.raises(_lib.SadError) as e:
+        _lib.sad_backward_noalloc(64, 64, 16, 0x10010, *fake[1:])  # records 16- but not 32-byte aligned
     assert e.value.status == _lib.SAD_ERR_INVALID_ARG
