@@ -607,10 +607,12 @@ __device__ __forceinline__ int pixel_softmax(const uint4 a, const uint4 b, const
             dropped += (id != EMPTY);
             continue;
         }
-        float px, py, A, B, C, b;
-        load_rank_fields(rec, id, px, py, A, B, C, b);
-        if (!(px >= 0.0f)) continue;
-        const float l = sad_logit(px, py, A, B, C, b, fx, fy);
+        // two loads, the second only for an active site: one 32-byte load
+        // per slot raised this kernel from 40 to 63 registers and slowed it
+        const float4 r0 = __ldg(rec + (size_t)id * REC_F4);
+        if (!(r0.x >= 0.0f)) continue;
+        const float2 r1 = __ldg(reinterpret_cast<const float2 *>(rec + (size_t)id * REC_F4 + 1));
+        const float l = sad_logit(r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, fx, fy);
         if (!isfinite(l)) continue;
         s.l[q] = l;
         s.valid |= 1u << q;
