@@ -140,13 +140,14 @@ __device__ __forceinline__ uint32_t inject_state(uint32_t seed, uint32_t pass, u
 // ---------------------------------------------------------------------------
 // per-thread top-8 list kept in registers
 // ---------------------------------------------------------------------------
-struct Top8 {
-    float l[K];
-    uint32_t id[K];
+template <int KN>
+struct TopN {
+    float l[KN];
+    uint32_t id[KN];
 
     __device__ __forceinline__ void clear() {
 #pragma unroll
-        for (int q = 0; q < K; ++q) {
+        for (int q = 0; q < KN; ++q) {
             l[q] = -__int_as_float(0x7f800000);  // -inf
             id[q] = EMPTY;
         }
@@ -154,13 +155,13 @@ struct Top8 {
     __device__ __forceinline__ bool has(uint32_t x) const {
         bool h = false;
 #pragma unroll
-        for (int q = 0; q < K; ++q) h |= (id[q] == x);
+        for (int q = 0; q < KN; ++q) h |= (id[q] == x);
         return h;
     }
     // insert a candidate known not to be in the list (bubble network)
     __device__ __forceinline__ void insert(float lv, uint32_t iv) {
 #pragma unroll
-        for (int q = 0; q < K; ++q) {
+        for (int q = 0; q < KN; ++q) {
             const bool a = ranks_above(lv, iv, l[q], id[q]);
             const float tl = a ? l[q] : lv;
             const uint32_t ti = a ? id[q] : iv;
@@ -171,9 +172,10 @@ struct Top8 {
         }
     }
     __device__ __forceinline__ bool beats_last(float lv, uint32_t iv) const {
-        return ranks_above(lv, iv, l[K - 1], id[K - 1]);
+        return ranks_above(lv, iv, l[KN - 1], id[KN - 1]);
     }
 };
+using Top8 = TopN<K>;
 
 // Sum v[0..NV-1] over each maximal run of lanes holding the same key (runs in
 // lane order; a warp covers 32 consecutive pixels of a row, and neighbouring

@@ -279,12 +279,12 @@ __device__ __forceinline__ float cand_logit(const float4 *__restrict__ rec, cons
 // >= N, inactive site, NaN logit, an id already held or repeated earlier in
 // the batch) become (-inf, EMPTY), which ranks below every candidate, and the
 // batch is sorted and merged; the network is skipped when no active lane has
-// a candidate that beats its 8th.  Without merge the candidates that beat
-// the 8th are inserted one by one: the JFA prepass keeps 4 entries and takes
-// few new ones per pass, and its kernel stays at 48 registers (5 blocks per
-// SM) without the network.
-template <int NB, bool F16, bool MERGE>
-__device__ __forceinline__ void offer_batch(Top8 &t, const uint32_t (&ids)[NB], const float4 *__restrict__ rec,
+// a candidate that beats its last entry.  Without merge the candidates that
+// beat the last entry are inserted one by one: the JFA prepass keeps 4
+// entries (KN = 4) and takes few new ones per pass, and its kernel fits 40
+// registers (6 blocks per SM) without the network.
+template <int NB, bool F16, bool MERGE, int KN = K>
+__device__ __forceinline__ void offer_batch(TopN<KN> &t, const uint32_t (&ids)[NB], const float4 *__restrict__ rec,
                                             const uint4 *__restrict__ c16, uint32_t N, float fx, float fy) {
     if constexpr (!MERGE) {
         float li[NB];
@@ -520,17 +520,19 @@ __global__ void __launch_bounds__(SITE_THREADS) pack_cand16_kernel(const float4 
 
 // One 3x3 flood pass of the optional JFA prepass (summary B.3): the 4 best
 // distinct candidates of the lists at (i + a k, j + b k), a, b in {-1, 0, 1},
-// go to slots 0-3; slots 4-7 are emptied.  LC as in propagate_kernel: 1 =
-// store the new lists' scores in lcache, 2 = also start from the own list's
-// stored scores (its 4 entries, in order) and offer only the 8 neighbours.
+// go to slots 0-3; slots 4-7 are emptied.  The prepass starts from the seed
+// pass, which leaves slots 1-7 empty, and every flood pass empties slots 4-7,
+// so a pass reads only the first plane (slots 0-3) of each list and keeps a
+// running top 4.  LC as in propagate_kernel: 1 = store the new lists' scores
+// in lcache, 2 = also start from the own list's stored scores (its 4
+// entries, in order) and offer only the 8 neighbours.
 template <int LC = 0>
-__global__ void __launch_bounds__(TILE_THREADS, 5) jfa3x3_kernel(const float4 *__restrict__ rec, uint32_t *table,
+__global__ void __launch_bounds__(TILE_THREADS, 6) jfa3x3_kernel(const float4 *__restrict__ rec, uint32_t *table,
                                                               int H, int W, float cs, int N, int jump, Counters *c,
                                                               float4 *__restrict__ lcache) {
     const uint32_t cur = c->cur, pass = c->pass_counter;
     const size_t P = (size_t)H * W;
     const uint4 *in0 = reinterpret_cast<const uint4 *>(table + cur * P * K);
-    const uint4 *in1 = in0 + P;
     uint4 *out0 = reinterpret_cast<uint4 *>(table + (cur ^ 1u) * P * K);
     uint4 *out1 = out0 + P;
     const int i = blockIdx.x * TILE_X + threadIdx.x;
@@ -538,7 +540,7 @@ __global__ void __launch_bounds__(TILE_THREADS, 5) jfa3x3_kernel(const float4 *_
     if (i < W && j < H) {
         const size_t p = (size_t)j * W + i;
         const float fx = ((float)i + 0.5f) * cs, fy = ((float)j + 0.5f) * cs;
-        Top8 t;
+        TopN<4> t;
         t.clear();
         if constexpr (LC == 2) {
             // the own list is the previous pass's top 4, sorted and distinct
@@ -559,9 +561,9 @@ __global__ void __launch_bounds__(TILE_THREADS, 5) jfa3x3_kernel(const float4 *_
             const int ni = i + (d % 3 - 1) * jump, nj = j + (d / 3 - 1) * jump;
             if (ni < 0 || ni >= W || nj < 0 || nj >= H) continue;
             const size_t pn = (size_t)nj * W + ni;
-            const uint4 a = in0[pn], b = in1[pn];
-            const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            offer_batch<8, false, false>(t, ids, rec, nullptr, (uint32_t)N, fx, fy);
+            const uint4 a = in0[pn];
+            const uint32_t ids[4] = {a.x, a.y, a.z, a.w};
+            offer_batch<4, false, false, 4>(t, ids, rec, nullptr, (uint32_t)N, fx, fy);
         }
         out0[p] = make_uint4(t.id[0], t.id[1], t.id[2], t.id[3]);
         out1[p] = make_uint4(EMPTY, EMPTY, EMPTY, EMPTY);
