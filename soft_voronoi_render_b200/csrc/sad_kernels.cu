@@ -281,8 +281,9 @@ __device__ __forceinline__ float cand_logit(const float4 *__restrict__ rec, cons
 // batch is sorted and merged; the network is skipped when no active lane has
 // a candidate that beats its last entry.  Without merge the candidates that
 // beat the last entry are inserted one by one: the JFA prepass keeps 4
-// entries (KN = 4) and takes few new ones per pass, and its kernel fits 40
-// registers (6 blocks per SM) without the network.
+// entries (KN = 4) and takes few new ones per pass; without the network its
+// kernel runs at 32 registers, 8 blocks per SM (a few bytes spill; measured
+// faster than 40 registers at 6 blocks and 47 at 5).
 template <int NB, bool F16, bool MERGE, int KN = K>
 __device__ __forceinline__ void offer_batch(TopN<KN> &t, const uint32_t (&ids)[NB], const float4 *__restrict__ rec,
                                             const uint4 *__restrict__ c16, uint32_t N, float fx, float fy) {
@@ -527,7 +528,7 @@ __global__ void __launch_bounds__(SITE_THREADS) pack_cand16_kernel(const float4 
 // in lcache, 2 = also start from the own list's stored scores (its 4
 // entries, in order) and offer only the 8 neighbours.
 template <int LC = 0>
-__global__ void __launch_bounds__(TILE_THREADS, 6) jfa3x3_kernel(const float4 *__restrict__ rec, uint32_t *table,
+__global__ void __launch_bounds__(TILE_THREADS, 8) jfa3x3_kernel(const float4 *__restrict__ rec, uint32_t *table,
                                                               int H, int W, float cs, int N, int jump, Counters *c,
                                                               float4 *__restrict__ lcache) {
     const uint32_t cur = c->cur, pass = c->pass_counter;
