@@ -449,7 +449,21 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
             const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
             offer_batch<8, F16, MERGE>(t, ids, rec, c16, (uint32_t)N, fx, fy);
         }
-        if (G > 0) {
+        if (G > 0 && G <= 4) {
+            // up to four injections: a half batch (no empty slots to check)
+            uint32_t h = inject_state(seed, pass, (uint32_t)p);
+            uint32_t ids[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (q < G) {
+                    h = xorshift32(h);
+                    ids[q] = __umulhi(h, (uint32_t)N);
+                } else {
+                    ids[q] = EMPTY;
+                }
+            }
+            offer_batch<4, F16, MERGE>(t, ids, rec, c16, (uint32_t)N, fx, fy);
+        } else if (G > 0) {
             uint32_t h = inject_state(seed, pass, (uint32_t)p);
 #pragma unroll 1
             for (int g0 = 0; g0 < G; g0 += 8) {
