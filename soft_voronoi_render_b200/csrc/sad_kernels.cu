@@ -283,8 +283,10 @@ __device__ __forceinline__ float cand_logit(const float4 *__restrict__ rec, cons
 // beat the last entry are inserted one by one: the JFA prepass keeps 4
 // entries (KN = 4) and takes few new ones per pass; without the network its
 // kernel runs at 32 registers, 8 blocks per SM (a few bytes spill; measured
-// faster than 40 registers at 6 blocks and 47 at 5).
-template <int NB, bool F16, bool MERGE, int KN = K>
+// faster than 40 registers at 6 blocks and 47 at 5).  DISTINCT: the batch
+// is known to hold no id twice (a list this library wrote), so the merge
+// skips the check of each id against the batch's earlier ones.
+template <int NB, bool F16, bool MERGE, int KN = K, bool DISTINCT = false>
 __device__ __forceinline__ void offer_batch(TopN<KN> &t, const uint32_t (&ids)[NB], const float4 *__restrict__ rec,
                                             const uint4 *__restrict__ c16, uint32_t N, float fx, float fy) {
     if constexpr (!MERGE) {
@@ -324,8 +326,10 @@ __device__ __forceinline__ void offer_batch(TopN<KN> &t, const uint32_t (&ids)[N
         if (q < NB) {
             const uint32_t x = ids[q];
             bool fresh = x < N && !t.has(x);
+            if constexpr (!DISTINCT) {
 #pragma unroll
-            for (int r = 0; r < q; ++r) fresh &= x != ids[r];
+                for (int r = 0; r < q; ++r) fresh &= x != ids[r];
+            }
             if (fresh) {
                 bool active;
                 const float lv = cand_logit<F16>(rec, c16, x, fx, fy, active);
@@ -366,6 +370,11 @@ __device__ __forceinline__ void take_own_list(Top8 &t, const uint4 a, const uint
             t.l[q] = v ? ls[q] : -__int_as_float(0x7f800000);
             t.id[q] = v ? ids[q] : EMPTY;
         }
+        // float32 ranking: the previous pass wrote this list, sorted and
+        // repeat-free, with these very scores (its empty slots, stored as
+        // -inf, at the end).  F16 stored it in float32 order beside the
+        // packed-record scores it ranks by, so it goes on to the check.
+        if constexpr (!F16) return;
     } else {
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -447,7 +456,9 @@ __global__ void __launch_bounds__(TILE_THREADS) propagate_kernel(const float4 *_
                 b = in1[pn];
             }
             const uint32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            offer_batch<8, F16, MERGE>(t, ids, rec, c16, (uint32_t)N, fx, fy);
+            // in a refresh (LC > 0) every list was written by the seed pass
+            // or by a pass of this kernel, so it holds no id twice
+            offer_batch<8, F16, MERGE, K, (LC > 0)>(t, ids, rec, c16, (uint32_t)N, fx, fy);
         }
         if (G > 0 && G <= 4) {
             // up to four injections: a half batch (no empty slots to check)

@@ -496,6 +496,11 @@ def test_propagate_equals_union_top8(orc, jump, G):
     tout = orc.propagate(H, W, rec, tin, jump, G, seed=77, pass_index=5)
     ref = _union_top8_reference(orc, H, W, rec, tin, jump, G, 77, 5)
     np.testing.assert_array_equal(tout, ref)
+    # a pass's lists hold no id twice, whatever its input held (the refresh's
+    # later passes rely on it: they read only lists written by a pass)
+    for row in tout:
+        v = row[row != SENT]
+        assert v.size == np.unique(v).size
 
 
 def test_propagate_with_rich_injection_converges_to_exact(orc):
