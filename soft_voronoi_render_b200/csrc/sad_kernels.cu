@@ -745,9 +745,15 @@ __global__ void __launch_bounds__(SITE_THREADS, 4) adam_kernel(float *__restrict
     const int i = blockIdx.x * SITE_THREADS + threadIdx.x;
     if (i < N) {
         const size_t n = (size_t)N;
-        float v[NPARAM];
+        // every load issued before the first use: one memory round trip
+        float v[NPARAM], gk[NPARAM], m1k[NPARAM], m2k[NPARAM];
 #pragma unroll
-        for (int k = 0; k < NPARAM; ++k) v[k] = prm[k * n + i];
+        for (int k = 0; k < NPARAM; ++k) {
+            v[k] = prm[k * n + i];
+            gk[k] = grads[k * n + i];
+            m1k[k] = m1[k * n + i];
+            m2k[k] = m2[k * n + i];
+        }
         // frozen sites keep their parameters (summary section 7)
         if (v[PX] >= 0.0f && !(frozen && frozen[i])) {
             // bias corrections 1 - beta^t, every thread its own (no barrier),
@@ -758,9 +764,9 @@ __global__ void __launch_bounds__(SITE_THREADS, 4) adam_kernel(float *__restrict
 #pragma unroll
             for (int k = 0; k < NPARAM; ++k) {
                 const float sig = (k == PX || k == PY || k == PR) ? sig_pos : 1.0f;
-                const float gh = grads[k * n + i] * sig;
-                const float mk = a.beta1 * m1[k * n + i] + (1.0f - a.beta1) * gh;
-                const float vk = a.beta2 * m2[k * n + i] + (1.0f - a.beta2) * gh * gh;
+                const float gh = gk[k] * sig;
+                const float mk = a.beta1 * m1k[k] + (1.0f - a.beta1) * gh;
+                const float vk = a.beta2 * m2k[k] + (1.0f - a.beta2) * gh * gh;
                 m1[k * n + i] = mk;
                 m2[k * n + i] = vk;
                 const float mh = mk * ibc1, vh = vk * ibc2;
