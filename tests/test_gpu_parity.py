@@ -123,6 +123,30 @@ def test_render_fixed_table_c1(torch_cuda):
     assert np.abs(img - ref).max() <= RENDER_ATOL
 
 
+def test_render_unsorted_table(torch_cuda):
+    """The render of lists in no particular order (random ids with repeats,
+    empty slots, ids beyond the capacity, an inactive site) agrees with the
+    oracle's."""
+    H, W, N = 40, 72, 500
+    prm = synth.uniform_sites(H, W, N, 12)
+    prm[0, 7] = -1.0
+    tgt = synth.make_image(H, W, 3, 0, 12)
+    st = synth.Stream(12, "render-unsorted")
+    table = st.integers(H * W * 8, N + 20).astype(np.uint32).reshape(H * W, 8)
+    table[st.uniform(H * W * 8).reshape(H * W, 8) < 0.15] = SENT
+    table[::5, 3] = table[::5, 1]
+    table[11] = SENT
+    s = make_ctx(torch_cuda, H, W, N, prm, tgt)
+    s.set_table(table)
+    img = s.render().cpu().numpy()
+    clean = table.copy()
+    clean[clean >= N] = SENT
+    ref = oracle.render(H, W, prm, clean)
+    assert np.abs(img - ref).max() <= RENDER_ATOL
+    st = s.stats()
+    assert st["empty_pixels"] >= 1 and st["dropped_ids"] >= 1
+
+
 @pytest.mark.parametrize("seed", [1, 2])
 def test_backward_c1(torch_cuda, seed):
     tgt, prm, w = synth.make_workload("c1", seed=seed)
