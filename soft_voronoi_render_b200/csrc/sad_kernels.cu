@@ -15,8 +15,9 @@
 //   jfa3x3_kernel       optional 3x3 flood prepass (summary B.3)
 //   tau_diffuse_kernel  Jacobi step on the ln tau gradients (summary B.6)
 //   target_u8_kernel    8-bit RGB -> planar float32 target
-// The fused steady-state pass (also the float backward) is in sad_fused.cu, budget control in
-// sad_densify.cu, the 16-byte site record in sad_pack.cu.
+// The fused steady-state pass (also the float backward) is in sad_fused_kernel.cuh with its
+// launchers in sad_fused.cu, budget control in sad_densify.cu, the 16-byte site record in
+// sad_pack.cu.
 #include <cuda_fp16.h>
 
 #include "sad_device.cuh"
