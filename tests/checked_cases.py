@@ -12,7 +12,8 @@ other cases take the default form), and once more with every block's first
 staging copy withheld (SAD_TEST_WITHHOLD_STAGING=1, read only by this
 build): each block's bounded wait for the copy runs out, the block reads its
 lists from global memory, the result is the same and staging_fallbacks
-counts one fallback per block.  Prints one JSON line."""
+counts one fallback per block.  Last, the full-size workload runs the
+same kinds of passes with the checks on.  Prints one JSON line."""
 import json
 import os
 import sys
@@ -91,7 +92,38 @@ def main():
         out["cases"] += 1
         out["check_failures"] += st["check_failures"]
         s.close()
+    out["full_size"] = full_size_case()
     print(json.dumps(out), flush=True)
+
+
+def full_size_case():
+    """The 2048 x 2048, N = 131,072 workload in the checked build: a refresh,
+    ten fitting iterations (where crowded tiles take the generic path), the
+    TMA-staged pass, the cached-list, statistics and order-independent
+    passes.  Returns the accesses the device-side checks refused."""
+    from soft_voronoi_render_b200 import (SAD_DETERMINISTIC, SAD_STAGING_LOADS, SAD_STAGING_TMA, SAD_STATS, Sad,
+                                          adam_cfg)
+    tgt, prm, w = synth.make_workload("c3", seed=1)
+    s = Sad(w.H, w.W, w.N, seed=1)
+    s.set_sites(prm)
+    s.set_target(tgt)
+    s.refresh(w.G)
+    cfg = adam_cfg(lr_pos=1e-3, lr_log_tau=1e-3, lr_r=1e-3, lr_color=5e-3, lr_theta=1e-3, lr_a=1e-3)
+    for _ in range(10):
+        s.fit_iteration(w.G, cfg)
+    s.set_list_staging(SAD_STAGING_TMA)
+    s.fit_pass(w.G)
+    s.set_list_staging(SAD_STAGING_LOADS)
+    s.grads.zero_()
+    s.fit_pass_cached()
+    s.grads.zero_()
+    s.backward(SAD_STATS)
+    s.grads.zero_()
+    s.backward(SAD_DETERMINISTIC)
+    st = s.stats()
+    assert st["staging_fallbacks"] == 0 and np.isfinite(s.loss())
+    s.close()
+    return st["check_failures"]
 
 
 if __name__ == "__main__":

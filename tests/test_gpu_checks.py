@@ -27,3 +27,5 @@ def test_checked_build_refuses_no_access():
     # two of the cases take the TMA-staged form (2 and 6 tiles); with their
     # first copies withheld every block fell back to plain loads
     assert res["withheld_fallbacks"] == 8, res
+    # the full-size workload, generic path included, refuses no access either
+    assert res["full_size"] == 0, res
